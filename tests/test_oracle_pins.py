@@ -1,0 +1,432 @@
+"""Pins for the CPU oracle: each check ties an oracle function to something other
+than itself -- values the SAGE paper prints, hand-worked examples, closed forms,
+invariants, library routines (NumPy, SciPy) and brute force on tiny inputs.
+
+Citations refer to "SAGE: Pushing 2-Bit Vector-Quantized LLMs toward Real-World
+Usability" by section / equation.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as fh:
+        return json.load(fh)
+
+
+def _fields(d_out, d_in, log2K, seed=0, **kw):
+    return synth.random_fields(np.random.default_rng(seed), d_out, d_in, log2K, **kw)
+
+
+# ---------------------------------------------------------------------------
+# fp16 conversions (IEEE binary16), pinned to NumPy's float16
+# ---------------------------------------------------------------------------
+
+def test_half_to_double_all_patterns():
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = h.view(np.float16).astype(np.float64)
+    got = oracle.halves_to_double(h)
+    finite = np.isfinite(ref)
+    assert np.array_equal(got[finite], ref[finite])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(np.isinf(got), np.isinf(ref))
+
+
+def test_double_to_half_rne():
+    g = np.random.default_rng(1)
+    xs = np.concatenate([
+        g.standard_normal(20000) * 10.0 ** g.integers(-9, 5, 20000),
+        # exact ties between neighbouring fp16 values (round half to even)
+        (np.arange(0, 2048, dtype=np.float64) + 0.5) * 2.0 ** -10,
+        (np.arange(1024, 2048, dtype=np.float64) + 0.5) * 2.0 ** -24,
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e-9, -2.0 ** -25, 2.0 ** -25 * 1.0000001],
+    ])
+    with np.errstate(over="ignore"):
+        ref = xs.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.double_to_half(v) for v in xs], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------------------
+# Bit budget (Sec. 1, Sec. 3.1 Eq. 3, Sec. 3.3 Eq. 7, App. A.6 Eq. 15)
+# ---------------------------------------------------------------------------
+
+def test_budget_printed_values():
+    gb = _gold("budget.json")
+    ex = gb["example_split"]
+    assert ex["signs"] + ex["index_bits"] + ex["radius_bits"] == gb["bits_per_subvector"]
+    for K, V in list(synth.SPLITS) + [tuple(c) for c in gb["eq7_candidates"]]:
+        assert int(np.log2(K)) + V == gb["eq7_index_plus_radius_bits"]
+        assert 8 + int(np.log2(K)) + V == gb["bits_per_subvector"]
+    N = 4096 * 4096
+    # codebook term excluded (b_c = 0): payload + fp16 grid
+    assert oracle.bpw(8, 18, 128, 0, 64, 16, N) == pytest.approx(gb["payload_bpw"] + 0.0, abs=1e-3)
+    assert oracle.bpw(8, 18, 128, 0, 64, 0, N) == pytest.approx(gb["payload_bpw"])
+    assert oracle.bpw(8, 18, 128, 16, 64, 0, N) == pytest.approx(gb["subtotal_bpw_before_codebook"])
+    assert oracle.bpw(8, 18, 128, 16, 64, 0, N) - oracle.bpw(8, 18, 128, 0, 64, 0, N) == \
+        pytest.approx(gb["fp16_grid_extra_bpw_at_G128"])
+    # the codebook term: K v b_c bits for N weights; 64 fp16 codewords are 1 KiB
+    cb_bits = (oracle.bpw(8, 18, 128, 16, 64, 16, N) - oracle.bpw(8, 18, 128, 16, 64, 0, N)) * N
+    assert cb_bits / 8 == pytest.approx(gb["codebook_K64_fp16_bytes"])
+    assert gb["group_size_G"] // 8 == gb["subvectors_per_group"]
+
+
+# ---------------------------------------------------------------------------
+# Packed layout v1 (the library's own format)
+# ---------------------------------------------------------------------------
+
+def test_unpack_hand_example():
+    gx = _gold("format_v1_example.json")
+    main = np.zeros(gx["main_words"], np.uint32)
+    meta = np.zeros(gx["meta_words"], np.uint32)
+    for k, v in gx["main_nonzero"].items():
+        main[int(k)] = int(v, 16)
+    for k, v in gx["meta_nonzero"].items():
+        meta[int(k)] = int(v, 16)
+    f = oracle.unpack_v1(gx["d_out"], gx["d_in"], gx["log2K"], main, meta)
+    exp = {k: np.zeros_like(v) for k, v in f.items()}
+    for e in gx["fields_nonzero"]:
+        exp["signs"][e["row"], e["j"]] = e["signs"]
+        exp["idx"][e["row"], e["j"]] = e["idx"]
+        exp["q"][e["row"], e["j"]] = e["q"]
+    for e in gx["grid_nonzero"]:
+        exp["mu"][e["row"], e["g"]] = int(e["mu"], 16)
+        exp["delta"][e["row"], e["g"]] = int(e["delta"], 16)
+    for k in f:
+        assert np.array_equal(f[k], exp[k]), k
+
+
+@pytest.mark.parametrize("log2K", [4, 5, 6, 7, 8])
+def test_unpack_is_a_bijection(log2K):
+    """Every packed bit of a (record, meta entry) maps to exactly one field bit and
+    every field bit is reached: flipping one packed bit changes one field bit."""
+    d_out, d_in = 16, 128
+    R8, S, G = 2, 16, 1
+    V = 10 - log2K
+    nmain, nmeta = S * R8 * 4, G * R8 * 8 * 2
+    base = oracle.unpack_v1(d_out, d_in, log2K, np.zeros(nmain, np.uint32), np.zeros(nmeta, np.uint32))
+    for k in base:
+        assert not base[k].any()
+    hit = set()
+
+    def field_bits(f):
+        bits = set()
+        for name, w in (("signs", 8), ("idx", log2K), ("q", V), ("mu", 16), ("delta", 16)):
+            a = f[name].astype(np.uint32)
+            for pos in zip(*np.nonzero(a)):
+                for b in range(w):
+                    if (int(a[pos]) >> b) & 1:
+                        bits.add((name, pos, b))
+        return bits
+
+    # main record (j=3, b=1) and meta entry (g=0, b=1)
+    for word in range(4):
+        for bit in range(32):
+            main = np.zeros(nmain, np.uint32)
+            main[(3 * R8 + 1) * 4 + word] = np.uint32(1 << bit)
+            fb = field_bits(oracle.unpack_v1(d_out, d_in, log2K, main, np.zeros(nmeta, np.uint32)))
+            assert len(fb) == 1, (word, bit, fb)
+            hit |= fb
+    for word in range(16):
+        for bit in range(32):
+            meta = np.zeros(nmeta, np.uint32)
+            meta[(1 * 8) * 2 + word] = np.uint32(1 << bit)
+            fb = field_bits(oracle.unpack_v1(d_out, d_in, log2K, np.zeros(nmain, np.uint32), meta))
+            assert len(fb) <= 1, (word, bit, fb)
+            hit |= fb
+    # 8 rows x (18 bits of subvector j=3) + 8 rows x 16 aux bits (only j=3's 2 counted) + grid
+    sv_bits = {h for h in hit if h[0] in ("signs", "idx", "q") and h[1][1] == 3}
+    assert len(sv_bits) == 8 * 18
+    grid_bits = {h for h in hit if h[0] in ("mu", "delta")}
+    assert len(grid_bits) == 8 * 32
+
+
+def test_unpack_all_ones():
+    for log2K in range(4, 9):
+        V = 10 - log2K
+        d_out, d_in = 8, 256
+        f = oracle.unpack_v1(d_out, d_in, log2K, np.full(32 * 4, 0xFFFFFFFF, np.uint32),
+                             np.full(2 * 8 * 2, 0xFFFFFFFF, np.uint32))
+        assert (f["signs"] == 255).all() and (f["idx"] == (1 << log2K) - 1).all()
+        assert (f["q"] == (1 << V) - 1).all()
+        assert (f["mu"] == 0xFFFF).all() and (f["delta"] == 0xFFFF).all()
+
+
+# ---------------------------------------------------------------------------
+# Reconstruction (Sec. 3.1 Eq. 1-2)
+# ---------------------------------------------------------------------------
+
+def _r_hat(f):
+    mu = f.mu.view(np.float16).astype(np.float64)
+    de = f.delta.view(np.float16).astype(np.float64)
+    g = np.arange(f.d_in // 8) // 16
+    return mu[:, g] + f.q.astype(np.float64) * de[:, g]
+
+
+def test_dequant_hand_value():
+    # mu = 0.125, delta = 2^-7, q = 14 -> r = 0.234375; c = 0.5; negative sign
+    f = _fields(1, 128, 4, seed=3)
+    f.mu[:] = 0x3000
+    f.delta[:] = 0x2000
+    f.q[:] = 14
+    f.idx[:] = 0
+    f.signs[:] = 0
+    f.signs[0, 0] = 0b00000100
+    f.codebook[0, :] = 0x3800
+    W = oracle.dequant(f)
+    assert W[0, 2] == -0.1171875
+    assert W[0, 3] == 0.1171875
+
+
+@pytest.mark.parametrize("log2K", [4, 6, 8])
+def test_dequant_norm_equals_radius(log2K):
+    """||w_hat|| = r_hat ||c_z|| for each subvector (signs do not change the norm),
+    and the generated unit codewords have ||c|| within 2^-10 of 1 (fp16 rounding)."""
+    f = _fields(24, 256, log2K, seed=log2K)
+    W = oracle.dequant(f).reshape(24, 32, 8)
+    cb = f.codebook.view(np.float16).astype(np.float64)
+    cnorm = np.sqrt((cb * cb).sum(1))
+    assert np.all(np.abs(cnorm - 1.0) <= 2.0 ** -10)
+    got = np.sqrt((W * W).sum(2))
+    exp = _r_hat(f) * cnorm[f.idx]
+    assert np.allclose(got, exp, rtol=1e-15, atol=0)
+    # magnitudes do not depend on the sign byte, and each sign bit flips one component
+    f2 = synth.Fields(**{**f.__dict__, "signs": f.signs ^ np.uint8(0xFF)})
+    W2 = oracle.dequant(f2).reshape(24, 32, 8)
+    assert np.array_equal(W2, -W)
+
+
+def test_dequant_zero_step_gives_common_radius():
+    """App. A.6: if all radii in a group coincide the reconstruction is their common
+    value; with delta = 0 every q decodes to mu."""
+    f = _fields(4, 256, 5, seed=7)
+    f.delta[:, 1] = 0
+    W = oracle.dequant(f).reshape(4, 32, 8)
+    mu = f.mu.view(np.float16).astype(np.float64)
+    cb = f.codebook.view(np.float16).astype(np.float64)
+    for o in range(4):
+        for j in range(16, 32):
+            assert np.linalg.norm(W[o, j]) == pytest.approx(mu[o, 1] * np.linalg.norm(cb[f.idx[o, j]]), rel=1e-15)
+
+
+def test_dequant_single_codeword_closed_form():
+    f = _fields(3, 128, 4, seed=11)
+    f.codebook[:] = 0
+    f.codebook[:, 0] = 0x3C00  # e_0 for every codeword
+    W = oracle.dequant(f).reshape(3, 16, 8)
+    s0 = np.where(f.signs & 1, -1.0, 1.0)
+    assert np.array_equal(W[:, :, 0], s0 * _r_hat(f))
+    assert not W[:, :, 1:].any()
+
+
+# ---------------------------------------------------------------------------
+# GEMV: y = W_hat x_perm (fp64), pinned to NumPy matmul and special cases
+# ---------------------------------------------------------------------------
+
+def test_gemv_matches_numpy_matmul():
+    f = _fields(40, 384, 7, seed=5)
+    f.perm = np.random.default_rng(9).permutation(384).astype(np.int32)
+    x = synth.activations(np.random.default_rng(10), 3, 384)
+    y, b = oracle.gemv(f, x)
+    W32 = oracle.dequant(f).astype(np.float32).astype(np.float64)
+    xp = x.view(np.float16).astype(np.float64)[:, f.perm]
+    assert np.allclose(y, xp @ W32.T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(b, np.abs(xp) @ np.abs(W32).T, rtol=1e-12)
+    assert np.all(np.abs(y) <= b * (1 + 1e-12))
+    # dense entry point agrees with the fields entry point
+    y2, b2 = oracle.gemv_dense(oracle.dequant(f), x, f.perm)
+    assert np.array_equal(y, y2) and np.array_equal(b, b2)
+    # row-subset evaluation agrees
+    y3, _ = oracle.gemv(f, x, rows=(7, 19))
+    assert np.array_equal(y3[:, 7:19], y[:, 7:19])
+
+
+def test_gemv_permutation_direction():
+    """Sec. 3.2/3.5: weights are stored in permuted column order and inference applies
+    the permutation to the activations, x_perm[p] = x[perm[p]].  A one-hot input on
+    original channel c selects the stored column p with perm[p] = c."""
+    f = _fields(16, 128, 6, seed=2)
+    f.perm = np.random.default_rng(4).permutation(128).astype(np.int32)
+    W = oracle.dequant(f)
+    for c in (0, 17, 127):
+        x = np.zeros((1, 128), np.float64)
+        x[0, c] = 1.0
+        y, _ = oracle.gemv(f, synth.f16_bits(x))
+        p = int(np.nonzero(f.perm == c)[0][0])
+        assert np.array_equal(y[0], W[:, p].astype(np.float32).astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# Encoder steps (Sec. 3.2-3.3, App. A.6)
+# ---------------------------------------------------------------------------
+
+def test_esg_hand_examples():
+    for case in _gold("esg_tiny.json")["cases"]:
+        assert oracle.esg_perm(np.array(case["energy"], float)).tolist() == case["perm"], case["name"]
+
+
+@pytest.mark.parametrize("d_in", [128, 2560, 9728])
+def test_esg_invariants(d_in):
+    e = np.random.default_rng(d_in).lognormal(0, 1.5, d_in)
+    perm = oracle.esg_perm(e)
+    assert sorted(perm.tolist()) == list(range(d_in))
+    m = d_in // 8
+    rank = np.empty(d_in, int)
+    rank[np.argsort(-e, kind="stable")] = np.arange(d_in)
+    P = perm.reshape(m, 8)
+    # position t of every subvector holds a channel of tier t (ranks [t m, (t+1) m))
+    assert np.all(rank[P] // m == np.arange(8)[None, :])
+    # energies decrease along the 8 positions of each subvector
+    assert np.all(np.diff(e[P], axis=1) <= 0)
+
+
+def test_omega_properties():
+    """Eq. 4: weights normalised to unit mean; equal energies give omega = 1."""
+    assert np.allclose(oracle.omega(np.full(8, 3.7), 0.75), 1.0, rtol=0, atol=1e-15)
+    g = np.random.default_rng(3)
+    for _ in range(20):
+        e = g.lognormal(0, 1.5, 8)
+        w = oracle.omega(e, 0.75)
+        assert w.mean() == pytest.approx(1.0, rel=1e-14)
+        assert np.allclose(w / w[0], (e / e[0]) ** 0.75, rtol=1e-12)
+        assert np.array_equal(np.argsort(w, kind="stable"), np.argsort(e, kind="stable"))
+
+
+def _unit_cb(g, K):
+    c = np.abs(g.standard_normal((K, 8)))
+    return c / np.linalg.norm(c, axis=1, keepdims=True)
+
+
+def test_assign_uniform_weights_is_cosine_rule():
+    """Sec. 3.1 / 3.2: with omega = 1 the assignment reduces to argmax_k d^T c_k and
+    the radius to r~ = |w|^T c_z."""
+    g = np.random.default_rng(5)
+    cb = _unit_cb(g, 16)
+    for _ in range(200):
+        p = np.abs(g.standard_normal(8))
+        z, r = oracle.assign(p, np.ones(8), cb)
+        d = p / np.linalg.norm(p)
+        assert z == int(np.argmax(cb @ d))
+        assert r == pytest.approx(float(p @ cb[z]), rel=1e-12)
+
+
+def test_error_decomposition_and_min_residual():
+    """App. A.6 Eq. 11: ||p - r c||^2 = ||p||^2 - (p^T c)^2 + (r - p^T c)^2 for unit c;
+    so the smallest continuous-radius residual is the largest cosine (both >= 0)."""
+    g = np.random.default_rng(6)
+    cb = _unit_cb(g, 32)
+    for _ in range(100):
+        p = np.abs(g.standard_normal(8))
+        r = g.uniform(0, 3)
+        c = cb[g.integers(32)]
+        lhs = np.sum((p - r * c) ** 2)
+        rhs = p @ p - (p @ c) ** 2 + (r - p @ c) ** 2
+        assert lhs == pytest.approx(rhs, rel=1e-12, abs=1e-12)
+        z, _ = oracle.assign(p, np.ones(8), cb)
+        resid = [np.sum((p - (p @ ck) * ck) ** 2) for ck in cb]
+        assert z == int(np.argmin(resid))
+
+
+def test_weighted_assign_brute_force():
+    """Eq. 6 against a numerical minimisation of Eq. 4 over the radius for every k."""
+    from scipy.optimize import minimize_scalar
+    g = np.random.default_rng(8)
+    cb = _unit_cb(g, 16)
+    for _ in range(60):
+        p = np.abs(g.standard_normal(8))
+        w = oracle.omega(g.lognormal(0, 1.5, 8), 0.75)
+        best = []
+        for ck in cb:
+            res = minimize_scalar(lambda r: float(np.sum(w * (p - r * ck) ** 2)),
+                                  bounds=(0.0, 10.0), method="bounded", options={"xatol": 1e-12})
+            best.append((res.fun, res.x))
+        losses = np.array([b[0] for b in best])
+        z, r = oracle.assign(p, w, cb)
+        if np.sort(losses)[1] - np.sort(losses)[0] > 1e-9:
+            assert z == int(np.argmin(losses))
+        assert r == pytest.approx(best[z][1], abs=1e-6)
+
+
+def test_assign_zero_vector():
+    z, r = oracle.assign(np.zeros(8), np.ones(8), _unit_cb(np.random.default_rng(1), 8))
+    assert (z, r) == (0, 0.0)
+
+
+def test_grid_and_quantize():
+    """Eq. 14 grid and Eq. 2 codes: q in range, group extremes at the ends, and the
+    decoded radius within half a step of the fitted one."""
+    # hand example: mu = 0.125, delta = 2^-7
+    assert oracle.quantize(0.2, 0x3000, 0x2000, 4) == 10       # 9.6 -> 10
+    assert oracle.quantize(0.1, 0x3000, 0x2000, 4) == 0        # below the grid
+    assert oracle.quantize(1.0, 0x3000, 0x2000, 4) == 15       # clipped
+    assert oracle.quantize(0.125 + 2.5 * 2 ** -7, 0x3000, 0x2000, 4) == 3  # tie rounds up
+    g = np.random.default_rng(12)
+    for V in (2, 3, 4, 5, 6):
+        for _ in range(50):
+            r = g.uniform(0.01, 0.5, 16)
+            mu16, de16 = oracle.grid(r, V)
+            mu, de = np.uint16(mu16).view(np.float16).astype(float), np.uint16(de16).view(np.float16).astype(float)
+            assert mu == pytest.approx(r.min(), rel=2 ** -11)
+            assert de == pytest.approx((r.max() - r.min()) / (2 ** V - 1), rel=2 ** -11)
+            q = np.array([oracle.quantize(x, mu16, de16, V) for x in r])
+            assert q.min() >= 0 and q.max() <= 2 ** V - 1
+            assert q[np.argmin(r)] == 0
+            assert q[np.argmax(r)] >= 2 ** V - 2
+            rec = mu + q * de
+            inside = (r >= mu) & (r <= mu + (2 ** V - 1) * de)
+            assert np.all(np.abs(rec - r)[inside] <= de / 2 * (1 + 1e-9) + 1e-12)
+    mu16, de16 = oracle.grid(np.full(16, 0.3), 4)
+    assert de16 == 0 and oracle.quantize(0.3, mu16, de16, 4) == 0
+
+
+def test_kmeans_recovers_planted_directions():
+    """With omega = 1 the update is spherical k-means; data drawn tightly around K
+    well-separated nonnegative unit directions must give those directions back."""
+    g = np.random.default_rng(13)
+    K = 8
+    centers = np.eye(8)
+    lab = g.integers(0, K, 4000)
+    P = np.abs(centers[lab] + 0.01 * g.standard_normal((4000, 8))) * g.uniform(0.5, 2, (4000, 1))
+    init = np.array([int(np.nonzero(lab == k)[0][0]) for k in range(K)])
+    cb = oracle.kmeans(P, np.ones_like(P), K, init, 10)
+    assert np.allclose(np.linalg.norm(cb, axis=1), 1.0, atol=1e-12)
+    assert (cb >= 0).all()
+    # fixed point of spherical k-means: each codeword is the normalised sum of its
+    # members' unit directions (the planted clusters are well separated)
+    D = P / np.linalg.norm(P, axis=1, keepdims=True)
+    exp = np.stack([D[lab == k].sum(0) for k in range(K)])
+    exp /= np.linalg.norm(exp, axis=1, keepdims=True)
+    assert np.allclose(cb, exp, rtol=0, atol=1e-12)
+    assert np.allclose(cb, centers, atol=2e-2)
+
+
+def test_kmeans_deterministic_and_optimal_assignment():
+    inp, _ = synth.config2(d_out=32, d_in=256, n_samples=512, iters=4, log2K=4)
+    a = oracle.encode(inp)
+    b = oracle.encode(inp)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+    assert np.array_equal(a["perm"], oracle.esg_perm(inp.energies))
+    cb = a["codebook"].view(np.float16).astype(np.float64)
+    assert (cb >= 0).all()
+    assert np.allclose(np.linalg.norm(cb, axis=1), 1.0, atol=2 ** -9)
+    # every stored index is Eq. 6-optimal for the stored codebook
+    Wp = inp.W[:, a["perm"]]
+    S = 256 // 8
+    for o in range(0, 32, 7):
+        for j in range(0, S, 5):
+            w8 = oracle.omega(inp.energies[a["perm"][8 * j:8 * j + 8]], 0.75)
+            p = np.abs(Wp[o, 8 * j:8 * j + 8])
+            z, _ = oracle.assign(p, w8, cb)
+            assert a["idx"][o, j] == z
+            s = int(sum(1 << i for i in range(8) if Wp[o, 8 * j + i] < 0))
+            assert a["signs"][o, j] == s
+    assert a["q"].max() <= 2 ** 6 - 1
