@@ -44,8 +44,8 @@ def lib():
             L.oracle_half_to_double.restype = f64
             L.oracle_double_to_half.argtypes = [f64]
             L.oracle_double_to_half.restype = u16
-            L.oracle_unpack_v1.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
-            L.oracle_unpack_v1.restype = i32
+            L.oracle_unpack.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
+            L.oracle_unpack.restype = i32
             L.oracle_dequant.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
             L.oracle_dequant.restype = None
             L.oracle_round_half.argtypes = [sz, P, P]
@@ -101,10 +101,11 @@ def halves_to_double(h: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Packed layout v1 and reconstruction
+# Packed layout and reconstruction
 # ---------------------------------------------------------------------------
 
-def unpack_v1(d_out, d_in, log2K, main_plane, meta_plane):
+def unpack(d_out, d_in, log2K, main_plane, meta_plane):
+    """Logical fields from the library's packed planes (format version 2)."""
     S, G = d_in // 8, d_in // 128
     main_plane = _c(main_plane, np.uint32).reshape(-1)
     meta_plane = _c(meta_plane, np.uint32).reshape(-1)
@@ -113,10 +114,10 @@ def unpack_v1(d_out, d_in, log2K, main_plane, meta_plane):
     q = np.zeros((d_out, S), np.uint8)
     mu = np.zeros((d_out, G), np.uint16)
     delta = np.zeros((d_out, G), np.uint16)
-    rc = lib().oracle_unpack_v1(d_out, d_in, log2K, _p(main_plane), _p(meta_plane),
+    rc = lib().oracle_unpack(d_out, d_in, log2K, _p(main_plane), _p(meta_plane),
                                 _p(signs), _p(idx), _p(q), _p(mu), _p(delta))
     if rc:
-        raise ValueError("oracle_unpack_v1: unsupported shape")
+        raise ValueError("oracle_unpack: unsupported shape")
     return dict(signs=signs, idx=idx, q=q, mu=mu, delta=delta)
 
 

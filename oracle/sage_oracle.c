@@ -18,8 +18,8 @@
  *   App. A.6 Eq. 14  mu_g = min r~, delta_g = (max r~ - mu_g) / (2^V - 1), groups of 16 subvectors
  *   App. A.6 Eq. 15  BPW = B/v + 2 b_g / G + K v b_c / N
  *
- * The packed layout decoded by oracle_unpack_v1 is the CUDA library's own
- * format "v1" (the paper fixes only the field widths); it is restated here from
+ * The packed layout decoded by oracle_unpack is the CUDA library's own format
+ * (version 2; the paper fixes only the field widths); it is restated here from
  * its written specification, independently of the library's packer.
  *
  * Parity status: every function below is pinned by tests/test_oracle_*.py
@@ -75,11 +75,14 @@ uint16_t oracle_double_to_half(double x) {
 }
 
 /* ------------------------------------------------------------------ */
-/* Packed format v1 (the library's layout), restated from its spec.    */
+/* Packed format v2 (the library's layout), restated from its spec.    */
 /*                                                                     */
-/* R8 = ceil(d_out / 8) row octets; S = d_in / 8 subvector columns.    */
-/* main: uint32 words, index ((j * R8) + b) * 4 + u.  Word u of the    */
-/*   record (j, b) holds row A = 8b + 2u and row B = 8b + 2u + 1:      */
+/* R8 = ceil(d_out / 8) row octets (octet b = rows 8b..8b+7); blocks   */
+/* of 32 octets (256 rows), block B holding n_B = min(32, R8 - 32B)    */
+/* octets.  S = d_in / 8 subvector columns, G = d_in / 128 groups.     */
+/* main: uint32 words.  Record (j, octet o of block B) is the 4 words  */
+/*   at B * S * 128 + (j * n_B + o) * 4.  Word u holds row A =         */
+/*   8(32B + o) + 2u and row B = row A + 1:                            */
 /*     z_A at bits [7, 7 + log2K)      q_A at bits [23 - V, 23)        */
 /*     z_B at bits [23, 23 + log2K)    q_B at bits [7 - V, 7)          */
 /*   six sign slots at the ascending positions p_0 < ... < p_5 of      */
@@ -87,10 +90,11 @@ uint16_t oracle_double_to_half(double x) {
 /*   Slots 0..2 carry row A's component pairs 0..2, slots 3..5 row B's; */
 /*   pair n = components (2n, 2n+1): bit p_k is the sign of 2n, bit    */
 /*   p_k + 16 the sign of 2n + 1.                                       */
-/* meta: 8-byte entries, index ((g * R8) + b) * 8 + t for row 8b + t:  */
+/* meta: 8-byte entries; entry (g, octet o of block B, row t) is at    */
+/*   entry index B * G * 256 + (g * n_B + o) * 8 + t:                  */
 /*   uint32 aux, uint16 mu, uint16 delta (little endian).              */
-/*   aux bit t = sign of component 6 of subvector 16g + t,             */
-/*   aux bit t + 16 = sign of component 7 of that subvector.           */
+/*   aux bit t' = sign of component 6 of subvector 16g + t',           */
+/*   aux bit t' + 16 = sign of component 7 of that subvector.          */
 /* Rows past d_out in the last octet are zero.                          */
 /* ------------------------------------------------------------------ */
 
@@ -111,7 +115,7 @@ static uint32_t getbits(uint32_t w, int lo, int n) {
     return (w >> lo) & ((1u << n) - 1u);
 }
 
-int oracle_unpack_v1(int d_out, int d_in, int log2K,
+int oracle_unpack(int d_out, int d_in, int log2K,
                      const uint32_t* main_plane, const uint32_t* meta_plane,
                      uint8_t* signs, uint16_t* idx, uint8_t* q,
                      uint16_t* mu, uint16_t* delta) {
@@ -120,9 +124,12 @@ int oracle_unpack_v1(int d_out, int d_in, int log2K,
     const int S = d_in / SV, G = d_in / 128, R8 = (d_out + 7) / 8;
     for (int o = 0; o < d_out; ++o) {
         const int b = o / 8, t = o % 8, u = t / 2, isB = t & 1;
+        const int blk = b / 32, ob = b % 32;
+        const int nB = (R8 - 32 * blk < 32) ? R8 - 32 * blk : 32;
+        const size_t main0 = (size_t)blk * S * 128, meta0 = (size_t)blk * G * 256;
         for (int j = 0; j < S; ++j) {
-            const uint32_t w = main_plane[((size_t)j * R8 + b) * 4 + u];
-            const uint32_t aux = meta_plane[(((size_t)(j / GROUP_SV) * R8 + b) * 8 + t) * 2];
+            const uint32_t w = main_plane[main0 + ((size_t)j * nB + ob) * 4 + u];
+            const uint32_t aux = meta_plane[(meta0 + ((size_t)(j / GROUP_SV) * nB + ob) * 8 + t) * 2];
             uint32_t z, qq;
             if (!isB) { z = getbits(w, 7, log2K);  qq = getbits(w, 23 - V, V); }
             else      { z = getbits(w, 23, log2K); qq = getbits(w, 7 - V, V); }
@@ -140,7 +147,7 @@ int oracle_unpack_v1(int d_out, int d_in, int log2K,
             q[(size_t)o * S + j] = (uint8_t)qq;
         }
         for (int g = 0; g < G; ++g) {
-            const uint32_t md = meta_plane[(((size_t)g * R8 + b) * 8 + t) * 2 + 1];
+            const uint32_t md = meta_plane[(meta0 + ((size_t)g * nB + ob) * 8 + t) * 2 + 1];
             mu[(size_t)o * G + g] = (uint16_t)(md & 0xffff);
             delta[(size_t)o * G + g] = (uint16_t)(md >> 16);
         }

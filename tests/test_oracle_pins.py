@@ -80,28 +80,28 @@ def test_budget_printed_values():
 
 
 # ---------------------------------------------------------------------------
-# Packed layout v1 (the library's own format)
+# Packed layout (the library's own format, version 2)
 # ---------------------------------------------------------------------------
 
 def test_unpack_hand_example():
-    gx = _gold("format_v1_example.json")
-    main = np.zeros(gx["main_words"], np.uint32)
-    meta = np.zeros(gx["meta_words"], np.uint32)
-    for k, v in gx["main_nonzero"].items():
-        main[int(k)] = int(v, 16)
-    for k, v in gx["meta_nonzero"].items():
-        meta[int(k)] = int(v, 16)
-    f = oracle.unpack_v1(gx["d_out"], gx["d_in"], gx["log2K"], main, meta)
-    exp = {k: np.zeros_like(v) for k, v in f.items()}
-    for e in gx["fields_nonzero"]:
-        exp["signs"][e["row"], e["j"]] = e["signs"]
-        exp["idx"][e["row"], e["j"]] = e["idx"]
-        exp["q"][e["row"], e["j"]] = e["q"]
-    for e in gx["grid_nonzero"]:
-        exp["mu"][e["row"], e["g"]] = int(e["mu"], 16)
-        exp["delta"][e["row"], e["g"]] = int(e["delta"], 16)
-    for k in f:
-        assert np.array_equal(f[k], exp[k]), k
+    for gx in _gold("format_example.json")["examples"]:
+        main = np.zeros(gx["main_words"], np.uint32)
+        meta = np.zeros(gx["meta_words"], np.uint32)
+        for k, v in gx["main_nonzero"].items():
+            main[int(k)] = int(v, 16)
+        for k, v in gx["meta_nonzero"].items():
+            meta[int(k)] = int(v, 16)
+        f = oracle.unpack(gx["d_out"], gx["d_in"], gx["log2K"], main, meta)
+        exp = {k: np.zeros_like(v) for k, v in f.items()}
+        for e in gx["fields_nonzero"]:
+            exp["signs"][e["row"], e["j"]] = e["signs"]
+            exp["idx"][e["row"], e["j"]] = e["idx"]
+            exp["q"][e["row"], e["j"]] = e["q"]
+        for e in gx["grid_nonzero"]:
+            exp["mu"][e["row"], e["g"]] = int(e["mu"], 16)
+            exp["delta"][e["row"], e["g"]] = int(e["delta"], 16)
+        for k in f:
+            assert np.array_equal(f[k], exp[k]), (gx["d_out"], k)
 
 
 @pytest.mark.parametrize("log2K", [4, 5, 6, 7, 8])
@@ -112,7 +112,7 @@ def test_unpack_is_a_bijection(log2K):
     R8, S, G = 2, 16, 1
     V = 10 - log2K
     nmain, nmeta = S * R8 * 4, G * R8 * 8 * 2
-    base = oracle.unpack_v1(d_out, d_in, log2K, np.zeros(nmain, np.uint32), np.zeros(nmeta, np.uint32))
+    base = oracle.unpack(d_out, d_in, log2K, np.zeros(nmain, np.uint32), np.zeros(nmeta, np.uint32))
     for k in base:
         assert not base[k].any()
     hit = set()
@@ -132,14 +132,14 @@ def test_unpack_is_a_bijection(log2K):
         for bit in range(32):
             main = np.zeros(nmain, np.uint32)
             main[(3 * R8 + 1) * 4 + word] = np.uint32(1 << bit)
-            fb = field_bits(oracle.unpack_v1(d_out, d_in, log2K, main, np.zeros(nmeta, np.uint32)))
+            fb = field_bits(oracle.unpack(d_out, d_in, log2K, main, np.zeros(nmeta, np.uint32)))
             assert len(fb) == 1, (word, bit, fb)
             hit |= fb
     for word in range(16):
         for bit in range(32):
             meta = np.zeros(nmeta, np.uint32)
             meta[(1 * 8) * 2 + word] = np.uint32(1 << bit)
-            fb = field_bits(oracle.unpack_v1(d_out, d_in, log2K, np.zeros(nmain, np.uint32), meta))
+            fb = field_bits(oracle.unpack(d_out, d_in, log2K, np.zeros(nmain, np.uint32), meta))
             assert len(fb) <= 1, (word, bit, fb)
             hit |= fb
     # 8 rows x (18 bits of subvector j=3) + 8 rows x 16 aux bits (only j=3's 2 counted) + grid
@@ -153,7 +153,7 @@ def test_unpack_all_ones():
     for log2K in range(4, 9):
         V = 10 - log2K
         d_out, d_in = 8, 256
-        f = oracle.unpack_v1(d_out, d_in, log2K, np.full(32 * 4, 0xFFFFFFFF, np.uint32),
+        f = oracle.unpack(d_out, d_in, log2K, np.full(32 * 4, 0xFFFFFFFF, np.uint32),
                              np.full(2 * 8 * 2, 0xFFFFFFFF, np.uint32))
         assert (f["signs"] == 255).all() and (f["idx"] == (1 << log2K) - 1).all()
         assert (f["q"] == (1 << V) - 1).all()
