@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark: batch-1 packed SAGE GEMV over a Qwen3-4B-shaped decoder layer on B200.
+
+A step is one decoder layer's seven packed linears at batch 1, launched as its
+four dependency stages (q|k|v, o, gate|up, down; one grouped GEMV launch each,
+chained with programmatic dependent launch).  Inputs are synthetic (seeded, see
+synth/), resident in HBM; every step reads a different copy of the layer's
+packed planes so the working set (>= 4 x the 126 MB L2) comes from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  ``value`` is the whole-job throughput in GB/s of
+packed bytes (codes + mu/delta + codebooks + x + y) per layer; ``us_per_layer``
+is the device time of one layer.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 packed VQ GEMV µs/layer and achieved HBM GB/s vs B200 peak"
+WORKLOAD = "Qwen3-4B-shaped decoder layer, 7 packed linears (q,k,v,o,gate,up,down), hidden 2560, batch 1"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------
+# Workload construction (product path only: synth + libsage)
+# ---------------------------------------------------------------------------
+
+def build_layer(replicas: int):
+    import torch
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    L = synth.config1()
+    base = {}
+    for f in L.mats:
+        f.perm = sage.sage_esg_permutation(L.energies[f.name])
+        base[f.name] = sage.PackedMatrix.from_fields(f)
+    layers = []
+    for r in range(replicas):
+        if r == 0:
+            layers.append(base)
+            continue
+        layers.append({n: sage.PackedMatrix(m.d_out, m.d_in, m.log2K, m.main.clone(), m.meta.clone(),
+                                            m.codebook.clone(), m.perm.clone() if m.perm is not None else None, n)
+                       for n, m in base.items()})
+    xs = {s[0]: torch.from_numpy(L.xs[s[0]].view(np.int16)).cuda() for s in synth.QWEN3_4B_STAGES}
+    return L, layers, xs
+
+
+def layer_bytes(mats, M=1):
+    """Algorithmic bytes of one layer: packed planes + codebooks + x + y (perm excluded)."""
+    tot = 0
+    perm = 0
+    for m in mats.values():
+        tot += m.packed_bytes + (1 << m.log2K) * 16 + M * m.d_in * 2 + M * m.d_out * 2
+        perm += m.d_in * 4 if m.perm is not None else 0
+    return tot, perm
+
+
+class LayerRunner:
+    """Pre-marshalled grouped launches for one layer replica."""
+
+    def __init__(self, mats, xs, ys, ws):
+        import synth
+        import bit_vector_quantized_sage_b200 as sage
+        self.calls = []
+        for stage in synth.QWEN3_4B_STAGES:
+            ms = [mats[n] for n in stage]
+            self.calls.append(sage.GroupedCall(ms, [xs[stage[0]]] * len(stage), [ys[n] for n in stage], 1, ws))
+
+    def __call__(self, stream=None):
+        for c in self.calls:
+            c(stream)
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/sage_clocks_{os.getpid()}.csv"
+        self.gpu = gpu_index
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _traffic_for(kernel_src_hash: str):
+    p = os.path.join(ROOT, "profiles", "gemv_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None, None
+    if d.get("source_sha256") != kernel_src_hash:
+        return None, d.get("source_sha256")
+    return d.get("traffic_bytes_per_launch"), d.get("source_sha256")
+
+
+def _kernel_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_vector_quantized_sage_b200", "csrc")
+    for n in ("sage_gemv.cu", "sage_device.cuh"):
+        h.update(open(os.path.join(csrc, n), "rb").read())
+    return h.hexdigest()
+
+
+def cpu_oracle_sample(rows_per_matrix: int = 256, seconds_cap: float = 60.0):
+    """Times the CPU oracle (unpack + fp32 reconstruction + fp64 matvec) on the first
+    ``rows_per_matrix`` rows of each of the layer's seven matrices, single-threaded.
+    Returns (GB/s of packed bytes, sample description, cores used)."""
+    import oracle
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    L = synth.config1()
+    tot_bytes, tot_s = 0, 0.0
+    for f in L.mats:
+        f.perm = sage.sage_esg_permutation(L.energies[f.name])
+        x = L.xs[[s for s in synth.QWEN3_4B_STAGES if f.name in s][0][0]]
+        R = min(rows_per_matrix, f.d_out)
+        # row-octet slice of the planes for the first R rows
+        sub = synth.Fields(R, f.d_in, f.log2K, f.signs[:R], f.idx[:R], f.q[:R], f.mu[:R], f.delta[:R],
+                           f.codebook, f.perm, f.name)
+        m_sub, t_sub = sage.sage_pack(R, f.d_in, f.log2K, sub.signs, sub.idx, sub.q, sub.mu, sub.delta)
+        t0 = time.perf_counter()
+        u = oracle.unpack(R, f.d_in, f.log2K, m_sub, t_sub)
+        g = synth.Fields(R, f.d_in, f.log2K, u["signs"], u["idx"], u["q"], u["mu"], u["delta"], f.codebook, f.perm)
+        oracle.gemv(g, x)
+        tot_s += time.perf_counter() - t0
+        mb, tb = sage.sage_packed_sizes(R, f.d_in, f.log2K)
+        tot_bytes += mb + tb + (1 << f.log2K) * 16 + f.d_in * 2 + R * 2
+        if tot_s > seconds_cap:
+            break
+    desc = f"first {rows_per_matrix} rows of each of the 7 layer matrices (unpack + reconstruct + fp64 matvec)"
+    return tot_bytes / tot_s / 1e9, desc, 1, tot_s
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        cpu_oracle_sample(rows_per_matrix=32)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        v, desc, cores, s = cpu_oracle_sample(rows_per_matrix=64)
+        vals.append(v)
+        secs += s
+    value = statistics.median(vals)
+    layer_b = 31_682_560  # packed layer bytes scale: reported per-layer time from the GB/s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; see synth/config1)",
+        "config": {"workload": WORKLOAD, "batch": 1, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "us_per_layer_extrapolated": layer_b / (value * 1e9) * 1e6,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_gpu(args):
+    import torch
+    import bit_vector_quantized_sage_b200 as sage
+    from bit_vector_quantized_sage_b200 import build as sage_build
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if rank == 0 or not os.path.exists(sage_build.LIB):
+        sage_build.build()
+    if dist is not None:
+        dist.barrier()
+    sage.load()
+
+    L, layers1, xs = build_layer(1)
+    one_layer_bytes, perm_bytes = layer_bytes(layers1[0])
+    replicas = max(2, int(np.ceil(4 * L2_BYTES / one_layer_bytes)) + 1)
+    _, layers, xs = build_layer(replicas)
+    ys = {f.name: torch.zeros((1, f.d_out), dtype=torch.int16, device="cuda") for f in L.mats}
+    ws = sage.Workspace(max(sage.sage_workspace_size(sage.SAGE_OP_GROUPED, [layers[0][n] for n in st], 1)
+                            for st in __import__("synth").QWEN3_4B_STAGES))
+    runners = [LayerRunner(lay, xs, ys, ws) for lay in layers]
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+
+    # ---- warm-up (eager) ----
+    for i in range(max(3, args.warmup)):
+        runners[i % replicas](stream)
+    torch.cuda.synchronize()
+    assert sage.sage_query_status(ws) == sage.SAGE_OK
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn(torch.cuda.current_stream())
+        return g
+
+    def time_graph(g, reps=1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    import synth
+    n_stage = len(synth.QWEN3_4B_STAGES)
+    stage_bytes = []
+    for stage in synth.QWEN3_4B_STAGES:
+        stage_bytes.append(sum(layers[0][n].packed_bytes + (1 << layers[0][n].log2K) * 16 +
+                               layers[0][n].d_in * 2 + layers[0][n].d_out * 2 for n in stage))
+
+    # ---- per-stage kernel time: one graph = the stage launched once per replica ----
+    stage_avg = []
+    with torch.cuda.stream(stream):
+        for s_i in range(n_stage):
+            g = capture(lambda st: [runners[r].calls[s_i](st) for r in range(replicas)])
+            for _ in range(3):
+                g.replay()
+            ms_s = time_graph(g, reps=max(1, 200 // replicas))
+            stage_avg.append(ms_s / (max(1, 200 // replicas) * replicas))
+            del g
+
+    # ---- timed region: one graph holding K layers back to back (rotating replicas) ----
+    with torch.cuda.stream(stream):
+        g_all = capture(lambda st: [runners[k % replicas](st) for k in range(args.steps)])
+        for _ in range(max(3, args.warmup // max(1, args.steps) + 1)):
+            g_all.replay()
+        torch.cuda.synchronize()
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    g_all.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert sage.sage_query_status(ws) == sage.SAGE_OK
+    us_per_layer = ms * 1e3 / args.steps
+    value = world * one_layer_bytes * args.steps / (ms * 1e-3) / 1e9
+    del g_all
+
+    # ---- end to end through the public API with host buffers (graph per step) ----
+    h_x = {k: torch.from_numpy(L.xs[k].view(np.int16)).pin_memory() for k in xs}
+    h_y = {n: torch.zeros(tuple(ys[n].shape), dtype=torch.int16).pin_memory() for n in ys}
+    h2d = sum(v.numel() * 2 for v in h_x.values())
+    d2h = sum(v.numel() * 2 for v in h_y.values())
+    e2e_steps = max(20, args.steps // 2)
+
+    def e2e_step(st, r):
+        for n, hx in h_x.items():
+            xs[n].copy_(hx, non_blocking=True)
+        runners[r](st)
+        for n, hy in h_y.items():
+            hy.copy_(ys[n], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        g_e2e = [capture(lambda st, r=r: e2e_step(st, r)) for r in range(replicas)]
+        for r in range(replicas):
+            g_e2e[r].replay()
+        torch.cuda.synchronize()
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_start.record(stream)
+        for k in range(e2e_steps):
+            g_e2e[k % replicas].replay()
+            stream.synchronize()          # the host reads the step's result
+        e_end.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
+    e2e_value = world * one_layer_bytes / (e2e_ms * 1e-3) / 1e9
+    del g_e2e
+
+    peak, peak_kind = _peaks()
+    achieved = sum(stage_bytes) / (sum(stage_avg) * 1e-3) / 1e9
+    traffic, _ = _traffic_for(_kernel_hash())
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, cores, secs = cpu_oracle_sample(rows_per_matrix=args.cpu_rows)
+        cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc,
+               "seconds": round(secs, 2)}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded; see synth/config1)",
+        "config": {"workload": WORKLOAD, "batch": 1, "stages": "q|k|v, o, gate|up, down (4 grouped launches)",
+                   "packed_bytes_per_layer": one_layer_bytes, "perm_bytes_per_layer": perm_bytes,
+                   "l2": f"inputs larger than L2: {replicas} rotating copies of the packed layer "
+                         f"({replicas * one_layer_bytes / 2**20:.0f} MiB)",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_layer": us_per_layer,
+        "hbm_fraction": value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "kernel": "gemv_kernel<1> (grouped packed GEMV)",
+                     "stage_us": [round(s * 1e3, 3) for s in stage_avg],
+                     "stage_bytes": stage_bytes},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_layer": e2e_ms * 1e3},
+        "gpu_launches": args.steps * n_stage,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

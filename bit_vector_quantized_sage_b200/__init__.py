@@ -1,0 +1,313 @@
+"""Python binding of libsage, the B200 (sm_100a) SAGE packed linear layer.
+
+Argument marshalling only: every computation runs in the compiled library
+(``libsage.so``, built in-tree by ``bit_vector_quantized_sage_b200.build``).
+Function names mirror the C ABI declared in ``include/sage.h``.  There is no
+fallback: if the library is missing or a CUDA device is absent the calls raise.
+
+PyTorch is used only to own device memory and streams (``tensor.data_ptr()``
+and ``torch.cuda.current_stream().cuda_stream`` are passed through).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage.so")
+
+SAGE_OK = 0
+SAGE_ERR_INVALID_ARGUMENT = 1
+SAGE_ERR_UNSUPPORTED = 2
+SAGE_ERR_MISALIGNED = 3
+SAGE_ERR_WORKSPACE = 4
+SAGE_ERR_CUDA = 5
+SAGE_ERR_TIMEOUT = 6
+
+SAGE_OP_GEMV, SAGE_OP_GEMM, SAGE_OP_MOE, SAGE_OP_GROUPED = 0, 1, 2, 3
+
+# Every extern "C" symbol declared in include/sage.h.
+EXPORTS = (
+    "sage_status_string", "sage_version", "sage_packed_sizes", "sage_pack", "sage_unpack",
+    "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
+    "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
+    "sage_query_status",
+)
+
+
+class SageError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} ({status})")
+
+
+class sage_matrix(C.Structure):
+    _fields_ = [
+        ("d_out", C.c_int32), ("d_in", C.c_int32), ("log2K", C.c_int32),
+        ("main", C.c_void_p), ("meta", C.c_void_p), ("codebook", C.c_void_p), ("perm", C.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Loads libsage.so and declares the argument types (raises if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"libsage.so not built ({path}); run python -m bit_vector_quantized_sage_b200.build")
+    L = C.CDLL(path)
+    P, I, SZ = C.c_void_p, C.c_int, C.c_size_t
+    MP = C.POINTER(sage_matrix)
+    sig = {
+        "sage_status_string": ([I], C.c_char_p),
+        "sage_version": ([], C.c_char_p),
+        "sage_packed_sizes": ([I, I, I, C.POINTER(SZ), C.POINTER(SZ)], I),
+        "sage_pack": ([I, I, I, P, P, P, P, P, P, P], I),
+        "sage_unpack": ([I, I, I, P, P, P, P, P, P, P], I),
+        "sage_esg_permutation": ([I, P, P], I),
+        "sage_encode": ([I, I, I, P, P, C.c_double, I, P, P, I, I, P, P, P, P, P, P, P], I),
+        "sage_workspace_size": ([I, MP, I, I, C.POINTER(SZ)], I),
+        "sage_gemv": ([MP, P, I, P, P, SZ, P], I),
+        "sage_gemv_grouped": ([MP, I, P, P, I, P, SZ, P], I),
+        "sage_gemm": ([MP, P, I, P, P, SZ, P], I),
+        "sage_moe_gemv": ([MP, I, P, P, I, P, P, P, SZ, P], I),
+        "sage_dequant": ([MP, P, P], I),
+        "sage_unpack_device": ([MP, P, P, P, P, P, P], I),
+        "sage_permute_x": ([P, P, I, I, P, P], I),
+        "sage_query_status": ([P, P], I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def status_string(s: int) -> str:
+    return load().sage_status_string(int(s)).decode()
+
+
+def version() -> str:
+    return load().sage_version().decode()
+
+
+def _check(fn: str, rc: int):
+    if rc != SAGE_OK:
+        raise SageError(fn, rc)
+
+
+def _np(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(C.c_void_p)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a torch tensor (or None / int passthrough)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# Host entry points
+# ---------------------------------------------------------------------------
+
+def sage_packed_sizes(d_out: int, d_in: int, log2K: int):
+    a, b = C.c_size_t(), C.c_size_t()
+    _check("sage_packed_sizes", load().sage_packed_sizes(d_out, d_in, log2K, C.byref(a), C.byref(b)))
+    return a.value, b.value
+
+
+def sage_pack(d_out, d_in, log2K, signs, idx, q, mu, delta):
+    """Packs fields (NumPy, storage order) into (main, meta) uint32 NumPy planes."""
+    mb, tb = sage_packed_sizes(d_out, d_in, log2K)
+    main = np.zeros(mb // 4, np.uint32)
+    meta = np.zeros(tb // 4, np.uint32)
+    s, ps = _np(signs, np.uint8)
+    i, pi = _np(idx, np.uint16)
+    qq, pq = _np(q, np.uint8)
+    m, pm = _np(mu, np.uint16)
+    d, pd = _np(delta, np.uint16)
+    _check("sage_pack", load().sage_pack(d_out, d_in, log2K, ps, pi, pq, pm, pd,
+                                          main.ctypes.data_as(C.c_void_p), meta.ctypes.data_as(C.c_void_p)))
+    return main, meta
+
+
+def sage_unpack(d_out, d_in, log2K, main, meta):
+    S, G = d_in // 8, d_in // 128
+    out = dict(signs=np.zeros((d_out, S), np.uint8), idx=np.zeros((d_out, S), np.uint16),
+               q=np.zeros((d_out, S), np.uint8), mu=np.zeros((d_out, G), np.uint16),
+               delta=np.zeros((d_out, G), np.uint16))
+    mn, pmn = _np(main, np.uint32)
+    mt, pmt = _np(meta, np.uint32)
+    _check("sage_unpack", load().sage_unpack(d_out, d_in, log2K, pmn, pmt,
+                                              *[out[k].ctypes.data_as(C.c_void_p)
+                                                for k in ("signs", "idx", "q", "mu", "delta")]))
+    return out
+
+
+def sage_esg_permutation(energy) -> np.ndarray:
+    e, pe = _np(energy, np.float64)
+    perm = np.zeros(e.size, np.int32)
+    _check("sage_esg_permutation", load().sage_esg_permutation(e.size, pe, perm.ctypes.data_as(C.c_void_p)))
+    return perm
+
+
+def sage_encode(W, energy, log2K: int, gamma: float, sample, init, iters: int, n_threads: int = 0):
+    """CPU encoder (ESG, weighted k-means, Eq. 6, Eq. 14, Eq. 2) -> dict of fields + perm + codebook."""
+    W, pW = _np(W, np.float64)
+    e, pe = _np(energy, np.float64)
+    sm, psm = _np(sample, np.int64)
+    it, pit = _np(init, np.int64)
+    d_out, d_in = W.shape
+    K, S, G = 1 << log2K, d_in // 8, d_in // 128
+    out = dict(perm=np.zeros(d_in, np.int32), codebook=np.zeros((K, 8), np.uint16),
+               signs=np.zeros((d_out, S), np.uint8), idx=np.zeros((d_out, S), np.uint16),
+               q=np.zeros((d_out, S), np.uint8), mu=np.zeros((d_out, G), np.uint16),
+               delta=np.zeros((d_out, G), np.uint16))
+    _check("sage_encode", load().sage_encode(
+        d_out, d_in, log2K, pW, pe, float(gamma), sm.size, psm, pit, iters, n_threads,
+        *[out[k].ctypes.data_as(C.c_void_p) for k in ("perm", "codebook", "signs", "idx", "q", "mu", "delta")]))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Device-side packed matrices
+# ---------------------------------------------------------------------------
+
+@dataclass
+class PackedMatrix:
+    """A packed matrix resident on the device (torch tensors own the memory)."""
+    d_out: int
+    d_in: int
+    log2K: int
+    main: "object"
+    meta: "object"
+    codebook: "object"
+    perm: "object" = None
+    name: str = ""
+
+    def desc(self) -> sage_matrix:
+        return sage_matrix(self.d_out, self.d_in, self.log2K, _ptr(self.main), _ptr(self.meta),
+                           _ptr(self.codebook), _ptr(self.perm) if self.perm is not None else None)
+
+    @property
+    def packed_bytes(self) -> int:
+        return self.main.numel() * 4 + self.meta.numel() * 4
+
+    @staticmethod
+    def from_planes(d_out, d_in, log2K, main, meta, codebook, perm=None, device="cuda", name=""):
+        import torch
+        t = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
+        return PackedMatrix(d_out, d_in, log2K, t(main, np.int32), t(meta, np.int32),
+                            t(np.asarray(codebook, np.uint16).reshape(-1), np.int16),
+                            t(np.asarray(perm, np.int32), np.int32) if perm is not None else None, name)
+
+    @staticmethod
+    def from_fields(f, device="cuda"):
+        main, meta = sage_pack(f.d_out, f.d_in, f.log2K, f.signs, f.idx, f.q, f.mu, f.delta)
+        return PackedMatrix.from_planes(f.d_out, f.d_in, f.log2K, main, meta, f.codebook, f.perm, device, f.name)
+
+
+def _mat_array(mats: Sequence[PackedMatrix]):
+    arr = (sage_matrix * len(mats))(*[m.desc() for m in mats])
+    return arr
+
+
+def sage_workspace_size(op: int, mats, M: int) -> int:
+    """Workspace bytes for one call of `op` over `mats` (one matrix, a grouped list or all experts)."""
+    if isinstance(mats, PackedMatrix):
+        mats = [mats]
+    arr = _mat_array(mats)
+    b = C.c_size_t()
+    _check("sage_workspace_size", load().sage_workspace_size(op, arr, len(mats), M, C.byref(b)))
+    return b.value
+
+
+class Workspace:
+    """Zero-initialised device workspace (status word + split-K scratch)."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        import torch
+        self.nbytes = int(max(256, nbytes))
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+
+def sage_gemv(A: PackedMatrix, x, M: int, y, ws: Workspace, stream=None):
+    d = A.desc()
+    _check("sage_gemv", load().sage_gemv(C.byref(d), _ptr(x), M, _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def sage_gemm(A: PackedMatrix, x, M: int, y, ws: Workspace, stream=None):
+    d = A.desc()
+    _check("sage_gemm", load().sage_gemm(C.byref(d), _ptr(x), M, _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+class GroupedCall:
+    """Pre-marshalled sage_gemv_grouped arguments (cheap to launch repeatedly)."""
+
+    def __init__(self, mats: Sequence[PackedMatrix], xs, ys, M: int, ws: Workspace):
+        self.n = len(mats)
+        self.arr = _mat_array(mats)
+        self.xs = (C.c_void_p * self.n)(*[_ptr(x) for x in xs])
+        self.ys = (C.c_void_p * self.n)(*[_ptr(y) for y in ys])
+        self.M = M
+        self.ws = ws
+        self.keep = (list(mats), list(xs), list(ys))
+
+    def __call__(self, stream=None):
+        _check("sage_gemv_grouped", load().sage_gemv_grouped(self.arr, self.n, self.xs, self.ys, self.M,
+                                                             self.ws.ptr, self.ws.nbytes, _stream(stream)))
+
+
+def sage_gemv_grouped(mats: Sequence[PackedMatrix], xs, ys, M: int, ws: Workspace, stream=None):
+    GroupedCall(mats, xs, ys, M, ws)(stream)
+
+
+def sage_moe_gemv(experts: Sequence[PackedMatrix], pair_expert, pair_xrow, n_pairs: int, x, y, ws: Workspace,
+                  stream=None):
+    arr = _mat_array(experts)
+    _check("sage_moe_gemv", load().sage_moe_gemv(arr, len(experts), _ptr(pair_expert), _ptr(pair_xrow), n_pairs,
+                                                 _ptr(x), _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def sage_dequant(A: PackedMatrix, W, stream=None):
+    d = A.desc()
+    _check("sage_dequant", load().sage_dequant(C.byref(d), _ptr(W), _stream(stream)))
+
+
+def sage_unpack_device(A: PackedMatrix, signs, idx, q, mu, delta, stream=None):
+    d = A.desc()
+    _check("sage_unpack_device", load().sage_unpack_device(C.byref(d), _ptr(signs), _ptr(idx), _ptr(q), _ptr(mu),
+                                                           _ptr(delta), _stream(stream)))
+
+
+def sage_permute_x(x, perm, M: int, d_in: int, x_perm, stream=None):
+    _check("sage_permute_x", load().sage_permute_x(_ptr(x), _ptr(perm), M, d_in, _ptr(x_perm), _stream(stream)))
+
+
+def sage_query_status(ws: Workspace, stream=None) -> int:
+    return int(load().sage_query_status(ws.ptr, _stream(stream)))

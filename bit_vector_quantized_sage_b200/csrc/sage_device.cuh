@@ -1,0 +1,171 @@
+// Device-side building blocks shared by the libsage kernels (sm_100a):
+// PTX wrappers for mbarriers, bulk (TMA) copies, PDL, and the decode of the
+// packed format v1 (see include/sage.h).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace sage {
+namespace dev {
+
+// ------------------------------------------------------------------------
+// Shared-memory addressing and loads
+// ------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+// ------------------------------------------------------------------------
+// mbarrier (CTA scope)
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Arrival that also raises the expected transaction byte count of the phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Gives up after roughly
+// `limit` polls (with nanosleep back-off after the first few thousand) and
+// returns false; callers then record a timeout in the status word and carry
+// on, so no wait can hang the GPU.
+constexpr uint32_t kWaitLimit = 1u << 22;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = kWaitLimit) {
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if (i > 2048) __nanosleep(64);
+    }
+    return false;
+}
+
+// ------------------------------------------------------------------------
+// Bulk asynchronous copy global -> shared (1-D TMA), completes on an mbarrier.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ------------------------------------------------------------------------
+// Programmatic dependent launch
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Device-scope atomic add with acquire-release semantics (returns the old value).
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ------------------------------------------------------------------------
+// Packed format v1 decode constants (per radius width V = 10 - log2K).
+// ------------------------------------------------------------------------
+template <int V>
+struct Fmt {
+    static constexpr int kLog2K = 10 - V;
+    // z occupies bits [7, 7 + log2K) of the (rotated) word -> byte offset z*128
+    static constexpr uint32_t kZMask = ((1u << kLog2K) - 1u) << 7;
+    // q occupies the top V mantissa bits [23 - V, 23): OR-ing 1.0f gives 1 + q/2^V
+    static constexpr uint32_t kQMask = ((1u << V) - 1u) << (23 - V);
+    // sign slots {0 .. 6-V} U {17-V .. 15}
+    __host__ __device__ static constexpr int slot(int k) { return k <= 6 - V ? k : (17 - V) + (k - (7 - V)); }
+};
+
+// XOR mask with the slot's two sign bits moved to bits 15 and 31 (the fp16
+// sign bits of a half2).
+template <int P>
+__device__ __forceinline__ uint32_t slot_mask(uint32_t w) {
+    return (w << (15 - P)) & 0x80008000u;
+}
+
+__device__ __forceinline__ uint32_t aux_mask(uint32_t aux, int t) {
+    return (aux << (15 - t)) & 0x80008000u;
+}
+
+__device__ __forceinline__ uint32_t rot16(uint32_t w) { return __funnelshift_l(w, w, 16); }
+
+// 1 + q / 2^V as fp32 bits, from a word whose bits [23-V, 23) hold q.
+template <int V>
+__device__ __forceinline__ float q_unit(uint32_t w) {
+    return __uint_as_float((w & Fmt<V>::kQMask) | 0x3F800000u);
+}
+
+// Plane offsets (format v2): blocks of 32 row octets stored contiguously.
+__device__ __forceinline__ int block_octets(int R8, int blk) { return min(32, R8 - blk * 32); }
+// uint32 word index of word u of the record (column j, local octet o) of block blk.
+__device__ __forceinline__ size_t main_word(int R8, int S, int blk, int j, int o, int u) {
+    return (size_t)blk * S * 128 + ((size_t)j * block_octets(R8, blk) + o) * 4 + u;
+}
+// 8-byte entry index of (group g, local octet o, row t) of block blk.
+__device__ __forceinline__ size_t meta_entry(int R8, int G, int blk, int g, int o, int t) {
+    return (size_t)blk * G * 256 + ((size_t)g * block_octets(R8, blk) + o) * 8 + t;
+}
+
+__device__ __forceinline__ __half2 u2h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
+__device__ __forceinline__ uint32_t h22u(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
+// (s (.) c) . x for one subvector: four half2 products with fp16 local
+// accumulation (the paper's Fig. 6a data path), returned in fp32.
+__device__ __forceinline__ float signed_dot(uint4 c, uint4 x) {
+    __half2 h = __hmul2(u2h2(c.x), u2h2(x.x));
+    h = __hfma2(u2h2(c.y), u2h2(x.y), h);
+    h = __hfma2(u2h2(c.z), u2h2(x.z), h);
+    h = __hfma2(u2h2(c.w), u2h2(x.w), h);
+    return __low2float(h) + __high2float(h);
+}
+
+}  // namespace dev
+}  // namespace sage

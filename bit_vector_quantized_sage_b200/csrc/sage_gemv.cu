@@ -1,0 +1,1043 @@
+// Packed SAGE GEMV for batch 1..8 on sm_100a (decode path, Sec. 3.5 and App. A.1
+// of "SAGE: Pushing 2-Bit Vector-Quantized LLMs toward Real-World Usability"),
+// its grouped multi-matrix form, and the grouped-expert MoE GEMV.
+//
+// Work decomposition (B200-first, not the paper's RTX 4090 tiling):
+//  * A "unit" is one subvector column j of one 256-row block (32 row octets) of
+//    one matrix: a 512-byte slab of the main plane.  The units of all matrices
+//    of a launch are flattened (matrix, block, j) and cut into one contiguous
+//    range per CTA of a persistent grid (one CTA per SM).  Dense launches are
+//    planned on the host (each matrix gets its own CTAs when that costs little
+//    balance); MoE launches are planned on the device from the routing.
+//  * Two producer warps per CTA.  The copy warp issues, at kernel start and
+//    before waiting on the preceding kernel (programmatic dependent launch),
+//    1-D bulk (TMA) copies of everything static the CTA needs: code records,
+//    grid/aux meta, the permutation slice and the raw codebook.  The activation
+//    warp waits for the preceding kernel, then gathers the ESG-permuted
+//    x_perm[p] = x[perm[p]] (Sec. 3.5 fuses this gather into the decode GEMV).
+//  * Decode warps: lane l owns row octet l of the 256-row block, so every
+//    16-byte record holds 8 of its rows; the warps split the columns.
+//  * Per subvector: the codeword address and the radius code each come out of
+//    one logic op (layout v1), the codeword is one conflict-free 128-bit shared
+//    load (8 bank-rotated replicas of the codebook), the signs are XORed into
+//    the fp16 sign bits, four half2 FMAs form (s (.) c) . x with fp16 local
+//    accumulation (Fig. 6a), and r = mu + q delta (Eq. 2) is applied once, fp32.
+//  * Rows whose columns are split between CTAs are combined deterministically:
+//    partial sums go to the workspace and the last CTA to finish a block adds
+//    them in CTA order (the paper's FP32 split-K combine for small grids).
+//    A CTA defers its outputs to the end so that no segment waits for another
+//    segment's global round trips.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "sage_device.cuh"
+#include "sage_internal.h"
+
+namespace sage {
+using namespace dev;
+
+namespace {
+
+constexpr int kMaxMats = 64;
+constexpr int kMaxExperts = 256;
+constexpr int kMaxPairsPerVirtual = 8;
+constexpr int kOct = 32;               // row octets per block (one per lane)
+constexpr int kBlockRows = kOct * 8;
+constexpr int kChunkJ = 16;            // a chunk lies inside one radius group
+constexpr int kMaxSegs = 4;            // segments stashed before outputs are flushed
+constexpr int kMaxPass = 4;            // chunks per pass (one ring half)
+constexpr int kMainSlot = kChunkJ * kOct * 16;  // 8 KB of code records
+constexpr int kMetaSlot = kOct * 64;            // 2 KB: one group of 256 rows
+constexpr int kPermSlot = kChunkJ * 8 * 4;      // 512 B
+
+template <int M>
+struct Cfg {
+    static constexpr int kW = 8;                       // decode warps
+    static constexpr int kThreads = (kW + 2) * 32;     // + copy warp + activation warp
+    static constexpr int kDecodeThreads = kW * 32;
+    static constexpr int kMinBlocks = (M <= 2) ? 2 : 1;  // room for the next kernel of a PDL chain
+    static constexpr int kXSlot = M * kChunkJ * 16;
+    static constexpr int kSlot = kMainSlot + kMetaSlot + kPermSlot + kXSlot;
+    static constexpr int kRed = kW * 8 * M * 32 * 4;
+    static constexpr int kStash = kMaxSegs * M * kBlockRows * 4;
+    static constexpr int kFixed = kRed + kStash + (4 * kMaxPass + 6) * 8 + 64 + 32 * 160;  // ... + segment table (kSegTab x kSegBytes)
+    // codebook replicas (K_max * 8 * 16) + 2 raw codebooks + ring + fixed
+    static int smem(int pass_chunks, int kmax) { return kmax * 128 + 2 * kmax * 16 + 2 * pass_chunks * kSlot + kFixed; }
+};
+
+// One matrix as the kernel sees it while working on one of its segments.
+struct MatView {
+    const uint32_t* main;
+    const uint32_t* meta;
+    const uint16_t* cb;
+    const int32_t* perm;
+    const uint16_t* x;      // activations, row stride d_in
+    uint16_t* y;            // outputs, row stride d_out
+    const int32_t* xrows;   // [Mk] activation row of batch slot m (null: m)
+    const int32_t* yrows;   // [Mk] output row of batch slot m (null: m)
+    long long unit0;
+    int d_out, d_in, log2K, R8, S, blk0, Mk;
+};
+
+struct DenseMat {
+    const uint32_t* main;
+    const uint32_t* meta;
+    const uint16_t* cb;
+    const int32_t* perm;
+    const uint16_t* x;
+    uint16_t* y;
+    long long unit0, units;
+    int d_out, d_in, log2K, blk0;
+    int cta0, ncta;        // CTAs [cta0, cta0 + ncta) own this matrix (per-matrix plans)
+};
+
+struct ExpertMat {
+    const uint32_t* main;
+    const uint32_t* meta;
+    const uint16_t* cb;
+    const int32_t* perm;
+    int log2K, pad;
+};
+
+struct Common {
+    int n_cta;
+    int M;                 // dense: batch; MoE: 0 (per virtual expert)
+    int pass_chunks;       // chunks per ring half
+    int kmax;              // largest codebook of the launch (replica area size)
+    uint32_t* status;
+    unsigned* counters;
+    float* partials;       // [n_cta][2][8][kBlockRows]
+};
+
+// CTA c covers units [first(c), first(c + 1)).  Stream-K plans split the
+// flattened units evenly; per-matrix plans give matrix k its own CTAs and
+// split its units evenly among them.  Both are plain arithmetic, so no
+// dependent parameter-space loads sit on any critical path.
+struct DenseParams {
+    Common c;
+    long long total_units;
+    int n_mats;
+    int per_matrix;
+    DenseMat mats[kMaxMats];
+};
+
+struct MoeRoute {
+    int n_virtual;
+    int pad[3];
+};
+struct MoeParams {
+    Common c;
+    int n_experts, d_out, d_in, n_pairs;
+    const uint16_t* x;
+    uint16_t* y;
+    const MoeRoute* route;         // ws
+    const int32_t* v_expert;       // ws [n_pairs]
+    const int32_t* v_xrows;        // ws [n_pairs][8]
+    const int32_t* v_yrows;        // ws [n_pairs][8]
+    const int32_t* v_count;        // ws [n_pairs]
+    ExpertMat experts[kMaxExperts];
+};
+
+struct DenseProblem {
+    const DenseParams& p;
+    __device__ long long total() const { return p.total_units; }
+    __device__ long long cta_begin(int c) const {
+        if (!p.per_matrix) return (long long)c * p.total_units / p.c.n_cta;
+        if (c >= p.c.n_cta) return p.total_units;
+        int k = 0;
+        while (k + 1 < p.n_mats && p.mats[k + 1].cta0 <= c) ++k;
+        const DenseMat& d = p.mats[k];
+        return d.unit0 + (long long)(c - d.cta0) * d.units / d.ncta;
+    }
+    __device__ int cta_of(long long u) const {
+        if (!p.per_matrix) return (int)(((u + 1) * p.c.n_cta + p.total_units - 1) / p.total_units) - 1;
+        int k = 0;
+        while (k + 1 < p.n_mats && p.mats[k + 1].unit0 <= u) ++k;
+        const DenseMat& d = p.mats[k];
+        return d.cta0 + (int)(((u - d.unit0 + 1) * d.ncta + d.units - 1) / d.units) - 1;
+    }
+    __device__ MatView view(long long u) const {
+        int k = 0;
+        while (k + 1 < p.n_mats && p.mats[k + 1].unit0 <= u) ++k;
+        const DenseMat& d = p.mats[k];
+        MatView v;
+        v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = d.x; v.y = d.y;
+        v.xrows = nullptr; v.yrows = nullptr; v.unit0 = d.unit0;
+        v.d_out = d.d_out; v.d_in = d.d_in; v.log2K = d.log2K;
+        v.R8 = (d.d_out + 7) >> 3; v.S = d.d_in >> 3;
+        v.blk0 = d.blk0; v.Mk = p.c.M;
+        return v;
+    }
+};
+
+struct MoeProblem {
+    const MoeParams& p;
+    __device__ int R8() const { return (p.d_out + 7) >> 3; }
+    __device__ long long upv() const { return (long long)((R8() + kOct - 1) / kOct) * (p.d_in >> 3); }
+    __device__ long long total() const { return (long long)__ldcg(&p.route->n_virtual) * upv(); }
+    __device__ long long cta_begin(int c) const { return (long long)c * total() / p.c.n_cta; }
+    __device__ int cta_of(long long u) const {
+        const long long t = total();
+        return (int)(((u + 1) * p.c.n_cta + t - 1) / t) - 1;
+    }
+    __device__ MatView view(long long u) const {
+        const long long per = upv();
+        const int vi = (int)(u / per);
+        const int e = __ldcg(p.v_expert + vi);
+        const ExpertMat& d = p.experts[e];
+        MatView v;
+        v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = p.x; v.y = p.y;
+        v.xrows = p.v_xrows + (size_t)vi * kMaxPairsPerVirtual;
+        v.yrows = p.v_yrows + (size_t)vi * kMaxPairsPerVirtual;
+        v.unit0 = (long long)vi * per;
+        v.d_out = p.d_out; v.d_in = p.d_in; v.log2K = d.log2K;
+        v.R8 = R8(); v.S = p.d_in >> 3;
+        v.blk0 = vi * ((v.R8 + kOct - 1) / kOct); v.Mk = __ldcg(p.v_count + vi);
+        return v;
+    }
+};
+
+// A segment: one matrix, one 256-row block, columns [ja, jb), plus what the
+// split-K combine needs.  Each CTA builds its segment table once, in shared
+// memory, so no role ever walks the parameter tables again.
+struct Seg {
+    MatView v;
+    unsigned* counter;      // split blocks: arrival counter
+    int blk, ja, jb, n_oct, n_chunks;
+    int full;               // the segment covers all columns of its block
+    int c_first, c_last;    // CTAs contributing to the block (split blocks)
+    int first_slot;         // partial-sum slot of c_first for this block
+    int my_slot;            // this CTA's partial-sum slot for this block
+};
+constexpr int kSegTab = 32;  // table capacity per round
+constexpr int kSegBytes = 160;  // shared-memory budget per table entry (Cfg::kFixed)
+static_assert(sizeof(Seg) <= kSegBytes, "segment table entry outgrew its shared-memory budget");
+
+template <class Problem>
+__device__ Seg make_seg(const Problem& P, long long u, long long u_end, long long cta_u0) {
+    Seg s;
+    s.v = P.view(u);
+    const long long local = u - s.v.unit0;
+    s.blk = (int)(local / s.v.S);
+    s.ja = (int)(local - (long long)s.blk * s.v.S);
+    const long long jb = (long long)s.ja + (u_end - u);
+    s.jb = (int)(jb < (long long)s.v.S ? jb : (long long)s.v.S);
+    s.n_oct = min(kOct, s.v.R8 - s.blk * kOct);
+    s.n_chunks = ((s.jb - 1) >> 4) - (s.ja >> 4) + 1;
+    s.full = (s.ja == 0 && s.jb == s.v.S);
+    s.counter = nullptr;
+    s.c_first = s.c_last = s.first_slot = s.my_slot = 0;
+    if (!s.full) {
+        const long long b0 = s.v.unit0 + (long long)s.blk * s.v.S;
+        s.c_first = P.cta_of(b0);
+        s.c_last = P.cta_of(b0 + s.v.S - 1);
+        s.first_slot = (P.cta_begin(s.c_first) >= b0) ? 0 : 1;
+        s.my_slot = (cta_u0 >= b0) ? 0 : 1;
+        s.counter = nullptr;
+    }
+    return s;
+}
+
+// Fills tab[0..n) with the segments of [u, u_end) (at most kSegTab); returns n
+// and the first unit not covered.
+template <class Problem>
+__device__ int build_segs(const Problem& P, const Common& C, long long u, long long u_end, long long cta_u0,
+                          Seg* tab, long long* u_next) {
+    int n = 0;
+    while (u < u_end && n < kSegTab) {
+        Seg s = make_seg(P, u, u_end, cta_u0);
+        if (!s.full) s.counter = C.counters + s.v.blk0 + s.blk;
+        tab[n++] = s;
+        u += s.jb - s.ja;
+    }
+    *u_next = u;
+    return n;
+}
+
+// Column range of chunk c of a segment (chunks are cut at group boundaries).
+__device__ __forceinline__ int2 chunk_cols(const Seg& s, int c) {
+    const int g = (s.ja >> 4) + c;
+    return make_int2(max(s.ja, g << 4), min(s.jb, (g + 1) << 4));
+}
+
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
+
+template <int M>
+struct Smem {
+    uint32_t cb0;     // codebook replicas: entry z*8 + r holds codeword z (16 bytes)
+    uint32_t ring0;   // shared address of the staging ring
+    int pc;           // chunks per ring half
+    int cbraw_bytes;
+    uint32_t cbraw0;
+    float* red;
+    float* stash;
+    uint64_t* bars;
+    int* bcast;
+    Seg* segs;
+    __device__ uint32_t slot(int h, int k) const { return ring0 + (h * pc + k) * Cfg<M>::kSlot; }
+    __device__ uint64_t* landed(int h, int k) const { return bars + h * kMaxPass + k; }
+    __device__ uint64_t* ready(int h, int k) const { return bars + 2 * kMaxPass + h * kMaxPass + k; }
+    __device__ uint64_t* pass_empty(int h) const { return bars + 4 * kMaxPass + h; }
+    __device__ uint64_t* cb_full(int h) const { return bars + 4 * kMaxPass + 2 + h; }
+    __device__ uint64_t* cb_empty(int h) const { return bars + 4 * kMaxPass + 4 + h; }
+};
+
+template <int M>
+__device__ __forceinline__ Smem<M> carve(uint8_t* base, int pc, int kmax) {
+    Smem<M> s;
+    s.pc = pc;
+    uint8_t* p = base;
+    s.cb0 = smem_u32(p); p += kmax * 128;
+    s.ring0 = smem_u32(p); p += 2 * pc * Cfg<M>::kSlot;
+    s.cbraw_bytes = kmax * 16;
+    s.cbraw0 = smem_u32(p); p += 2 * kmax * 16;
+    s.red = reinterpret_cast<float*>(p); p += Cfg<M>::kRed;
+    s.stash = reinterpret_cast<float*>(p); p += Cfg<M>::kStash;
+    s.segs = reinterpret_cast<Seg*>(p); p += kSegTab * sizeof(Seg);
+    s.bars = reinterpret_cast<uint64_t*>(p); p += (4 * kMaxPass + 6) * 8;
+    s.bcast = reinterpret_cast<int*>(p);
+    return s;
+}
+
+// Per-role progress that persists across segment-table rounds.
+struct RoleState {
+    int q;     // pass counter (ring phases)
+    int s;     // segment counter (codebook phases)
+};
+
+// ------------------------------------------------------------------------
+// Copy warp: bulk copies of everything static, issued ahead of the decode.
+// ------------------------------------------------------------------------
+template <int M>
+__device__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+    const int lane = threadIdx.x & 31;
+    for (int si = 0; si < n_seg; ++si, ++st.s) {
+        const Seg& g = sm.segs[si];
+        const int s = st.s;
+        if (s >= 2 && !mbar_wait(sm.cb_empty(s & 1), ((s >> 1) - 1) & 1)) flag(C.status, kDevTimeout);
+        const uint32_t cbb = (uint32_t)(16u << g.v.log2K);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(sm.cb_full(s & 1), cbb);
+            bulk_g2s(sm.cbraw0 + (s & 1) * sm.cbraw_bytes, g.v.cb, cbb, sm.cb_full(s & 1));
+        }
+        const int n_pass = (g.n_chunks + sm.pc - 1) / sm.pc;
+        const int n_oct = g.n_oct, R8 = g.v.R8, S = g.v.S, G = g.v.d_in >> 7, blk = g.blk;
+        for (int t = 0; t < n_pass; ++t, ++st.q) {
+            const int q = st.q, h = q & 1;
+            if (q >= 2 && !mbar_wait(sm.pass_empty(h), ((q >> 1) - 1) & 1)) flag(C.status, kDevTimeout);
+            for (int k = 0; k < sm.pc; ++k) {
+                const int c = t * sm.pc + k;
+                if (c >= g.n_chunks) {
+                    if (lane == 0) mbar_arrive(sm.landed(h, k));
+                    continue;
+                }
+                const int2 cc = chunk_cols(g, c);
+                const int nj = cc.y - cc.x;
+                const uint32_t tx = (uint32_t)(nj * n_oct * 16 + n_oct * 64 + (g.v.perm ? nj * 32 : 0));
+                if (lane == 0) mbar_arrive_expect_tx(sm.landed(h, k), tx);
+                __syncwarp();
+                const uint32_t dst = sm.slot(h, k);
+                if (lane == 0)  // the chunk's records: one contiguous range of the block
+                    bulk_g2s(dst, g.v.main + main_word(R8, S, blk, cc.x, 0, 0), nj * n_oct * 16, sm.landed(h, k));
+                if (lane == 16)
+                    bulk_g2s(dst + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0), n_oct * 64,
+                             sm.landed(h, k));
+                if (lane == 17 && g.v.perm)
+                    bulk_g2s(dst + kMainSlot + kMetaSlot, g.v.perm + cc.x * 8, nj * 32, sm.landed(h, k));
+            }
+        }
+    }
+}
+
+template <int M>
+__device__ void copy_drain(const Common& C, const Smem<M>& sm, const RoleState& st) {
+    // The CTA may not exit while bulk copies are in flight.
+    for (int qq = max(0, st.q - 2); qq < st.q; ++qq)
+        for (int k = 0; k < sm.pc; ++k)
+            if (!mbar_wait(sm.landed(qq & 1, k), (qq >> 1) & 1)) flag(C.status, kDevTimeout);
+}
+
+// ------------------------------------------------------------------------
+// Activation warp: x_perm for every chunk (after the preceding kernel).
+// ------------------------------------------------------------------------
+template <int M>
+__device__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+    const int lane = threadIdx.x & 31;
+    for (int si = 0; si < n_seg; ++si) {
+        const Seg& g = sm.segs[si];
+        const int n_pass = (g.n_chunks + sm.pc - 1) / sm.pc;
+        const uint16_t* xbase = g.v.x;
+        const int32_t* xrows = g.v.xrows;
+        const int32_t* perm = g.v.perm;
+        const int d_in = g.v.d_in, Mk = g.v.Mk;
+        for (int t = 0; t < n_pass; ++t, ++st.q) {
+            const int q = st.q, h = q & 1;
+            const int c0 = t * sm.pc, c1 = min(g.n_chunks, c0 + sm.pc);
+            for (int c = c0; c < c1; ++c)  // the permutation slices must have landed
+                if (!mbar_wait(sm.landed(h, c - c0), (q >> 1) & 1)) flag(C.status, kDevTimeout);
+            const int pa = chunk_cols(g, c0).x, pb = chunk_cols(g, c1 - 1).y;
+            const int ncol = pb - pa, total = Mk * ncol;
+            // All loads of a round are issued before any store, so a pass costs
+            // one memory round trip per 128 (batch row, column) pairs.
+            for (int e0 = 0; e0 < total; e0 += 4 * 32) {
+                uint4 val[4];
+                uint32_t dst[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int e = e0 + r * 32 + lane;
+                    dst[r] = 0xffffffffu;
+                    if (e < total) {
+                        const int m = e / ncol, j = pa + (e - m * ncol);
+                        const int k = (j >> 4) - (pa >> 4);
+                        const int i = j - max(pa, (j >> 4) << 4);
+                        const uint32_t base = sm.slot(h, k);
+                        const int xr_idx = xrows ? __ldcg(xrows + m) : m;
+                        const uint16_t* xr = xbase + (size_t)xr_idx * d_in;
+                        if (perm) {
+                            const uint32_t sp = base + kMainSlot + kMetaSlot + i * 32;
+                            const uint4 pa4 = lds128(sp), pb4 = lds128(sp + 16);
+                            val[r].x = (uint32_t)xr[pa4.x] | ((uint32_t)xr[pa4.y] << 16);
+                            val[r].y = (uint32_t)xr[pa4.z] | ((uint32_t)xr[pa4.w] << 16);
+                            val[r].z = (uint32_t)xr[pb4.x] | ((uint32_t)xr[pb4.y] << 16);
+                            val[r].w = (uint32_t)xr[pb4.z] | ((uint32_t)xr[pb4.w] << 16);
+                        } else {
+                            val[r] = *reinterpret_cast<const uint4*>(xr + j * 8);
+                        }
+                        dst[r] = base + kMainSlot + kMetaSlot + kPermSlot + (m * kChunkJ + i) * 16;
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (dst[r] != 0xffffffffu) sts128(dst[r], val[r]);
+            }
+            for (int k = 0; k < sm.pc; ++k) mbar_arrive(sm.ready(h, k));
+        }
+    }
+}
+
+// ------------------------------------------------------------------------
+// Decode warps.
+// ------------------------------------------------------------------------
+struct VDec {            // per-split decode constants (radius width V = 10 - log2K)
+    uint32_t zmask, qmask;
+    uint32_t sh0, sh1, sh2, sh3, sh4, sh5;   // 15 - (sign slot position)
+    float vscale;
+};
+
+__device__ __forceinline__ VDec vdec(int log2K) {
+    const int V = 10 - log2K;
+    VDec d;
+    d.zmask = ((1u << log2K) - 1u) << 7;
+    d.qmask = ((1u << V) - 1u) << (23 - V);
+    // slot k sits at bit k for k <= 6 - V, else at bit 10 + k
+    auto sh = [&](int k) { return (uint32_t)(k <= 6 - V ? 15 - k : 5 - k); };
+    d.sh0 = sh(0); d.sh1 = sh(1); d.sh2 = sh(2); d.sh3 = sh(3); d.sh4 = sh(4); d.sh5 = sh(5);
+    d.vscale = (float)(1 << V);
+    return d;
+}
+
+template <int M>
+__device__ __forceinline__ void decode_record(const VDec& d, uint4 rec, const uint32_t (&aux)[8], uint32_t sh_aux,
+                                              const float (&mup)[8], const float (&dlp)[8], uint32_t cbsel,
+                                              const uint4 (&xv)[M], float (&acc)[8][M]) {
+    const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint32_t wa = wv[u];
+        const uint32_t wb = rot16(wa);
+        {   // row A = 2u: z at [7, 7 + log2K), q at [23 - V, 23) of wa; signs in slots 0..2
+            uint4 c = lds128(cbsel + (wa & d.zmask));
+            c.x ^= (wa << d.sh0) & 0x80008000u;
+            c.y ^= (wa << d.sh1) & 0x80008000u;
+            c.z ^= (wa << d.sh2) & 0x80008000u;
+            c.w ^= (aux[2 * u] << sh_aux) & 0x80008000u;
+            const float r = fmaf(__uint_as_float((wa & d.qmask) | 0x3F800000u), dlp[2 * u], mup[2 * u]);
+#pragma unroll
+            for (int m = 0; m < M; ++m) acc[2 * u][m] = fmaf(r, signed_dot(c, xv[m]), acc[2 * u][m]);
+        }
+        {   // row B = 2u + 1: the same fields after a 16-bit rotation; signs in slots 3..5
+            uint4 c = lds128(cbsel + (wb & d.zmask));
+            c.x ^= (wa << d.sh3) & 0x80008000u;
+            c.y ^= (wa << d.sh4) & 0x80008000u;
+            c.z ^= wa & 0x80008000u;  // slot 5 sits at bit 15 for every split
+            c.w ^= (aux[2 * u + 1] << sh_aux) & 0x80008000u;
+            const float r = fmaf(__uint_as_float((wb & d.qmask) | 0x3F800000u), dlp[2 * u + 1], mup[2 * u + 1]);
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                acc[2 * u + 1][m] = fmaf(r, signed_dot(c, xv[m]), acc[2 * u + 1][m]);
+        }
+    }
+}
+
+// Decode this warp's share of one pass (columns [pa, pb) of segment g).
+template <int M, int MS>
+__device__ __forceinline__ void decode_pass(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int h,
+                                            uint32_t parity, int pa, int pb, int warp, int lane, float (&acc)[8][M]) {
+    constexpr int W = Cfg<MS>::kW;
+    const int n = pb - pa;
+    const int ra = pa + (warp * n) / W, rb = pa + ((warp + 1) * n) / W;
+    const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
+    const int n_oct = g.n_oct;
+    const bool active = lane < n_oct;
+    uint32_t aux[8];
+    float mup[8], dlp[8];
+    int kcur = -1, gcur = -1;
+    uint32_t base = 0;
+    int j0 = 0;
+    for (int j = ra; j < rb; ++j) {
+        const int k = (j >> 4) - (pa >> 4);
+        if (k != kcur) {
+            if (!mbar_wait(sm.landed(h, k), parity)) flag(C.status, kDevTimeout);
+            if (!mbar_wait(sm.ready(h, k), parity)) flag(C.status, kDevTimeout);
+            kcur = k;
+            base = sm.slot(h, k);
+            j0 = max(pa, (j >> 4) << 4);
+        }
+        if (!active) continue;
+        if ((j >> 4) != gcur) {
+            gcur = j >> 4;
+            const uint32_t a = base + kMainSlot + lane * 64;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint4 q = lds128(a + e * 16);
+                aux[2 * e] = q.x;
+                aux[2 * e + 1] = q.z;
+                const float2 m0 = __half22float2(u2h2(q.y));
+                const float2 m1 = __half22float2(u2h2(q.w));
+                dlp[2 * e] = m0.y * d.vscale;
+                mup[2 * e] = m0.x - dlp[2 * e];
+                dlp[2 * e + 1] = m1.y * d.vscale;
+                mup[2 * e + 1] = m1.x - dlp[2 * e + 1];
+            }
+        }
+        const int i = j - j0;
+        const uint4 rec = lds128(base + (i * n_oct + lane) * 16);
+        uint4 xv[M];
+        const uint32_t sx = base + kMainSlot + kMetaSlot + kPermSlot;
+#pragma unroll
+        for (int m = 0; m < M; ++m) xv[m] = lds128(sx + (m * kChunkJ + i) * 16);
+        decode_record<M>(d, rec, aux, (uint32_t)(15 - (j & 15)), mup, dlp, cbsel, xv, acc);
+    }
+}
+
+// Writes (or combines) the outputs of the pending segments tab[i0 .. i0 + n).
+// Split blocks: every contributor stores its partial sums, the CTA's writes are
+// published with one release atomic per block, and the contributor that sees
+// the count complete (acquire) adds all partials in CTA order.
+template <int M>
+__device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
+    constexpr int DT = Cfg<M>::kDecodeThreads;
+    const int tid = threadIdx.x;
+    const int cta = blockIdx.x;
+    const int l = tid & 31, r = tid >> 5;
+    const int row_local = l * 8 + r;
+    bool any_partial = false;
+    for (int i = 0; i < n; ++i) {
+        const Seg& g = sm.segs[i0 + i];
+        const int row = g.blk * kBlockRows + row_local;
+        const float* st = sm.stash + (size_t)i * M * kBlockRows;
+        if (g.full) {
+            if (tid < kBlockRows && row < g.v.d_out) {
+#pragma unroll
+                for (int m = 0; m < M; ++m)
+                    if (m < g.v.Mk) {
+                        const int yr = g.v.yrows ? __ldcg(g.v.yrows + m) : m;
+                        g.v.y[(size_t)yr * g.v.d_out + row] = __half_as_ushort(__float2half_rn(st[m * kBlockRows + row_local]));
+                    }
+            }
+        } else {
+            any_partial = true;
+            float* part = C.partials + ((size_t)(cta * 2 + g.my_slot) * 8) * kBlockRows;
+            if (tid < kBlockRows)
+#pragma unroll
+                for (int m = 0; m < M; ++m) part[m * kBlockRows + row_local] = st[m * kBlockRows + row_local];
+        }
+    }
+    if (!any_partial) return;  // uniform across the decode threads
+    named_barrier(1, DT);      // every partial store of the CTA precedes the release below
+    if (tid < n) {
+        const Seg& g = sm.segs[i0 + tid];
+        int last = 0;
+        if (!g.full) {
+            const unsigned old = atom_add_acq_rel_gpu(g.counter, 1u);
+            last = (old == (unsigned)(g.c_last - g.c_first));
+            if (last) *reinterpret_cast<volatile unsigned*>(g.counter) = 0u;  // restore for the next call
+        }
+        sm.bcast[tid] = last;
+    }
+    named_barrier(1, DT);
+    for (int i = 0; i < n; ++i) {
+        const Seg& g = sm.segs[i0 + i];
+        if (!sm.bcast[i]) continue;
+        const int row = g.blk * kBlockRows + row_local;
+        if (tid < kBlockRows && row < g.v.d_out) {
+            const int c_first = g.c_first, c_last = g.c_last, first_slot = g.first_slot;
+            float tot[M];
+#pragma unroll
+            for (int m = 0; m < M; ++m) tot[m] = 0.f;
+            for (int c0 = c_first; c0 <= c_last; c0 += 8) {
+                float v[8][M];   // up to 8 contributors' loads in flight at once
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int c = c0 + k;
+                    const int sp = (c == c_first) ? first_slot : 0;
+                    const float* src = C.partials + ((size_t)(c * 2 + sp) * 8) * kBlockRows + row_local;
+#pragma unroll
+                    for (int m = 0; m < M; ++m) v[k][m] = (c <= c_last) ? __ldcg(src + m * kBlockRows) : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+#pragma unroll
+                    for (int m = 0; m < M; ++m) tot[m] += v[k][m];
+            }
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                if (m < g.v.Mk) {
+                    const int yr = g.v.yrows ? __ldcg(g.v.yrows + m) : m;
+                    g.v.y[(size_t)yr * g.v.d_out + row] = __half_as_ushort(__float2half_rn(tot[m]));
+                }
+        }
+    }
+    named_barrier(1, DT);  // bcast reuse
+}
+
+// Decodes one segment with compile-time batch MK (<= MS, the launch's stash
+// stride) and leaves its 256 x MS results in stash slot `slot`.
+template <int MK, int MS>
+__device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, int q0, int slot) {
+    constexpr int W = Cfg<MS>::kW, DT = Cfg<MS>::kDecodeThreads;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const VDec d = vdec(g.v.log2K);
+    float acc[8][MK];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int m = 0; m < MK; ++m) acc[r][m] = 0.f;
+    const int n_pass = (g.n_chunks + sm.pc - 1) / sm.pc;
+    int q = q0;
+    for (int t = 0; t < n_pass; ++t, ++q) {
+        const int h = q & 1;
+        const int2 first = chunk_cols(g, t * sm.pc);
+        const int2 last = chunk_cols(g, min(g.n_chunks, (t + 1) * sm.pc) - 1);
+        decode_pass<MK, MS>(sm, C, g, d, h, (q >> 1) & 1, first.x, last.y, warp, lane, acc);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.pass_empty(h));
+    }
+    // reduce the warps' partial sums in a fixed order into the stash
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int m = 0; m < MK; ++m) sm.red[((warp * 8 + r) * MK + m) * 32 + lane] = acc[r][m];
+    named_barrier(1, DT);
+    if (tid < kBlockRows) {
+        const int l = tid & 31, r = tid >> 5;
+        for (int m = 0; m < MS; ++m) {
+            float sum = 0.f;
+            if (m < MK) {
+#pragma unroll
+                for (int w = 0; w < W; ++w) sum += sm.red[((w * 8 + r) * MK + m) * 32 + l];
+            }
+            sm.stash[((size_t)slot * MS + m) * kBlockRows + l * 8 + r] = sum;
+        }
+    }
+    named_barrier(1, DT);
+}
+
+template <int MLO, int M>
+__device__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+    constexpr int DT = Cfg<M>::kDecodeThreads;
+    const int tid = threadIdx.x;
+    int npend = 0, i_pend = 0;
+    const uint16_t* cur_cb = nullptr;
+    for (int si = 0; si < n_seg; ++si, ++st.s) {
+        const Seg& g = sm.segs[si];
+        const int s = st.s;
+        if (!mbar_wait(sm.cb_full(s & 1), (s >> 1) & 1)) flag(C.status, kDevTimeout);
+        if (g.v.cb != cur_cb) {  // build the 8 bank-rotated replicas from the raw copy
+            if (cur_cb) named_barrier(1, DT);
+            const int K = 1 << g.v.log2K;
+            const uint32_t raw = sm.cbraw0 + (s & 1) * sm.cbraw_bytes;
+            for (int e = tid; e < K * 8; e += DT) sts128(sm.cb0 + e * 16, lds128(raw + (e >> 3) * 16));
+            named_barrier(1, DT);
+            cur_cb = g.v.cb;
+        }
+        if (tid == 0) mbar_arrive(sm.cb_empty(s & 1));
+        if constexpr (MLO == M) {
+            segment_body<M, M>(sm, C, g, st.q, npend);
+        } else {
+            switch (g.v.Mk) {
+                case 1: segment_body<1, M>(sm, C, g, st.q, npend); break;
+                case 2: segment_body<2, M>(sm, C, g, st.q, npend); break;
+                case 3: segment_body<3, M>(sm, C, g, st.q, npend); break;
+                case 4: segment_body<4, M>(sm, C, g, st.q, npend); break;
+                case 5: segment_body<5, M>(sm, C, g, st.q, npend); break;
+                case 6: segment_body<6, M>(sm, C, g, st.q, npend); break;
+                case 7: segment_body<7, M>(sm, C, g, st.q, npend); break;
+                default: segment_body<8, M>(sm, C, g, st.q, npend); break;
+            }
+        }
+        st.q += (g.n_chunks + sm.pc - 1) / sm.pc;
+        ++npend;
+        if (npend == kMaxSegs || si + 1 == n_seg) {
+            flush<M>(C, sm, i_pend, npend);
+            npend = 0;
+            i_pend = si + 1;
+        }
+    }
+}
+
+template <int MLO, int M, class Problem>
+__device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* smem_raw, bool plan_needs_wait) {
+    const Smem<M> sm = carve<M>(smem_raw, C.pass_chunks, C.kmax);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        for (int h = 0; h < 2; ++h) {
+            for (int k = 0; k < kMaxPass; ++k) {
+                mbar_init(sm.landed(h, k), 1);
+                mbar_init(sm.ready(h, k), 32);
+            }
+            mbar_init(sm.pass_empty(h), Cfg<M>::kW);
+            mbar_init(sm.cb_full(h), 1);
+            mbar_init(sm.cb_empty(h), 1);
+        }
+        fence_mbar_init();
+    }
+    pdl_launch_dependents();
+    if (plan_needs_wait) pdl_wait();  // the plan itself depends on preceding work
+    __shared__ long long s_next;
+    __shared__ int s_nseg;
+    const long long total = P.total();
+    const long long u0 = total > 0 ? P.cta_begin(blockIdx.x) : 0;
+    const long long u1 = total > 0 ? P.cta_begin(blockIdx.x + 1) : 0;
+    RoleState st{0, 0};
+    bool waited = plan_needs_wait;
+    for (long long u = u0; u < u1;) {
+        if (tid == 0) s_nseg = build_segs(P, C, u, u1, u0, sm.segs, &s_next);
+        __syncthreads();
+        const int n_seg = s_nseg;
+        if (warp == Cfg<M>::kW) {
+            copy_warp<M>(C, sm, n_seg, st);
+        } else if (warp == Cfg<M>::kW + 1) {
+            if (!waited) pdl_wait();  // activations may come from the preceding kernel
+            waited = true;
+            act_warp<M>(C, sm, n_seg, st);
+        } else {
+            decode_warps<MLO, M>(C, sm, n_seg, st);
+        }
+        u = s_next;
+        __syncthreads();  // the segment table is rebuilt for the next round
+    }
+    if (warp == Cfg<M>::kW) copy_drain<M>(C, sm, st);
+    if (warp == Cfg<M>::kW + 1 && !waited) pdl_wait();
+}
+
+template <int M>
+__global__ void __launch_bounds__(Cfg<M>::kThreads, Cfg<M>::kMinBlocks) gemv_kernel(const __grid_constant__ DenseParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const DenseProblem P{p};
+    run<M, M>(P, p.c, smem_raw, false);
+}
+
+// Virtual experts carry 1..8 pairs; each segment dispatches on its own count.
+__global__ void __launch_bounds__(Cfg<kMaxPairsPerVirtual>::kThreads, 1) moe_kernel(const __grid_constant__ MoeParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const MoeProblem P{p};
+    run<1, kMaxPairsPerVirtual>(P, p.c, smem_raw, true);
+}
+
+// Groups the (pair -> expert) routing into virtual experts of at most 8 pairs,
+// in expert order and, within an expert, pair order (deterministic).
+__global__ void moe_route_kernel(const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs, int n_experts,
+                                 MoeRoute* route, int32_t* v_expert, int32_t* v_xrows, int32_t* v_yrows,
+                                 int32_t* v_count, uint32_t* status) {
+    pdl_wait();
+    extern __shared__ int s_cnt[];  // [n_experts]
+    for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    for (int q = threadIdx.x; q < n_pairs; q += blockDim.x) {
+        const int e = pair_expert[q];
+        if (e >= 0 && e < n_experts) atomicAdd(&s_cnt[e], 1);
+        else atomicOr(status, kDevUnsupported);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int nv = 0;
+        for (int e = 0; e < n_experts; ++e) {
+            const int c = s_cnt[e];
+            s_cnt[e] = nv;  // first virtual index of expert e
+            nv += (c + kMaxPairsPerVirtual - 1) / kMaxPairsPerVirtual;
+        }
+        route->n_virtual = nv;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
+        int vi = s_cnt[e], k = 0;
+        for (int q = 0; q < n_pairs; ++q) {
+            if (pair_expert[q] != e) continue;
+            if (k == kMaxPairsPerVirtual) { ++vi; k = 0; }
+            v_expert[vi] = e;
+            v_xrows[(size_t)vi * kMaxPairsPerVirtual + k] = pair_xrow[q];
+            v_yrows[(size_t)vi * kMaxPairsPerVirtual + k] = q;
+            v_count[vi] = ++k;
+        }
+    }
+    pdl_launch_dependents();
+}
+
+int g_sm_count = 0;
+std::once_flag g_once;
+
+int sm_count() {
+    std::call_once(g_once, [] {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (g_sm_count <= 0) g_sm_count = 148;
+    });
+    return g_sm_count;
+}
+
+long long units_of(const sage_matrix& A) {
+    const int R8 = (A.d_out + 7) / 8;
+    return (long long)((R8 + kOct - 1) / kOct) * (A.d_in / 8);
+}
+int blocks_of(const sage_matrix& A) { return ((A.d_out + 7) / 8 + kOct - 1) / kOct; }
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// CTA counts per matrix for a dense launch.  If giving every matrix its own
+// CTAs keeps the largest CTA within 6% of an even split of all units, each
+// matrix gets its own CTAs (one codebook per CTA, fewer segments); otherwise
+// the plan is plain stream-K over the flattened units (returns empty).
+std::vector<int> per_matrix_shares(const std::vector<long long>& units, int n_cta) {
+    long long total = 0;
+    for (long long u : units) total += u;
+    const int n_mat = (int)units.size();
+    if (n_mat == 1 || n_mat > n_cta) return {};
+    std::vector<int> share((size_t)n_mat);
+    int given = 0;
+    for (int k = 0; k < n_mat; ++k) {
+        share[k] = std::max(1, (int)((double)units[k] * n_cta / total));
+        given += share[k];
+    }
+    while (given < n_cta) {  // hand out the rest to the most loaded matrix
+        int best = 0;
+        for (int k = 1; k < n_mat; ++k)
+            if ((double)units[k] / share[k] > (double)units[best] / share[best]) best = k;
+        ++share[best];
+        ++given;
+    }
+    if (given > n_cta) return {};
+    double worst = 0;
+    for (int k = 0; k < n_mat; ++k) {
+        if (share[k] > units[k]) return {};
+        worst = std::max(worst, (double)units[k] / share[k]);
+    }
+    if (worst > 1.06 * (double)total / n_cta) return {};
+    return share;
+}
+
+// Chunks per ring half: the whole CTA range when it fits, keeping the CTA's
+// shared memory under ~110 KB so that two CTAs (this kernel's and the next
+// kernel's in a PDL chain) can share an SM.
+template <int M>
+int pass_chunks_for(long long max_units_per_cta, int kmax) {
+    const long long chunks = (max_units_per_cta + kChunkJ - 1) / kChunkJ + 2;
+    int pc = (int)std::min<long long>(kMaxPass, std::max<long long>(1, (chunks + 1) / 2));
+    const int budget = (Cfg<M>::kMinBlocks > 1 ? 110 : 220) * 1024;
+    while (pc > 1 && Cfg<M>::smem(pc, kmax) > budget) --pc;
+    return pc;
+}
+
+// Raises the kernel's dynamic shared memory limit when a launch needs more
+// than any earlier one (callers hold the launch mutex).
+template <class K>
+bool ensure_smem(K kernel, int bytes, int& configured) {
+    if (bytes <= configured) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    configured = bytes;
+    return true;
+}
+
+template <class K, class Params>
+int launch_pdl(K kernel, const Params& p, int grid, int threads, int smem, sage_stream_t stream) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+
+template <int M>
+int launch_m(const GemvJob* jobs, int n, void* ws, sage_stream_t stream) {
+    static DenseParams p;  // large: keep off the stack
+    static std::mutex mu;
+    static int configured = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    std::vector<long long> units((size_t)n);
+    long long unit = 0;
+    int blk = 0, kmax = 16;
+    for (int i = 0; i < n; ++i) {
+        const sage_matrix& A = jobs[i].A;
+        kmax = std::max(kmax, 1 << A.log2K);
+        DenseMat& d = p.mats[i];
+        d.main = A.main; d.meta = A.meta; d.cb = A.codebook; d.perm = A.perm;
+        d.x = jobs[i].x; d.y = jobs[i].y;
+        d.d_out = A.d_out; d.d_in = A.d_in; d.log2K = A.log2K;
+        d.unit0 = unit; d.blk0 = blk;
+        units[i] = units_of(A);
+        unit += units[i];
+        blk += blocks_of(A);
+    }
+    const int n_cta = (int)std::max<long long>(1, std::min<long long>(sm_count(), unit / 4));
+    const std::vector<int> share = per_matrix_shares(units, n_cta);
+    long long widest = 0;
+    p.per_matrix = share.empty() ? 0 : 1;
+    int cta = 0;
+    for (int i = 0; i < n; ++i) {
+        p.mats[i].units = units[i];
+        p.mats[i].cta0 = cta;
+        p.mats[i].ncta = share.empty() ? 0 : share[i];
+        cta += p.mats[i].ncta;
+        if (!share.empty()) widest = std::max(widest, (units[i] + share[i] - 1) / share[i]);
+    }
+    if (share.empty()) widest = (unit + n_cta - 1) / n_cta;
+    p.n_mats = n;
+    p.total_units = unit;
+    p.c.n_cta = n_cta;
+    p.c.M = M;
+    p.c.pass_chunks = pass_chunks_for<M>(widest, kmax);
+    p.c.kmax = kmax;
+    if (!ensure_smem(gemv_kernel<M>, Cfg<M>::smem(p.c.pass_chunks, kmax), configured)) return SAGE_ERR_CUDA;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.c.status = reinterpret_cast<uint32_t*>(w);
+    p.c.counters = reinterpret_cast<unsigned*>(w + kWsHeader);
+    p.c.partials = reinterpret_cast<float*>(w + kWsHeader + round256((size_t)blk * 4));
+    return launch_pdl(gemv_kernel<M>, p, n_cta, Cfg<M>::kThreads, Cfg<M>::smem(p.c.pass_chunks, kmax), stream);
+}
+
+}  // namespace
+
+size_t gemv_workspace_bytes(const sage_matrix* mats, int n, int M) {
+    (void)M;
+    long long units = 0;
+    int blk = 0;
+    for (int i = 0; i < n; ++i) { units += units_of(mats[i]); blk += blocks_of(mats[i]); }
+    const int n_cta = (int)std::max<long long>(1, std::min<long long>(sm_count(), units / 4));
+    return kWsHeader + round256((size_t)blk * 4) + (size_t)n_cta * 2 * 8 * kBlockRows * sizeof(float);
+}
+
+int launch_gemv(const GemvJob* jobs, int n, int M, void* ws, size_t ws_bytes, sage_stream_t stream) {
+    if (n > kMaxMats) return SAGE_ERR_UNSUPPORTED;
+    std::vector<sage_matrix> mats((size_t)n);
+    for (int i = 0; i < n; ++i) mats[i] = jobs[i].A;
+    if (ws_bytes < gemv_workspace_bytes(mats.data(), n, M)) return SAGE_ERR_WORKSPACE;
+    switch (M) {
+        case 1: return launch_m<1>(jobs, n, ws, stream);
+        case 2: return launch_m<2>(jobs, n, ws, stream);
+        case 3: return launch_m<3>(jobs, n, ws, stream);
+        case 4: return launch_m<4>(jobs, n, ws, stream);
+        case 5: return launch_m<5>(jobs, n, ws, stream);
+        case 6: return launch_m<6>(jobs, n, ws, stream);
+        case 7: return launch_m<7>(jobs, n, ws, stream);
+        case 8: return launch_m<8>(jobs, n, ws, stream);
+        default: return SAGE_ERR_UNSUPPORTED;
+    }
+}
+
+// MoE workspace: header | route | v_expert | v_xrows | v_yrows | v_count | counters | partials
+namespace {
+struct MoeWs {
+    size_t route, v_expert, v_xrows, v_yrows, v_count, counters, partials, total;
+};
+MoeWs moe_ws_layout(int n_pairs, int d_out, int n_cta) {
+    MoeWs L;
+    size_t o = kWsHeader;
+    L.route = o; o += 256;
+    L.v_expert = o; o += round256((size_t)n_pairs * 4);
+    L.v_xrows = o; o += round256((size_t)n_pairs * kMaxPairsPerVirtual * 4);
+    L.v_yrows = o; o += round256((size_t)n_pairs * kMaxPairsPerVirtual * 4);
+    L.v_count = o; o += round256((size_t)n_pairs * 4);
+    const int nblk = ((d_out + 7) / 8 + kOct - 1) / kOct;
+    L.counters = o; o += round256((size_t)n_pairs * nblk * 4);
+    L.partials = o; o += (size_t)n_cta * 2 * 8 * kBlockRows * sizeof(float);
+    L.total = o;
+    return L;
+}
+}  // namespace
+
+size_t moe_workspace_bytes(const sage_matrix* experts, int n_experts, int n_pairs) {
+    (void)n_experts;
+    return moe_ws_layout(std::max(1, n_pairs), experts[0].d_out, sm_count()).total;
+}
+
+int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_expert, const int32_t* pair_xrow,
+               int n_pairs, const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream) {
+    constexpr int MV = kMaxPairsPerVirtual;
+    if (n_experts > kMaxExperts) return SAGE_ERR_UNSUPPORTED;
+    const int n_cta = sm_count();
+    const MoeWs L = moe_ws_layout(n_pairs, experts[0].d_out, n_cta);
+    if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    static MoeParams p;
+    static std::mutex mu;
+    static int configured = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    p.c.n_cta = n_cta;
+    p.c.M = 0;
+    int kmax = 16;
+    for (int e = 0; e < n_experts; ++e) kmax = std::max(kmax, 1 << experts[e].log2K);
+    p.c.kmax = kmax;
+    p.c.pass_chunks = pass_chunks_for<MV>(1 << 30, kmax);
+    if (!ensure_smem(moe_kernel, Cfg<MV>::smem(p.c.pass_chunks, kmax), configured)) return SAGE_ERR_CUDA;
+    p.c.status = reinterpret_cast<uint32_t*>(w);
+    p.c.counters = reinterpret_cast<unsigned*>(w + L.counters);
+    p.c.partials = reinterpret_cast<float*>(w + L.partials);
+    p.n_experts = n_experts;
+    p.d_out = experts[0].d_out;
+    p.d_in = experts[0].d_in;
+    p.n_pairs = n_pairs;
+    p.x = x;
+    p.y = y;
+    p.route = reinterpret_cast<const MoeRoute*>(w + L.route);
+    p.v_expert = reinterpret_cast<const int32_t*>(w + L.v_expert);
+    p.v_xrows = reinterpret_cast<const int32_t*>(w + L.v_xrows);
+    p.v_yrows = reinterpret_cast<const int32_t*>(w + L.v_yrows);
+    p.v_count = reinterpret_cast<const int32_t*>(w + L.v_count);
+    for (int e = 0; e < n_experts; ++e) {
+        p.experts[e].main = experts[e].main;
+        p.experts[e].meta = experts[e].meta;
+        p.experts[e].cb = experts[e].codebook;
+        p.experts[e].perm = experts[e].perm;
+        p.experts[e].log2K = experts[e].log2K;
+    }
+    {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = (size_t)n_experts * sizeof(int);
+        cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, moe_route_kernel, pair_expert, pair_xrow, n_pairs, n_experts,
+                               reinterpret_cast<MoeRoute*>(w + L.route), reinterpret_cast<int32_t*>(w + L.v_expert),
+                               reinterpret_cast<int32_t*>(w + L.v_xrows), reinterpret_cast<int32_t*>(w + L.v_yrows),
+                               reinterpret_cast<int32_t*>(w + L.v_count), p.c.status) != cudaSuccess)
+            return SAGE_ERR_CUDA;
+    }
+    return launch_pdl(moe_kernel, p, n_cta, Cfg<MV>::kThreads, Cfg<MV>::smem(p.c.pass_chunks, kmax), stream);
+}
+
+}  // namespace sage

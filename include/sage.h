@@ -1,0 +1,211 @@
+/*
+ * sage.h -- C ABI of libsage, a B200 (sm_100a) implementation of the SAGE
+ * packed linear layer y = W_hat x computed straight from 2.25-bit codes.
+ *
+ * Method: "SAGE: Pushing 2-Bit Vector-Quantized LLMs toward Real-World
+ * Usability" (Yan et al.).  Each row of W is cut into subvectors of v = 8
+ * input channels (in ESG-permuted order); a subvector is rebuilt as
+ *     w_hat = r_hat * (s (.) c_z),   r_hat = mu_g + q * delta_g      (Sec. 3.1, Eq. 1-2)
+ * with s the 8 stored signs, c_z one of K nonnegative unit fp16 codewords of a
+ * per-matrix codebook, and (mu_g, delta_g) an fp16 radius grid shared by the
+ * 16 consecutive subvectors (G = 128 weights) of a row group (App. A.6,
+ * Eq. 14).  A subvector costs v + log2 K + V = 18 bits (Eq. 3) for every
+ * split (K, V) with log2 K + V = 10 (Sec. 3.3); the layout below keeps the
+ * paper's "16-bit main word plus two auxiliary bits" per subvector (Sec. 3.5).
+ *
+ * Conventions
+ *  - Every function returns a sage_status (int).  Argument errors are detected
+ *    on the host before anything is enqueued; no compute call enqueues work
+ *    after returning an error.
+ *  - Device pointers are allocated and owned by the caller.  The library never
+ *    allocates device memory and never synchronises the host with the device in
+ *    compute calls; work is enqueued on the caller's stream.
+ *  - fp16 values cross the ABI as uint16_t bit patterns (IEEE binary16).
+ *  - Compute calls take a caller-allocated device workspace of at least
+ *    sage_workspace_size() bytes, zero-filled once before first use (cudaMemset).
+ *    Its first 256 bytes hold a device status word; the library restores every
+ *    other byte it uses to its initial state, so the workspace may be reused
+ *    across calls on one stream.  Calls that share a workspace must not overlap
+ *    on the device.
+ *  - Device pointers must be 16-byte aligned (SAGE_ERR_MISALIGNED otherwise).
+ *
+ * ------------------------------------------------------------------------
+ * Packed format v2 (this library's layout; the paper gives only the widths)
+ * ------------------------------------------------------------------------
+ *  d_in % 128 == 0, 4 <= log2K <= 8, V = 10 - log2K, K = 2^log2K.
+ *  Subvector column j = 0 .. S-1 (S = d_in/8) covers storage columns
+ *  8j .. 8j+7; group g = j / 16 (G = d_in/128 groups).  R8 = ceil(d_out/8)
+ *  row octets; octet b holds rows 8b .. 8b+7 (rows >= d_out are padding and
+ *  must be zero).  Octets form blocks of 32 (256 rows); block B holds
+ *  n_B = min(32, R8 - 32B) octets and is stored contiguously, so one block's
+ *  columns [ja, jb) are one contiguous range of both planes.
+ *
+ *  main plane (uint32 words): the 16-byte record of (column j, local octet o
+ *    of block B) is words B*S*128 + (j*n_B + o)*4 .. +3.  Word u holds row
+ *    A = 8(32B + o) + 2u and row B = row A + 1:
+ *      z_A  bits [7, 7 + log2K)        q_A  bits [23 - V, 23)
+ *      z_B  bits [23, 23 + log2K)      q_B  bits [7 - V, 7)
+ *      six sign slots at the ascending bit positions p_0 < ... < p_5 of
+ *      {0 .. 6 - V} U {17 - V .. 15}; slot k owns bits p_k and p_k + 16.
+ *      Slots 0..2 hold row A's component pairs 0..2, slots 3..5 row B's;
+ *      pair n is components (2n, 2n + 1): bit p_k = sign of component 2n,
+ *      bit p_k + 16 = sign of component 2n + 1 (1 = negative).
+ *  meta plane: 8-byte entries; entry (group g, local octet o of block B,
+ *    row t of the octet) is entry B*G*256 + (g*n_B + o)*8 + t =
+ *    { uint32_t aux; uint16_t mu; uint16_t delta; } (little endian):
+ *      aux bit t' = sign of component 6 of subvector 16g + t',
+ *      aux bit t' + 16 = sign of component 7 of that subvector (t' = 0..15);
+ *      mu, delta = fp16 grid of (row, group).
+ *  Per 128 weights: 32 B main + 8 B meta = 2.50 bits per weight (Eq. 15).
+ *  codebook: fp16 codebook[K][8] (16 bytes per codeword).
+ *  perm: int32_t perm[d_in], storage column p holds original input channel
+ *    perm[p]; the layer computes y = W_hat * x_perm with x_perm[p] = x[perm[p]]
+ *    (Sec. 3.2 Eq. 5 and Sec. 3.5).  NULL means the identity.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SAGE_FORMAT_VERSION 2
+
+typedef struct CUstream_st* sage_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad enum */
+    SAGE_ERR_UNSUPPORTED = 2,      /* shape / split / batch outside what is implemented */
+    SAGE_ERR_MISALIGNED = 3,       /* a device pointer is not 16-byte aligned */
+    SAGE_ERR_WORKSPACE = 4,        /* workspace missing or smaller than sage_workspace_size() */
+    SAGE_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch or query) */
+    SAGE_ERR_TIMEOUT = 6           /* a device-side bounded wait gave up (see sage_query_status) */
+} sage_status;
+
+/* One packed matrix (all pointers are device pointers; perm may be NULL). */
+typedef struct {
+    int32_t d_out, d_in, log2K;
+    const uint32_t* main;      /* main plane, sage_packed_sizes() bytes */
+    const uint32_t* meta;      /* meta plane */
+    const uint16_t* codebook;  /* fp16 [K][8] */
+    const int32_t* perm;       /* [d_in] or NULL */
+} sage_matrix;
+
+/* Operation selector for sage_workspace_size(). */
+enum { SAGE_OP_GEMV = 0, SAGE_OP_GEMM = 1, SAGE_OP_MOE = 2, SAGE_OP_GROUPED = 3 };
+
+/* Human-readable name of a status code (static storage). */
+const char* sage_status_string(int status);
+
+/* Library build string and format version. */
+const char* sage_version(void);
+
+/* Bytes of the main and meta planes of a d_out x d_in matrix (format v2).
+ * Errors: INVALID_ARGUMENT (null outputs, d_out < 1), UNSUPPORTED (d_in % 128,
+ * log2K outside 4..8). */
+int sage_packed_sizes(int d_out, int d_in, int log2K, size_t* main_bytes, size_t* meta_bytes);
+
+/* HOST.  Packs logical fields into the v2 planes (host buffers).
+ * signs/idx/q: [d_out][d_in/8] row-major, storage column order (Sec. 3.1:
+ *   bit i of signs = 1 when component i is negative; idx < K; q < 2^V);
+ * mu/delta: fp16 bits [d_out][d_in/128].  main_out/meta_out: sage_packed_sizes
+ * bytes, fully written (padding rows zero).  Errors: INVALID_ARGUMENT (null,
+ * idx or q out of range), UNSUPPORTED (shape/split). */
+int sage_pack(int d_out, int d_in, int log2K,
+              const uint8_t* signs, const uint16_t* idx, const uint8_t* q,
+              const uint16_t* mu, const uint16_t* delta,
+              uint32_t* main_out, uint32_t* meta_out);
+
+/* HOST.  Inverse of sage_pack (same shapes). */
+int sage_unpack(int d_out, int d_in, int log2K,
+                const uint32_t* main_plane, const uint32_t* meta_plane,
+                uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu, uint16_t* delta);
+
+/* HOST.  ESG permutation (Sec. 3.2, Eq. 5): channels sorted by decreasing
+ * energy (ties: lower channel first) into 8 tiers of d_in/8; storage position
+ * 8j + t takes the j-th channel of tier t.  perm_out: [d_in].
+ * Errors: INVALID_ARGUMENT (null), UNSUPPORTED (d_in % 8). */
+int sage_esg_permutation(int d_in, const double* energy, int32_t* perm_out);
+
+/* HOST.  Per-matrix SAGE initialisation (Algorithm 1's per-matrix half, App.
+ * A.7, for one fixed (K, V)): ESG permutation (Eq. 5), activation weights
+ * (Eq. 4, exponent gamma), weighted spherical k-means over the listed sample
+ * subvectors (Sec. 3.2; `iters` iterations, codewords initialised to the
+ * directions of sample[init[k]]), fp16 codebook, Eq. 6 assignment of every
+ * subvector, fp16 grid per group (Eq. 14) and radius codes (Eq. 2).
+ * W: fp64 [d_out][d_in] original channel order; energy: [d_in];
+ * sample: subvector ids o*(d_in/8)+j (n_samples); init: K positions into
+ * sample.  Outputs as in sage_pack plus perm_out [d_in] and codebook_out
+ * (fp16 [K][8]).  n_threads <= 0 uses all hardware threads.
+ * Errors: INVALID_ARGUMENT, UNSUPPORTED. */
+int sage_encode(int d_out, int d_in, int log2K, const double* W, const double* energy, double gamma,
+                int n_samples, const int64_t* sample, const int64_t* init, int iters, int n_threads,
+                int32_t* perm_out, uint16_t* codebook_out,
+                uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu, uint16_t* delta);
+
+/* Device workspace bytes for one call of `op` over the n matrices `mats`
+ * (host array: the single matrix of sage_gemv / sage_gemm, all matrices of a
+ * sage_gemv_grouped call, or all experts of a sage_moe_gemv call) at batch M
+ * (for SAGE_OP_MOE: the pair count).  Always >= 256.
+ * Errors: INVALID_ARGUMENT. */
+int sage_workspace_size(int op, const sage_matrix* mats, int n, int M, size_t* bytes);
+
+/* y[M][d_out] = W_hat x_perm for M in 1..8 (Sec. 3.5 decode GEMV; App. A.1):
+ * x: fp16 [M][d_in] original channel order (device); y: fp16 [M][d_out].
+ * fp32 accumulation; deterministic (identical bits on every run).
+ * Errors: INVALID_ARGUMENT, UNSUPPORTED (M outside 1..8), MISALIGNED,
+ * WORKSPACE, CUDA. */
+int sage_gemv(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y,
+              void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* One launch over n matrices (host array `mats`), each with its own input
+ * xs[i] ([M][d_in_i]) and output ys[i] ([M][d_out_i]), M in 1..8 -- e.g. the
+ * q|k|v or gate|up projections of a decoder layer.  Same numerics as
+ * sage_gemv.  n <= 64.  Errors: as sage_gemv. */
+int sage_gemv_grouped(const sage_matrix* mats, int n, const uint16_t* const* xs, uint16_t* const* ys,
+                      int M, void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* y = W_hat x_perm for any M >= 1 (Sec. 3.5 prefill GEMM; App. A.1):
+ * M <= 8 runs the GEMV kernel; M >= 9 permutes x once and runs the
+ * tcgen05/TMEM tensor-core kernel (fp16 operands, fp32 accumulation).
+ * Errors: as sage_gemv (UNSUPPORTED for M > 256). */
+int sage_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y,
+              void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* Grouped-expert GEMV for a mixture-of-experts layer: for every pair p,
+ * y[p] = W_hat_{pair_expert[p]} x_perm[pair_xrow[p]].  experts: host array of
+ * n_experts matrices sharing d_out and d_in (each with its own split,
+ * codebook and perm); pair_expert / pair_xrow: device int32 [n_pairs];
+ * x: fp16 [rows][d_in]; y: fp16 [n_pairs][d_out].  Each expert's planes are
+ * read once per call whatever the number of its pairs (at most 16 pairs per
+ * expert).  Errors: as sage_gemv; UNSUPPORTED for > 16 pairs on one expert is
+ * reported through the status word (SAGE_ERR_UNSUPPORTED). */
+int sage_moe_gemv(const sage_matrix* experts, int n_experts,
+                  const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs,
+                  const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* Test hook: fp16 reconstruction W[d_out][d_in] (storage column order),
+ * computed by the same device decode as the kernels (Eq. 1-2). */
+int sage_dequant(const sage_matrix* A, uint16_t* W, sage_stream_t stream);
+
+/* Test hook: device unpack of the logical fields (shapes as sage_pack). */
+int sage_unpack_device(const sage_matrix* A, uint8_t* signs, uint16_t* idx, uint8_t* q,
+                       uint16_t* mu, uint16_t* delta, sage_stream_t stream);
+
+/* x_perm[m][p] = x[m][perm[p]] (fp16, device), the prefill reorder of Sec. 3.5. */
+int sage_permute_x(const uint16_t* x, const int32_t* perm, int M, int d_in, uint16_t* x_perm,
+                   sage_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the workspace status word.
+ * Returns SAGE_OK, SAGE_ERR_TIMEOUT (a bounded device wait gave up),
+ * SAGE_ERR_UNSUPPORTED (a device-side limit was exceeded) or SAGE_ERR_CUDA. */
+int sage_query_status(void* ws, sage_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_H_ */
