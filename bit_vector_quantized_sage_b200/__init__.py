@@ -35,7 +35,7 @@ EXPORTS = (
     "sage_status_string", "sage_version", "sage_packed_sizes", "sage_pack", "sage_unpack",
     "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
-    "sage_query_status",
+    "sage_query_status", "sage_gemv_static",
 )
 
 
@@ -82,6 +82,7 @@ def load(path: str = LIB_PATH):
         "sage_unpack_device": ([MP, P, P, P, P, P, P], I),
         "sage_permute_x": ([P, P, I, I, P, P], I),
         "sage_query_status": ([P, P], I),
+        "sage_gemv_static": ([MP, P, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -259,6 +260,13 @@ class Workspace:
 def sage_gemv(A: PackedMatrix, x, M: int, y, ws: Workspace, stream=None):
     d = A.desc()
     _check("sage_gemv", load().sage_gemv(C.byref(d), _ptr(x), M, _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def sage_gemv_static(A: PackedMatrix, x, M: int, y, stream=None):
+    """sage_gemv with the library's built-in 4 MiB scratch instead of a workspace
+    (for callers that cannot allocate; calls on one device must not overlap)."""
+    d = A.desc()
+    _check("sage_gemv_static", load().sage_gemv_static(C.byref(d), _ptr(x), M, _ptr(y), _stream(stream)))
 
 
 def sage_gemm(A: PackedMatrix, x, M: int, y, ws: Workspace, stream=None):

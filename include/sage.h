@@ -162,6 +162,32 @@ int sage_workspace_size(int op, const sage_matrix* mats, int n, int M, size_t* b
 int sage_gemv(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y,
               void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* sage_gemv without a workspace argument.  The SAGE paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory or
+ * hand the library a workspace at the point of the call (allocator-free
+ * plugins, custom ops whose framework owns all device memory).  It allocates
+ * nothing: its scratch is a 4 MiB array compiled into libsage (one per device,
+ * resident while the library's device code is loaded), and it runs the same
+ * kernel with the same numerics as sage_gemv (identical y bits).
+ *   - Limit: the scratch of the call, as sage_workspace_size(SAGE_OP_GEMV, ...)
+ *     would report it, must fit in 4 MiB.  About 2.4 MiB go to split-K partial
+ *     sums on a 148-SM GPU; the rest holds one 4-byte counter per 256 output
+ *     rows, so any d_out up to about 400,000 rows fits.  Larger shapes return
+ *     SAGE_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call outside any CUDA stream
+ *     capture.
+ *   - Calls on one device share the scratch: they must not overlap.  Two calls
+ *     in flight at once (different streams, or different host threads without
+ *     ordering) race on it and give wrong results.
+ *   - The status word and counters in the scratch start at zero and every
+ *     completed call leaves them at zero.  A bounded device wait that gives up
+ *     (SAGE_ERR_TIMEOUT under sage_gemv) is not reported by this entry point:
+ *     use sage_gemv with a workspace where that report is needed.
+ * Errors: as sage_gemv, with WORKSPACE meaning "shape beyond the 4 MiB
+ * scratch". */
+int sage_gemv_static(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y, sage_stream_t stream);
+
 /* One launch over n matrices (host array `mats`), each with its own input
  * xs[i] ([M][d_in_i]) and output ys[i] ([M][d_out_i]), M in 1..8 -- e.g. the
  * q|k|v or gate|up projections of a decoder layer.  Same numerics as
