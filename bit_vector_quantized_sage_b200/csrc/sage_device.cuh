@@ -84,6 +84,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 // Bulk asynchronous copy global -> shared (1-D TMA), completes on an mbarrier.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 // ------------------------------------------------------------------------
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// its later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),

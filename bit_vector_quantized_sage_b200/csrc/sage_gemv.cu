@@ -48,24 +48,29 @@ constexpr int kOct = 32;               // row octets per block (one per lane)
 constexpr int kBlockRows = kOct * 8;
 constexpr int kChunkJ = 16;            // a chunk lies inside one radius group
 constexpr int kMaxSegs = 4;            // segments stashed before outputs are flushed
-constexpr int kMaxPass = 4;            // chunks per pass (one ring half)
 constexpr int kMainSlot = kChunkJ * kOct * 16;  // 8 KB of code records
 constexpr int kMetaSlot = kOct * 64;            // 2 KB: one group of 256 rows
-constexpr int kPermSlot = kChunkJ * 8 * 4;      // 512 B
+constexpr int kSlot = kMainSlot + kMetaSlot;    // one ring slot = one chunk
+constexpr int kMaxSlots = 16;                   // ring depth limit
+constexpr int kSegTab = 32;                     // segment-table capacity per round
+constexpr int kSegBytes = 160;                  // shared memory per table entry
 
 template <int M>
 struct Cfg {
     static constexpr int kW = 8;                       // decode warps
     static constexpr int kThreads = (kW + 2) * 32;     // + copy warp + activation warp
     static constexpr int kDecodeThreads = kW * 32;
-    static constexpr int kMinBlocks = (M <= 2) ? 2 : 1;  // room for the next kernel of a PDL chain
-    static constexpr int kXSlot = M * kChunkJ * 16;
-    static constexpr int kSlot = kMainSlot + kMetaSlot + kPermSlot + kXSlot;
+    // Columns per activation window: x_perm for a window is gathered in one go.
+    static constexpr int kXW = (M == 1) ? 256 : (M == 2) ? 128 : (M <= 4) ? 64 : 32;
+    static constexpr int kXBuf = kXW * M * 16;         // one window of x_perm, [m][column]
+    static constexpr int kPermBuf = kXW * 32;          // the window's permutation entries
+    static constexpr int kPosInfo = kXW * 4;           // (segment, column) of each window position
     static constexpr int kRed = kW * 8 * M * 32 * 4;
     static constexpr int kStash = kMaxSegs * M * kBlockRows * 4;
-    static constexpr int kFixed = kRed + kStash + (4 * kMaxPass + 6) * 8 + 64 + 32 * 160;  // ... + segment table (kSegTab x kSegBytes)
+    static constexpr int kBars = (2 * kMaxSlots + 9) * 8;
+    static constexpr int kFixed = 2 * kXBuf + kPermBuf + kPosInfo + kRed + kStash + kSegTab * kSegBytes + kBars + 64;
     // codebook replicas (K_max * 8 * 16) + 2 raw codebooks + ring + fixed
-    static int smem(int pass_chunks, int kmax) { return kmax * 128 + 2 * kmax * 16 + 2 * pass_chunks * kSlot + kFixed; }
+    static int smem(int slots, int kmax) { return kmax * 128 + 2 * kmax * 16 + slots * kSlot + kFixed; }
 };
 
 // One matrix as the kernel sees it while working on one of its segments.
@@ -105,7 +110,7 @@ struct ExpertMat {
 struct Common {
     int n_cta;
     int M;                 // dense: batch; MoE: 0 (per virtual expert)
-    int pass_chunks;       // chunks per ring half
+    int slots;             // ring depth (chunks in flight)
     int kmax;              // largest codebook of the launch (replica area size)
     uint32_t* status;
     unsigned* counters;
@@ -212,8 +217,6 @@ struct Seg {
     int first_slot;         // partial-sum slot of c_first for this block
     int my_slot;            // this CTA's partial-sum slot for this block
 };
-constexpr int kSegTab = 32;  // table capacity per round
-constexpr int kSegBytes = 160;  // shared-memory budget per table entry (Cfg::kFixed)
 static_assert(sizeof(Seg) <= kSegBytes, "segment table entry outgrew its shared-memory budget");
 
 template <class Problem>
@@ -265,51 +268,100 @@ __device__ __forceinline__ int2 chunk_cols(const Seg& s, int c) {
 
 __device__ __forceinline__ void flag(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
 
+// Set when any bounded wait of the CTA gives up; later waits then return at
+// once, so a CTA whose pipeline is stuck ends after one wait limit.
+__shared__ int s_abort;
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Common& C) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if (i > 2048) {
+            if (*reinterpret_cast<volatile int*>(&s_abort)) return false;
+            __nanosleep(64);
+        }
+    }
+    *reinterpret_cast<volatile int*>(&s_abort) = 1;
+    flag(C.status, kDevTimeout);
+    return false;
+}
+
 template <int M>
 struct Smem {
     uint32_t cb0;     // codebook replicas: entry z*8 + r holds codeword z (16 bytes)
-    uint32_t ring0;   // shared address of the staging ring
-    int pc;           // chunks per ring half
+    uint32_t ring0;   // shared address of the chunk ring
+    int slots;        // ring depth
     int cbraw_bytes;
-    uint32_t cbraw0;
+    uint32_t cbraw0;  // two raw codebooks (double buffer across segments)
+    uint32_t xbuf0;   // two activation windows, each [m][kXW] x 16 bytes
+    uint32_t perm0;   // permutation entries of the window being gathered, [kXW] x 32 bytes
+    uint32_t* posinfo;  // per window position: segment index << 24 | column j
     float* red;
     float* stash;
     uint64_t* bars;
     int* bcast;
     Seg* segs;
-    __device__ uint32_t slot(int h, int k) const { return ring0 + (h * pc + k) * Cfg<M>::kSlot; }
-    __device__ uint64_t* landed(int h, int k) const { return bars + h * kMaxPass + k; }
-    __device__ uint64_t* ready(int h, int k) const { return bars + 2 * kMaxPass + h * kMaxPass + k; }
-    __device__ uint64_t* pass_empty(int h) const { return bars + 4 * kMaxPass + h; }
-    __device__ uint64_t* cb_full(int h) const { return bars + 4 * kMaxPass + 2 + h; }
-    __device__ uint64_t* cb_empty(int h) const { return bars + 4 * kMaxPass + 4 + h; }
+    __device__ uint32_t slot(int t) const { return ring0 + (uint32_t)(t % slots) * kSlot; }
+    __device__ uint64_t* full(int t) const { return bars + (t % slots); }
+    __device__ uint64_t* empty(int t) const { return bars + kMaxSlots + (t % slots); }
+    __device__ uint64_t* cb_full(int h) const { return bars + 2 * kMaxSlots + h; }
+    __device__ uint64_t* cb_empty(int h) const { return bars + 2 * kMaxSlots + 2 + h; }
+    __device__ uint64_t* x_full(int h) const { return bars + 2 * kMaxSlots + 4 + h; }
+    __device__ uint64_t* x_empty(int h) const { return bars + 2 * kMaxSlots + 6 + h; }
+    __device__ uint64_t* perm_full() const { return bars + 2 * kMaxSlots + 8; }
+    __device__ uint32_t xwin(int w) const { return xbuf0 + (uint32_t)(w & 1) * Cfg<M>::kXBuf; }
 };
 
 template <int M>
-__device__ __forceinline__ Smem<M> carve(uint8_t* base, int pc, int kmax) {
+__device__ __forceinline__ Smem<M> carve(uint8_t* base, int slots, int kmax) {
     Smem<M> s;
-    s.pc = pc;
+    s.slots = slots;
     uint8_t* p = base;
     s.cb0 = smem_u32(p); p += kmax * 128;
-    s.ring0 = smem_u32(p); p += 2 * pc * Cfg<M>::kSlot;
+    s.ring0 = smem_u32(p); p += slots * kSlot;
     s.cbraw_bytes = kmax * 16;
     s.cbraw0 = smem_u32(p); p += 2 * kmax * 16;
+    s.xbuf0 = smem_u32(p); p += 2 * Cfg<M>::kXBuf;
+    s.perm0 = smem_u32(p); p += Cfg<M>::kPermBuf;
+    s.posinfo = reinterpret_cast<uint32_t*>(p); p += Cfg<M>::kPosInfo;
     s.red = reinterpret_cast<float*>(p); p += Cfg<M>::kRed;
     s.stash = reinterpret_cast<float*>(p); p += Cfg<M>::kStash;
-    s.segs = reinterpret_cast<Seg*>(p); p += kSegTab * sizeof(Seg);
-    s.bars = reinterpret_cast<uint64_t*>(p); p += (4 * kMaxPass + 6) * 8;
+    s.segs = reinterpret_cast<Seg*>(p); p += kSegTab * kSegBytes;
+    s.bars = reinterpret_cast<uint64_t*>(p); p += (2 * kMaxSlots + 9) * 8;
     s.bcast = reinterpret_cast<int*>(p);
     return s;
 }
 
+// Activation windows.  The chunks of a CTA are laid end to end; a window holds
+// up to kXW of their columns (a chunk never straddles two windows) and every
+// segment-table round starts a new window.  The activation warp and the
+// decode warps apply these same two rules, so they agree on where each
+// chunk's x_perm sits without talking to each other.
+struct WinPos {
+    int win;    // window index (its buffer is win & 1)
+    int wpos;   // columns already placed in the window
+};
+__device__ __forceinline__ int win_place(WinPos& w, int nj, int xw) {
+    if (w.wpos + nj > xw) { ++w.win; w.wpos = 0; }
+    const int p = w.wpos;
+    w.wpos += nj;
+    return p;
+}
+__device__ __forceinline__ void win_break(WinPos& w) {
+    if (w.wpos > 0) { ++w.win; w.wpos = 0; }
+}
+
 // Per-role progress that persists across segment-table rounds.
 struct RoleState {
-    int q;     // pass counter (ring phases)
-    int s;     // segment counter (codebook phases)
+    int t;      // chunk counter (ring slots and phases)
+    int s;      // segment counter (codebook phases)
+    WinPos w;   // activation window placement
+    int cur_win;  // decode warps: the x window they hold (-1: none)
 };
 
 // ------------------------------------------------------------------------
-// Copy warp: bulk copies of everything static, issued ahead of the decode.
+// Copy warp: bulk copies of codebooks and code chunks into the ring, issued
+// as far ahead as the ring allows (before and independent of the wait on the
+// preceding kernel: nothing it reads is written by that kernel).
 // ------------------------------------------------------------------------
 template <int M>
 __device__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
@@ -317,105 +369,131 @@ __device__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleSta
     for (int si = 0; si < n_seg; ++si, ++st.s) {
         const Seg& g = sm.segs[si];
         const int s = st.s;
-        if (s >= 2 && !mbar_wait(sm.cb_empty(s & 1), ((s >> 1) - 1) & 1)) flag(C.status, kDevTimeout);
+        if (s >= 2) wait_bar(sm.cb_empty(s & 1), ((s >> 1) - 1) & 1, C);
         const uint32_t cbb = (uint32_t)(16u << g.v.log2K);
         if (lane == 0) {
             mbar_arrive_expect_tx(sm.cb_full(s & 1), cbb);
             bulk_g2s(sm.cbraw0 + (s & 1) * sm.cbraw_bytes, g.v.cb, cbb, sm.cb_full(s & 1));
         }
-        const int n_pass = (g.n_chunks + sm.pc - 1) / sm.pc;
         const int n_oct = g.n_oct, R8 = g.v.R8, S = g.v.S, G = g.v.d_in >> 7, blk = g.blk;
-        for (int t = 0; t < n_pass; ++t, ++st.q) {
-            const int q = st.q, h = q & 1;
-            if (q >= 2 && !mbar_wait(sm.pass_empty(h), ((q >> 1) - 1) & 1)) flag(C.status, kDevTimeout);
-            for (int k = 0; k < sm.pc; ++k) {
-                const int c = t * sm.pc + k;
-                if (c >= g.n_chunks) {
-                    if (lane == 0) mbar_arrive(sm.landed(h, k));
-                    continue;
-                }
+        for (int c = 0; c < g.n_chunks; ++c, ++st.t) {
+            const int t = st.t;
+            if (t >= sm.slots) wait_bar(sm.empty(t), ((t / sm.slots) - 1) & 1, C);
+            if (lane == 0) {
                 const int2 cc = chunk_cols(g, c);
                 const int nj = cc.y - cc.x;
-                const uint32_t tx = (uint32_t)(nj * n_oct * 16 + n_oct * 64 + (g.v.perm ? nj * 32 : 0));
-                if (lane == 0) mbar_arrive_expect_tx(sm.landed(h, k), tx);
-                __syncwarp();
-                const uint32_t dst = sm.slot(h, k);
-                if (lane == 0)  // the chunk's records: one contiguous range of the block
-                    bulk_g2s(dst, g.v.main + main_word(R8, S, blk, cc.x, 0, 0), nj * n_oct * 16, sm.landed(h, k));
-                if (lane == 16)
-                    bulk_g2s(dst + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0), n_oct * 64,
-                             sm.landed(h, k));
-                if (lane == 17 && g.v.perm)
-                    bulk_g2s(dst + kMainSlot + kMetaSlot, g.v.perm + cc.x * 8, nj * 32, sm.landed(h, k));
+                const uint32_t mb = (uint32_t)(nj * n_oct * 16), tb = (uint32_t)(n_oct * 64);
+                mbar_arrive_expect_tx(sm.full(t), mb + tb);
+                // the chunk's records: one contiguous range of the block; its group's meta entries
+                bulk_g2s(sm.slot(t), g.v.main + main_word(R8, S, blk, cc.x, 0, 0), mb, sm.full(t));
+                bulk_g2s(sm.slot(t) + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0), tb,
+                         sm.full(t));
             }
         }
     }
 }
 
+// The CTA may not exit while bulk copies are in flight.
 template <int M>
 __device__ void copy_drain(const Common& C, const Smem<M>& sm, const RoleState& st) {
-    // The CTA may not exit while bulk copies are in flight.
-    for (int qq = max(0, st.q - 2); qq < st.q; ++qq)
-        for (int k = 0; k < sm.pc; ++k)
-            if (!mbar_wait(sm.landed(qq & 1, k), (qq >> 1) & 1)) flag(C.status, kDevTimeout);
+    for (int t = max(0, st.t - sm.slots); t < st.t; ++t)
+        wait_bar(sm.full(t), (t / sm.slots) & 1, C);
 }
 
 // ------------------------------------------------------------------------
-// Activation warp: x_perm for every chunk (after the preceding kernel).
+// Activation warp: x_perm[m][p] = x[m][perm[p]] for one window of columns
+// (Sec. 3.5 fuses this gather into the decode GEMV).  The permutation entries
+// are bulk-copied first -- for the first window before the wait on the
+// preceding kernel, since only x comes from that kernel -- so after the wait
+// the gather costs one round trip per window.
 // ------------------------------------------------------------------------
 template <int M>
-__device__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+__device__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
+    constexpr int XW = Cfg<M>::kXW;
     const int lane = threadIdx.x & 31;
+    fence_proxy_async_smem();  // earlier reads of the permutation buffer precede the copies below
+    int si = si0, c = c0, wlen = 0;
+    for (int k = 0; k < nch; ++k) {
+        const Seg& g = sm.segs[si];
+        const int2 cc = chunk_cols(g, c);
+        const int nj = cc.y - cc.x;
+        if (g.v.perm && lane == 0) {
+            mbar_expect_tx(sm.perm_full(), (uint32_t)(nj * 32));
+            bulk_g2s(sm.perm0 + wlen * 32, g.v.perm + cc.x * 8, (uint32_t)(nj * 32), sm.perm_full());
+        }
+        if (lane < nj) sm.posinfo[wlen + lane] = ((uint32_t)si << 24) | (uint32_t)(cc.x + lane);
+        wlen += nj;
+        if (++c == g.n_chunks) { c = 0; ++si; }
+    }
+    if (lane == 0) mbar_arrive(sm.perm_full());
+    if (!waited) {
+        pdl_wait();  // x may be written by the preceding kernel
+        waited = true;
+    }
+    wait_bar(sm.perm_full(), w & 1, C);
+    if (w >= 2) wait_bar(sm.x_empty(w & 1), ((w >> 1) - 1) & 1, C);
+    __syncwarp();
+    const uint32_t xb = sm.xwin(w);
+    const int total = M * wlen;
+    // All loads of a round are issued before any store: one memory round trip
+    // per 256 (batch row, column) pairs.
+    for (int e0 = 0; e0 < total; e0 += 8 * 32) {
+        uint4 val[8];
+        uint32_t dst[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int e = e0 + r * 32 + lane;
+            dst[r] = 0xffffffffu;
+            if (e < total) {
+                const int m = e / wlen, p = e - m * wlen;
+                const uint32_t info = sm.posinfo[p];
+                const Seg& g = sm.segs[info >> 24];
+                const int j = (int)(info & 0xffffffu);
+                if (m < g.v.Mk) {
+                    const int xr_idx = g.v.xrows ? __ldcg(g.v.xrows + m) : m;
+                    const unsigned short* xr =
+                        reinterpret_cast<const unsigned short*>(g.v.x) + (size_t)xr_idx * g.v.d_in;
+                    if (g.v.perm) {
+                        const uint32_t sp = sm.perm0 + p * 32;
+                        const uint4 pa = lds128(sp), pb = lds128(sp + 16);
+                        val[r].x = (uint32_t)__ldcg(xr + pa.x) | ((uint32_t)__ldcg(xr + pa.y) << 16);
+                        val[r].y = (uint32_t)__ldcg(xr + pa.z) | ((uint32_t)__ldcg(xr + pa.w) << 16);
+                        val[r].z = (uint32_t)__ldcg(xr + pb.x) | ((uint32_t)__ldcg(xr + pb.y) << 16);
+                        val[r].w = (uint32_t)__ldcg(xr + pb.z) | ((uint32_t)__ldcg(xr + pb.w) << 16);
+                    } else {
+                        val[r] = __ldcg(reinterpret_cast<const uint4*>(xr + j * 8));
+                    }
+                    dst[r] = xb + (m * XW + p) * 16;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            if (dst[r] != 0xffffffffu) sts128(dst[r], val[r]);
+    }
+    mbar_arrive(sm.x_full(w & 1));  // all 32 lanes, each after its own stores
+}
+
+template <int M>
+__device__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st, bool& waited) {
+    win_break(st.w);
+    int pend = -1, si0 = 0, c0 = 0, nch = 0;
     for (int si = 0; si < n_seg; ++si) {
         const Seg& g = sm.segs[si];
-        const int n_pass = (g.n_chunks + sm.pc - 1) / sm.pc;
-        const uint16_t* xbase = g.v.x;
-        const int32_t* xrows = g.v.xrows;
-        const int32_t* perm = g.v.perm;
-        const int d_in = g.v.d_in, Mk = g.v.Mk;
-        for (int t = 0; t < n_pass; ++t, ++st.q) {
-            const int q = st.q, h = q & 1;
-            const int c0 = t * sm.pc, c1 = min(g.n_chunks, c0 + sm.pc);
-            for (int c = c0; c < c1; ++c)  // the permutation slices must have landed
-                if (!mbar_wait(sm.landed(h, c - c0), (q >> 1) & 1)) flag(C.status, kDevTimeout);
-            const int pa = chunk_cols(g, c0).x, pb = chunk_cols(g, c1 - 1).y;
-            const int ncol = pb - pa, total = Mk * ncol;
-            // All loads of a round are issued before any store, so a pass costs
-            // one memory round trip per 128 (batch row, column) pairs.
-            for (int e0 = 0; e0 < total; e0 += 4 * 32) {
-                uint4 val[4];
-                uint32_t dst[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int e = e0 + r * 32 + lane;
-                    dst[r] = 0xffffffffu;
-                    if (e < total) {
-                        const int m = e / ncol, j = pa + (e - m * ncol);
-                        const int k = (j >> 4) - (pa >> 4);
-                        const int i = j - max(pa, (j >> 4) << 4);
-                        const uint32_t base = sm.slot(h, k);
-                        const int xr_idx = xrows ? __ldcg(xrows + m) : m;
-                        const uint16_t* xr = xbase + (size_t)xr_idx * d_in;
-                        if (perm) {
-                            const uint32_t sp = base + kMainSlot + kMetaSlot + i * 32;
-                            const uint4 pa4 = lds128(sp), pb4 = lds128(sp + 16);
-                            val[r].x = (uint32_t)xr[pa4.x] | ((uint32_t)xr[pa4.y] << 16);
-                            val[r].y = (uint32_t)xr[pa4.z] | ((uint32_t)xr[pa4.w] << 16);
-                            val[r].z = (uint32_t)xr[pb4.x] | ((uint32_t)xr[pb4.y] << 16);
-                            val[r].w = (uint32_t)xr[pb4.z] | ((uint32_t)xr[pb4.w] << 16);
-                        } else {
-                            val[r] = *reinterpret_cast<const uint4*>(xr + j * 8);
-                        }
-                        dst[r] = base + kMainSlot + kMetaSlot + kPermSlot + (m * kChunkJ + i) * 16;
-                    }
-                }
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    if (dst[r] != 0xffffffffu) sts128(dst[r], val[r]);
+        for (int c = 0; c < g.n_chunks; ++c) {
+            const int2 cc = chunk_cols(g, c);
+            win_place(st.w, cc.y - cc.x, Cfg<M>::kXW);
+            if (st.w.win != pend) {
+                if (nch) fill_window<M>(C, sm, pend, si0, c0, nch, waited);
+                pend = st.w.win;
+                si0 = si;
+                c0 = c;
+                nch = 0;
             }
-            for (int k = 0; k < sm.pc; ++k) mbar_arrive(sm.ready(h, k));
+            ++nch;
         }
     }
+    if (nch) fill_window<M>(C, sm, pend, si0, c0, nch, waited);
 }
 
 // ------------------------------------------------------------------------
@@ -472,33 +550,23 @@ __device__ __forceinline__ void decode_record(const VDec& d, uint4 rec, const ui
     }
 }
 
-// Decode this warp's share of one pass (columns [pa, pb) of segment g).
+// Decodes this warp's columns of ring chunk t (chunk c of segment g): columns
+// warp, warp + W, ... of the chunk, against the x_perm window at xw, where the
+// chunk's first column sits at window position pos.
 template <int M, int MS>
-__device__ __forceinline__ void decode_pass(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int h,
-                                            uint32_t parity, int pa, int pb, int warp, int lane, float (&acc)[8][M]) {
-    constexpr int W = Cfg<MS>::kW;
-    const int n = pb - pa;
-    const int ra = pa + (warp * n) / W, rb = pa + ((warp + 1) * n) / W;
-    const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
+__device__ __forceinline__ void decode_chunk(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int t,
+                                             int c, uint32_t xw, int pos, int warp, int lane, float (&acc)[8][M]) {
+    constexpr int W = Cfg<MS>::kW, XW = Cfg<MS>::kXW;
+    const int2 cc = chunk_cols(g, c);
+    const int nj = cc.y - cc.x;
+    wait_bar(sm.full(t), (t / sm.slots) & 1, C);
     const int n_oct = g.n_oct;
-    const bool active = lane < n_oct;
-    uint32_t aux[8];
-    float mup[8], dlp[8];
-    int kcur = -1, gcur = -1;
-    uint32_t base = 0;
-    int j0 = 0;
-    for (int j = ra; j < rb; ++j) {
-        const int k = (j >> 4) - (pa >> 4);
-        if (k != kcur) {
-            if (!mbar_wait(sm.landed(h, k), parity)) flag(C.status, kDevTimeout);
-            if (!mbar_wait(sm.ready(h, k), parity)) flag(C.status, kDevTimeout);
-            kcur = k;
-            base = sm.slot(h, k);
-            j0 = max(pa, (j >> 4) << 4);
-        }
-        if (!active) continue;
-        if ((j >> 4) != gcur) {
-            gcur = j >> 4;
+    if (warp < nj && lane < n_oct) {
+        const uint32_t base = sm.slot(t);
+        const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
+        uint32_t aux[8];
+        float mup[8], dlp[8];
+        {   // the group's grid and aux signs for this lane's 8 rows
             const uint32_t a = base + kMainSlot + lane * 64;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -513,14 +581,17 @@ __device__ __forceinline__ void decode_pass(const Smem<MS>& sm, const Common& C,
                 mup[2 * e + 1] = m1.x - dlp[2 * e + 1];
             }
         }
-        const int i = j - j0;
-        const uint4 rec = lds128(base + (i * n_oct + lane) * 16);
-        uint4 xv[M];
-        const uint32_t sx = base + kMainSlot + kMetaSlot + kPermSlot;
+        for (int i = warp; i < nj; i += W) {
+            const int j = cc.x + i;
+            const uint4 rec = lds128(base + (i * n_oct + lane) * 16);
+            uint4 xv[M];
 #pragma unroll
-        for (int m = 0; m < M; ++m) xv[m] = lds128(sx + (m * kChunkJ + i) * 16);
-        decode_record<M>(d, rec, aux, (uint32_t)(15 - (j & 15)), mup, dlp, cbsel, xv, acc);
+            for (int m = 0; m < M; ++m) xv[m] = lds128(xw + (m * XW + pos + i) * 16);
+            decode_record<M>(d, rec, aux, (uint32_t)(15 - (j & 15)), mup, dlp, cbsel, xv, acc);
+        }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(t));
 }
 
 // Writes (or combines) the outputs of the pending segments tab[i0 .. i0 + n).
@@ -578,10 +649,11 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
             float tot[M];
 #pragma unroll
             for (int m = 0; m < M; ++m) tot[m] = 0.f;
-            for (int c0 = c_first; c0 <= c_last; c0 += 8) {
-                float v[8][M];   // up to 8 contributors' loads in flight at once
+            constexpr int NF = (M <= 2) ? 16 : 8;  // contributors' loads in flight at once
+            for (int c0 = c_first; c0 <= c_last; c0 += NF) {
+                float v[NF][M];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                for (int k = 0; k < NF; ++k) {
                     const int c = c0 + k;
                     const int sp = (c == c_first) ? first_slot : 0;
                     const float* src = C.partials + ((size_t)(c * 2 + sp) * 8) * kBlockRows + row_local;
@@ -589,7 +661,7 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
                     for (int m = 0; m < M; ++m) v[k][m] = (c <= c_last) ? __ldcg(src + m * kBlockRows) : 0.f;
                 }
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
+                for (int k = 0; k < NF; ++k)
 #pragma unroll
                     for (int m = 0; m < M; ++m) tot[m] += v[k][m];
             }
@@ -607,7 +679,7 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
 // Decodes one segment with compile-time batch MK (<= MS, the launch's stash
 // stride) and leaves its 256 x MS results in stash slot `slot`.
 template <int MK, int MS>
-__device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, int q0, int slot) {
+__device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st, int slot) {
     constexpr int W = Cfg<MS>::kW, DT = Cfg<MS>::kDecodeThreads;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const VDec d = vdec(g.v.log2K);
@@ -616,16 +688,24 @@ __device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, c
     for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int m = 0; m < MK; ++m) acc[r][m] = 0.f;
-    const int n_pass = (g.n_chunks + sm.pc - 1) / sm.pc;
-    int q = q0;
-    for (int t = 0; t < n_pass; ++t, ++q) {
-        const int h = q & 1;
-        const int2 first = chunk_cols(g, t * sm.pc);
-        const int2 last = chunk_cols(g, min(g.n_chunks, (t + 1) * sm.pc) - 1);
-        decode_pass<MK, MS>(sm, C, g, d, h, (q >> 1) & 1, first.x, last.y, warp, lane, acc);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sm.pass_empty(h));
+    int t = st.t, cur = st.cur_win;
+    WinPos w = st.w;
+    for (int c = 0; c < g.n_chunks; ++c, ++t) {
+        const int2 cc = chunk_cols(g, c);
+        const int pos = win_place(w, cc.y - cc.x, Cfg<MS>::kXW);
+        if (w.win != cur) {  // release the previous x window, wait for this one
+            if (cur >= 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sm.x_empty(cur & 1));
+            }
+            wait_bar(sm.x_full(w.win & 1), (w.win >> 1) & 1, C);
+            cur = w.win;
+        }
+        decode_chunk<MK, MS>(sm, C, g, d, t, c, sm.xwin(w.win), pos, warp, lane, acc);
     }
+    st.t = t;
+    st.cur_win = cur;
+    st.w = w;
     // reduce the warps' partial sums in a fixed order into the stash
 #pragma unroll
     for (int r = 0; r < 8; ++r)
@@ -638,7 +718,7 @@ __device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, c
             float sum = 0.f;
             if (m < MK) {
 #pragma unroll
-                for (int w = 0; w < W; ++w) sum += sm.red[((w * 8 + r) * MK + m) * 32 + l];
+                for (int w2 = 0; w2 < W; ++w2) sum += sm.red[((w2 * 8 + r) * MK + m) * 32 + l];
             }
             sm.stash[((size_t)slot * MS + m) * kBlockRows + l * 8 + r] = sum;
         }
@@ -652,10 +732,11 @@ __device__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, Role
     const int tid = threadIdx.x;
     int npend = 0, i_pend = 0;
     const uint16_t* cur_cb = nullptr;
+    win_break(st.w);
     for (int si = 0; si < n_seg; ++si, ++st.s) {
         const Seg& g = sm.segs[si];
         const int s = st.s;
-        if (!mbar_wait(sm.cb_full(s & 1), (s >> 1) & 1)) flag(C.status, kDevTimeout);
+        wait_bar(sm.cb_full(s & 1), (s >> 1) & 1, C);
         if (g.v.cb != cur_cb) {  // build the 8 bank-rotated replicas from the raw copy
             if (cur_cb) named_barrier(1, DT);
             const int K = 1 << g.v.log2K;
@@ -666,20 +747,19 @@ __device__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, Role
         }
         if (tid == 0) mbar_arrive(sm.cb_empty(s & 1));
         if constexpr (MLO == M) {
-            segment_body<M, M>(sm, C, g, st.q, npend);
+            segment_body<M, M>(sm, C, g, st, npend);
         } else {
             switch (g.v.Mk) {
-                case 1: segment_body<1, M>(sm, C, g, st.q, npend); break;
-                case 2: segment_body<2, M>(sm, C, g, st.q, npend); break;
-                case 3: segment_body<3, M>(sm, C, g, st.q, npend); break;
-                case 4: segment_body<4, M>(sm, C, g, st.q, npend); break;
-                case 5: segment_body<5, M>(sm, C, g, st.q, npend); break;
-                case 6: segment_body<6, M>(sm, C, g, st.q, npend); break;
-                case 7: segment_body<7, M>(sm, C, g, st.q, npend); break;
-                default: segment_body<8, M>(sm, C, g, st.q, npend); break;
+                case 1: segment_body<1, M>(sm, C, g, st, npend); break;
+                case 2: segment_body<2, M>(sm, C, g, st, npend); break;
+                case 3: segment_body<3, M>(sm, C, g, st, npend); break;
+                case 4: segment_body<4, M>(sm, C, g, st, npend); break;
+                case 5: segment_body<5, M>(sm, C, g, st, npend); break;
+                case 6: segment_body<6, M>(sm, C, g, st, npend); break;
+                case 7: segment_body<7, M>(sm, C, g, st, npend); break;
+                default: segment_body<8, M>(sm, C, g, st, npend); break;
             }
         }
-        st.q += (g.n_chunks + sm.pc - 1) / sm.pc;
         ++npend;
         if (npend == kMaxSegs || si + 1 == n_seg) {
             flush<M>(C, sm, i_pend, npend);
@@ -691,19 +771,23 @@ __device__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, Role
 
 template <int MLO, int M, class Problem>
 __device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* smem_raw, bool plan_needs_wait) {
-    const Smem<M> sm = carve<M>(smem_raw, C.pass_chunks, C.kmax);
+    const Smem<M> sm = carve<M>(smem_raw, C.slots, C.kmax);
     const int tid = threadIdx.x, warp = tid >> 5;
+    constexpr int W = Cfg<M>::kW;
     if (tid == 0) {
+        for (int k = 0; k < kMaxSlots; ++k) {
+            mbar_init(sm.bars + k, 1);              // full: copy warp arrival + bytes
+            mbar_init(sm.bars + kMaxSlots + k, W);  // empty: one arrival per decode warp
+        }
         for (int h = 0; h < 2; ++h) {
-            for (int k = 0; k < kMaxPass; ++k) {
-                mbar_init(sm.landed(h, k), 1);
-                mbar_init(sm.ready(h, k), 32);
-            }
-            mbar_init(sm.pass_empty(h), Cfg<M>::kW);
             mbar_init(sm.cb_full(h), 1);
             mbar_init(sm.cb_empty(h), 1);
+            mbar_init(sm.x_full(h), 32);
+            mbar_init(sm.x_empty(h), W);
         }
+        mbar_init(sm.perm_full(), 1);
         fence_mbar_init();
+        s_abort = 0;
     }
     pdl_launch_dependents();
     if (plan_needs_wait) pdl_wait();  // the plan itself depends on preceding work
@@ -712,30 +796,28 @@ __device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* 
     const long long total = P.total();
     const long long u0 = total > 0 ? P.cta_begin(blockIdx.x) : 0;
     const long long u1 = total > 0 ? P.cta_begin(blockIdx.x + 1) : 0;
-    RoleState st{0, 0};
+    RoleState st{0, 0, {0, 0}, -1};
     bool waited = plan_needs_wait;
     for (long long u = u0; u < u1;) {
         if (tid == 0) s_nseg = build_segs(P, C, u, u1, u0, sm.segs, &s_next);
         __syncthreads();
         const int n_seg = s_nseg;
-        if (warp == Cfg<M>::kW) {
+        if (warp == W) {
             copy_warp<M>(C, sm, n_seg, st);
-        } else if (warp == Cfg<M>::kW + 1) {
-            if (!waited) pdl_wait();  // activations may come from the preceding kernel
-            waited = true;
-            act_warp<M>(C, sm, n_seg, st);
+        } else if (warp == W + 1) {
+            act_warp<M>(C, sm, n_seg, st, waited);
         } else {
             decode_warps<MLO, M>(C, sm, n_seg, st);
         }
         u = s_next;
         __syncthreads();  // the segment table is rebuilt for the next round
     }
-    if (warp == Cfg<M>::kW) copy_drain<M>(C, sm, st);
-    if (warp == Cfg<M>::kW + 1 && !waited) pdl_wait();
+    if (warp == W) copy_drain<M>(C, sm, st);
+    if (warp == W + 1 && !waited) pdl_wait();
 }
 
 template <int M>
-__global__ void __launch_bounds__(Cfg<M>::kThreads, Cfg<M>::kMinBlocks) gemv_kernel(const __grid_constant__ DenseParams p) {
+__global__ void __launch_bounds__(Cfg<M>::kThreads, 1) gemv_kernel(const __grid_constant__ DenseParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const DenseProblem P{p};
     run<M, M>(P, p.c, smem_raw, false);
@@ -839,16 +921,15 @@ std::vector<int> per_matrix_shares(const std::vector<long long>& units, int n_ct
     return share;
 }
 
-// Chunks per ring half: the whole CTA range when it fits, keeping the CTA's
-// shared memory under ~110 KB so that two CTAs (this kernel's and the next
-// kernel's in a PDL chain) can share an SM.
+// Ring depth: as many chunk slots as fit next to the fixed shared memory (one
+// CTA per SM), at most one more than the widest CTA's chunk count.
+constexpr int kSmemBudget = 226 * 1024;  // 227 KB per CTA less static shared memory
 template <int M>
-int pass_chunks_for(long long max_units_per_cta, int kmax) {
+int slots_for(long long max_units_per_cta, int kmax) {
     const long long chunks = (max_units_per_cta + kChunkJ - 1) / kChunkJ + 2;
-    int pc = (int)std::min<long long>(kMaxPass, std::max<long long>(1, (chunks + 1) / 2));
-    const int budget = (Cfg<M>::kMinBlocks > 1 ? 110 : 220) * 1024;
-    while (pc > 1 && Cfg<M>::smem(pc, kmax) > budget) --pc;
-    return pc;
+    int n = (int)std::min<long long>(kMaxSlots, std::max<long long>(2, chunks));
+    while (n > 2 && Cfg<M>::smem(n, kmax) > kSmemBudget) --n;
+    return n;
 }
 
 // Raises the kernel's dynamic shared memory limit when a launch needs more
@@ -915,14 +996,14 @@ int launch_m(const GemvJob* jobs, int n, void* ws, sage_stream_t stream) {
     p.total_units = unit;
     p.c.n_cta = n_cta;
     p.c.M = M;
-    p.c.pass_chunks = pass_chunks_for<M>(widest, kmax);
+    p.c.slots = slots_for<M>(widest, kmax);
     p.c.kmax = kmax;
-    if (!ensure_smem(gemv_kernel<M>, Cfg<M>::smem(p.c.pass_chunks, kmax), configured)) return SAGE_ERR_CUDA;
+    if (!ensure_smem(gemv_kernel<M>, Cfg<M>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     p.c.status = reinterpret_cast<uint32_t*>(w);
     p.c.counters = reinterpret_cast<unsigned*>(w + kWsHeader);
     p.c.partials = reinterpret_cast<float*>(w + kWsHeader + round256((size_t)blk * 4));
-    return launch_pdl(gemv_kernel<M>, p, n_cta, Cfg<M>::kThreads, Cfg<M>::smem(p.c.pass_chunks, kmax), stream);
+    return launch_pdl(gemv_kernel<M>, p, n_cta, Cfg<M>::kThreads, Cfg<M>::smem(p.c.slots, kmax), stream);
 }
 
 }  // namespace
@@ -997,8 +1078,8 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
     int kmax = 16;
     for (int e = 0; e < n_experts; ++e) kmax = std::max(kmax, 1 << experts[e].log2K);
     p.c.kmax = kmax;
-    p.c.pass_chunks = pass_chunks_for<MV>(1 << 30, kmax);
-    if (!ensure_smem(moe_kernel, Cfg<MV>::smem(p.c.pass_chunks, kmax), configured)) return SAGE_ERR_CUDA;
+    p.c.slots = slots_for<MV>(1 << 30, kmax);
+    if (!ensure_smem(moe_kernel, Cfg<MV>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
     p.c.status = reinterpret_cast<uint32_t*>(w);
     p.c.counters = reinterpret_cast<unsigned*>(w + L.counters);
     p.c.partials = reinterpret_cast<float*>(w + L.partials);
@@ -1037,7 +1118,7 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
                                reinterpret_cast<int32_t*>(w + L.v_count), p.c.status) != cudaSuccess)
             return SAGE_ERR_CUDA;
     }
-    return launch_pdl(moe_kernel, p, n_cta, Cfg<MV>::kThreads, Cfg<MV>::smem(p.c.pass_chunks, kmax), stream);
+    return launch_pdl(moe_kernel, p, n_cta, Cfg<MV>::kThreads, Cfg<MV>::smem(p.c.slots, kmax), stream);
 }
 
 }  // namespace sage
