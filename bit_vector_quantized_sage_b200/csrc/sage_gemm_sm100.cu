@@ -1,16 +1,505 @@
-// tcgen05 / TMEM tensor-core path for M >= 9 (placeholder until the kernel lands).
+// Tensor-core path of the packed SAGE layer for batch M >= 9 on sm_100a
+// (the prefill GEMM of Sec. 3.5 / App. A.1 of "SAGE: Pushing 2-Bit
+// Vector-Quantized LLMs toward Real-World Usability": W_hat tiles are
+// reconstructed into shared memory and multiplied there, so the decode is
+// amortised over the whole batch).
+//
+//   y[m][o] = sum_p W_hat[o][p] x_perm[m][p],  M <= 256.
+//
+// Two kernels per call:
+//  * tile_x_kernel writes x_perm (Sec. 3.5: the activations are reordered once
+//    per projection) straight into the tcgen05 K-major operand layout, zero
+//    padded to N = M rounded up to 16, so every 64-column slab of it is one
+//    contiguous bulk copy.
+//  * gemm_kernel: one CTA per (256-row block, part of the input columns).  A
+//    copy warp bulk-copies the block's packed chunks (16 subvector columns =
+//    one radius group) and the x_perm slabs; eight decode warps rebuild each
+//    64-column slab of W_hat (Eq. 1-2: r_hat (s (.) c_z), r_hat = mu + q delta,
+//    rounded to fp16) into shared memory; one thread issues tcgen05.mma
+//    (kind::f16, M = 128, N, K = 16) for the two 128-row halves into two fp32
+//    accumulators in tensor memory and commits to an mbarrier that frees the
+//    slab's buffers.  The epilogue reads the accumulators with tcgen05.ld.
+//    A block split over several CTAs is combined deterministically: every part
+//    stores fp32 partial sums and the last part to arrive adds them in order.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <mutex>
+
+#include "sage_device.cuh"
 #include "sage_internal.h"
 
 namespace sage {
+using namespace dev;
 
-size_t gemm_workspace_bytes(const sage_matrix* A, int M) {
-    return kWsHeader + (size_t)M * A->d_in * 2 + 256;
+namespace {
+
+constexpr int kGW = 8;                        // decode warps
+constexpr int kGThreads = (kGW + 1) * 32;     // + copy warp
+constexpr int kGDecodeThreads = kGW * 32;
+constexpr int kGOct = 32;                     // row octets per block
+constexpr int kGChunkJ = 16;                  // subvector columns per chunk (one radius group)
+constexpr int kGSlabJ = 8;                    // subvector columns per MMA slab (64 input channels)
+constexpr int kGCodeSlot = kGChunkJ * kGOct * 16 + kGOct * 64;  // records + meta of one chunk
+constexpr int kGCodeSlots = 4;
+constexpr int kASbo = 1040;                   // bytes between 8-row core-matrix groups of A (padded: no bank conflicts)
+constexpr int kAHalf = 16 * kASbo;            // one 128-row half of an A slab
+constexpr int kASlab = 2 * kAHalf;            // 256 rows x 64 channels, fp16
+constexpr int kBSbo = 1024;                   // B: 8 core matrices of 8 rows x 16 bytes per 8 batch rows
+
+// ------------------------------------------------------------------------
+// tcgen05 / TMEM primitives (PTX ISA, sm_100a).
+// ------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, fp16 inputs, fp32 accumulation.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrives (once) on the mbarrier when every MMA this thread issued so far is complete.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-int launch_gemm(const sage_matrix*, const uint16_t*, int, uint16_t*, void*, size_t, sage_stream_t) {
-    return SAGE_ERR_UNSUPPORTED;
+// Shared-memory matrix descriptor, K-major, no swizzle: core matrices of
+// 8 rows x 16 bytes; lbo = bytes between the two K-adjacent core matrices of
+// one MMA, sbo = bytes between 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);  // descriptor version 1
+}
+// Instruction descriptor of kind::f16: fp32 D, fp16 A and B, both K-major, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void gflag(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
+
+// Set when a bounded wait of the CTA gives up; later waits then return at once.
+__shared__ int s_gabort;
+
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if (i > 2048) {
+            if (*reinterpret_cast<volatile int*>(&s_gabort)) return false;
+            __nanosleep(64);
+        }
+    }
+    *reinterpret_cast<volatile int*>(&s_gabort) = 1;
+    gflag(status, kDevTimeout);
+    return false;
+}
+
+// ------------------------------------------------------------------------
+// x_perm in the B-operand layout: slab s (input channels 64s .. 64s+63) is
+// [n / 8][kb = 0..7][n % 8] x 16 bytes, 16 bytes = channels 64s + 8kb .. +7
+// of batch row n; rows n >= M are zero.
+// ------------------------------------------------------------------------
+__global__ void tile_x_kernel(const uint16_t* x, const int32_t* perm, int M, int n_pad, int d_in, uint4* xt) {
+    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long per_slab = (long long)n_pad * 8;
+    if (id >= per_slab * (d_in / 64)) return;
+    const int s = (int)(id / per_slab);
+    const int w = (int)(id - (long long)s * per_slab);
+    const int ng = w >> 6, kb = (w >> 3) & 7, r = w & 7;
+    const int n = ng * 8 + r, k0 = s * 64 + kb * 8;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (n < M) {
+        const uint16_t* xr = x + (size_t)n * d_in;
+        if (perm) {
+            const int4 pa = __ldg(reinterpret_cast<const int4*>(perm + k0));
+            const int4 pb = __ldg(reinterpret_cast<const int4*>(perm + k0 + 4));
+            o.x = (uint32_t)xr[pa.x] | ((uint32_t)xr[pa.y] << 16);
+            o.y = (uint32_t)xr[pa.z] | ((uint32_t)xr[pa.w] << 16);
+            o.z = (uint32_t)xr[pb.x] | ((uint32_t)xr[pb.y] << 16);
+            o.w = (uint32_t)xr[pb.z] | ((uint32_t)xr[pb.w] << 16);
+        } else {
+            o = *reinterpret_cast<const uint4*>(xr + k0);
+        }
+    }
+    xt[id] = o;
+}
+
+struct GemmParams {
+    const uint32_t* main;
+    const uint32_t* meta;
+    const uint16_t* cb;
+    const uint4* xt;        // x_perm in the B-operand layout (tile_x_kernel)
+    uint16_t* y;            // [M][d_out]
+    float* partials;        // [n_blocks * parts][n_pad][256]
+    unsigned* counters;     // [n_blocks], zero between calls
+    uint32_t* status;
+    int d_out, d_in, log2K, M;
+    int n_pad;              // M rounded up to 16: the MMA's N
+    int n_alloc;            // TMEM columns per accumulator (power of two >= max(32, n_pad))
+    int parts;              // CTAs per block (split over the input columns)
+    int b_slots;            // x_perm slabs in flight
+};
+
+struct GemmSmem {
+    uint32_t cb0, cbraw, code0, a0, b0;
+    uint32_t b_bytes;
+    uint64_t* bars;
+    uint32_t* taddr_slot;
+    int* bcast;
+    __device__ uint64_t* code_full(int t) const { return bars + (t % kGCodeSlots); }
+    __device__ uint64_t* code_empty(int t) const { return bars + kGCodeSlots + (t % kGCodeSlots); }
+    __device__ uint64_t* cb_full() const { return bars + 2 * kGCodeSlots; }
+    __device__ uint64_t* b_full(int s, int nb) const { return bars + 2 * kGCodeSlots + 1 + (s % nb); }
+    __device__ uint64_t* mma_done(int s, int nb) const { return bars + 2 * kGCodeSlots + 1 + 8 + (s % nb); }
+};
+
+__host__ __device__ inline int gemm_smem_bytes(int K, int n_pad, int b_slots) {
+    return K * 128 + K * 16 + kGCodeSlots * kGCodeSlot + 2 * kASlab + b_slots * n_pad * 128 +
+           (2 * kGCodeSlots + 1 + 16) * 8 + 64;
+}
+
+// Rebuilds the 8 rows of octet o for subvector column w of a slab (Eq. 1-2),
+// rounded to fp16, into the A operand: core matrix (o % 16, w) of half o / 16.
+__device__ __forceinline__ void decode_to_a(const VDec& d, uint4 rec, const uint32_t (&aux)[8], uint32_t sh_aux,
+                                            const float (&mup)[8], const float (&dlp)[8], uint32_t cbsel,
+                                            uint32_t dst) {
+    const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int t = 2 * u + half;
+            const uint32_t wa = wv[u];
+            const uint32_t wf = half ? rot16(wa) : wa;  // (z, q) field word of this row
+            uint4 c = lds128(cbsel + (wf & d.zmask));
+            if (!half) {
+                c.x ^= (wa << d.sh0) & 0x80008000u;
+                c.y ^= (wa << d.sh1) & 0x80008000u;
+                c.z ^= (wa << d.sh2) & 0x80008000u;
+            } else {
+                c.x ^= (wa << d.sh3) & 0x80008000u;
+                c.y ^= (wa << d.sh4) & 0x80008000u;
+                c.z ^= wa & 0x80008000u;  // slot 5 sits at bit 15 for every split
+            }
+            c.w ^= (aux[t] << sh_aux) & 0x80008000u;
+            const float r = fmaf(__uint_as_float((wf & d.qmask) | 0x3F800000u), dlp[t], mup[t]);
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 cf = __half22float2(u2h2(cw[k]));
+                o[k] = h22u(__floats2half2_rn(r * cf.x, r * cf.y));
+            }
+            sts128(dst + t * 16, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int blk = blockIdx.x / p.parts, part = blockIdx.x - blk * p.parts;
+    const int R8 = (p.d_out + 7) >> 3, S = p.d_in >> 3, G = p.d_in >> 7;
+    const int n_oct = block_octets(R8, blk);
+    const int g0 = part * G / p.parts, g1 = (part + 1) * G / p.parts;
+    const int n_chunk = g1 - g0, n_slab = 2 * n_chunk;
+    const int K = 1 << p.log2K, NB = p.b_slots;
+
+    GemmSmem sm;
+    {
+        uint8_t* q = smem_raw;
+        sm.cb0 = smem_u32(q); q += K * 128;
+        sm.cbraw = smem_u32(q); q += K * 16;
+        sm.code0 = smem_u32(q); q += kGCodeSlots * kGCodeSlot;
+        sm.a0 = smem_u32(q); q += 2 * kASlab;
+        sm.b_bytes = (uint32_t)p.n_pad * 128;
+        sm.b0 = smem_u32(q); q += NB * sm.b_bytes;
+        sm.bars = reinterpret_cast<uint64_t*>(q); q += (2 * kGCodeSlots + 1 + 16) * 8;
+        sm.taddr_slot = reinterpret_cast<uint32_t*>(q); q += 16;
+        sm.bcast = reinterpret_cast<int*>(q);
+    }
+    if (tid == 0) {
+        for (int k = 0; k < kGCodeSlots; ++k) {
+            mbar_init(sm.code_full(k), 1);
+            mbar_init(sm.code_empty(k), kGW);
+        }
+        mbar_init(sm.cb_full(), 1);
+        for (int k = 0; k < 8; ++k) {
+            mbar_init(sm.bars + 2 * kGCodeSlots + 1 + k, 1);      // b_full
+            mbar_init(sm.bars + 2 * kGCodeSlots + 1 + 8 + k, 1);  // mma_done (tcgen05.commit)
+        }
+        fence_mbar_init();
+        s_gabort = 0;
+    }
+    const uint32_t tcols = 2u * (uint32_t)p.n_alloc;
+    if (warp == 0) {
+        tmem_alloc(smem_u32(sm.taddr_slot), tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t taddr = *sm.taddr_slot;
+
+    if (warp == kGW) {
+        // ---------------- copy warp ----------------
+        if (lane == 0) {
+            mbar_arrive_expect_tx(sm.cb_full(), (uint32_t)K * 16);
+            bulk_g2s(sm.cbraw, p.cb, (uint32_t)K * 16, sm.cb_full());
+            const uint32_t mb = (uint32_t)(kGChunkJ * n_oct * 16), tb = (uint32_t)(n_oct * 64);
+            for (int t = 0; t < n_chunk; ++t) {
+                if (t >= kGCodeSlots) gwait(sm.code_empty(t), ((t / kGCodeSlots) - 1) & 1, p.status);
+                const int g = g0 + t;
+                const uint32_t dst = sm.code0 + (uint32_t)(t % kGCodeSlots) * kGCodeSlot;
+                mbar_arrive_expect_tx(sm.code_full(t), mb + tb);
+                bulk_g2s(dst, p.main + main_word(R8, S, blk, g * kGChunkJ, 0, 0), mb, sm.code_full(t));
+                bulk_g2s(dst + kGChunkJ * kGOct * 16, p.meta + 2 * meta_entry(R8, G, blk, g, 0, 0), tb,
+                         sm.code_full(t));
+                for (int h = 0; h < 2; ++h) {
+                    const int s = 2 * t + h;
+                    if (s >= NB) gwait(sm.mma_done(s, NB), ((s / NB) - 1) & 1, p.status);
+                    mbar_arrive_expect_tx(sm.b_full(s, NB), sm.b_bytes);
+                    bulk_g2s(sm.b0 + (uint32_t)(s % NB) * sm.b_bytes, p.xt + (size_t)(2 * g + h) * p.n_pad * 8,
+                             sm.b_bytes, sm.b_full(s, NB));
+                }
+            }
+        }
+    } else {
+        // ---------------- decode warps (+ MMA issue by thread 0) ----------------
+        gwait(sm.cb_full(), 0, p.status);
+        for (int e = tid; e < K * 8; e += kGDecodeThreads) sts128(sm.cb0 + e * 16, lds128(sm.cbraw + (e >> 3) * 16));
+        named_barrier(1, kGDecodeThreads);
+        const VDec d = vdec(p.log2K);
+        const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
+        const uint32_t idesc = idesc_f16(p.n_pad);
+        const bool active = lane < n_oct;
+        for (int t = 0; t < n_chunk; ++t) {
+            gwait(sm.code_full(t), (t / kGCodeSlots) & 1, p.status);
+            const uint32_t slot = sm.code0 + (uint32_t)(t % kGCodeSlots) * kGCodeSlot;
+            uint32_t aux[8];
+            float mup[8], dlp[8];
+            if (active) {
+                const uint32_t a = slot + kGChunkJ * kGOct * 16 + lane * 64;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint4 q = lds128(a + e * 16);
+                    aux[2 * e] = q.x;
+                    aux[2 * e + 1] = q.z;
+                    const float2 m0 = __half22float2(u2h2(q.y));
+                    const float2 m1 = __half22float2(u2h2(q.w));
+                    dlp[2 * e] = m0.y * d.vscale;
+                    mup[2 * e] = m0.x - dlp[2 * e];
+                    dlp[2 * e + 1] = m1.y * d.vscale;
+                    mup[2 * e + 1] = m1.x - dlp[2 * e + 1];
+                }
+            }
+            for (int h = 0; h < 2; ++h) {
+                const int s = 2 * t + h;
+                // the A buffer of slab s was last read by the MMAs of slab s - 2
+                if (s >= 2) gwait(sm.mma_done(s - 2, NB), ((s - 2) / NB) & 1, p.status);
+                const int jl = h * kGSlabJ + warp;  // column of the chunk
+                const uint32_t dst = sm.a0 + (uint32_t)(s & 1) * kASlab + (uint32_t)(lane >> 4) * kAHalf +
+                                     (uint32_t)(lane & 15) * kASbo + (uint32_t)warp * 128;
+                if (active) {
+                    const uint4 rec = lds128(slot + (jl * n_oct + lane) * 16);
+                    decode_to_a(d, rec, aux, (uint32_t)(15 - jl), mup, dlp, cbsel, dst);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) sts128(dst + r * 16, make_uint4(0, 0, 0, 0));
+                }
+                fence_proxy_async_smem();  // the generic-proxy writes above are read by the tensor core
+                named_barrier(1, kGDecodeThreads);
+                if (tid == 0) {
+                    gwait(sm.b_full(s, NB), (s / NB) & 1, p.status);
+                    tc_fence_after();
+                    const uint32_t a_base = sm.a0 + (uint32_t)(s & 1) * kASlab;
+                    const uint32_t b_base = sm.b0 + (uint32_t)(s % NB) * sm.b_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = smem_desc(b_base + kk * 256, 128, kBSbo);
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf)
+                            mma_f16(taddr + (uint32_t)(hf * p.n_alloc), smem_desc(a_base + hf * kAHalf + kk * 256, 128, kASbo),
+                                    bd, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(sm.mma_done(s, NB));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sm.code_empty(t));
+        }
+        // ---------------- epilogue ----------------
+        gwait(sm.mma_done(n_slab - 1, NB), ((n_slab - 1) / NB) & 1, p.status);
+        tc_fence_after();
+        const int q4 = warp & 3, hf = warp >> 2;
+        const int row_local = hf * 128 + q4 * 32 + lane;
+        const int row = blk * 256 + row_local;
+        const uint32_t tw = taddr + (uint32_t)(hf * p.n_alloc) + ((uint32_t)(q4 * 32) << 16);
+        float* mypart = p.partials + (size_t)blockIdx.x * p.n_pad * 256;
+        for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
+            float v[16];
+            tmem_ld16(tw + (uint32_t)c0, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int n = c0 + i;
+                if (n < p.M) {
+                    if (p.parts == 1) {
+                        if (row < p.d_out) p.y[(size_t)n * p.d_out + row] = __half_as_ushort(__float2half_rn(v[i]));
+                    } else {
+                        mypart[(size_t)n * 256 + row_local] = v[i];
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        if (p.parts > 1) {
+            named_barrier(1, kGDecodeThreads);  // every partial store of the CTA precedes the release below
+            if (tid == 0) {
+                const unsigned old = atom_add_acq_rel_gpu(p.counters + blk, 1u);
+                const int last = old == (unsigned)(p.parts - 1);
+                if (last) *reinterpret_cast<volatile unsigned*>(p.counters + blk) = 0u;  // ready for the next call
+                *sm.bcast = last;
+            }
+            named_barrier(1, kGDecodeThreads);
+            if (*sm.bcast && row < p.d_out) {
+                const float* base = p.partials + (size_t)blk * p.parts * p.n_pad * 256 + row_local;
+                for (int n = 0; n < p.M; ++n) {
+                    float tot = 0.f;
+                    for (int k = 0; k < p.parts; ++k) tot += __ldcg(base + ((size_t)k * p.n_pad + n) * 256);
+                    p.y[(size_t)n * p.d_out + row] = __half_as_ushort(__float2half_rn(tot));
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(taddr, tcols);
+    }
+}
+
+}  // namespace
+
+namespace {
+
+int gemm_sm_count() {
+    static std::once_flag once;
+    static int n = 0;
+    std::call_once(once, [] {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    });
+    return n;
+}
+
+size_t round256g(size_t b) { return (b + 255) / 256 * 256; }
+
+// Launch plan and workspace layout of one sage_gemm call:
+//   status header | counters [n_blocks] | x_perm tiles | partial sums (split blocks only)
+struct GemmPlan {
+    int n_pad, n_alloc, parts, b_slots, n_blocks, smem;
+    size_t off_counters, off_xt, off_part, total;
+};
+
+constexpr int kGemmSmemBudget = 226 * 1024;
+
+GemmPlan gemm_plan(const sage_matrix* A, int M) {
+    GemmPlan g;
+    g.n_pad = (M + 15) / 16 * 16;
+    g.n_alloc = 32;
+    while (g.n_alloc < g.n_pad) g.n_alloc *= 2;
+    const int R8 = (A->d_out + 7) / 8;
+    g.n_blocks = (R8 + kGOct - 1) / kGOct;
+    const int G = A->d_in / 128;
+    g.parts = std::max(1, std::min(gemm_sm_count() / g.n_blocks, G / 2));
+    const int K = 1 << A->log2K;
+    g.b_slots = 2;
+    while (g.b_slots < 8 && gemm_smem_bytes(K, g.n_pad, g.b_slots + 1) <= kGemmSmemBudget) ++g.b_slots;
+    g.smem = gemm_smem_bytes(K, g.n_pad, g.b_slots);
+    size_t o = kWsHeader;
+    g.off_counters = o;
+    o += round256g((size_t)g.n_blocks * 4);
+    g.off_xt = o;
+    o += round256g((size_t)(A->d_in / 64) * g.n_pad * 128);
+    g.off_part = o;
+    if (g.parts > 1) o += (size_t)g.n_blocks * g.parts * g.n_pad * 256 * sizeof(float);
+    g.total = o;
+    return g;
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(const sage_matrix* A, int M) { return gemm_plan(A, M).total; }
+
+int launch_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y, void* ws, size_t ws_bytes,
+                sage_stream_t stream) {
+    if (M < 9 || M > 256) return SAGE_ERR_UNSUPPORTED;
+    const GemmPlan g = gemm_plan(A, M);
+    if (ws_bytes < g.total) return SAGE_ERR_WORKSPACE;
+    if (g.smem > kGemmSmemBudget) return SAGE_ERR_UNSUPPORTED;
+    static std::mutex mu;
+    static int configured = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (g.smem > configured) {
+            if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem) != cudaSuccess)
+                return SAGE_ERR_CUDA;
+            configured = g.smem;
+        }
+    }
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint4* xt = reinterpret_cast<uint4*>(w + g.off_xt);
+    const long long n_xt = (long long)(A->d_in / 64) * g.n_pad * 8;
+    tile_x_kernel<<<(unsigned)((n_xt + 255) / 256), 256, 0, s>>>(x, A->perm, M, g.n_pad, A->d_in, xt);
+    if (cudaGetLastError() != cudaSuccess) return SAGE_ERR_CUDA;
+    GemmParams p;
+    p.main = A->main;
+    p.meta = A->meta;
+    p.cb = A->codebook;
+    p.xt = xt;
+    p.y = y;
+    p.partials = reinterpret_cast<float*>(w + g.off_part);
+    p.counters = reinterpret_cast<unsigned*>(w + g.off_counters);
+    p.status = reinterpret_cast<uint32_t*>(w);
+    p.d_out = A->d_out;
+    p.d_in = A->d_in;
+    p.log2K = A->log2K;
+    p.M = M;
+    p.n_pad = g.n_pad;
+    p.n_alloc = g.n_alloc;
+    p.parts = g.parts;
+    p.b_slots = g.b_slots;
+    gemm_kernel<<<(unsigned)(g.n_blocks * g.parts), kGThreads, (size_t)g.smem, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 }  // namespace sage

@@ -499,24 +499,6 @@ __device__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleStat
 // ------------------------------------------------------------------------
 // Decode warps.
 // ------------------------------------------------------------------------
-struct VDec {            // per-split decode constants (radius width V = 10 - log2K)
-    uint32_t zmask, qmask;
-    uint32_t sh0, sh1, sh2, sh3, sh4, sh5;   // 15 - (sign slot position)
-    float vscale;
-};
-
-__device__ __forceinline__ VDec vdec(int log2K) {
-    const int V = 10 - log2K;
-    VDec d;
-    d.zmask = ((1u << log2K) - 1u) << 7;
-    d.qmask = ((1u << V) - 1u) << (23 - V);
-    // slot k sits at bit k for k <= 6 - V, else at bit 10 + k
-    auto sh = [&](int k) { return (uint32_t)(k <= 6 - V ? 15 - k : 5 - k); };
-    d.sh0 = sh(0); d.sh1 = sh(1); d.sh2 = sh(2); d.sh3 = sh(3); d.sh4 = sh(4); d.sh5 = sh(5);
-    d.vscale = (float)(1 << V);
-    return d;
-}
-
 template <int M>
 __device__ __forceinline__ void decode_record(const VDec& d, uint4 rec, const uint32_t (&aux)[8], uint32_t sh_aux,
                                               const float (&mup)[8], const float (&dlp)[8], uint32_t cbsel,
