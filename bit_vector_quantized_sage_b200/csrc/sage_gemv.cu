@@ -111,6 +111,7 @@ struct Common {
     int n_cta;
     int M;                 // dense: batch; MoE: 0 (per virtual expert)
     int slots;             // ring depth (chunks in flight)
+    int n_wg;              // decode warp groups (1, 2 or 4); chunk t goes to group t % n_wg
     int kmax;              // largest codebook of the launch (replica area size)
     uint32_t* status;
     unsigned* counters;
@@ -121,11 +122,14 @@ struct Common {
 // flattened units evenly; per-matrix plans give matrix k its own CTAs and
 // split its units evenly among them.  Both are plain arithmetic, so no
 // dependent parameter-space loads sit on any critical path.
+constexpr int kMaxCta = 256;
+
 struct DenseParams {
     Common c;
     long long total_units;
     int n_mats;
     int per_matrix;
+    int cta_start[kMaxCta + 1];   // first unit of each CTA; cta_start[n_cta] = total_units
     DenseMat mats[kMaxMats];
 };
 
@@ -146,28 +150,27 @@ struct MoeParams {
     ExpertMat experts[kMaxExperts];
 };
 
+// The CTA start table and the matrix descriptors are read from shared-memory
+// copies: dependent loads from the parameter space miss the constant cache.
 struct DenseProblem {
     const DenseParams& p;
+    const int* cs;        // shared copy of p.cta_start
+    const DenseMat* ms;   // shared copy of p.mats
     __device__ long long total() const { return p.total_units; }
-    __device__ long long cta_begin(int c) const {
-        if (!p.per_matrix) return (long long)c * p.total_units / p.c.n_cta;
-        if (c >= p.c.n_cta) return p.total_units;
-        int k = 0;
-        while (k + 1 < p.n_mats && p.mats[k + 1].cta0 <= c) ++k;
-        const DenseMat& d = p.mats[k];
-        return d.unit0 + (long long)(c - d.cta0) * d.units / d.ncta;
-    }
-    __device__ int cta_of(long long u) const {
-        if (!p.per_matrix) return (int)(((u + 1) * p.c.n_cta + p.total_units - 1) / p.total_units) - 1;
-        int k = 0;
-        while (k + 1 < p.n_mats && p.mats[k + 1].unit0 <= u) ++k;
-        const DenseMat& d = p.mats[k];
-        return d.cta0 + (int)(((u - d.unit0 + 1) * d.ncta + d.units - 1) / d.units) - 1;
+    __device__ long long cta_begin(int c) const { return cs[min(c, p.c.n_cta)]; }
+    __device__ int cta_of(long long u) const {  // the CTA whose range holds unit u
+        int lo = 0, hi = p.c.n_cta - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cs[mid] <= u) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
     }
     __device__ MatView view(long long u) const {
         int k = 0;
-        while (k + 1 < p.n_mats && p.mats[k + 1].unit0 <= u) ++k;
-        const DenseMat& d = p.mats[k];
+        while (k + 1 < p.n_mats && ms[k + 1].unit0 <= u) ++k;
+        const DenseMat& d = ms[k];
         MatView v;
         v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = d.x; v.y = d.y;
         v.xrows = nullptr; v.yrows = nullptr; v.unit0 = d.unit0;
@@ -223,9 +226,9 @@ template <class Problem>
 __device__ Seg make_seg(const Problem& P, long long u, long long u_end, long long cta_u0) {
     Seg s;
     s.v = P.view(u);
-    const long long local = u - s.v.unit0;
-    s.blk = (int)(local / s.v.S);
-    s.ja = (int)(local - (long long)s.blk * s.v.S);
+    const int local = (int)(u - s.v.unit0);  // unit counts fit in 32 bits (checked on the host)
+    s.blk = local / s.v.S;
+    s.ja = local - s.blk * s.v.S;
     const long long jb = (long long)s.ja + (u_end - u);
     s.jb = (int)(jb < (long long)s.v.S ? jb : (long long)s.v.S);
     s.n_oct = min(kOct, s.v.R8 - s.blk * kOct);
@@ -299,10 +302,11 @@ struct Smem {
     float* stash;
     uint64_t* bars;
     int* bcast;
+    int* wlen0;       // length of the first activation window
     Seg* segs;
-    __device__ uint32_t slot(int t) const { return ring0 + (uint32_t)(t % slots) * kSlot; }
-    __device__ uint64_t* full(int t) const { return bars + (t % slots); }
-    __device__ uint64_t* empty(int t) const { return bars + kMaxSlots + (t % slots); }
+    __device__ uint32_t slot_addr(int k) const { return ring0 + (uint32_t)k * kSlot; }
+    __device__ uint64_t* full(int k) const { return bars + k; }
+    __device__ uint64_t* empty(int k) const { return bars + kMaxSlots + k; }
     __device__ uint64_t* cb_full(int h) const { return bars + 2 * kMaxSlots + h; }
     __device__ uint64_t* cb_empty(int h) const { return bars + 2 * kMaxSlots + 2 + h; }
     __device__ uint64_t* x_full(int h) const { return bars + 2 * kMaxSlots + 4 + h; }
@@ -328,6 +332,7 @@ __device__ __forceinline__ Smem<M> carve(uint8_t* base, int slots, int kmax) {
     s.segs = reinterpret_cast<Seg*>(p); p += kSegTab * kSegBytes;
     s.bars = reinterpret_cast<uint64_t*>(p); p += (2 * kMaxSlots + 9) * 8;
     s.bcast = reinterpret_cast<int*>(p);
+    s.wlen0 = s.bcast + 8;
     return s;
 }
 
@@ -350,9 +355,18 @@ __device__ __forceinline__ void win_break(WinPos& w) {
     if (w.wpos > 0) { ++w.win; w.wpos = 0; }
 }
 
+__device__ __forceinline__ void ring_next(int& slot, int& ph, int slots) {
+    if (++slot == slots) {
+        slot = 0;
+        ph ^= 1;
+    }
+}
+
 // Per-role progress that persists across segment-table rounds.
 struct RoleState {
-    int t;      // chunk counter (ring slots and phases)
+    int t;      // chunk counter
+    int slot;   // ring slot of chunk t (t % slots, kept incrementally)
+    int ph;     // phase parity of that slot for chunk t ((t / slots) & 1)
     int s;      // segment counter (codebook phases)
     WinPos w;   // activation window placement
     int cur_win;  // decode warps: the x window they hold (-1: none)
@@ -376,18 +390,18 @@ __device__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleSta
             bulk_g2s(sm.cbraw0 + (s & 1) * sm.cbraw_bytes, g.v.cb, cbb, sm.cb_full(s & 1));
         }
         const int n_oct = g.n_oct, R8 = g.v.R8, S = g.v.S, G = g.v.d_in >> 7, blk = g.blk;
-        for (int c = 0; c < g.n_chunks; ++c, ++st.t) {
-            const int t = st.t;
-            if (t >= sm.slots) wait_bar(sm.empty(t), ((t / sm.slots) - 1) & 1, C);
+        for (int c = 0; c < g.n_chunks; ++c, ++st.t, ring_next(st.slot, st.ph, sm.slots)) {
+            const int k = st.slot;
+            if (st.t >= sm.slots) wait_bar(sm.empty(k), st.ph ^ 1, C);
             if (lane == 0) {
                 const int2 cc = chunk_cols(g, c);
                 const int nj = cc.y - cc.x;
                 const uint32_t mb = (uint32_t)(nj * n_oct * 16), tb = (uint32_t)(n_oct * 64);
-                mbar_arrive_expect_tx(sm.full(t), mb + tb);
+                mbar_arrive_expect_tx(sm.full(k), mb + tb);
                 // the chunk's records: one contiguous range of the block; its group's meta entries
-                bulk_g2s(sm.slot(t), g.v.main + main_word(R8, S, blk, cc.x, 0, 0), mb, sm.full(t));
-                bulk_g2s(sm.slot(t) + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0), tb,
-                         sm.full(t));
+                bulk_g2s(sm.slot_addr(k), g.v.main + main_word(R8, S, blk, cc.x, 0, 0), mb, sm.full(k));
+                bulk_g2s(sm.slot_addr(k) + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0), tb,
+                         sm.full(k));
             }
         }
     }
@@ -396,8 +410,7 @@ __device__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleSta
 // The CTA may not exit while bulk copies are in flight.
 template <int M>
 __device__ void copy_drain(const Common& C, const Smem<M>& sm, const RoleState& st) {
-    for (int t = max(0, st.t - sm.slots); t < st.t; ++t)
-        wait_bar(sm.full(t), (t / sm.slots) & 1, C);
+    for (int t = max(0, st.t - sm.slots); t < st.t; ++t) wait_bar(sm.full(t % sm.slots), (t / sm.slots) & 1, C);
 }
 
 // ------------------------------------------------------------------------
@@ -407,42 +420,19 @@ __device__ void copy_drain(const Common& C, const Smem<M>& sm, const RoleState& 
 // preceding kernel, since only x comes from that kernel -- so after the wait
 // the gather costs one round trip per window.
 // ------------------------------------------------------------------------
-template <int M>
-__device__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
+// Gathers x_perm for window positions e = gi, gi + gn, ... of the (batch row,
+// position) pairs of a window of wlen positions into the window buffer xb.
+// All loads of a round are issued before any store.
+template <int M, int B>
+__device__ __forceinline__ void gather_x(const Smem<M>& sm, int wlen, uint32_t xb, int gi, int gn) {
     constexpr int XW = Cfg<M>::kXW;
-    const int lane = threadIdx.x & 31;
-    fence_proxy_async_smem();  // earlier reads of the permutation buffer precede the copies below
-    int si = si0, c = c0, wlen = 0;
-    for (int k = 0; k < nch; ++k) {
-        const Seg& g = sm.segs[si];
-        const int2 cc = chunk_cols(g, c);
-        const int nj = cc.y - cc.x;
-        if (g.v.perm && lane == 0) {
-            mbar_expect_tx(sm.perm_full(), (uint32_t)(nj * 32));
-            bulk_g2s(sm.perm0 + wlen * 32, g.v.perm + cc.x * 8, (uint32_t)(nj * 32), sm.perm_full());
-        }
-        if (lane < nj) sm.posinfo[wlen + lane] = ((uint32_t)si << 24) | (uint32_t)(cc.x + lane);
-        wlen += nj;
-        if (++c == g.n_chunks) { c = 0; ++si; }
-    }
-    if (lane == 0) mbar_arrive(sm.perm_full());
-    if (!waited) {
-        pdl_wait();  // x may be written by the preceding kernel
-        waited = true;
-    }
-    wait_bar(sm.perm_full(), w & 1, C);
-    if (w >= 2) wait_bar(sm.x_empty(w & 1), ((w >> 1) - 1) & 1, C);
-    __syncwarp();
-    const uint32_t xb = sm.xwin(w);
     const int total = M * wlen;
-    // All loads of a round are issued before any store: one memory round trip
-    // per 256 (batch row, column) pairs.
-    for (int e0 = 0; e0 < total; e0 += 8 * 32) {
-        uint4 val[8];
-        uint32_t dst[8];
+    for (int e0 = 0; e0 < total; e0 += B * gn) {
+        uint4 val[B];
+        uint32_t dst[B];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int e = e0 + r * 32 + lane;
+        for (int r = 0; r < B; ++r) {
+            const int e = e0 + r * gn + gi;
             dst[r] = 0xffffffffu;
             if (e < total) {
                 const int m = e / wlen, p = e - m * wlen;
@@ -468,8 +458,51 @@ __device__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, 
             }
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int r = 0; r < B; ++r)
             if (dst[r] != 0xffffffffu) sts128(dst[r], val[r]);
+    }
+}
+
+// Named barriers besides the decode warps' own (id 1): the activation and
+// copy warps (id 3) and the activation and decode warps (id 2).
+constexpr int kBarPermIssued = 3;
+constexpr int kBarFirstWindow = 2;
+
+template <int M>
+__device__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
+    const int lane = threadIdx.x & 31;
+    fence_proxy_async_smem();  // earlier reads of the permutation buffer precede the copies below
+    int si = si0, c = c0, wlen = 0;
+    for (int k = 0; k < nch; ++k) {
+        const Seg& g = sm.segs[si];
+        const int2 cc = chunk_cols(g, c);
+        const int nj = cc.y - cc.x;
+        if (g.v.perm && lane == 0) {
+            mbar_expect_tx(sm.perm_full(), (uint32_t)(nj * 32));
+            bulk_g2s(sm.perm0 + wlen * 32, g.v.perm + cc.x * 8, (uint32_t)(nj * 32), sm.perm_full());
+        }
+        if (lane < nj) sm.posinfo[wlen + lane] = ((uint32_t)si << 24) | (uint32_t)(cc.x + lane);
+        wlen += nj;
+        if (++c == g.n_chunks) { c = 0; ++si; }
+    }
+    if (lane == 0) mbar_arrive(sm.perm_full());
+    // The first window's permutation entries go ahead of the code chunks in the
+    // copy queue: the copy warp starts once they are issued.
+    if (w == 0) named_barrier(kBarPermIssued, 64);
+    if (!waited) {
+        pdl_wait();  // x may be written by the preceding kernel
+        waited = true;
+    }
+    wait_bar(sm.perm_full(), w & 1, C);
+    if (w >= 2) wait_bar(sm.x_empty(w & 1), ((w >> 1) - 1) & 1, C);
+    __syncwarp();
+    if (w == 0) {  // the decode warps, idle until now, help with the first window
+        if (lane == 0) *sm.wlen0 = wlen;
+        named_barrier(kBarFirstWindow, 32 + Cfg<M>::kDecodeThreads);
+        gather_x<M, 2>(sm, wlen, sm.xwin(0), Cfg<M>::kDecodeThreads + lane, 32 + Cfg<M>::kDecodeThreads);
+        named_barrier(kBarFirstWindow, 32 + Cfg<M>::kDecodeThreads);
+    } else {
+        gather_x<M, 8>(sm, wlen, sm.xwin(w), lane, 32);
     }
     mbar_arrive(sm.x_full(w & 1));  // all 32 lanes, each after its own stores
 }
@@ -532,48 +565,76 @@ __device__ __forceinline__ void decode_record(const VDec& d, uint4 rec, const ui
     }
 }
 
-// Decodes this warp's columns of ring chunk t (chunk c of segment g): columns
-// warp, warp + W, ... of the chunk, against the x_perm window at xw, where the
-// chunk's first column sits at window position pos.
+// Loads the grid / aux meta of this lane's octet (64 bytes at a) without bank
+// conflicts: lane pairs start at rotated 16-byte quarters, and the four
+// quarters are rotated back into place with selects.
+__device__ __forceinline__ void load_meta(uint32_t a, int lane, uint4 (&q)[4]) {
+    const int r = (lane >> 1) & 3;
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = lds128(a + (uint32_t)((k + r) & 3) * 16);  // v[k] = quarter (k + r) & 3
+    uint4 u[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {  // quarter e sits in v[(e - r) & 3]: rotate right by r
+        const uint4 a1 = (r & 1) ? v[(e + 3) & 3] : v[e];
+        const uint4 a2 = (r & 1) ? v[(e + 1) & 3] : v[(e + 2) & 3];
+        u[e] = (r & 2) ? a2 : a1;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = u[e];
+}
+
+// Decodes this warp's columns of one ring chunk (chunk c of segment g, in
+// ring slot k with phase parity ph): columns lw, lw + wpg, ... of the chunk,
+// against the x_perm window at xw, where the chunk's first column sits at
+// window position pos.
 template <int M, int MS>
-__device__ __forceinline__ void decode_chunk(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int t,
-                                             int c, uint32_t xw, int pos, int warp, int lane, float (&acc)[8][M]) {
-    constexpr int W = Cfg<MS>::kW, XW = Cfg<MS>::kXW;
+__device__ __forceinline__ void decode_chunk(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int k,
+                                             int ph, int c, uint32_t xw, int pos, int lw, int wpg, int lane,
+                                             float (&acc)[8][M]) {
+    constexpr int XW = Cfg<MS>::kXW;
     const int2 cc = chunk_cols(g, c);
     const int nj = cc.y - cc.x;
-    wait_bar(sm.full(t), (t / sm.slots) & 1, C);
+    wait_bar(sm.full(k), ph, C);
     const int n_oct = g.n_oct;
-    if (warp < nj && lane < n_oct) {
-        const uint32_t base = sm.slot(t);
+    if (lw < nj && lane < n_oct) {
+        const uint32_t base = sm.slot_addr(k);
         const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
         uint32_t aux[8];
         float mup[8], dlp[8];
         {   // the group's grid and aux signs for this lane's 8 rows
-            const uint32_t a = base + kMainSlot + lane * 64;
+            uint4 q[4];
+            load_meta(base + kMainSlot + lane * 64, lane, q);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const uint4 q = lds128(a + e * 16);
-                aux[2 * e] = q.x;
-                aux[2 * e + 1] = q.z;
-                const float2 m0 = __half22float2(u2h2(q.y));
-                const float2 m1 = __half22float2(u2h2(q.w));
+                aux[2 * e] = q[e].x;
+                aux[2 * e + 1] = q[e].z;
+                const float2 m0 = __half22float2(u2h2(q[e].y));
+                const float2 m1 = __half22float2(u2h2(q[e].w));
                 dlp[2 * e] = m0.y * d.vscale;
                 mup[2 * e] = m0.x - dlp[2 * e];
                 dlp[2 * e + 1] = m1.y * d.vscale;
                 mup[2 * e + 1] = m1.x - dlp[2 * e + 1];
             }
         }
-        for (int i = warp; i < nj; i += W) {
+        auto column = [&](int i) {
             const int j = cc.x + i;
             const uint4 rec = lds128(base + (i * n_oct + lane) * 16);
             uint4 xv[M];
 #pragma unroll
             for (int m = 0; m < M; ++m) xv[m] = lds128(xw + (m * XW + pos + i) * 16);
             decode_record<M>(d, rec, aux, (uint32_t)(15 - (j & 15)), mup, dlp, cbsel, xv, acc);
+        };
+        if constexpr (M <= 4) {  // two columns in flight where registers allow
+#pragma unroll 2
+            for (int i = lw; i < nj; i += wpg) column(i);
+        } else {
+#pragma unroll 1
+            for (int i = lw; i < nj; i += wpg) column(i);
         }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.empty(t));
+    if (lane == 0) mbar_arrive(sm.empty(k));
 }
 
 // Writes (or combines) the outputs of the pending segments tab[i0 .. i0 + n).
@@ -670,9 +731,10 @@ __device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, c
     for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int m = 0; m < MK; ++m) acc[r][m] = 0.f;
-    int t = st.t, cur = st.cur_win;
+    int t = st.t, k = st.slot, ph = st.ph, cur = st.cur_win;
     WinPos w = st.w;
-    for (int c = 0; c < g.n_chunks; ++c, ++t) {
+    const int wpg = W / C.n_wg, grp = warp / wpg, lw = warp - grp * wpg;
+    for (int c = 0; c < g.n_chunks; ++c, ++t, ring_next(k, ph, sm.slots)) {
         const int2 cc = chunk_cols(g, c);
         const int pos = win_place(w, cc.y - cc.x, Cfg<MS>::kXW);
         if (w.win != cur) {  // release the previous x window, wait for this one
@@ -680,12 +742,21 @@ __device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, c
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sm.x_empty(cur & 1));
             }
-            wait_bar(sm.x_full(w.win & 1), (w.win >> 1) & 1, C);
+            if (w.win == 0) {  // the first window is gathered together with the activation warp
+                pdl_wait();
+                named_barrier(kBarFirstWindow, 32 + DT);
+                gather_x<MS, 2>(sm, *sm.wlen0, sm.xwin(0), tid, 32 + DT);
+                named_barrier(kBarFirstWindow, 32 + DT);
+            } else {
+                wait_bar(sm.x_full(w.win & 1), (w.win >> 1) & 1, C);
+            }
             cur = w.win;
         }
-        decode_chunk<MK, MS>(sm, C, g, d, t, c, sm.xwin(w.win), pos, warp, lane, acc);
+        if ((t & (C.n_wg - 1)) == grp) decode_chunk<MK, MS>(sm, C, g, d, k, ph, c, sm.xwin(w.win), pos, lw, wpg, lane, acc);
     }
     st.t = t;
+    st.slot = k;
+    st.ph = ph;
     st.cur_win = cur;
     st.w = w;
     // reduce the warps' partial sums in a fixed order into the stash
@@ -759,7 +830,7 @@ __device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* 
     if (tid == 0) {
         for (int k = 0; k < kMaxSlots; ++k) {
             mbar_init(sm.bars + k, 1);              // full: copy warp arrival + bytes
-            mbar_init(sm.bars + kMaxSlots + k, W);  // empty: one arrival per decode warp
+            mbar_init(sm.bars + kMaxSlots + k, W / C.n_wg);  // empty: one arrival per warp of the chunk's group
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(sm.cb_full(h), 1);
@@ -778,13 +849,14 @@ __device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* 
     const long long total = P.total();
     const long long u0 = total > 0 ? P.cta_begin(blockIdx.x) : 0;
     const long long u1 = total > 0 ? P.cta_begin(blockIdx.x + 1) : 0;
-    RoleState st{0, 0, {0, 0}, -1};
+    RoleState st{0, 0, 0, 0, {0, 0}, -1};
     bool waited = plan_needs_wait;
     for (long long u = u0; u < u1;) {
         if (tid == 0) s_nseg = build_segs(P, C, u, u1, u0, sm.segs, &s_next);
         __syncthreads();
         const int n_seg = s_nseg;
         if (warp == W) {
+            if (u == u0) named_barrier(kBarPermIssued, 64);  // after the first window's permutation copies
             copy_warp<M>(C, sm, n_seg, st);
         } else if (warp == W + 1) {
             act_warp<M>(C, sm, n_seg, st, waited);
@@ -801,7 +873,12 @@ __device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* 
 template <int M>
 __global__ void __launch_bounds__(Cfg<M>::kThreads, 1) gemv_kernel(const __grid_constant__ DenseParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    const DenseProblem P{p};
+    __shared__ int s_cs[kMaxCta + 1];
+    __shared__ DenseMat s_ms[kMaxMats];
+    for (int i = threadIdx.x; i <= p.c.n_cta; i += blockDim.x) s_cs[i] = p.cta_start[i];
+    for (int i = threadIdx.x; i < p.n_mats; i += blockDim.x) s_ms[i] = p.mats[i];
+    __syncthreads();
+    const DenseProblem P{p, s_cs, s_ms};
     run<M, M>(P, p.c, smem_raw, false);
 }
 
@@ -906,13 +983,18 @@ std::vector<int> per_matrix_shares(const std::vector<long long>& units, int n_ct
 // Ring depth: as many chunk slots as fit next to the fixed shared memory (one
 // CTA per SM), at most one more than the widest CTA's chunk count.
 constexpr int kSmemBudget = 226 * 1024;  // 227 KB per CTA less static shared memory
+constexpr int kDenseStatic = (kMaxCta + 1) * 4 + kMaxMats * (int)sizeof(DenseMat);  // gemv_kernel's staged tables
 template <int M>
-int slots_for(long long max_units_per_cta, int kmax) {
+int slots_for(long long max_units_per_cta, int kmax, int budget) {
     const long long chunks = (max_units_per_cta + kChunkJ - 1) / kChunkJ + 2;
     int n = (int)std::min<long long>(kMaxSlots, std::max<long long>(2, chunks));
-    while (n > 2 && Cfg<M>::smem(n, kmax) > kSmemBudget) --n;
+    while (n > 2 && Cfg<M>::smem(n, kmax) > budget) --n;
     return n;
 }
+
+// Decode warp groups: a chunk is decoded by one group, so that a warp handles
+// several columns per ring slot; each group needs two slots in flight.
+int wg_for(int slots) { return slots >= 8 ? 4 : slots >= 4 ? 2 : 1; }
 
 // Raises the kernel's dynamic shared memory limit when a launch needs more
 // than any earlier one (callers hold the launch mutex).
@@ -961,7 +1043,8 @@ int launch_m(const GemvJob* jobs, int n, void* ws, sage_stream_t stream) {
         unit += units[i];
         blk += blocks_of(A);
     }
-    const int n_cta = (int)std::max<long long>(1, std::min<long long>(sm_count(), unit / 4));
+    if (unit >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+    const int n_cta = (int)std::max<long long>(1, std::min<long long>(std::min(sm_count(), kMaxCta), unit / 4));
     const std::vector<int> share = per_matrix_shares(units, n_cta);
     long long widest = 0;
     p.per_matrix = share.empty() ? 0 : 1;
@@ -977,8 +1060,22 @@ int launch_m(const GemvJob* jobs, int n, void* ws, sage_stream_t stream) {
     p.n_mats = n;
     p.total_units = unit;
     p.c.n_cta = n_cta;
+    for (int c = 0; c <= n_cta; ++c) {
+        long long b;
+        if (c == n_cta) {
+            b = unit;
+        } else if (share.empty()) {
+            b = (long long)c * unit / n_cta;
+        } else {
+            int k = 0;
+            while (k + 1 < n && p.mats[k + 1].cta0 <= c) ++k;
+            b = p.mats[k].unit0 + (long long)(c - p.mats[k].cta0) * p.mats[k].units / p.mats[k].ncta;
+        }
+        p.cta_start[c] = (int)b;
+    }
     p.c.M = M;
-    p.c.slots = slots_for<M>(widest, kmax);
+    p.c.slots = slots_for<M>(widest, kmax, kSmemBudget - kDenseStatic);
+    p.c.n_wg = wg_for(p.c.slots);
     p.c.kmax = kmax;
     if (!ensure_smem(gemv_kernel<M>, Cfg<M>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
@@ -1060,7 +1157,8 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
     int kmax = 16;
     for (int e = 0; e < n_experts; ++e) kmax = std::max(kmax, 1 << experts[e].log2K);
     p.c.kmax = kmax;
-    p.c.slots = slots_for<MV>(1 << 30, kmax);
+    p.c.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget);
+    p.c.n_wg = wg_for(p.c.slots);
     if (!ensure_smem(moe_kernel, Cfg<MV>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
     p.c.status = reinterpret_cast<uint32_t*>(w);
     p.c.counters = reinterpret_cast<unsigned*>(w + L.counters);
