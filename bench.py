@@ -201,6 +201,110 @@ def cpu_oracle_sample(rows_per_matrix: int = 256, seconds_cap: float = 60.0):
     return tot_bytes / tot_s / 1e9, desc, 1, tot_s
 
 
+def _peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["bf16_tflops"]), "measured (bf16 burst; fp16 dense has the same nominal rate)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def _timed_calls(fn, stream, reps, flush):
+    """Median device time (ms) of one fn call with L2 flushed before each call.
+    The call is captured once in a CUDA graph; the flush is enqueued first, so
+    the host side of the replay overlaps it and the events bracket device work
+    only."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(torch.cuda.current_stream())
+    g.replay()
+    times = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del g
+    return statistics.median(times)
+
+
+def bench_gemm(stream, flush, reps=20):
+    """Config 3: 4096 -> 12288, (K,V) = (32,5); batch 1-8 through the GEMV
+    kernel, 16-128 through the tcgen05 path (sage_gemm).  Per batch: device us,
+    TFLOP/s against the measured dense fp16 peak and GB/s of packed bytes."""
+    import torch
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    f, _ = synth.config3(1)
+    A = sage.PackedMatrix.from_fields(f)
+    peak, kind = _peak_tflops()
+    hbm, _ = _peaks()
+    out = []
+    for M in (1, 2, 4, 8, 16, 32, 64, 128):
+        _, xb = synth.config3(M)
+        x = torch.from_numpy(xb.view(np.int16)).cuda()
+        y = torch.zeros((M, f.d_out), dtype=torch.int16, device="cuda")
+        ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_GEMM, A, M))
+        fn = lambda st: sage.sage_gemm(A, x, M, y, ws, st)
+        for _ in range(3):
+            fn(stream)
+        ms = _timed_calls(fn, stream, reps, flush)
+        assert sage.sage_query_status(ws) == sage.SAGE_OK
+        flops = 2.0 * M * f.d_out * f.d_in
+        nbytes = A.packed_bytes + 32 * 16 + M * f.d_in * 2 + M * f.d_out * 2
+        tf = flops / (ms * 1e-3) / 1e12
+        out.append({"M": M, "path": "gemv" if M <= 8 else "tcgen05", "us": round(ms * 1e3, 2),
+                    "tflops": round(tf, 1), "tensor_frac": round(tf / peak, 4),
+                    "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
+    return {"workload": "4096->12288 up-projection, (K,V)=(32,5), L2 flushed before each call",
+            "peak_tflops": peak, "peak_kind": kind, "points": out}
+
+
+def bench_moe(stream, flush, reps=20):
+    """Config 4: 128 experts, gate 2048 -> 768 and down 768 -> 2048, top-8,
+    T tokens; one sage_moe_gemv call per projection."""
+    import torch
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    hbm, _ = _peaks()
+    out = []
+    for proj in (0, 2):
+        packed = None
+        for T in (1, 4, 16):
+            spec = synth.config4(T)
+            if packed is None:
+                packed = [sage.PackedMatrix.from_fields(spec.expert(e, proj)) for e in range(synth.MOE_EXPERTS)]
+            n_pairs = T * synth.MOE_TOPK
+            pe = torch.from_numpy(spec.routes.reshape(-1).astype(np.int32)).cuda()
+            if proj < 2:
+                xb, xrow = spec.x, np.repeat(np.arange(T, dtype=np.int32), synth.MOE_TOPK)
+            else:
+                xb, xrow = spec.x_down, np.arange(n_pairs, dtype=np.int32)
+            x = torch.from_numpy(xb.view(np.int16)).cuda()
+            xr = torch.from_numpy(xrow).cuda()
+            d_out = synth.MOE_PROJ[proj][1]
+            y = torch.zeros((n_pairs, d_out), dtype=torch.int16, device="cuda")
+            ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_MOE, packed, n_pairs))
+            fn = lambda st: sage.sage_moe_gemv(packed, pe, xr, n_pairs, x, y, ws, st)
+            for _ in range(3):
+                fn(stream)
+            ms = _timed_calls(fn, stream, reps, flush)
+            assert sage.sage_query_status(ws) == sage.SAGE_OK
+            active = np.unique(spec.routes)
+            nbytes = sum(packed[e].packed_bytes + (1 << packed[e].log2K) * 16 for e in active)
+            nbytes += xb.nbytes + n_pairs * d_out * 2
+            out.append({"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size),
+                        "us": round(ms * 1e3, 2), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                        "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
+    return {"workload": "128 experts, top-8, one projection per call, L2 flushed before each call", "points": out}
+
+
 def run_reference(args):
     ws, rank, _ = _dist()
     if rank != 0:
@@ -355,6 +459,14 @@ def run_gpu(args):
     e2e_value = world * one_layer_bytes / (e2e_ms * 1e-3) / 1e9
     del g_e2e
 
+    extra = {}
+    if rank == 0 and not args.no_extra:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        with torch.cuda.stream(stream):
+            extra["gemm_config3"] = bench_gemm(stream, flush)
+            extra["moe_config4"] = bench_moe(stream, flush)
+        del flush
+
     peak, peak_kind = _peaks()
     achieved = sum(stage_bytes) / (sum(stage_avg) * 1e-3) / 1e9
     traffic, _ = _traffic_for(_kernel_hash())
@@ -385,6 +497,7 @@ def run_gpu(args):
         "gpu_launches": args.steps * n_stage,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "extra": extra,
     }
     if rank == 0:
         print(json.dumps(line))
@@ -402,6 +515,7 @@ def main():
     ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the batch sweep and MoE measurements")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -23,6 +23,18 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
@@ -191,6 +203,25 @@ __device__ __forceinline__ VDec vdec(int log2K) {
     d.sh0 = sh(0); d.sh1 = sh(1); d.sh2 = sh(2); d.sh3 = sh(3); d.sh4 = sh(4); d.sh5 = sh(5);
     d.vscale = (float)(1 << V);
     return d;
+}
+
+// Loads the grid / aux meta of this lane's octet (64 bytes at a) without bank
+// conflicts: lane pairs start at rotated 16-byte quarters, and the four
+// quarters are rotated back into place with selects.
+__device__ __forceinline__ void load_meta(uint32_t a, int lane, uint4 (&q)[4]) {
+    const int r = (lane >> 1) & 3;
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = lds128(a + (uint32_t)((k + r) & 3) * 16);  // v[k] = quarter (k + r) & 3
+    uint4 u[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {  // quarter e sits in v[(e - r) & 3]: rotate right by r
+        const uint4 a1 = (r & 1) ? v[(e + 3) & 3] : v[e];
+        const uint4 a2 = (r & 1) ? v[(e + 1) & 3] : v[(e + 2) & 3];
+        u[e] = (r & 2) ? a2 : a1;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = u[e];
 }
 
 }  // namespace dev

@@ -34,15 +34,15 @@ using namespace dev;
 
 namespace {
 
-constexpr int kGW = 8;                        // decode warps
-constexpr int kGThreads = (kGW + 1) * 32;     // + copy warp
+constexpr int kGW = 16;                       // decode warps: two per (slab column, record half)
+constexpr int kGThreads = (kGW + 2) * 32;     // + copy warp + MMA warp
 constexpr int kGDecodeThreads = kGW * 32;
 constexpr int kGOct = 32;                     // row octets per block
 constexpr int kGChunkJ = 16;                  // subvector columns per chunk (one radius group)
 constexpr int kGSlabJ = 8;                    // subvector columns per MMA slab (64 input channels)
 constexpr int kGCodeSlot = kGChunkJ * kGOct * 16 + kGOct * 64;  // records + meta of one chunk
 constexpr int kGCodeSlots = 4;
-constexpr int kASbo = 1040;                   // bytes between 8-row core-matrix groups of A (padded: no bank conflicts)
+constexpr int kASbo = 1024;                   // bytes between 8-row core-matrix groups of A
 constexpr int kAHalf = 16 * kASbo;            // one 128-row half of an A slab
 constexpr int kASlab = 2 * kAHalf;            // 256 rows x 64 channels, fp16
 constexpr int kBSbo = 1024;                   // B: 8 core matrices of 8 rows x 16 bytes per 8 batch rows
@@ -104,6 +104,25 @@ __host__ __device__ constexpr uint32_t idesc_f16(int n) {
 
 __device__ __forceinline__ void gflag(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
 
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory offset in the CTA of the cluster with the given rank.
+__device__ __forceinline__ uint32_t map_cluster(uint32_t addr, int rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 // Set when a bounded wait of the CTA gives up; later waits then return at once.
 __shared__ int s_gabort;
 
@@ -156,14 +175,14 @@ struct GemmParams {
     const uint16_t* cb;
     const uint4* xt;        // x_perm in the B-operand layout (tile_x_kernel)
     uint16_t* y;            // [M][d_out]
-    float* partials;        // [n_blocks * parts][n_pad][256]
-    unsigned* counters;     // [n_blocks], zero between calls
     uint32_t* status;
     int d_out, d_in, log2K, M;
     int n_pad;              // M rounded up to 16: the MMA's N
     int n_alloc;            // TMEM columns per accumulator (power of two >= max(32, n_pad))
-    int parts;              // CTAs per block (split over the input columns)
+    int parts;              // CTAs per block (split over the input columns), one cluster
+    int red_cols;           // batch columns per round of the cluster reduction
     int b_slots;            // x_perm slabs in flight
+    int a_slots;            // decoded W_hat slabs in flight (2 .. kMaxASlots)
 };
 
 struct GemmSmem {
@@ -177,48 +196,37 @@ struct GemmSmem {
     __device__ uint64_t* cb_full() const { return bars + 2 * kGCodeSlots; }
     __device__ uint64_t* b_full(int s, int nb) const { return bars + 2 * kGCodeSlots + 1 + (s % nb); }
     __device__ uint64_t* mma_done(int s, int nb) const { return bars + 2 * kGCodeSlots + 1 + 8 + (s % nb); }
+    __device__ uint64_t* a_full(int s, int na) const { return bars + 2 * kGCodeSlots + 1 + 16 + (s % na); }
 };
 
-__host__ __device__ inline int gemm_smem_bytes(int K, int n_pad, int b_slots) {
-    return K * 128 + K * 16 + kGCodeSlots * kGCodeSlot + 2 * kASlab + b_slots * n_pad * 128 +
-           (2 * kGCodeSlots + 1 + 16) * 8 + 64;
+constexpr int kMaxASlots = 4;
+__host__ __device__ inline int gemm_smem_bytes(int K, int n_pad, int a_slots, int b_slots) {
+    return K * 128 + K * 16 + kGCodeSlots * kGCodeSlot + a_slots * kASlab + b_slots * n_pad * 128 +
+           (2 * kGCodeSlots + 1 + 16 + kMaxASlots) * 8 + 64;
 }
 
-// Rebuilds the 8 rows of octet o for subvector column w of a slab (Eq. 1-2),
-// rounded to fp16, into the A operand: core matrix (o % 16, w) of half o / 16.
-__device__ __forceinline__ void decode_to_a(const VDec& d, uint4 rec, const uint32_t (&aux)[8], uint32_t sh_aux,
-                                            const float (&mup)[8], const float (&dlp)[8], uint32_t cbsel,
-                                            uint32_t dst) {
-    const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
+// Rebuilds one subvector of one row (Eq. 1-2), rounded to fp16: w is the
+// record word holding the row, odd selects the row's half of it (rows 2u and
+// 2u + 1 share word u), s0..s2 are the row's sign-slot shifts, and the aux
+// signs come from the row's group word at bit `col`.
+__device__ __forceinline__ uint4 decode_sv(const VDec& d, uint32_t w, bool odd, uint32_t s0, uint32_t s1,
+                                           uint32_t s2, uint32_t aux, uint32_t sh_aux, float mp, float dl,
+                                           uint32_t cbsel) {
+    const uint32_t wf = odd ? rot16(w) : w;  // (z, q) field word of this row
+    uint4 c = lds128(cbsel + (wf & d.zmask));
+    c.x ^= (w << s0) & 0x80008000u;
+    c.y ^= (w << s1) & 0x80008000u;
+    c.z ^= (w << s2) & 0x80008000u;
+    c.w ^= (aux << sh_aux) & 0x80008000u;
+    const float r = fmaf(__uint_as_float((wf & d.qmask) | 0x3F800000u), dl, mp);
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int t = 2 * u + half;
-            const uint32_t wa = wv[u];
-            const uint32_t wf = half ? rot16(wa) : wa;  // (z, q) field word of this row
-            uint4 c = lds128(cbsel + (wf & d.zmask));
-            if (!half) {
-                c.x ^= (wa << d.sh0) & 0x80008000u;
-                c.y ^= (wa << d.sh1) & 0x80008000u;
-                c.z ^= (wa << d.sh2) & 0x80008000u;
-            } else {
-                c.x ^= (wa << d.sh3) & 0x80008000u;
-                c.y ^= (wa << d.sh4) & 0x80008000u;
-                c.z ^= wa & 0x80008000u;  // slot 5 sits at bit 15 for every split
-            }
-            c.w ^= (aux[t] << sh_aux) & 0x80008000u;
-            const float r = fmaf(__uint_as_float((wf & d.qmask) | 0x3F800000u), dlp[t], mup[t]);
-            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 cf = __half22float2(u2h2(cw[k]));
-                o[k] = h22u(__floats2half2_rn(r * cf.x, r * cf.y));
-            }
-            sts128(dst + t * 16, make_uint4(o[0], o[1], o[2], o[3]));
-        }
+    for (int k = 0; k < 4; ++k) {
+        const float2 cf = __half22float2(u2h2(cw[k]));
+        o[k] = h22u(__floats2half2_rn(r * cf.x, r * cf.y));
     }
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -229,7 +237,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
     const int n_oct = block_octets(R8, blk);
     const int g0 = part * G / p.parts, g1 = (part + 1) * G / p.parts;
     const int n_chunk = g1 - g0, n_slab = 2 * n_chunk;
-    const int K = 1 << p.log2K, NB = p.b_slots;
+    const int K = 1 << p.log2K, NB = p.b_slots, NA = p.a_slots;
 
     GemmSmem sm;
     {
@@ -237,10 +245,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
         sm.cb0 = smem_u32(q); q += K * 128;
         sm.cbraw = smem_u32(q); q += K * 16;
         sm.code0 = smem_u32(q); q += kGCodeSlots * kGCodeSlot;
-        sm.a0 = smem_u32(q); q += 2 * kASlab;
+        sm.a0 = smem_u32(q); q += NA * kASlab;
         sm.b_bytes = (uint32_t)p.n_pad * 128;
         sm.b0 = smem_u32(q); q += NB * sm.b_bytes;
-        sm.bars = reinterpret_cast<uint64_t*>(q); q += (2 * kGCodeSlots + 1 + 16) * 8;
+        sm.bars = reinterpret_cast<uint64_t*>(q); q += (2 * kGCodeSlots + 1 + 16 + kMaxASlots) * 8;
         sm.taddr_slot = reinterpret_cast<uint32_t*>(q); q += 16;
         sm.bcast = reinterpret_cast<int*>(q);
     }
@@ -254,6 +262,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
             mbar_init(sm.bars + 2 * kGCodeSlots + 1 + k, 1);      // b_full
             mbar_init(sm.bars + 2 * kGCodeSlots + 1 + 8 + k, 1);  // mma_done (tcgen05.commit)
         }
+        for (int k = 0; k < kMaxASlots; ++k) mbar_init(sm.a_full(k, kMaxASlots), kGW);  // one arrival per decode warp
         fence_mbar_init();
         s_gabort = 0;
     }
@@ -267,6 +276,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
     tc_fence_after();
     const uint32_t taddr = *sm.taddr_slot;
 
+    bool wait_last = false;
     if (warp == kGW) {
         // ---------------- copy warp ----------------
         if (lane == 0) {
@@ -290,111 +300,182 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
                 }
             }
         }
+    } else if (warp == kGW + 1) {
+        // ---------------- MMA warp: one thread issues the tensor-core work ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16(p.n_pad);
+            for (int s = 0; s < n_slab; ++s) {
+                gwait(sm.a_full(s, NA), (s / NA) & 1, p.status);
+                gwait(sm.b_full(s, NB), (s / NB) & 1, p.status);
+                tc_fence_after();
+                const uint32_t a_base = sm.a0 + (uint32_t)(s % NA) * kASlab;
+                const uint32_t b_base = sm.b0 + (uint32_t)(s % NB) * sm.b_bytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bd = smem_desc(b_base + kk * 256, 128, kBSbo);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf)
+                        mma_f16(taddr + (uint32_t)(hf * p.n_alloc), smem_desc(a_base + hf * kAHalf + kk * 256, 128, kASbo),
+                                bd, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(sm.mma_done(s, NB));
+            }
+        }
     } else {
-        // ---------------- decode warps (+ MMA issue by thread 0) ----------------
+        // ---------------- decode warps ----------------
         gwait(sm.cb_full(), 0, p.status);
         for (int e = tid; e < K * 8; e += kGDecodeThreads) sts128(sm.cb0 + e * 16, lds128(sm.cbraw + (e >> 3) * 16));
         named_barrier(1, kGDecodeThreads);
         const VDec d = vdec(p.log2K);
-        const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
-        const uint32_t idesc = idesc_f16(p.n_pad);
-        const bool active = lane < n_oct;
+        // Thread <-> one row of the block: rows 32 (warp % 8) + lane; warps 0-7
+        // and 8-15 take slab columns 0-3 and 4-7.  The 8 lanes of a quarter warp
+        // hold the 8 rows of one octet, so their 16-byte stores land in 8
+        // different bank groups and their codeword loads hit 8 different replicas.
+        const int r = 32 * (warp & 7) + lane, o = r >> 3, tr = r & 7;
+        const int cw = warp >> 3;
+        const bool odd = tr & 1;
+        const bool active = o < n_oct;
+        const uint32_t cbsel = sm.cb0 + ((uint32_t)tr << 4);
+        const uint32_t s0 = odd ? d.sh3 : d.sh0, s1 = odd ? d.sh4 : d.sh1, s2 = odd ? d.sh5 : d.sh2;
+        const uint32_t a_row = (uint32_t)(r >> 7) * kAHalf + (uint32_t)((r & 127) >> 3) * kASbo + (uint32_t)tr * 16;
         for (int t = 0; t < n_chunk; ++t) {
             gwait(sm.code_full(t), (t / kGCodeSlots) & 1, p.status);
             const uint32_t slot = sm.code0 + (uint32_t)(t % kGCodeSlots) * kGCodeSlot;
-            uint32_t aux[8];
-            float mup[8], dlp[8];
-            if (active) {
-                const uint32_t a = slot + kGChunkJ * kGOct * 16 + lane * 64;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint4 q = lds128(a + e * 16);
-                    aux[2 * e] = q.x;
-                    aux[2 * e + 1] = q.z;
-                    const float2 m0 = __half22float2(u2h2(q.y));
-                    const float2 m1 = __half22float2(u2h2(q.w));
-                    dlp[2 * e] = m0.y * d.vscale;
-                    mup[2 * e] = m0.x - dlp[2 * e];
-                    dlp[2 * e + 1] = m1.y * d.vscale;
-                    mup[2 * e + 1] = m1.x - dlp[2 * e + 1];
-                }
+            uint32_t aux = 0;
+            float mp = 0.f, dl = 0.f;
+            if (active) {  // this row's group entry: aux signs, mu, delta
+                const uint2 e = lds64(slot + kGChunkJ * kGOct * 16 + (uint32_t)(o * 8 + tr) * 8);
+                aux = e.x;
+                const float2 md = __half22float2(u2h2(e.y));
+                dl = md.y * d.vscale;
+                mp = md.x - dl;
             }
             for (int h = 0; h < 2; ++h) {
                 const int s = 2 * t + h;
-                // the A buffer of slab s was last read by the MMAs of slab s - 2
-                if (s >= 2) gwait(sm.mma_done(s - 2, NB), ((s - 2) / NB) & 1, p.status);
-                const int jl = h * kGSlabJ + warp;  // column of the chunk
-                const uint32_t dst = sm.a0 + (uint32_t)(s & 1) * kASlab + (uint32_t)(lane >> 4) * kAHalf +
-                                     (uint32_t)(lane & 15) * kASbo + (uint32_t)warp * 128;
-                if (active) {
-                    const uint4 rec = lds128(slot + (jl * n_oct + lane) * 16);
-                    decode_to_a(d, rec, aux, (uint32_t)(15 - jl), mup, dlp, cbsel, dst);
-                } else {
+                // the A buffer of slab s was last read by the MMAs of slab s - NA
+                if (s >= NA) gwait(sm.mma_done(s - NA, NB), ((s - NA) / NB) & 1, p.status);
+                const uint32_t a_slab = sm.a0 + (uint32_t)(s % NA) * kASlab + a_row;
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) sts128(dst + r * 16, make_uint4(0, 0, 0, 0));
+                for (int i = 0; i < 4; ++i) {
+                    const int wc = 4 * cw + i;          // slab column
+                    const int jl = h * kGSlabJ + wc;    // chunk column
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (active) {
+                        const uint32_t w = lds32(slot + (uint32_t)(jl * n_oct + o) * 16 + (uint32_t)(tr >> 1) * 4);
+                        v = decode_sv(d, w, odd, s0, s1, s2, aux, (uint32_t)(15 - jl), mp, dl, cbsel);
+                    }
+                    sts128(a_slab + (uint32_t)wc * 128, v);
                 }
                 fence_proxy_async_smem();  // the generic-proxy writes above are read by the tensor core
-                named_barrier(1, kGDecodeThreads);
-                if (tid == 0) {
-                    gwait(sm.b_full(s, NB), (s / NB) & 1, p.status);
-                    tc_fence_after();
-                    const uint32_t a_base = sm.a0 + (uint32_t)(s & 1) * kASlab;
-                    const uint32_t b_base = sm.b0 + (uint32_t)(s % NB) * sm.b_bytes;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = smem_desc(b_base + kk * 256, 128, kBSbo);
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf)
-                            mma_f16(taddr + (uint32_t)(hf * p.n_alloc), smem_desc(a_base + hf * kAHalf + kk * 256, 128, kASbo),
-                                    bd, idesc, (s > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(sm.mma_done(s, NB));
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sm.a_full(s, NA));
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.code_empty(t));
         }
         // ---------------- epilogue ----------------
+        wait_last = true;
+    }
+    if (warp < 8 && wait_last) {
         gwait(sm.mma_done(n_slab - 1, NB), ((n_slab - 1) / NB) & 1, p.status);
         tc_fence_after();
-        const int q4 = warp & 3, hf = warp >> 2;
-        const int row_local = hf * 128 + q4 * 32 + lane;
+    }
+    const int q4 = warp & 3, hf = (warp >> 2) & 1;
+    const int row_local = hf * 128 + q4 * 32 + lane;
+    const uint32_t tw = taddr + (uint32_t)(hf * p.n_alloc) + ((uint32_t)(q4 * 32) << 16);
+    if (p.parts == 1) {
         const int row = blk * 256 + row_local;
-        const uint32_t tw = taddr + (uint32_t)(hf * p.n_alloc) + ((uint32_t)(q4 * 32) << 16);
-        float* mypart = p.partials + (size_t)blockIdx.x * p.n_pad * 256;
-        for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
-            float v[16];
-            tmem_ld16(tw + (uint32_t)c0, v);
+        if (warp < 8) {
+            for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
+                float v[16];
+                tmem_ld16(tw + (uint32_t)c0, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int n = c0 + i;
-                if (n < p.M) {
-                    if (p.parts == 1) {
-                        if (row < p.d_out) p.y[(size_t)n * p.d_out + row] = __half_as_ushort(__float2half_rn(v[i]));
+                for (int i = 0; i < 16; ++i) {
+                    const int n = c0 + i;
+                    if (n < p.M && row < p.d_out) p.y[(size_t)n * p.d_out + row] = __half_as_ushort(__float2half_rn(v[i]));
+                }
+            }
+            tc_fence_before();
+        }
+    } else {
+        // The parts of a block form one thread-block cluster.  Round by round over
+        // the batch columns, every part stages its fp32 accumulator in its own
+        // (now idle) operand buffers; then part r adds the parts' values, in part
+        // order, for rows [256 r / parts, 256 (r + 1) / parts) through distributed
+        // shared memory and writes those rows of y.
+        const uint32_t red0 = sm.code0;
+        const int nc = p.red_cols;
+        // part r reduces the row quads [64 r / parts, 64 (r + 1) / parts)
+        const int qA = part * 64 / p.parts, qB = (part + 1) * 64 / p.parts, nq = qB - qA;
+        const bool vec_y = (p.d_out & 3) == 0;
+        for (int n0 = 0; n0 < p.M; n0 += nc) {
+            const int n1 = min(p.M, n0 + nc);
+            if (warp < 8) {
+                for (int c0 = n0 & ~15; c0 < n1; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tw + (uint32_t)c0, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int n = c0 + i;
+                        if (n >= n0 && n < n1) sts_f32(red0 + (uint32_t)((n - n0) * 256 + row_local) * 4, v[i]);
+                    }
+                }
+                tc_fence_before();
+            }
+            cluster_sync();
+            const int total = nq * (n1 - n0);
+            for (int e0 = tid; e0 < total; e0 += 2 * kGThreads) {
+                float4 acc[2];
+                uint32_t off[2];
+                bool ok[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int e = e0 + u * kGThreads;
+                    ok[u] = e < total;
+                    const int c = ok[u] ? e / nq : 0, q = qA + (ok[u] ? e - c * nq : 0);
+                    off[u] = red0 + (uint32_t)(c * 256 + q * 4) * 4;
+                    acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                for (int k0 = 0; k0 < p.parts; k0 += 4) {  // parts in order, four at a time in flight
+                    float4 t[2][4];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            t[u][k] = (ok[u] && k0 + k < p.parts) ? ld_cluster_v4(map_cluster(off[u], k0 + k))
+                                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            acc[u].x += t[u][k].x;
+                            acc[u].y += t[u][k].y;
+                            acc[u].z += t[u][k].z;
+                            acc[u].w += t[u][k].w;
+                        }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (!ok[u]) continue;
+                    const int e = e0 + u * kGThreads, c = e / nq, q = qA + (e - c * nq);
+                    const int row = blk * 256 + q * 4;
+                    uint16_t* yr = p.y + (size_t)(n0 + c) * p.d_out + row;
+                    const uint16_t h0 = __half_as_ushort(__float2half_rn(acc[u].x));
+                    const uint16_t h1 = __half_as_ushort(__float2half_rn(acc[u].y));
+                    const uint16_t h2 = __half_as_ushort(__float2half_rn(acc[u].z));
+                    const uint16_t h3 = __half_as_ushort(__float2half_rn(acc[u].w));
+                    if (vec_y && row + 3 < p.d_out) {
+                        *reinterpret_cast<uint2*>(yr) = make_uint2((uint32_t)h0 | ((uint32_t)h1 << 16),
+                                                                   (uint32_t)h2 | ((uint32_t)h3 << 16));
                     } else {
-                        mypart[(size_t)n * 256 + row_local] = v[i];
+                        if (row < p.d_out) yr[0] = h0;
+                        if (row + 1 < p.d_out) yr[1] = h1;
+                        if (row + 2 < p.d_out) yr[2] = h2;
+                        if (row + 3 < p.d_out) yr[3] = h3;
                     }
                 }
             }
-        }
-        tc_fence_before();
-        if (p.parts > 1) {
-            named_barrier(1, kGDecodeThreads);  // every partial store of the CTA precedes the release below
-            if (tid == 0) {
-                const unsigned old = atom_add_acq_rel_gpu(p.counters + blk, 1u);
-                const int last = old == (unsigned)(p.parts - 1);
-                if (last) *reinterpret_cast<volatile unsigned*>(p.counters + blk) = 0u;  // ready for the next call
-                *sm.bcast = last;
-            }
-            named_barrier(1, kGDecodeThreads);
-            if (*sm.bcast && row < p.d_out) {
-                const float* base = p.partials + (size_t)blk * p.parts * p.n_pad * 256 + row_local;
-                for (int n = 0; n < p.M; ++n) {
-                    float tot = 0.f;
-                    for (int k = 0; k < p.parts; ++k) tot += __ldcg(base + ((size_t)k * p.n_pad + n) * 256);
-                    p.y[(size_t)n * p.d_out + row] = __half_as_ushort(__float2half_rn(tot));
-                }
-            }
+            cluster_sync();  // the remote reads are done before the buffers are reused or the CTA exits
         }
     }
     __syncthreads();
@@ -423,10 +504,10 @@ int gemm_sm_count() {
 size_t round256g(size_t b) { return (b + 255) / 256 * 256; }
 
 // Launch plan and workspace layout of one sage_gemm call:
-//   status header | counters [n_blocks] | x_perm tiles | partial sums (split blocks only)
+//   status header | x_perm tiles
 struct GemmPlan {
-    int n_pad, n_alloc, parts, b_slots, n_blocks, smem;
-    size_t off_counters, off_xt, off_part, total;
+    int n_pad, n_alloc, parts, a_slots, b_slots, n_blocks, smem, red_cols;
+    size_t off_xt, total;
 };
 
 constexpr int kGemmSmemBudget = 226 * 1024;
@@ -439,18 +520,23 @@ GemmPlan gemm_plan(const sage_matrix* A, int M) {
     const int R8 = (A->d_out + 7) / 8;
     g.n_blocks = (R8 + kGOct - 1) / kGOct;
     const int G = A->d_in / 128;
-    g.parts = std::max(1, std::min(gemm_sm_count() / g.n_blocks, G / 2));
+    // parts of a block run as one cluster (at most 8: portable cluster size)
+    g.parts = std::max(1, std::min(std::min(8, gemm_sm_count() / g.n_blocks), G / 2));
     const int K = 1 << A->log2K;
-    g.b_slots = 2;
-    while (g.b_slots < 8 && gemm_smem_bytes(K, g.n_pad, g.b_slots + 1) <= kGemmSmemBudget) ++g.b_slots;
-    g.smem = gemm_smem_bytes(K, g.n_pad, g.b_slots);
+    // The decoded-slab ring as deep as fits, then the x_perm ring.  The x_perm
+    // ring is at least as deep: a slab's mma_done barrier is then never two
+    // phases ahead of a decode warp that waits on it.
+    g.a_slots = kMaxASlots;
+    while (g.a_slots > 2 && gemm_smem_bytes(K, g.n_pad, g.a_slots, g.a_slots) > kGemmSmemBudget) --g.a_slots;
+    g.b_slots = g.a_slots;
+    while (g.b_slots < 8 && gemm_smem_bytes(K, g.n_pad, g.a_slots, g.b_slots + 1) <= kGemmSmemBudget) ++g.b_slots;
+    g.smem = gemm_smem_bytes(K, g.n_pad, g.a_slots, g.b_slots);
+    // the cluster reduction stages 256 fp32 per batch column in the code ring and operand buffers
+    const int staging = kGCodeSlots * kGCodeSlot + g.a_slots * kASlab + g.b_slots * g.n_pad * 128;
+    g.red_cols = std::min(g.n_pad, staging / 1024 / 16 * 16);
     size_t o = kWsHeader;
-    g.off_counters = o;
-    o += round256g((size_t)g.n_blocks * 4);
     g.off_xt = o;
     o += round256g((size_t)(A->d_in / 64) * g.n_pad * 128);
-    g.off_part = o;
-    if (g.parts > 1) o += (size_t)g.n_blocks * g.parts * g.n_pad * 256 * sizeof(float);
     g.total = o;
     return g;
 }
@@ -487,8 +573,6 @@ int launch_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y, voi
     p.cb = A->codebook;
     p.xt = xt;
     p.y = y;
-    p.partials = reinterpret_cast<float*>(w + g.off_part);
-    p.counters = reinterpret_cast<unsigned*>(w + g.off_counters);
     p.status = reinterpret_cast<uint32_t*>(w);
     p.d_out = A->d_out;
     p.d_in = A->d_in;
@@ -497,9 +581,34 @@ int launch_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y, voi
     p.n_pad = g.n_pad;
     p.n_alloc = g.n_alloc;
     p.parts = g.parts;
+    p.red_cols = g.red_cols;
+    p.a_slots = g.a_slots;
     p.b_slots = g.b_slots;
-    gemm_kernel<<<(unsigned)(g.n_blocks * g.parts), kGThreads, (size_t)g.smem, s>>>(p);
-    return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(kGThreads);
+    cfg.dynamicSmemBytes = (size_t)g.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // The largest cluster (parts per block) for which every block's cluster is
+    // resident at once: a second wave would double the time.
+    int parts = g.parts;
+    for (; parts > 1; --parts) {
+        attr[0].val.clusterDim.x = (unsigned)parts;
+        cfg.gridDim = dim3((unsigned)(g.n_blocks * parts));
+        int active = 0;
+        if (cudaOccupancyMaxActiveClusters(&active, (const void*)gemm_kernel, &cfg) == cudaSuccess && active >= g.n_blocks)
+            break;
+    }
+    (void)cudaGetLastError();
+    p.parts = parts;
+    attr[0].val.clusterDim.x = (unsigned)parts;
+    cfg.gridDim = dim3((unsigned)(g.n_blocks * parts));
+    return cudaLaunchKernelEx(&cfg, gemm_kernel, p) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 }  // namespace sage

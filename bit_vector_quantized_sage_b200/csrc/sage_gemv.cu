@@ -181,21 +181,36 @@ struct DenseProblem {
     }
 };
 
+// The routing results this CTA needs (virtual-expert count, and the expert
+// and pair count of the virtual experts its range touches, with their
+// descriptors) are staged in shared memory once, after the routing kernel.
+constexpr int kMoeCache = 32;
+struct MoeStage {
+    long long total;
+    int vi0, nvi;
+    int v_expert[kMoeCache];
+    int v_count[kMoeCache];
+    ExpertMat emat[kMoeCache];
+};
+
 struct MoeProblem {
     const MoeParams& p;
+    const MoeStage& st;
     __device__ int R8() const { return (p.d_out + 7) >> 3; }
     __device__ long long upv() const { return (long long)((R8() + kOct - 1) / kOct) * (p.d_in >> 3); }
-    __device__ long long total() const { return (long long)__ldcg(&p.route->n_virtual) * upv(); }
-    __device__ long long cta_begin(int c) const { return (long long)c * total() / p.c.n_cta; }
+    __device__ long long total() const { return st.total; }
+    __device__ long long cta_begin(int c) const { return (long long)c * st.total / p.c.n_cta; }
     __device__ int cta_of(long long u) const {
-        const long long t = total();
+        const long long t = st.total;
         return (int)(((u + 1) * p.c.n_cta + t - 1) / t) - 1;
     }
     __device__ MatView view(long long u) const {
         const long long per = upv();
         const int vi = (int)(u / per);
-        const int e = __ldcg(p.v_expert + vi);
-        const ExpertMat& d = p.experts[e];
+        const int k = vi - st.vi0;
+        const bool cached = k >= 0 && k < st.nvi;
+        const int e = cached ? st.v_expert[k] : __ldcg(p.v_expert + vi);
+        const ExpertMat& d = cached ? st.emat[k] : p.experts[e];
         MatView v;
         v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = p.x; v.y = p.y;
         v.xrows = p.v_xrows + (size_t)vi * kMaxPairsPerVirtual;
@@ -203,7 +218,8 @@ struct MoeProblem {
         v.unit0 = (long long)vi * per;
         v.d_out = p.d_out; v.d_in = p.d_in; v.log2K = d.log2K;
         v.R8 = R8(); v.S = p.d_in >> 3;
-        v.blk0 = vi * ((v.R8 + kOct - 1) / kOct); v.Mk = __ldcg(p.v_count + vi);
+        v.blk0 = vi * ((v.R8 + kOct - 1) / kOct);
+        v.Mk = cached ? st.v_count[k] : __ldcg(p.v_count + vi);
         return v;
     }
 };
@@ -565,25 +581,6 @@ __device__ __forceinline__ void decode_record(const VDec& d, uint4 rec, const ui
     }
 }
 
-// Loads the grid / aux meta of this lane's octet (64 bytes at a) without bank
-// conflicts: lane pairs start at rotated 16-byte quarters, and the four
-// quarters are rotated back into place with selects.
-__device__ __forceinline__ void load_meta(uint32_t a, int lane, uint4 (&q)[4]) {
-    const int r = (lane >> 1) & 3;
-    uint4 v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = lds128(a + (uint32_t)((k + r) & 3) * 16);  // v[k] = quarter (k + r) & 3
-    uint4 u[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {  // quarter e sits in v[(e - r) & 3]: rotate right by r
-        const uint4 a1 = (r & 1) ? v[(e + 3) & 3] : v[e];
-        const uint4 a2 = (r & 1) ? v[(e + 1) & 3] : v[(e + 2) & 3];
-        u[e] = (r & 2) ? a2 : a1;
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) q[e] = u[e];
-}
-
 // Decodes this warp's columns of one ring chunk (chunk c of segment g, in
 // ring slot k with phase parity ph): columns lw, lw + wpg, ... of the chunk,
 // against the x_perm window at xw, where the chunk's first column sits at
@@ -885,7 +882,26 @@ __global__ void __launch_bounds__(Cfg<M>::kThreads, 1) gemv_kernel(const __grid_
 // Virtual experts carry 1..8 pairs; each segment dispatches on its own count.
 __global__ void __launch_bounds__(Cfg<kMaxPairsPerVirtual>::kThreads, 1) moe_kernel(const __grid_constant__ MoeParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    const MoeProblem P{p};
+    __shared__ MoeStage st;
+    pdl_wait();  // the routing comes from the preceding kernel
+    if (threadIdx.x == 0) {
+        const long long per = (long long)(((p.d_out + 7) / 8 + kOct - 1) / kOct) * (p.d_in >> 3);
+        st.total = (long long)__ldcg(&p.route->n_virtual) * per;
+        const long long u0 = (long long)blockIdx.x * st.total / p.c.n_cta;
+        const long long u1 = (long long)(blockIdx.x + 1) * st.total / p.c.n_cta;
+        st.vi0 = (int)(u0 / per);
+        st.nvi = u1 > u0 ? (int)min((long long)kMoeCache, (u1 - 1) / per - st.vi0 + 1) : 0;
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < st.nvi) {
+        const int vi = st.vi0 + threadIdx.x;
+        const int e = __ldcg(p.v_expert + vi);
+        st.v_expert[threadIdx.x] = e;
+        st.v_count[threadIdx.x] = __ldcg(p.v_count + vi);
+        st.emat[threadIdx.x] = p.experts[e];
+    }
+    __syncthreads();
+    const MoeProblem P{p, st};
     run<1, kMaxPairsPerVirtual>(P, p.c, smem_raw, true);
 }
 
@@ -1157,7 +1173,7 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
     int kmax = 16;
     for (int e = 0; e < n_experts; ++e) kmax = std::max(kmax, 1 << experts[e].log2K);
     p.c.kmax = kmax;
-    p.c.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget);
+    p.c.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget - (int)sizeof(MoeStage));
     p.c.n_wg = wg_for(p.c.slots);
     if (!ensure_smem(moe_kernel, Cfg<MV>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
     p.c.status = reinterpret_cast<uint32_t*>(w);
