@@ -394,7 +394,7 @@ struct RoleState {
 // preceding kernel: nothing it reads is written by that kernel).
 // ------------------------------------------------------------------------
 template <int M>
-__device__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+__device__ __forceinline__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
     const int lane = threadIdx.x & 31;
     for (int si = 0; si < n_seg; ++si, ++st.s) {
         const Seg& g = sm.segs[si];
@@ -485,7 +485,7 @@ constexpr int kBarPermIssued = 3;
 constexpr int kBarFirstWindow = 2;
 
 template <int M>
-__device__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
+__device__ __forceinline__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
     const int lane = threadIdx.x & 31;
     fence_proxy_async_smem();  // earlier reads of the permutation buffer precede the copies below
     int si = si0, c = c0, wlen = 0;
@@ -524,7 +524,7 @@ __device__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, 
 }
 
 template <int M>
-__device__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st, bool& waited) {
+__device__ __forceinline__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st, bool& waited) {
     win_break(st.w);
     int pend = -1, si0 = 0, c0 = 0, nch = 0;
     for (int si = 0; si < n_seg; ++si) {
@@ -719,7 +719,8 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
 // Decodes one segment with compile-time batch MK (<= MS, the launch's stash
 // stride) and leaves its 256 x MS results in stash slot `slot`.
 template <int MK, int MS>
-__device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st, int slot) {
+__device__ __forceinline__ void segment_body_impl(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st,
+                                                  int slot) {
     constexpr int W = Cfg<MS>::kW, DT = Cfg<MS>::kDecodeThreads;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const VDec d = vdec(g.v.log2K);
@@ -776,8 +777,16 @@ __device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, c
     named_barrier(1, DT);
 }
 
+// Out-of-line instance for launches whose segments have different batch
+// sizes (the MoE kernel dispatches on each segment's); a dense launch inlines
+// its single instance.
+template <int MK, int MS>
+__device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st, int slot) {
+    segment_body_impl<MK, MS>(sm, C, g, st, slot);
+}
+
 template <int MLO, int M>
-__device__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+__device__ __forceinline__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
     constexpr int DT = Cfg<M>::kDecodeThreads;
     const int tid = threadIdx.x;
     int npend = 0, i_pend = 0;
@@ -797,7 +806,7 @@ __device__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, Role
         }
         if (tid == 0) mbar_arrive(sm.cb_empty(s & 1));
         if constexpr (MLO == M) {
-            segment_body<M, M>(sm, C, g, st, npend);
+            segment_body_impl<M, M>(sm, C, g, st, npend);
         } else {
             switch (g.v.Mk) {
                 case 1: segment_body<1, M>(sm, C, g, st, npend); break;
