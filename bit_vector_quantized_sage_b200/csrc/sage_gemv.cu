@@ -459,15 +459,18 @@ __device__ __forceinline__ void gather_x(const Smem<M>& sm, int wlen, uint32_t x
                     const int xr_idx = g.v.xrows ? __ldcg(g.v.xrows + m) : m;
                     const unsigned short* xr =
                         reinterpret_cast<const unsigned short*>(g.v.x) + (size_t)xr_idx * g.v.d_in;
+                    // x is read-only while this kernel runs and is first read here,
+                    // after the wait on the kernel that wrote it: the scattered
+                    // 2-byte reads go through L1, which holds the whole row.
                     if (g.v.perm) {
                         const uint32_t sp = sm.perm0 + p * 32;
                         const uint4 pa = lds128(sp), pb = lds128(sp + 16);
-                        val[r].x = (uint32_t)__ldcg(xr + pa.x) | ((uint32_t)__ldcg(xr + pa.y) << 16);
-                        val[r].y = (uint32_t)__ldcg(xr + pa.z) | ((uint32_t)__ldcg(xr + pa.w) << 16);
-                        val[r].z = (uint32_t)__ldcg(xr + pb.x) | ((uint32_t)__ldcg(xr + pb.y) << 16);
-                        val[r].w = (uint32_t)__ldcg(xr + pb.z) | ((uint32_t)__ldcg(xr + pb.w) << 16);
+                        val[r].x = (uint32_t)__ldg(xr + pa.x) | ((uint32_t)__ldg(xr + pa.y) << 16);
+                        val[r].y = (uint32_t)__ldg(xr + pa.z) | ((uint32_t)__ldg(xr + pa.w) << 16);
+                        val[r].z = (uint32_t)__ldg(xr + pb.x) | ((uint32_t)__ldg(xr + pb.y) << 16);
+                        val[r].w = (uint32_t)__ldg(xr + pb.z) | ((uint32_t)__ldg(xr + pb.w) << 16);
                     } else {
-                        val[r] = __ldcg(reinterpret_cast<const uint4*>(xr + j * 8));
+                        val[r] = __ldg(reinterpret_cast<const uint4*>(xr + j * 8));
                     }
                     dst[r] = xb + (m * XW + p) * 16;
                 }
