@@ -65,7 +65,8 @@ struct Cfg {
     static constexpr int kXBuf = kXW * M * 16;         // one window of x_perm, [m][column]
     static constexpr int kPermBuf = kXW * 32;          // the window's permutation entries
     static constexpr int kPosInfo = kXW * 4;           // (segment, column) of each window position
-    static constexpr int kRed = kW * 8 * M * 32 * 4;
+    // cross-warp reduction buffer: only the MoE kernel's segment body (batch 8) uses one
+    static constexpr int kRed = (M == kMaxPairsPerVirtual) ? kW * 8 * M * 32 * 4 : 0;
     static constexpr int kStash = kMaxSegs * M * kBlockRows * 4;
     static constexpr int kBars = (2 * kMaxSlots + 9) * 8;
     static constexpr int kFixed = 2 * kXBuf + kPermBuf + kPosInfo + kRed + kStash + kSegTab * kSegBytes + kBars + 64;
@@ -637,6 +638,55 @@ __device__ __forceinline__ void decode_chunk(const Smem<MS>& sm, const Common& C
     if (lane == 0) mbar_arrive(sm.empty(k));
 }
 
+// Decodes one ring chunk (chunk c of segment g, ring slot k, phase parity ph)
+// with one thread per row of the 256-row block: row 32 warp + lane, i.e. the
+// 8 lanes of a quarter warp hold the 8 rows of one octet.  Per row the grid
+// and aux signs are one 8-byte entry; per (row, column) the fields are the
+// row's half of one record word, and the codeword comes from the replica of
+// the row's position in its octet (no bank conflicts).  acc[m] accumulates the
+// row's output for batch row m.
+template <int M, int MS>
+__device__ __forceinline__ void decode_rows(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int k,
+                                            int ph, int c, uint32_t xw, int pos, int warp, int lane, float (&acc)[M]) {
+    constexpr int XW = Cfg<MS>::kXW;
+    const int2 cc = chunk_cols(g, c);
+    const int nj = cc.y - cc.x;
+    wait_bar(sm.full(k), ph, C);
+    const int n_oct = g.n_oct;
+    const int o = (warp << 2) + (lane >> 3), tr = lane & 7;
+    if (o < n_oct) {
+        const uint32_t base = sm.slot_addr(k);
+        const uint2 e = lds64(base + kMainSlot + (uint32_t)(o * 8 + tr) * 8);
+        const float2 md = __half22float2(u2h2(e.y));
+        const float dl = md.y * d.vscale, mp = md.x - dl;
+        const uint32_t aux = e.x;
+        const bool odd = tr & 1;
+        const uint32_t s0 = odd ? d.sh3 : d.sh0, s1 = odd ? d.sh4 : d.sh1, s2 = odd ? d.sh5 : d.sh2;
+        const uint32_t cbsel = sm.cb0 + ((uint32_t)tr << 4);
+        const uint32_t wbase = base + (uint32_t)o * 16 + (uint32_t)(tr >> 1) * 4;
+        const uint32_t rstride = (uint32_t)n_oct * 16;
+        const uint32_t xbase = xw + (uint32_t)pos * 16;
+#pragma unroll 4
+        for (int i = 0; i < nj; ++i) {
+            const uint32_t w = lds32(wbase + (uint32_t)i * rstride);
+            const uint32_t wf = odd ? rot16(w) : w;  // (z, q) field word of this row
+            uint4 cw = lds128(cbsel + (wf & d.zmask));
+            cw.x ^= (w << s0) & 0x80008000u;
+            cw.y ^= (w << s1) & 0x80008000u;
+            cw.z ^= (w << s2) & 0x80008000u;
+            cw.w ^= (aux << (uint32_t)(15 - ((cc.x + i) & 15))) & 0x80008000u;
+            const float r = fmaf(__uint_as_float((wf & d.qmask) | 0x3F800000u), dl, mp);
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const uint4 xv = lds128(xbase + (uint32_t)(m * XW + i) * 16);
+                acc[m] = fmaf(r, signed_dot(cw, xv), acc[m]);
+            }
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.empty(k));
+}
+
 // Writes (or combines) the outputs of the pending segments tab[i0 .. i0 + n).
 // Split blocks: every contributor stores its partial sums, the CTA's writes are
 // published with one release atomic per block, and the contributor that sees
@@ -724,6 +774,59 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
 template <int MK, int MS>
 __device__ __forceinline__ void segment_body_impl(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st,
                                                   int slot) {
+    constexpr int DT = Cfg<MS>::kDecodeThreads;
+    static_assert(Cfg<MS>::kW * 32 == kBlockRows, "one decode thread per block row");
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const VDec d = vdec(g.v.log2K);
+    float acc[MK];
+#pragma unroll
+    for (int m = 0; m < MK; ++m) acc[m] = 0.f;
+    int t = st.t, k = st.slot, ph = st.ph, cur = st.cur_win;
+    WinPos w = st.w;
+    for (int c = 0; c < g.n_chunks; ++c, ++t, ring_next(k, ph, sm.slots)) {
+        const int2 cc = chunk_cols(g, c);
+        const int pos = win_place(w, cc.y - cc.x, Cfg<MS>::kXW);
+        if (w.win != cur) {  // release the previous x window, wait for this one
+            if (cur >= 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sm.x_empty(cur & 1));
+            }
+            if (w.win == 0) {  // the first window is gathered together with the activation warp
+                pdl_wait();
+                named_barrier(kBarFirstWindow, 32 + DT);
+                gather_x<MS, 2>(sm, *sm.wlen0, sm.xwin(0), tid, 32 + DT);
+                named_barrier(kBarFirstWindow, 32 + DT);
+            } else {
+                wait_bar(sm.x_full(w.win & 1), (w.win >> 1) & 1, C);
+            }
+            cur = w.win;
+        }
+        decode_rows<MK, MS>(sm, C, g, d, k, ph, c, sm.xwin(w.win), pos, warp, lane, acc);
+    }
+    st.t = t;
+    st.slot = k;
+    st.ph = ph;
+    st.cur_win = cur;
+    st.w = w;
+    // each thread owns one row: its sums go straight to the stash
+    const int row = 32 * warp + lane;
+#pragma unroll
+    for (int m = 0; m < MS; ++m) {
+        float v = 0.f;
+#pragma unroll
+        for (int mm = 0; mm < MK; ++mm)
+            if (mm == m) v = acc[mm];
+        sm.stash[((size_t)slot * MS + m) * kBlockRows + row] = v;
+    }
+    named_barrier(1, DT);
+}
+
+// The MoE kernel's segment body: lane <-> row octet, warps split each chunk's
+// columns within warp groups, and the warps' partial sums are reduced through
+// shared memory.  (Dense launches use segment_body_impl: one thread per row.)
+template <int MK, int MS>
+__device__ __forceinline__ void segment_body_octets(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st,
+                                                  int slot) {
     constexpr int W = Cfg<MS>::kW, DT = Cfg<MS>::kDecodeThreads;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const VDec d = vdec(g.v.log2K);
@@ -781,11 +884,10 @@ __device__ __forceinline__ void segment_body_impl(const Smem<MS>& sm, const Comm
 }
 
 // Out-of-line instance for launches whose segments have different batch
-// sizes (the MoE kernel dispatches on each segment's); a dense launch inlines
-// its single instance.
+// sizes (the MoE kernel dispatches on each segment's).
 template <int MK, int MS>
 __device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st, int slot) {
-    segment_body_impl<MK, MS>(sm, C, g, st, slot);
+    segment_body_octets<MK, MS>(sm, C, g, st, slot);
 }
 
 template <int MLO, int M>
@@ -1103,7 +1205,7 @@ int launch_m(const GemvJob* jobs, int n, void* ws, sage_stream_t stream) {
     }
     p.c.M = M;
     p.c.slots = slots_for<M>(widest, kmax, kSmemBudget - kDenseStatic);
-    p.c.n_wg = wg_for(p.c.slots);
+    p.c.n_wg = 1;  // dense launches: every decode warp works on every chunk (one thread per block row)
     p.c.kmax = kmax;
     if (!ensure_smem(gemv_kernel<M>, Cfg<M>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
