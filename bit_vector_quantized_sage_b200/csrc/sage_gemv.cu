@@ -9,16 +9,22 @@
 //    range per CTA of a persistent grid (one CTA per SM).  Dense launches are
 //    planned on the host (each matrix gets its own CTAs when that costs little
 //    balance); MoE launches are planned on the device from the routing.
-//  * Two producer warps per CTA.  The copy warp issues, at kernel start and
-//    before waiting on the preceding kernel (programmatic dependent launch),
-//    1-D bulk (TMA) copies of everything static the CTA needs: code records,
-//    grid/aux meta, the permutation slice and the raw codebook.  The activation
-//    warp waits for the preceding kernel, then gathers the ESG-permuted
-//    x_perm[p] = x[perm[p]] (Sec. 3.5 fuses this gather into the decode GEMV).
-//  * Decode warps: lane l owns row octet l of the 256-row block, so every
-//    16-byte record holds 8 of its rows; the warps split the columns.
+//  * Two producer warps per CTA.  The copy warp bulk-copies (1-D TMA) the
+//    codebooks and, chunk by chunk (16 columns = one radius group), the code
+//    records and grid/aux meta into a ring of shared-memory slots, without
+//    waiting on the preceding kernel (programmatic dependent launch): none of
+//    it is written there.  The activation warp gathers the ESG-permuted
+//    x_perm[p] = x[perm[p]] window by window (Sec. 3.5 fuses this gather into
+//    the decode GEMV); the permutation entries are copied before the wait on
+//    the preceding kernel, only x after it.
+//  * Decode warps (dense launches): one thread per row of the 256-row block
+//    for the whole segment; it reads its row's half of a record word per
+//    column and accumulates the row's outputs itself.  The MoE kernel keeps
+//    an octet-per-lane body: lane l decodes the 16-byte record of row octet l
+//    (8 rows) per column, and the warps' partial sums are reduced in shared
+//    memory.
 //  * Per subvector: the codeword address and the radius code each come out of
-//    one logic op (layout v1), the codeword is one conflict-free 128-bit shared
+//    one logic op (format v2), the codeword is one conflict-free 128-bit shared
 //    load (8 bank-rotated replicas of the codebook), the signs are XORed into
 //    the fp16 sign bits, four half2 FMAs form (s (.) c) . x with fp16 local
 //    accumulation (Fig. 6a), and r = mu + q delta (Eq. 2) is applied once, fp32.
@@ -666,7 +672,7 @@ __device__ __forceinline__ void decode_rows(const Smem<MS>& sm, const Common& C,
         const uint32_t wbase = base + (uint32_t)o * 16 + (uint32_t)(tr >> 1) * 4;
         const uint32_t rstride = (uint32_t)n_oct * 16;
         const uint32_t xbase = xw + (uint32_t)pos * 16;
-#pragma unroll 4
+#pragma unroll 8
         for (int i = 0; i < nj; ++i) {
             const uint32_t w = lds32(wbase + (uint32_t)i * rstride);
             const uint32_t wf = odd ? rot16(w) : w;  // (z, q) field word of this row
