@@ -197,7 +197,8 @@ def cpu_oracle_sample(rows_per_matrix: int = 256, seconds_cap: float = 60.0):
         tot_bytes += mb + tb + (1 << f.log2K) * 16 + f.d_in * 2 + R * 2
         if tot_s > seconds_cap:
             break
-    desc = f"first {rows_per_matrix} rows of each of the 7 layer matrices (unpack + reconstruct + fp64 matvec)"
+    desc = (f"first {rows_per_matrix} rows of each of the 7 layer matrices" if rows_per_matrix < 9728
+            else "the whole layer, all 7 matrices") + " (unpack + reconstruct + fp64 matvec, single thread)"
     return tot_bytes / tot_s / 1e9, desc, 1, tot_s
 
 
@@ -313,7 +314,7 @@ def run_reference(args):
         cpu_oracle_sample(rows_per_matrix=32)
     vals, secs = [], 0.0
     for _ in range(args.steps):
-        v, desc, cores, s = cpu_oracle_sample(rows_per_matrix=64)
+        v, desc, cores, s = cpu_oracle_sample(rows_per_matrix=256)
         vals.append(v)
         secs += s
     value = statistics.median(vals)
@@ -513,7 +514,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
-    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--cpu-rows", type=int, default=1 << 30,
+                    help="rows per matrix in the CPU-oracle baseline sample (default: the whole layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the batch sweep and MoE measurements")
     args = ap.parse_args()
