@@ -46,6 +46,22 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's time is its slowest rank's: all-reduce MAX of a per-rank time
+    (no-op on one process)."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank runs its own replica of the step."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -420,14 +436,10 @@ def run_gpu(args):
     if dist is not None:
         dist.barrier()
     clk = clocks.stop()
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dist, "cuda")
     assert sage.sage_query_status(ws) == sage.SAGE_OK
     us_per_layer = ms * 1e3 / args.steps
-    value = world * one_layer_bytes * args.steps / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, one_layer_bytes, args.steps, ms)
     del g_all
 
     # ---- end to end through the public API with host buffers (graph per step) ----
@@ -456,8 +468,8 @@ def run_gpu(args):
             stream.synchronize()          # the host reads the step's result
         e_end.record(stream)
         torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / e2e_steps
-    e2e_value = world * one_layer_bytes / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / e2e_steps, dist, "cuda")
+    e2e_value = whole_job_gbs(world, one_layer_bytes, 1, e2e_ms)
     del g_e2e
 
     extra = {}
