@@ -60,6 +60,10 @@ constexpr int kSlot = kMainSlot + kMetaSlot;    // one ring slot = one chunk
 constexpr int kMaxSlots = 16;                   // ring depth limit
 constexpr int kSegTab = 32;                     // segment-table capacity per round
 constexpr int kSegBytes = 160;                  // shared memory per table entry
+// Named barriers besides the decode warps' own (id 1): the activation and
+// copy warps (id 3) and the activation and decode warps (id 2).
+constexpr int kBarPermIssued = 3;
+constexpr int kBarFirstWindow = 2;
 
 template <int M>
 struct Cfg {
@@ -259,15 +263,22 @@ __device__ Seg make_seg(const Problem& P, long long u, long long u_end, long lon
     s.full = (s.ja == 0 && s.jb == s.v.S);
     s.counter = nullptr;
     s.c_first = s.c_last = s.first_slot = s.my_slot = 0;
-    if (!s.full) {
-        const long long b0 = s.v.unit0 + (long long)s.blk * s.v.S;
-        s.c_first = P.cta_of(b0);
-        s.c_last = P.cta_of(b0 + s.v.S - 1);
-        s.first_slot = (P.cta_begin(s.c_first) >= b0) ? 0 : 1;
-        s.my_slot = (cta_u0 >= b0) ? 0 : 1;
-        s.counter = nullptr;
-    }
+    (void)cta_u0;
     return s;
+}
+
+// Split-K bookkeeping of a segment whose block is shared with other CTAs:
+// the contributing CTAs, the partial-sum slots and the arrival counter.  Run
+// by one lane per segment, in parallel, after the segments are laid out.
+template <class Problem>
+__device__ void seg_split_info(const Problem& P, const Common& C, Seg& s, long long cta_u0) {
+    if (s.full) return;
+    const long long b0 = s.v.unit0 + (long long)s.blk * s.v.S;
+    s.c_first = P.cta_of(b0);
+    s.c_last = P.cta_of(b0 + s.v.S - 1);
+    s.first_slot = (P.cta_begin(s.c_first) >= b0) ? 0 : 1;
+    s.my_slot = (cta_u0 >= b0) ? 0 : 1;
+    s.counter = C.counters + s.v.blk0 + s.blk;
 }
 
 // Fills tab[0..n) with the segments of [u, u_end) (at most kSegTab); returns n
@@ -277,9 +288,8 @@ __device__ int build_segs(const Problem& P, const Common& C, long long u, long l
                           Seg* tab, long long* u_next) {
     int n = 0;
     while (u < u_end && n < kSegTab) {
-        Seg s = make_seg(P, u, u_end, cta_u0);
-        if (!s.full) s.counter = C.counters + s.v.blk0 + s.blk;
-        tab[n++] = s;
+        tab[n++] = make_seg(P, u, u_end, cta_u0);
+        const Seg& s = tab[n - 1];
         u += s.jb - s.ja;
     }
     *u_next = u;
@@ -401,7 +411,8 @@ struct RoleState {
 // preceding kernel: nothing it reads is written by that kernel).
 // ------------------------------------------------------------------------
 template <int M>
-__device__ __forceinline__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
+__device__ __forceinline__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st,
+                                          bool first_round) {
     const int lane = threadIdx.x & 31;
     for (int si = 0; si < n_seg; ++si, ++st.s) {
         const Seg& g = sm.segs[si];
@@ -412,6 +423,9 @@ __device__ __forceinline__ void copy_warp(const Common& C, const Smem<M>& sm, in
             mbar_arrive_expect_tx(sm.cb_full(s & 1), cbb);
             bulk_g2s(sm.cbraw0 + (s & 1) * sm.cbraw_bytes, g.v.cb, cbb, sm.cb_full(s & 1));
         }
+        // the first codebook goes first; then the first window's permutation
+        // entries (activation warp) ahead of the code chunks
+        if (first_round && si == 0) named_barrier(kBarPermIssued, 64);
         const int n_oct = g.n_oct, R8 = g.v.R8, S = g.v.S, G = g.v.d_in >> 7, blk = g.blk;
         for (int c = 0; c < g.n_chunks; ++c, ++st.t, ring_next(st.slot, st.ph, sm.slots)) {
             const int k = st.slot;
@@ -489,10 +503,6 @@ __device__ __forceinline__ void gather_x(const Smem<M>& sm, int wlen, uint32_t x
     }
 }
 
-// Named barriers besides the decode warps' own (id 1): the activation and
-// copy warps (id 3) and the activation and decode warps (id 2).
-constexpr int kBarPermIssued = 3;
-constexpr int kBarFirstWindow = 2;
 
 template <int M>
 __device__ __forceinline__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
@@ -969,12 +979,15 @@ __device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* 
     RoleState st{0, 0, 0, 0, {0, 0}, -1};
     bool waited = plan_needs_wait;
     for (long long u = u0; u < u1;) {
-        if (tid == 0) s_nseg = build_segs(P, C, u, u1, u0, sm.segs, &s_next);
+        if (warp == 0) {  // lane 0 lays the segments out, then one lane per segment adds the split-K data
+            if ((tid & 31) == 0) s_nseg = build_segs(P, C, u, u1, u0, sm.segs, &s_next);
+            __syncwarp();
+            for (int i = tid & 31; i < s_nseg; i += 32) seg_split_info(P, C, sm.segs[i], u0);
+        }
         __syncthreads();
         const int n_seg = s_nseg;
         if (warp == W) {
-            if (u == u0) named_barrier(kBarPermIssued, 64);  // after the first window's permutation copies
-            copy_warp<M>(C, sm, n_seg, st);
+            copy_warp<M>(C, sm, n_seg, st, u == u0);
         } else if (warp == W + 1) {
             act_warp<M>(C, sm, n_seg, st, waited);
         } else {
