@@ -436,9 +436,10 @@ __device__ __forceinline__ void copy_warp(const Common& C, const Smem<M>& sm, in
                 const uint32_t mb = (uint32_t)(nj * n_oct * 16), tb = (uint32_t)(n_oct * 64);
                 mbar_arrive_expect_tx(sm.full(k), mb + tb);
                 // the chunk's records: one contiguous range of the block; its group's meta entries
-                bulk_g2s(sm.slot_addr(k), g.v.main + main_word(R8, S, blk, cc.x, 0, 0), mb, sm.full(k));
-                bulk_g2s(sm.slot_addr(k) + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0), tb,
-                         sm.full(k));
+                const uint64_t pol = l2_evict_first();
+                bulk_g2s_stream(sm.slot_addr(k), g.v.main + main_word(R8, S, blk, cc.x, 0, 0), mb, sm.full(k), pol);
+                bulk_g2s_stream(sm.slot_addr(k) + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0),
+                                tb, sm.full(k), pol);
             }
         }
     }
