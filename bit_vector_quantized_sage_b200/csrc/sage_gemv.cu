@@ -683,21 +683,28 @@ __device__ __forceinline__ void decode_rows(const Smem<MS>& sm, const Common& C,
         const uint32_t wbase = base + (uint32_t)o * 16 + (uint32_t)(tr >> 1) * 4;
         const uint32_t rstride = (uint32_t)n_oct * 16;
         const uint32_t xbase = xw + (uint32_t)pos * 16;
-#pragma unroll 8
-        for (int i = 0; i < nj; ++i) {
+        // column i of the chunk; its sign bit 7 is aux bit (cc.x + i) % 16
+        auto column = [&](int i, uint32_t aux_shift) {
             const uint32_t w = lds32(wbase + (uint32_t)i * rstride);
             const uint32_t wf = odd ? rot16(w) : w;  // (z, q) field word of this row
             uint4 cw = lds128(cbsel + (wf & d.zmask));
             cw.x ^= (w << s0) & 0x80008000u;
             cw.y ^= (w << s1) & 0x80008000u;
             cw.z ^= (w << s2) & 0x80008000u;
-            cw.w ^= (aux << (uint32_t)(15 - ((cc.x + i) & 15))) & 0x80008000u;
+            cw.w ^= (aux << aux_shift) & 0x80008000u;
             const float r = fmaf(__uint_as_float((wf & d.qmask) | 0x3F800000u), dl, mp);
 #pragma unroll
             for (int m = 0; m < M; ++m) {
                 const uint4 xv = lds128(xbase + (uint32_t)(m * XW + i) * 16);
                 acc[m] = fmaf(r, signed_dot(cw, xv), acc[m]);
             }
+        };
+        if (nj == kChunkJ) {  // a whole radius group (cc.x % 16 == 0): fixed trip count, constant shifts
+#pragma unroll 8
+            for (int i = 0; i < kChunkJ; ++i) column(i, (uint32_t)(15 - i));
+        } else {
+#pragma unroll 4
+            for (int i = 0; i < nj; ++i) column(i, (uint32_t)(15 - ((cc.x + i) & 15)));
         }
     }
     __syncwarp();
