@@ -92,8 +92,8 @@ struct MatView {
     const int32_t* perm;
     const uint16_t* x;      // activations, row stride d_in
     uint16_t* y;            // outputs, row stride d_out
-    const int32_t* xrows;   // [Mk] activation row of batch slot m (null: m)
-    const int32_t* yrows;   // [Mk] output row of batch slot m (null: m)
+    const int32_t* xrows;   // [Mk] activation row of batch slot m (null: m); shared or global memory
+    const int32_t* yrows;   // [Mk] output row of batch slot m (null: m); shared or global memory
     long long unit0;
     int d_out, d_in, log2K, R8, S, blk0, Mk;
 };
@@ -201,6 +201,8 @@ struct MoeStage {
     int vi0, nvi;
     int v_expert[kMoeCache];
     int v_count[kMoeCache];
+    int v_xrows[kMoeCache][kMaxPairsPerVirtual];  // activation / output rows of the cached virtual experts
+    int v_yrows[kMoeCache][kMaxPairsPerVirtual];
     ExpertMat emat[kMoeCache];
 };
 
@@ -224,8 +226,8 @@ struct MoeProblem {
         const ExpertMat& d = cached ? st.emat[k] : p.experts[e];
         MatView v;
         v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = p.x; v.y = p.y;
-        v.xrows = p.v_xrows + (size_t)vi * kMaxPairsPerVirtual;
-        v.yrows = p.v_yrows + (size_t)vi * kMaxPairsPerVirtual;
+        v.xrows = cached ? st.v_xrows[k] : p.v_xrows + (size_t)vi * kMaxPairsPerVirtual;
+        v.yrows = cached ? st.v_yrows[k] : p.v_yrows + (size_t)vi * kMaxPairsPerVirtual;
         v.unit0 = (long long)vi * per;
         v.d_out = p.d_out; v.d_in = p.d_in; v.log2K = d.log2K;
         v.R8 = R8(); v.S = p.d_in >> 3;
@@ -234,6 +236,12 @@ struct MoeProblem {
         return v;
     }
 };
+
+// Batch-slot row of a virtual expert: from the CTA's staged copy in shared
+// memory, or (experts outside the staged range) from the workspace in L2.
+__device__ __forceinline__ int row_at(const int32_t* rows, int m) {
+    return __isShared(rows) ? rows[m] : __ldcg(rows + m);
+}
 
 // A segment: one matrix, one 256-row block, columns [ja, jb), plus what the
 // split-K combine needs.  Each CTA builds its segment table once, in shared
@@ -478,7 +486,7 @@ __device__ __forceinline__ void gather_x(const Smem<M>& sm, int wlen, uint32_t x
                 const Seg& g = sm.segs[info >> 24];
                 const int j = (int)(info & 0xffffffu);
                 if (m < g.v.Mk) {
-                    const int xr_idx = g.v.xrows ? __ldcg(g.v.xrows + m) : m;
+                    const int xr_idx = g.v.xrows ? row_at(g.v.xrows, m) : m;
                     const unsigned short* xr =
                         reinterpret_cast<const unsigned short*>(g.v.x) + (size_t)xr_idx * g.v.d_in;
                     // x is read-only while this kernel runs and is first read here,
@@ -732,7 +740,7 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
 #pragma unroll
                 for (int m = 0; m < M; ++m)
                     if (m < g.v.Mk) {
-                        const int yr = g.v.yrows ? __ldcg(g.v.yrows + m) : m;
+                        const int yr = g.v.yrows ? row_at(g.v.yrows, m) : m;
                         g.v.y[(size_t)yr * g.v.d_out + row] = __half_as_ushort(__float2half_rn(st[m * kBlockRows + row_local]));
                     }
             }
@@ -741,7 +749,8 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
             float* part = C.partials + ((size_t)(cta * 2 + g.my_slot) * 8) * kBlockRows;
             if (tid < kBlockRows)
 #pragma unroll
-                for (int m = 0; m < M; ++m) part[m * kBlockRows + row_local] = st[m * kBlockRows + row_local];
+                for (int m = 0; m < M; ++m)
+                    if (m < g.v.Mk) part[m * kBlockRows + row_local] = st[m * kBlockRows + row_local];
         }
     }
     if (!any_partial) return;  // uniform across the decode threads
@@ -762,7 +771,7 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
         if (!sm.bcast[i]) continue;
         const int row = g.blk * kBlockRows + row_local;
         if (tid < kBlockRows && row < g.v.d_out) {
-            const int c_first = g.c_first, c_last = g.c_last, first_slot = g.first_slot;
+            const int c_first = g.c_first, c_last = g.c_last, first_slot = g.first_slot, mk = g.v.Mk;
             float tot[M];
 #pragma unroll
             for (int m = 0; m < M; ++m) tot[m] = 0.f;
@@ -775,7 +784,7 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
                     const int sp = (c == c_first) ? first_slot : 0;
                     const float* src = C.partials + ((size_t)(c * 2 + sp) * 8) * kBlockRows + row_local;
 #pragma unroll
-                    for (int m = 0; m < M; ++m) v[k][m] = (c <= c_last) ? __ldcg(src + m * kBlockRows) : 0.f;
+                    for (int m = 0; m < M; ++m) v[k][m] = (c <= c_last && m < mk) ? __ldcg(src + m * kBlockRows) : 0.f;
                 }
 #pragma unroll
                 for (int k = 0; k < NF; ++k)
@@ -785,7 +794,7 @@ __device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
 #pragma unroll
             for (int m = 0; m < M; ++m)
                 if (m < g.v.Mk) {
-                    const int yr = g.v.yrows ? __ldcg(g.v.yrows + m) : m;
+                    const int yr = g.v.yrows ? row_at(g.v.yrows, m) : m;
                     g.v.y[(size_t)yr * g.v.d_out + row] = __half_as_ushort(__float2half_rn(tot[m]));
                 }
         }
@@ -1040,6 +1049,11 @@ __global__ void __launch_bounds__(Cfg<kMaxPairsPerVirtual>::kThreads, 1) moe_ker
         st.v_expert[threadIdx.x] = e;
         st.v_count[threadIdx.x] = __ldcg(p.v_count + vi);
         st.emat[threadIdx.x] = p.experts[e];
+    }
+    for (int i = threadIdx.x; i < st.nvi * kMaxPairsPerVirtual; i += blockDim.x) {
+        const size_t src = (size_t)st.vi0 * kMaxPairsPerVirtual + i;
+        st.v_xrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_xrows + src);
+        st.v_yrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_yrows + src);
     }
     __syncthreads();
     const MoeProblem P{p, st};
