@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -125,8 +126,10 @@ class Clocks:
 
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/sage_clocks_{os.getpid()}.csv"
+        # SAGE_CLOCKS_DIR keeps the raw samples (one CSV per rank); default: a temp file
+        d = os.environ.get("SAGE_CLOCKS_DIR")
+        self.path = (os.path.join(d, f"clocks_rank{gpu_index}.csv") if d and os.path.isdir(d)
+                     else os.path.join(tempfile.gettempdir(), f"sage_clocks_{os.getpid()}_{gpu_index}.csv"))
         self.gpu = gpu_index
 
     def start(self):
