@@ -708,8 +708,13 @@ __device__ __forceinline__ void decode_rows(const Smem<MS>& sm, const Common& C,
             }
         };
         if (nj == kChunkJ) {  // a whole radius group (cc.x % 16 == 0): fixed trip count, constant shifts
+            if constexpr (M == 1) {  // the whole chunk in one schedule (no spills at batch 1)
+#pragma unroll
+                for (int i = 0; i < kChunkJ; ++i) column(i, (uint32_t)(15 - i));
+            } else {
 #pragma unroll 8
-            for (int i = 0; i < kChunkJ; ++i) column(i, (uint32_t)(15 - i));
+                for (int i = 0; i < kChunkJ; ++i) column(i, (uint32_t)(15 - i));
+            }
         } else {
 #pragma unroll 4
             for (int i = 0; i < nj; ++i) column(i, (uint32_t)(15 - ((cc.x + i) & 15)));
