@@ -430,3 +430,63 @@ def test_kmeans_deterministic_and_optimal_assignment():
             s = int(sum(1 << i for i in range(8) if Wp[o, 8 * j + i] < 0))
             assert a["signs"][o, j] == s
     assert a["q"].max() <= 2 ** 6 - 1
+
+
+def _kmeans_case(seed=21, n=600, K=6):
+    """Nonnegative subvector magnitudes with unequal per-channel weights."""
+    g = np.random.default_rng(seed)
+    P = np.abs(g.standard_normal((n, 8))) * g.uniform(0.2, 3.0, (n, 1))
+    Wt = g.uniform(0.25, 4.0, (n, 8))
+    init = g.choice(n, K, replace=False).astype(np.int64)
+    return P, Wt, K, init
+
+
+def test_kmeans_invariant_to_power_of_two_scaling():
+    """Eq. 6 picks a direction, not a length: scaling every subvector, or every
+    weight, by a power of two changes no assignment and no normalised
+    centroid, so the codebook is bit-identical."""
+    P, Wt, K, init = _kmeans_case()
+    ref = oracle.kmeans(P, Wt, K, init, 5)
+    assert np.array_equal(oracle.kmeans(P * 4.0, Wt, K, init, 5), ref)
+    assert np.array_equal(oracle.kmeans(P * 0.125, Wt, K, init, 5), ref)
+    assert np.array_equal(oracle.kmeans(P, Wt * 8.0, K, init, 5), ref)
+
+
+def test_kmeans_single_cluster_is_a_fixed_point_after_one_step():
+    """K = 1: every subvector joins the only cluster, so the first update is
+    final and further iterations repeat it exactly."""
+    P, Wt, _, init = _kmeans_case(K=1)
+    one = oracle.kmeans(P, Wt, 1, init[:1], 1)
+    assert np.array_equal(oracle.kmeans(P, Wt, 1, init[:1], 6), one)
+    assert np.isclose(np.linalg.norm(one), 1.0, atol=1e-12) and (one >= 0).all()
+
+
+def test_kmeans_equivariant_to_sample_order_and_channel_order():
+    """Reordering the sampled subvectors (with the initial picks following them)
+    leaves the codebook unchanged; permuting the 8 channels of every subvector
+    and weight permutes the codebook's channels the same way (up to rounding
+    of the reordered sums)."""
+    P, Wt, K, init = _kmeans_case()
+    ref = oracle.kmeans(P, Wt, K, init, 5)
+    g = np.random.default_rng(5)
+    order = g.permutation(P.shape[0])
+    where = np.empty_like(order)
+    where[order] = np.arange(order.size)
+    got = oracle.kmeans(P[order], Wt[order], K, where[init], 5)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+    sigma = g.permutation(8)
+    got = oracle.kmeans(P[:, sigma], Wt[:, sigma], K, init, 5)
+    assert np.allclose(got, ref[:, sigma], rtol=0, atol=1e-12)
+
+
+def test_kmeans_channel_without_weight_gets_zero_component():
+    """The update weights each channel of a member's unit direction by that
+    channel's omega (reading of Sec. 3.4 / App. A.7): a channel whose weight
+    is zero in every sample contributes nothing, so after one step every
+    codeword has a zero there."""
+    P, Wt, K, init = _kmeans_case()
+    Wt = Wt.copy()
+    Wt[:, 3] = 0.0
+    cb = oracle.kmeans(P, Wt, K, init, 2)
+    assert np.all(cb[:, 3] == 0.0)
+    assert np.allclose(np.linalg.norm(cb, axis=1), 1.0, atol=1e-12)
