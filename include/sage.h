@@ -60,7 +60,10 @@
  *  codebook: fp16 codebook[K][8] (16 bytes per codeword).
  *  perm: int32_t perm[d_in], storage column p holds original input channel
  *    perm[p]; the layer computes y = W_hat * x_perm with x_perm[p] = x[perm[p]]
- *    (Sec. 3.2 Eq. 5 and Sec. 3.5).  NULL means the identity.
+ *    (Sec. 3.2 Eq. 5 and Sec. 3.5).  NULL means the identity.  The entries
+ *    must be a permutation of 0 .. d_in - 1; device arrays are not read on
+ *    the host, so this is not checked (an entry out of range reads outside
+ *    the row of x).
  */
 #ifndef SAGE_H_
 #define SAGE_H_
@@ -206,10 +209,15 @@ int sage_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y,
  * y[p] = W_hat_{pair_expert[p]} x_perm[pair_xrow[p]].  experts: host array of
  * n_experts matrices sharing d_out and d_in (each with its own split,
  * codebook and perm); pair_expert / pair_xrow: device int32 [n_pairs];
- * x: fp16 [rows][d_in]; y: fp16 [n_pairs][d_out].  Each expert's planes are
- * read once per call whatever the number of its pairs (at most 16 pairs per
- * expert).  Errors: as sage_gemv; UNSUPPORTED for > 16 pairs on one expert is
- * reported through the status word (SAGE_ERR_UNSUPPORTED). */
+ * x: fp16 [rows][d_in]; y: fp16 [n_pairs][d_out].  The pairs of one expert
+ * are grouped (on the device, in pair order) into virtual matrices of at most
+ * 8 pairs, and each virtual matrix reads the expert's planes once: an expert
+ * with up to 8 pairs is read once per call.  pair_xrow entries must be rows
+ * of x (not checked on the host).  Errors: as sage_gemv, plus UNSUPPORTED
+ * for n_experts > 256 or n_pairs > 4096 and for experts that differ in d_out
+ * or d_in; a pair_expert entry outside [0, n_experts) sets
+ * SAGE_ERR_UNSUPPORTED in the status word and that pair's output is not
+ * written. */
 int sage_moe_gemv(const sage_matrix* experts, int n_experts,
                   const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs,
                   const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream);
