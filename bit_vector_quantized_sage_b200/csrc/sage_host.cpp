@@ -75,7 +75,7 @@ const char* sage_version(void) { return "libsage sm_100a, packed format v2"; }
 int sage_packed_sizes(int d_out, int d_in, int log2K, size_t* main_bytes, size_t* meta_bytes) {
     if (!main_bytes || !meta_bytes || d_out < 1 || d_in < 1) return SAGE_ERR_INVALID_ARGUMENT;
     if (d_in % 128 || log2K < 4 || log2K > 8) return SAGE_ERR_UNSUPPORTED;
-    const size_t R8 = (size_t)(d_out + 7) / 8;
+    const size_t R8 = ((size_t)d_out + 7) / 8;
     *main_bytes = (size_t)(d_in / kSV) * R8 * 16;
     *meta_bytes = (size_t)(d_in / 128) * R8 * 8 * 8;
     return SAGE_OK;

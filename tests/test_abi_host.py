@@ -155,3 +155,15 @@ def test_host_argument_errors_before_launch(lib):
     assert L.sage_workspace_size(sage.SAGE_OP_GROUPED, arr, 2, 1, C.byref(b)) == sage.SAGE_OK
     assert b.value >= one
     del pe
+
+
+def test_packed_sizes_closed_form_up_to_int_max(lib):
+    """Plane sizes are ceil(d_out / 8) octets x (d_in / 8) records of 16 B, and
+    ceil(d_out / 8) x (d_in / 128) groups of 8 rows x 8 B, computed without
+    overflow up to the largest int row count."""
+    a, b = C.c_size_t(), C.c_size_t()
+    for d_out, d_in in ((1, 128), (257, 2560), (2 ** 31 - 1, 128), (2 ** 31 - 8, 4096)):
+        assert lib.sage_packed_sizes(d_out, d_in, 6, C.byref(a), C.byref(b)) == sage.SAGE_OK
+        r8 = (d_out + 7) // 8
+        assert a.value == r8 * (d_in // 8) * 16
+        assert b.value == r8 * (d_in // 128) * 64
