@@ -418,7 +418,7 @@ int sage_moe_gemv(const sage_matrix* experts, int n_experts, const int32_t* pair
                   int n_pairs, const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream) {
     if (!experts || n_experts < 1 || !pair_expert || !pair_xrow || n_pairs < 1 || !x || !y)
         return SAGE_ERR_INVALID_ARGUMENT;
-    if (n_experts > 512 || n_pairs > 4096) return SAGE_ERR_UNSUPPORTED;
+    if (n_experts > 256 || n_pairs > 4096) return SAGE_ERR_UNSUPPORTED;
     for (int e = 0; e < n_experts; ++e) {
         int rc = check_matrix(&experts[e]);
         if (rc) return rc;

@@ -143,6 +143,9 @@ def test_host_argument_errors_before_launch(lib):
     pe = (C.c_int32 * 4)()
     arr = (sage.sage_matrix * 2)(mat(), mat(d_out=32))
     assert L.sage_moe_gemv(arr, 2, 0x600000, 0x700000, 4, x, y, wsp16, 1 << 20, None) == sage.SAGE_ERR_UNSUPPORTED
+    # limits checked before the expert array is read: 256 experts, 4096 pairs
+    assert L.sage_moe_gemv(arr, 257, 0x600000, 0x700000, 4, x, y, wsp16, 1 << 20, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert L.sage_moe_gemv(arr, 2, 0x600000, 0x700000, 4097, x, y, wsp16, 1 << 20, None) == sage.SAGE_ERR_UNSUPPORTED
     xs = (C.c_void_p * 2)(x, x)
     ys = (C.c_void_p * 2)(y, None)
     assert L.sage_gemv_grouped(arr, 2, xs, ys, 1, wsp16, 1 << 20, None) == sage.SAGE_ERR_INVALID_ARGUMENT
