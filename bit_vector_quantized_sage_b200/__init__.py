@@ -35,7 +35,7 @@ EXPORTS = (
     "sage_status_string", "sage_version", "sage_packed_sizes", "sage_pack", "sage_unpack",
     "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
-    "sage_query_status", "sage_gemv_static",
+    "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
 )
 
 
@@ -50,6 +50,17 @@ class sage_matrix(C.Structure):
         ("d_out", C.c_int32), ("d_in", C.c_int32), ("log2K", C.c_int32),
         ("main", C.c_void_p), ("meta", C.c_void_p), ("codebook", C.c_void_p), ("perm", C.c_void_p),
     ]
+
+
+class sage_decoder_layer(C.Structure):
+    _fields_ = [(n, sage_matrix) for n in ("q", "k", "v", "o", "gate", "up", "down")] + [
+        ("attn_norm", C.c_void_p), ("mlp_norm", C.c_void_p),
+        ("n_heads", C.c_int32), ("n_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("eps", C.c_float),
+    ]
+
+
+class sage_decoder_outputs(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("q", "k", "v", "o", "gate", "up", "down", "h_out")]
 
 
 _lib = None
@@ -83,6 +94,9 @@ def load(path: str = LIB_PATH):
         "sage_permute_x": ([P, P, I, I, P, P], I),
         "sage_query_status": ([P, P], I),
         "sage_gemv_static": ([MP, P, I, P, P], I),
+        "sage_decoder_layer_workspace_size": ([C.POINTER(sage_decoder_layer), I, C.POINTER(SZ)], I),
+        "sage_decoder_layer_forward": ([C.POINTER(sage_decoder_layer), P, I, C.POINTER(sage_decoder_outputs), P, SZ,
+                                        P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -319,3 +333,37 @@ def sage_permute_x(x, perm, M: int, d_in: int, x_perm, stream=None):
 
 def sage_query_status(ws: Workspace, stream=None) -> int:
     return int(load().sage_query_status(ws.ptr, _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Fused decoder layer (one launch of the four dependent projection stages)
+# ---------------------------------------------------------------------------
+
+class DecoderLayer:
+    """Pre-marshalled sage_decoder_layer_forward arguments.
+
+    mats: dict name -> PackedMatrix for q, k, v, o, gate, up, down; attn_norm /
+    mlp_norm: fp16 device tensors [hidden]; outputs: dict name -> fp16 device
+    tensors for q, k, v, o, gate, up, down, h_out ([M][...])."""
+
+    NAMES = ("q", "k", "v", "o", "gate", "up", "down")
+
+    def __init__(self, mats, attn_norm, mlp_norm, n_heads: int, n_kv_heads: int, head_dim: int, eps: float,
+                 outputs, M: int, ws: "Workspace" = None):
+        self.L = sage_decoder_layer(*[mats[n].desc() for n in self.NAMES], _ptr(attn_norm), _ptr(mlp_norm),
+                                    n_heads, n_kv_heads, head_dim, float(eps))
+        self.out = sage_decoder_outputs(*[_ptr(outputs[n]) for n in self.NAMES + ("h_out",)])
+        self.M = M
+        self.ws = ws if ws is not None else Workspace(self.workspace_size())
+        self.keep = (mats, attn_norm, mlp_norm, outputs)
+
+    def workspace_size(self) -> int:
+        b = C.c_size_t()
+        _check("sage_decoder_layer_workspace_size",
+               load().sage_decoder_layer_workspace_size(C.byref(self.L), self.M, C.byref(b)))
+        return b.value
+
+    def __call__(self, h, stream=None):
+        _check("sage_decoder_layer_forward",
+               load().sage_decoder_layer_forward(C.byref(self.L), _ptr(h), self.M, C.byref(self.out), self.ws.ptr,
+                                                 self.ws.nbytes, _stream(stream)))

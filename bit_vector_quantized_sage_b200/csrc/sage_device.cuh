@@ -1,6 +1,6 @@
 // Device-side building blocks shared by the libsage kernels (sm_100a):
-// PTX wrappers for mbarriers, bulk (TMA) copies, PDL, and the decode of the
-// packed format v1 (see include/sage.h).
+// PTX wrappers for mbarriers, bulk (TMA) copies, PDL, acquire/release
+// accesses, and the decode constants of the packed format v2 (include/sage.h).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -134,11 +134,31 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Device-scope atomic add with acquire-release semantics (returns the old value).
+// ------------------------------------------------------------------------
+// Device-scope atomics and ordered accesses
+// ------------------------------------------------------------------------
+// Atomic add with acquire-release semantics (returns the old value).
 __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
     unsigned old;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
+}
+
+// Release increment: every write of this thread that precedes it (and, after
+// a CTA barrier, of the threads that reached the barrier first) becomes
+// visible to an acquire load that sees the new value.
+__device__ __forceinline__ void red_add_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
@@ -146,7 +166,7 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
 }
 
 // ------------------------------------------------------------------------
-// Packed format v1 decode constants (per radius width V = 10 - log2K).
+// Packed format v2 decode constants (per radius width V = 10 - log2K).
 // ------------------------------------------------------------------------
 template <int V>
 struct Fmt {
@@ -192,23 +212,21 @@ __device__ __forceinline__ size_t meta_entry(int R8, int G, int blk, int g, int 
 __device__ __forceinline__ __half2 u2h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
 __device__ __forceinline__ uint32_t h22u(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-// (s (.) c) . x for one subvector: four half2 products with fp16 local
-// accumulation (the paper's Fig. 6a data path), returned in fp32.
-__device__ __forceinline__ float signed_dot(uint4 c, uint4 x) {
-    __half2 h = __hmul2(u2h2(c.x), u2h2(x.x));
-    h = __hfma2(u2h2(c.y), u2h2(x.y), h);
-    h = __hfma2(u2h2(c.z), u2h2(x.z), h);
-    h = __hfma2(u2h2(c.w), u2h2(x.w), h);
-    return __low2float(h) + __high2float(h);
-}
-
 // Per-split decode constants of format v2 (radius width V = 10 - log2K),
 // chosen at run time so one kernel serves every split of a launch.
-struct VDec {            // per-split decode constants (radius width V = 10 - log2K)
+struct VDec {
     uint32_t zmask, qmask;
-    uint32_t sh0, sh1, sh2, sh3, sh4, sh5;   // 15 - (sign slot position)
-    float vscale;
+    uint32_t sh0, sh1, sh2, sh3, sh4, sh5;   // 15 - (sign slot position); slot 5 sits at bit 15 (sh5 = 0)
+    uint32_t m0, m1, m2, m3, m4;             // 2^sh0 .. 2^sh4: the same shifts as multiplies
+    uint32_t m16;                            // 2^16
+    float vscale;                            // 2^V
 };
+
+__device__ __forceinline__ uint32_t opaque(uint32_t v) {
+    uint32_t r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
 
 __device__ __forceinline__ VDec vdec(int log2K) {
     const int V = 10 - log2K;
@@ -218,27 +236,13 @@ __device__ __forceinline__ VDec vdec(int log2K) {
     // slot k sits at bit k for k <= 6 - V, else at bit 10 + k
     auto sh = [&](int k) { return (uint32_t)(k <= 6 - V ? 15 - k : 5 - k); };
     d.sh0 = sh(0); d.sh1 = sh(1); d.sh2 = sh(2); d.sh3 = sh(3); d.sh4 = sh(4); d.sh5 = sh(5);
+    // The multipliers are passed through an opaque move, so that the compiler
+    // keeps the multiplies (FMA pipe) instead of turning them back into shifts.
+    d.m0 = opaque(1u << d.sh0); d.m1 = opaque(1u << d.sh1); d.m2 = opaque(1u << d.sh2);
+    d.m3 = opaque(1u << d.sh3); d.m4 = opaque(1u << d.sh4);
+    d.m16 = opaque(1u << 16);
     d.vscale = (float)(1 << V);
     return d;
-}
-
-// Loads the grid / aux meta of this lane's octet (64 bytes at a) without bank
-// conflicts: lane pairs start at rotated 16-byte quarters, and the four
-// quarters are rotated back into place with selects.
-__device__ __forceinline__ void load_meta(uint32_t a, int lane, uint4 (&q)[4]) {
-    const int r = (lane >> 1) & 3;
-    uint4 v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = lds128(a + (uint32_t)((k + r) & 3) * 16);  // v[k] = quarter (k + r) & 3
-    uint4 u[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {  // quarter e sits in v[(e - r) & 3]: rotate right by r
-        const uint4 a1 = (r & 1) ? v[(e + 3) & 3] : v[e];
-        const uint4 a2 = (r & 1) ? v[(e + 1) & 3] : v[(e + 2) & 3];
-        u[e] = (r & 2) ? a2 : a1;
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) q[e] = u[e];
 }
 
 }  // namespace dev

@@ -489,17 +489,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
 
 namespace {
 
-int gemm_sm_count() {
-    static std::once_flag once;
-    static int n = 0;
-    std::call_once(once, [] {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    });
-    return n;
-}
+int gemm_sm_count() { return current_sm_count(); }
 
 size_t round256g(size_t b) { return (b + 255) / 256 * 256; }
 
@@ -551,16 +541,8 @@ int launch_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y, voi
     const GemmPlan g = gemm_plan(A, M);
     if (ws_bytes < g.total) return SAGE_ERR_WORKSPACE;
     if (g.smem > kGemmSmemBudget) return SAGE_ERR_UNSUPPORTED;
-    static std::mutex mu;
-    static int configured = 0;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        if (g.smem > configured) {
-            if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, g.smem) != cudaSuccess)
-                return SAGE_ERR_CUDA;
-            configured = g.smem;
-        }
-    }
+    static SmemLimit limit;
+    if (!limit.ensure(gemm_kernel, g.smem)) return SAGE_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint4* xt = reinterpret_cast<uint4*>(w + g.off_xt);

@@ -1,38 +1,44 @@
-// Packed SAGE GEMV for batch 1..8 on sm_100a (decode path, Sec. 3.5 and App. A.1
-// of "SAGE: Pushing 2-Bit Vector-Quantized LLMs toward Real-World Usability"),
-// its grouped multi-matrix form, and the grouped-expert MoE GEMV.
+// Packed SAGE GEMV engine for batch 1..8 on sm_100a: the decode path of
+// "SAGE: Pushing 2-Bit Vector-Quantized LLMs toward Real-World Usability"
+// (Sec. 3.5 and App. A.1, Fig. 6a), run as one persistent launch over a list
+// of dependent stages (a stage is one GEMV or several GEMVs sharing a launch,
+// e.g. the q|k|v projections), and the grouped-expert MoE GEMV on the same
+// body.
 //
 // Work decomposition (B200-first, not the paper's RTX 4090 tiling):
-//  * A "unit" is one subvector column j of one 256-row block (32 row octets) of
-//    one matrix: a 512-byte slab of the main plane.  The units of all matrices
-//    of a launch are flattened (matrix, block, j) and cut into one contiguous
-//    range per CTA of a persistent grid (one CTA per SM).  Dense launches are
-//    planned on the host (each matrix gets its own CTAs when that costs little
-//    balance); MoE launches are planned on the device from the routing.
-//  * Two producer warps per CTA.  The copy warp bulk-copies (1-D TMA) the
-//    codebooks and, chunk by chunk (16 columns = one radius group), the code
-//    records and grid/aux meta into a ring of shared-memory slots, without
-//    waiting on the preceding kernel (programmatic dependent launch): none of
-//    it is written there.  The activation warp gathers the ESG-permuted
-//    x_perm[p] = x[perm[p]] window by window (Sec. 3.5 fuses this gather into
-//    the decode GEMV); the permutation entries are copied before the wait on
-//    the preceding kernel, only x after it.
-//  * Decode warps (dense launches): one thread per row of the 256-row block
-//    for the whole segment; it reads its row's half of a record word per
-//    column and accumulates the row's outputs itself.  The MoE kernel keeps
-//    an octet-per-lane body: lane l decodes the 16-byte record of row octet l
-//    (8 rows) per column, and the warps' partial sums are reduced in shared
-//    memory.
-//  * Per subvector: the codeword address and the radius code each come out of
-//    one logic op (format v2), the codeword is one conflict-free 128-bit shared
-//    load (8 bank-rotated replicas of the codebook), the signs are XORed into
-//    the fp16 sign bits, four half2 FMAs form (s (.) c) . x with fp16 local
-//    accumulation (Fig. 6a), and r = mu + q delta (Eq. 2) is applied once, fp32.
+//  * A "unit" is one subvector column j of one 256-row block (32 row octets)
+//    of one matrix: a 512-byte slab of the main plane.  The units of a stage
+//    are flattened (matrix, block, j) and cut into one contiguous range per
+//    CTA of a persistent grid (one CTA per SM); every stage is spread over
+//    every CTA.
+//  * The copy warp bulk-copies (1-D TMA) codebooks and, chunk by chunk (16
+//    columns = one radius group), the code records and grid/aux meta into a
+//    ring of shared-memory slots.  It runs ahead across segments and stages:
+//    the packed planes never depend on earlier work, so the next stage's codes
+//    stream in while the current stage finishes.
+//  * The gather warp builds the ESG-permuted activations x_perm[p] = x[perm[p]]
+//    window by window (Sec. 3.5 fuses this gather into the decode GEMV; the
+//    fused prologues -- RMSNorm, residual + RMSNorm, SiLU(gate) * up, and the
+//    single-position attention read of v -- are applied to the gathered values).
+//    The first window of each stage is gathered by the gather and decode warps
+//    together, after the stage's inputs are ready.
+//  * 8 decode warps: warp w holds row pairs 32 (w % 4) .. 32 (w % 4) + 31 of the
+//    256-row block (one 32-bit record word = two rows per thread) and columns
+//    8 (w / 4) .. 8 (w / 4) + 7 of each chunk.  Per subvector: the codeword
+//    address is one logic op on the word (format v2), the codeword one
+//    conflict-free 128-bit load from the replica of the thread's lane position
+//    (8 bank-rotated replicas of the codebook), the signs are XORed into the
+//    fp16 sign bits, four half2 products with fp16 accumulation form
+//    (s (.) c) . x (Fig. 6a), and r = mu + q delta (Eq. 2) scales it once, in
+//    fp32, into the row's fp32 accumulator.
+//  * Overflow guard for the fp16 local sums: each window's largest |x| decides
+//    a power-of-two prescale (x / 2^k, k <= 2) that keeps every partial sum of
+//    a subvector finite; the radius carries 2^k back.  Powers of two are exact.
 //  * Rows whose columns are split between CTAs are combined deterministically:
 //    partial sums go to the workspace and the last CTA to finish a block adds
-//    them in CTA order (the paper's FP32 split-K combine for small grids).
-//    A CTA defers its outputs to the end so that no segment waits for another
-//    segment's global round trips.
+//    them in CTA order.  A block whose final outputs are written bumps its
+//    stage's completion count; a stage that reads an earlier stage's outputs
+//    waits for that count (acquire), so dependent stages need no relaunch.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -41,310 +47,202 @@
 
 #include "sage_device.cuh"
 #include "sage_internal.h"
+#include "sage_engine.h"
 
 namespace sage {
 using namespace dev;
 
 namespace {
 
-constexpr int kMaxMats = 64;
-constexpr int kMaxExperts = 256;
-constexpr int kMaxPairsPerVirtual = 8;
-constexpr int kOct = 32;               // row octets per block (one per lane)
-constexpr int kBlockRows = kOct * 8;
-constexpr int kChunkJ = 16;            // a chunk lies inside one radius group
-constexpr int kMaxSegs = 4;            // segments stashed before outputs are flushed
-constexpr int kMainSlot = kChunkJ * kOct * 16;  // 8 KB of code records
-constexpr int kMetaSlot = kOct * 64;            // 2 KB: one group of 256 rows
+constexpr int kOct = 32;               // row octets per block
+constexpr int kBlockRows = kOct * 8;   // 256
+constexpr int kChunkJ = 32;            // a chunk is two radius groups (aligned)
+constexpr int kMainSlot = kChunkJ * kOct * 16;  // 16 KB of code records
+constexpr int kMetaSlot = 2 * kOct * 64;        // 4 KB: two groups of 256 rows
 constexpr int kSlot = kMainSlot + kMetaSlot;    // one ring slot = one chunk
-constexpr int kMaxSlots = 16;                   // ring depth limit
-constexpr int kSegTab = 32;                     // segment-table capacity per round
-constexpr int kSegBytes = 160;                  // shared memory per table entry
-// Named barriers besides the decode warps' own (id 1): the activation and
-// copy warps (id 3) and the activation and decode warps (id 2).
-constexpr int kBarPermIssued = 3;
-constexpr int kBarFirstWindow = 2;
+constexpr int kMaxSlots = 16;
+constexpr int kDW = 8;                          // decode warps: 4 row quarters x 2 column parts
+constexpr int kParts = kDW / 4;                 // column parts of a chunk (one radius group each)
+constexpr int kDT = kDW * 32;                   // decode threads
+constexpr int kGT = kDT + 32;                   // threads of a cooperative gather
+constexpr int kThreads = kDT + 96;              // + copy, gather and epilogue warps
+constexpr int kCopyWarp = kDW, kGatherWarp = kDW + 1, kEpiWarp = kDW + 2;
+constexpr int kStashSlots = 4;                  // segments between the decode and epilogue warps (at most)
+constexpr int kBarDecode = 1, kBarGather = 2;   // named barriers (0 is __syncthreads)
+constexpr int kXBufBytes = 8192;                // one activation window buffer
+constexpr int kMaxXW = 512;                     // window columns at batch 1
+constexpr int kPermBuf = kMaxXW * 32;           // the window's permutation entries
+constexpr int kMoeCache = 32;                   // virtual experts staged per CTA
+constexpr int kMaxPairsPerVirtual = 8;
+
+// Codebook replicas: codeword z of replica r at byte z*128 + r*16.  Static
+// shared memory has a link-time address, so a codeword's address is one logic
+// op on the record word plus the load's immediate offset.
+__shared__ __align__(1024) uint4 g_rep[256 * 8];
+
+// Codeword at byte offset `off` of the replicas (z * 128 + r * 16).  A plain
+// C++ load, so the array's shared-memory address becomes the instruction's
+// immediate offset.
+__device__ __forceinline__ uint4 cw_load(uint32_t off) {
+    return *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(g_rep) + off);
+}
 
 template <int M>
 struct Cfg {
-    static constexpr int kW = 8;                       // decode warps
-    static constexpr int kThreads = (kW + 2) * 32;     // + copy warp + activation warp
-    static constexpr int kDecodeThreads = kW * 32;
-    // Columns per activation window: x_perm for a window is gathered in one go.
-    static constexpr int kXW = (M == 1) ? 256 : (M == 2) ? 128 : (M <= 4) ? 64 : 32;
-    static constexpr int kXBuf = kXW * M * 16;         // one window of x_perm, [m][column]
-    static constexpr int kPermBuf = kXW * 32;          // the window's permutation entries
-    static constexpr int kPosInfo = kXW * 4;           // (segment, column) of each window position
-    // cross-warp reduction buffer: only the MoE kernel's segment body (batch 8) uses one
-    static constexpr int kRed = (M == kMaxPairsPerVirtual) ? kW * 8 * M * 32 * 4 : 0;
-    static constexpr int kStash = kMaxSegs * M * kBlockRows * 4;
-    static constexpr int kBars = (2 * kMaxSlots + 9) * 8;
-    static constexpr int kFixed = 2 * kXBuf + kPermBuf + kPosInfo + kRed + kStash + kSegTab * kSegBytes + kBars + 64;
-    // codebook replicas (K_max * 8 * 16) + 2 raw codebooks + ring + fixed
-    static int smem(int slots, int kmax) { return kmax * 128 + 2 * kmax * 16 + slots * kSlot + kFixed; }
+    static constexpr int kXW = kXBufBytes / (16 * M);    // window columns
+    static constexpr int kSlots = M <= 2 ? kStashSlots : M <= 4 ? 2 : 1;  // stash ring depth
+    static constexpr int kStash = kSlots * kParts * M * kBlockRows * 4;  // [slot][column part][m][row]
 };
 
-// One matrix as the kernel sees it while working on one of its segments.
-struct MatView {
+// ------------------------------------------------------------------------
+// Problem sources: where a stage's jobs (one matrix with its input and output
+// binding each) come from.  Dense launches carry them in the kernel
+// parameters; the MoE launch reads virtual experts from the routing result.
+// ------------------------------------------------------------------------
+struct JobView {
     const uint32_t* main;
     const uint32_t* meta;
     const uint16_t* cb;
     const int32_t* perm;
-    const uint16_t* x;      // activations, row stride d_in
-    uint16_t* y;            // outputs, row stride d_out
-    const int32_t* xrows;   // [Mk] activation row of batch slot m (null: m); shared or global memory
-    const int32_t* yrows;   // [Mk] output row of batch slot m (null: m); shared or global memory
-    long long unit0;
-    int d_out, d_in, log2K, R8, S, blk0, Mk;
+    const uint16_t* x;    // plain-prologue input rows, stride d_in
+    uint16_t* y;          // output rows, stride d_out
+    const int* xrows;     // batch slot -> input row (null: slot m reads row m); shared memory
+    const int* yrows;     // batch slot -> output row (null: slot m writes row m); shared memory
+    int unit0, d_out, d_in, log2K, S, R8, blk0, Mk, id;
 };
 
-struct DenseMat {
-    const uint32_t* main;
-    const uint32_t* meta;
-    const uint16_t* cb;
-    const int32_t* perm;
-    const uint16_t* x;
-    uint16_t* y;
-    long long unit0, units;
-    int d_out, d_in, log2K, blk0;
-    int cta0, ncta;        // CTAs [cta0, cta0 + ncta) own this matrix (per-matrix plans)
-};
-
-struct ExpertMat {
-    const uint32_t* main;
-    const uint32_t* meta;
-    const uint16_t* cb;
-    const int32_t* perm;
-    int log2K, pad;
-};
-
-struct Common {
-    int n_cta;
-    int M;                 // dense: batch; MoE: 0 (per virtual expert)
-    int slots;             // ring depth (chunks in flight)
-    int n_wg;              // decode warp groups (1, 2 or 4); chunk t goes to group t % n_wg
-    int kmax;              // largest codebook of the launch (replica area size)
-    uint32_t* status;
-    unsigned* counters;
-    float* partials;       // [n_cta][2][8][kBlockRows]
-};
-
-// CTA c covers units [first(c), first(c + 1)).  Stream-K plans split the
-// flattened units evenly; per-matrix plans give matrix k its own CTAs and
-// split its units evenly among them.  Both are plain arithmetic, so no
-// dependent parameter-space loads sit on any critical path.
-constexpr int kMaxCta = 256;
-
-struct DenseParams {
-    Common c;
-    long long total_units;
-    int n_mats;
-    int per_matrix;
-    int cta_start[kMaxCta + 1];   // first unit of each CTA; cta_start[n_cta] = total_units
-    DenseMat mats[kMaxMats];
-};
-
-struct MoeRoute {
-    int n_virtual;
-    int pad[3];
-};
-struct MoeParams {
-    Common c;
-    int n_experts, d_out, d_in, n_pairs;
-    const uint16_t* x;
-    uint16_t* y;
-    const MoeRoute* route;         // ws
-    const int32_t* v_expert;       // ws [n_pairs]
-    const int32_t* v_xrows;        // ws [n_pairs][8]
-    const int32_t* v_yrows;        // ws [n_pairs][8]
-    const int32_t* v_count;        // ws [n_pairs]
-    ExpertMat experts[kMaxExperts];
-};
-
-// The CTA start table and the matrix descriptors are read from shared-memory
-// copies: dependent loads from the parameter space miss the constant cache.
-struct DenseProblem {
-    const DenseParams& p;
-    const int* cs;        // shared copy of p.cta_start
-    const DenseMat* ms;   // shared copy of p.mats
-    __device__ long long total() const { return p.total_units; }
-    __device__ long long cta_begin(int c) const { return cs[min(c, p.c.n_cta)]; }
-    __device__ int cta_of(long long u) const {  // the CTA whose range holds unit u
-        int lo = 0, hi = p.c.n_cta - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (cs[mid] <= u) lo = mid;
-            else hi = mid - 1;
-        }
-        return lo;
+struct DenseSrc {
+    static constexpr bool kVarBatch = false;
+    const EngineParams& p;
+    __device__ int n_stages() const { return p.n_stages; }
+    __device__ const EngineStage& stage(int s) const { return p.st[s]; }
+    __device__ int units(int s) const { return p.st[s].units; }
+    __device__ JobView job_at(int s, int u) const {
+        const EngineStage& st = p.st[s];
+        int k = st.job0;
+        while (k + 1 < st.job0 + st.n_jobs && p.jobs[k + 1].unit0 <= u) ++k;
+        return job(k);
     }
-    __device__ MatView view(long long u) const {
-        int k = 0;
-        while (k + 1 < p.n_mats && ms[k + 1].unit0 <= u) ++k;
-        const DenseMat& d = ms[k];
-        MatView v;
+    __device__ JobView job(int k) const {
+        const EngineJob& d = p.jobs[k];
+        JobView v;
         v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = d.x; v.y = d.y;
-        v.xrows = nullptr; v.yrows = nullptr; v.unit0 = d.unit0;
-        v.d_out = d.d_out; v.d_in = d.d_in; v.log2K = d.log2K;
-        v.R8 = (d.d_out + 7) >> 3; v.S = d.d_in >> 3;
-        v.blk0 = d.blk0; v.Mk = p.c.M;
+        v.xrows = nullptr; v.yrows = nullptr;
+        v.unit0 = d.unit0; v.d_out = d.d_out; v.d_in = d.d_in; v.log2K = d.log2K;
+        v.S = d.d_in >> 3; v.R8 = (d.d_out + 7) >> 3; v.blk0 = d.blk0; v.Mk = p.M; v.id = k;
         return v;
     }
 };
 
-// The routing results this CTA needs (virtual-expert count, and the expert
-// and pair count of the virtual experts its range touches, with their
-// descriptors) are staged in shared memory once, after the routing kernel.
-constexpr int kMoeCache = 32;
+// The MoE routing result this CTA needs (virtual-expert ids, pair counts and
+// row lists of the virtual experts its range touches) is staged in shared
+// memory once, after the routing kernel.
 struct MoeStage {
-    long long total;
-    int vi0, nvi;
+    int n_virtual, units, vi0, nvi, overflow;
     int v_expert[kMoeCache];
     int v_count[kMoeCache];
-    int v_xrows[kMoeCache][kMaxPairsPerVirtual];  // activation / output rows of the cached virtual experts
+    int v_xrows[kMoeCache][kMaxPairsPerVirtual];
     int v_yrows[kMoeCache][kMaxPairsPerVirtual];
-    ExpertMat emat[kMoeCache];
 };
 
-struct MoeProblem {
+struct MoeSrc {
+    static constexpr bool kVarBatch = true;
     const MoeParams& p;
-    const MoeStage& st;
-    __device__ int R8() const { return (p.d_out + 7) >> 3; }
-    __device__ long long upv() const { return (long long)((R8() + kOct - 1) / kOct) * (p.d_in >> 3); }
-    __device__ long long total() const { return st.total; }
-    __device__ long long cta_begin(int c) const { return (long long)c * st.total / p.c.n_cta; }
-    __device__ int cta_of(long long u) const {
-        const long long t = st.total;
-        return (int)(((u + 1) * p.c.n_cta + t - 1) / t) - 1;
-    }
-    __device__ MatView view(long long u) const {
-        const long long per = upv();
-        const int vi = (int)(u / per);
-        const int k = vi - st.vi0;
-        const bool cached = k >= 0 && k < st.nvi;
-        const int e = cached ? st.v_expert[k] : __ldcg(p.v_expert + vi);
-        const ExpertMat& d = cached ? st.emat[k] : p.experts[e];
-        MatView v;
+    const MoeStage& ms;
+    __device__ int n_stages() const { return 1; }
+    __device__ const EngineStage& stage(int) const { return p.st; }
+    __device__ int units(int) const { return ms.units; }
+    __device__ int upv() const { return ((((p.d_out + 7) >> 3) + kOct - 1) / kOct) * (p.d_in >> 3); }
+    __device__ JobView job_at(int, int u) const { return job(u / upv()); }
+    __device__ JobView job(int vi) const {
+        const int k = vi - ms.vi0;  // always staged: a CTA only touches its own range
+        const int e = ms.v_expert[k];
+        const EngineExpert& d = p.experts[e];
+        JobView v;
         v.main = d.main; v.meta = d.meta; v.cb = d.cb; v.perm = d.perm; v.x = p.x; v.y = p.y;
-        v.xrows = cached ? st.v_xrows[k] : p.v_xrows + (size_t)vi * kMaxPairsPerVirtual;
-        v.yrows = cached ? st.v_yrows[k] : p.v_yrows + (size_t)vi * kMaxPairsPerVirtual;
-        v.unit0 = (long long)vi * per;
+        v.xrows = ms.v_xrows[k]; v.yrows = ms.v_yrows[k];
         v.d_out = p.d_out; v.d_in = p.d_in; v.log2K = d.log2K;
-        v.R8 = R8(); v.S = p.d_in >> 3;
+        v.S = p.d_in >> 3; v.R8 = (p.d_out + 7) >> 3;
+        v.unit0 = vi * upv();
         v.blk0 = vi * ((v.R8 + kOct - 1) / kOct);
-        v.Mk = cached ? st.v_count[k] : __ldcg(p.v_count + vi);
+        v.Mk = ms.v_count[k];
+        v.id = vi;
         return v;
     }
 };
 
-// Batch-slot row of a virtual expert: from the CTA's staged copy in shared
-// memory, or (experts outside the staged range) from the workspace in L2.
-__device__ __forceinline__ int row_at(const int32_t* rows, int m) {
-    return __isShared(rows) ? rows[m] : __ldcg(rows + m);
+// Balanced split of `units` over n_cta CTAs: the first units % n_cta CTAs
+// take one unit more.  32-bit arithmetic only.
+__device__ __forceinline__ int cta_begin(int units, int n_cta, int c) {
+    const int q = units / n_cta, r = units - q * n_cta;
+    return q * c + min(c, r);
+}
+// The CTA whose range [cta_begin(c), cta_begin(c + 1)) holds unit u.
+__device__ __forceinline__ int cta_of(int units, int n_cta, int u) {
+    const int q = units / n_cta, r = units - q * n_cta;
+    const int big = (q + 1) * r;  // units held by the CTAs that take q + 1
+    return u < big ? u / (q + 1) : r + (u - big) / q;
 }
 
-// A segment: one matrix, one 256-row block, columns [ja, jb), plus what the
-// split-K combine needs.  Each CTA builds its segment table once, in shared
-// memory, so no role ever walks the parameter tables again.
+// A segment: one job, one 256-row block, columns [ja, jb) of a CTA's range.
 struct Seg {
-    MatView v;
-    unsigned* counter;      // split blocks: arrival counter
-    int blk, ja, jb, n_oct, n_chunks;
-    int full;               // the segment covers all columns of its block
-    int c_first, c_last;    // CTAs contributing to the block (split blocks)
-    int first_slot;         // partial-sum slot of c_first for this block
-    int my_slot;            // this CTA's partial-sum slot for this block
+    JobView v;
+    int blk, ja, jb, n_oct;
+    bool full;
 };
-static_assert(sizeof(Seg) <= kSegBytes, "segment table entry outgrew its shared-memory budget");
 
-template <class Problem>
-__device__ Seg make_seg(const Problem& P, long long u, long long u_end, long long cta_u0) {
-    Seg s;
-    s.v = P.view(u);
-    const int local = (int)(u - s.v.unit0);  // unit counts fit in 32 bits (checked on the host)
-    s.blk = local / s.v.S;
-    s.ja = local - s.blk * s.v.S;
-    const long long jb = (long long)s.ja + (u_end - u);
-    s.jb = (int)(jb < (long long)s.v.S ? jb : (long long)s.v.S);
-    s.n_oct = min(kOct, s.v.R8 - s.blk * kOct);
-    s.n_chunks = ((s.jb - 1) >> 4) - (s.ja >> 4) + 1;
-    s.full = (s.ja == 0 && s.jb == s.v.S);
-    s.counter = nullptr;
-    s.c_first = s.c_last = s.first_slot = s.my_slot = 0;
-    (void)cta_u0;
-    return s;
+template <class Src>
+__device__ __forceinline__ Seg make_seg(const Src& src, int s, int u, int u1) {
+    Seg g;
+    g.v = src.job_at(s, u);
+    const int local = u - g.v.unit0;
+    g.blk = local / g.v.S;
+    g.ja = local - g.blk * g.v.S;
+    g.jb = min(g.v.S, g.ja + (u1 - u));
+    g.n_oct = min(kOct, g.v.R8 - g.blk * kOct);
+    g.full = (g.ja == 0 && g.jb == g.v.S);
+    return g;
 }
 
-// Split-K bookkeeping of a segment whose block is shared with other CTAs:
-// the contributing CTAs, the partial-sum slots and the arrival counter.  Run
-// by one lane per segment, in parallel, after the segments are laid out.
-template <class Problem>
-__device__ void seg_split_info(const Problem& P, const Common& C, Seg& s, long long cta_u0) {
-    if (s.full) return;
-    const long long b0 = s.v.unit0 + (long long)s.blk * s.v.S;
-    s.c_first = P.cta_of(b0);
-    s.c_last = P.cta_of(b0 + s.v.S - 1);
-    s.first_slot = (P.cta_begin(s.c_first) >= b0) ? 0 : 1;
-    s.my_slot = (cta_u0 >= b0) ? 0 : 1;
-    s.counter = C.counters + s.v.blk0 + s.blk;
+// Columns [x, y) of chunk c (chunks are cut at 32-column boundaries, i.e.
+// every other radius-group boundary).
+__device__ __forceinline__ int2 chunk_cols(const Seg& g, int c) {
+    const int k = (g.ja >> 5) + c;
+    return make_int2(max(g.ja, k << 5), min(g.jb, (k + 1) << 5));
 }
-
-// Fills tab[0..n) with the segments of [u, u_end) (at most kSegTab); returns n
-// and the first unit not covered.
-template <class Problem>
-__device__ int build_segs(const Problem& P, const Common& C, long long u, long long u_end, long long cta_u0,
-                          Seg* tab, long long* u_next) {
-    int n = 0;
-    while (u < u_end && n < kSegTab) {
-        tab[n++] = make_seg(P, u, u_end, cta_u0);
-        const Seg& s = tab[n - 1];
-        u += s.jb - s.ja;
-    }
-    *u_next = u;
-    return n;
-}
-
-// Column range of chunk c of a segment (chunks are cut at group boundaries).
-__device__ __forceinline__ int2 chunk_cols(const Seg& s, int c) {
-    const int g = (s.ja >> 4) + c;
-    return make_int2(max(s.ja, g << 4), min(s.jb, (g + 1) << 4));
-}
+__device__ __forceinline__ int n_chunks(const Seg& g) { return ((g.jb - 1) >> 5) - (g.ja >> 5) + 1; }
 
 __device__ __forceinline__ void flag(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
 
-// Set when any bounded wait of the CTA gives up; later waits then return at
-// once, so a CTA whose pipeline is stuck ends after one wait limit.
-__shared__ int s_abort;
+// A segment decoded but not yet written out (its sums wait in the stash).
+struct Pending {
+    Seg g;
+    int stage;
+    int first;   // the CTA's first segment of the stage (split-K slot 0)
+};
+static_assert(sizeof(Pending) <= 192, "pending-segment table entry outgrew its shared memory");
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Common& C) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_test(bar, parity)) return true;
-        if (i > 2048) {
-            if (*reinterpret_cast<volatile int*>(&s_abort)) return false;
-            __nanosleep(64);
-        }
-    }
-    *reinterpret_cast<volatile int*>(&s_abort) = 1;
-    flag(C.status, kDevTimeout);
-    return false;
-}
-
-template <int M>
+// ------------------------------------------------------------------------
+// Shared memory
+// ------------------------------------------------------------------------
 struct Smem {
-    uint32_t cb0;     // codebook replicas: entry z*8 + r holds codeword z (16 bytes)
-    uint32_t ring0;   // shared address of the chunk ring
-    int slots;        // ring depth
+    uint32_t cb0;       // codebook replicas (g_rep)
+    uint32_t ring0;     // chunk ring
+    uint32_t cbraw0;    // two raw codebooks
     int cbraw_bytes;
-    uint32_t cbraw0;  // two raw codebooks (double buffer across segments)
-    uint32_t xbuf0;   // two activation windows, each [m][kXW] x 16 bytes
-    uint32_t perm0;   // permutation entries of the window being gathered, [kXW] x 32 bytes
-    uint32_t* posinfo;  // per window position: segment index << 24 | column j
-    float* red;
-    float* stash;
+    uint32_t xbuf0;     // two activation windows
+    uint32_t perm0;     // the window's permutation entries (8 int32 per column)
+    int slots;
+    uint32_t* posinfo;  // per window position: job << 20 | column j
+    const int32_t** posperm;  // per window position: its 8 permutation entries (null: identity)
+    float* stash;       // [slot][column part][M][256] decode sums awaiting the epilogue
+    float* red;         // [kGT / 32][8] cooperative reductions
     uint64_t* bars;
-    int* bcast;
-    int* wlen0;       // length of the first activation window
-    Seg* segs;
+    int* misc;          // [0..1] window shift k per buffer, [2] abort flag, [3] window max |x| bits,
+                        // [8] window length, [9] batch rows per window, [10] first window gathered,
+                        // [16..24) flush flags
+    float* inv_rms;     // [8] per batch row
+    struct Pending* pend;  // segments awaiting their flush (written by decode thread 0)
     __device__ uint32_t slot_addr(int k) const { return ring0 + (uint32_t)k * kSlot; }
     __device__ uint64_t* full(int k) const { return bars + k; }
     __device__ uint64_t* empty(int k) const { return bars + kMaxSlots + k; }
@@ -353,38 +251,87 @@ struct Smem {
     __device__ uint64_t* x_full(int h) const { return bars + 2 * kMaxSlots + 4 + h; }
     __device__ uint64_t* x_empty(int h) const { return bars + 2 * kMaxSlots + 6 + h; }
     __device__ uint64_t* perm_full() const { return bars + 2 * kMaxSlots + 8; }
-    __device__ uint32_t xwin(int w) const { return xbuf0 + (uint32_t)(w & 1) * Cfg<M>::kXBuf; }
+    __device__ uint64_t* st_full(int k) const { return bars + 2 * kMaxSlots + 9 + k; }
+    __device__ uint64_t* st_empty(int k) const { return bars + 2 * kMaxSlots + 9 + kStashSlots + k; }
+    __device__ uint32_t xwin(int w) const { return xbuf0 + (uint32_t)(w & 1) * kXBufBytes; }
+    __device__ volatile int* abort_flag() const { return misc + 2; }
 };
+constexpr int kBars = 2 * kMaxSlots + 9 + 2 * kStashSlots;
+
+constexpr int kPendBytes = kStashSlots * 192;  // pending-segment table (sizeof(Pending) <= 192)
 
 template <int M>
-__device__ __forceinline__ Smem<M> carve(uint8_t* base, int slots, int kmax) {
-    Smem<M> s;
+constexpr int fixed_smem() {
+    return 2 * kXBufBytes + kPermBuf + kMaxXW * 4 + kMaxXW * 8 + Cfg<M>::kStash + (kGT / 32) * 8 * 4 + kBars * 8 +
+           64 * 4 + 8 * 4 + kPendBytes;
+}
+// Dynamic shared memory of a launch: raw codebooks + ring + fixed buffers.
+template <int M>
+int smem_bytes(int slots, int kmax) {
+    return 2 * kmax * 16 + slots * kSlot + fixed_smem<M>();
+}
+
+template <int M>
+__device__ Smem carve(uint8_t* base, int slots, int kmax) {
+    Smem s;
     s.slots = slots;
+    s.cb0 = smem_u32(g_rep);
     uint8_t* p = base;
-    s.cb0 = smem_u32(p); p += kmax * 128;
     s.ring0 = smem_u32(p); p += slots * kSlot;
     s.cbraw_bytes = kmax * 16;
     s.cbraw0 = smem_u32(p); p += 2 * kmax * 16;
-    s.xbuf0 = smem_u32(p); p += 2 * Cfg<M>::kXBuf;
-    s.perm0 = smem_u32(p); p += Cfg<M>::kPermBuf;
-    s.posinfo = reinterpret_cast<uint32_t*>(p); p += Cfg<M>::kPosInfo;
-    s.red = reinterpret_cast<float*>(p); p += Cfg<M>::kRed;
+    s.xbuf0 = smem_u32(p); p += 2 * kXBufBytes;
+    s.perm0 = smem_u32(p); p += kPermBuf;
+    s.posinfo = reinterpret_cast<uint32_t*>(p); p += kMaxXW * 4;
+    s.posperm = reinterpret_cast<const int32_t**>(p); p += kMaxXW * 8;
     s.stash = reinterpret_cast<float*>(p); p += Cfg<M>::kStash;
-    s.segs = reinterpret_cast<Seg*>(p); p += kSegTab * kSegBytes;
-    s.bars = reinterpret_cast<uint64_t*>(p); p += (2 * kMaxSlots + 9) * 8;
-    s.bcast = reinterpret_cast<int*>(p);
-    s.wlen0 = s.bcast + 8;
+    s.red = reinterpret_cast<float*>(p); p += (kGT / 32) * 8 * 4;
+    s.bars = reinterpret_cast<uint64_t*>(p); p += kBars * 8;
+    s.misc = reinterpret_cast<int*>(p); p += 64 * 4;
+    s.inv_rms = reinterpret_cast<float*>(p); p += 8 * 4;
+    s.pend = reinterpret_cast<Pending*>(p);
     return s;
 }
 
-// Activation windows.  The chunks of a CTA are laid end to end; a window holds
-// up to kXW of their columns (a chunk never straddles two windows) and every
-// segment-table round starts a new window.  The activation warp and the
-// decode warps apply these same two rules, so they agree on where each
-// chunk's x_perm sits without talking to each other.
+__device__ __forceinline__ bool wait_bar(const Smem& sm, uint64_t* bar, uint32_t parity, uint32_t* status) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if (i > 2048) {
+            if (*sm.abort_flag()) return false;
+            __nanosleep(64);
+        }
+    }
+    *sm.abort_flag() = 1;
+    flag(status, kDevTimeout);
+    return false;
+}
+
+// Bounded wait until *cnt >= target (acquire).  One thread polls.
+__device__ __forceinline__ bool wait_count(const Smem& sm, const unsigned* cnt, unsigned target, uint32_t* status) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (ld_acquire_gpu(cnt) >= target) return true;
+        if (*sm.abort_flag()) return false;
+        __nanosleep(i < 64 ? 32 : 128);
+    }
+    *sm.abort_flag() = 1;
+    flag(status, kDevTimeout);
+    return false;
+}
+
+__device__ __forceinline__ void ring_next(int& slot, int& ph, int slots) {
+    if (++slot == slots) {
+        slot = 0;
+        ph ^= 1;
+    }
+}
+
+// Activation windows: the chunks of a CTA's stage range are laid end to end;
+// a window holds up to `xw` of their columns (a chunk never straddles two
+// windows) and every stage starts a new window.  The gather warp and the
+// decode warps apply these rules identically.
 struct WinPos {
-    int win;    // window index (its buffer is win & 1)
-    int wpos;   // columns already placed in the window
+    int win;   // global window index (buffer win & 1)
+    int wpos;  // columns placed in the window so far
 };
 __device__ __forceinline__ int win_place(WinPos& w, int nj, int xw) {
     if (w.wpos + nj > xw) { ++w.win; w.wpos = 0; }
@@ -396,679 +343,777 @@ __device__ __forceinline__ void win_break(WinPos& w) {
     if (w.wpos > 0) { ++w.win; w.wpos = 0; }
 }
 
-__device__ __forceinline__ void ring_next(int& slot, int& ph, int slots) {
-    if (++slot == slots) {
-        slot = 0;
-        ph ^= 1;
+// ------------------------------------------------------------------------
+// Copy warp
+// ------------------------------------------------------------------------
+// Chunks requested before the launch's first activation window is gathered:
+// the permutation entries, x and the kernel parameters must not queue behind
+// the CTA's whole share of the packed planes.
+constexpr int kStartChunks = 2;
+
+template <class Src>
+__device__ void copy_role(const Src& src, const Smem& sm, uint32_t* status, int n_cta) {
+    const int lane = threadIdx.x & 31;
+    int t = 0, slot = 0, ph = 0, ncb = 0;
+    bool throttled = true;
+    const uint16_t* cur_cb = nullptr;
+    const uint64_t pol = l2_evict_first();
+    for (int s = 0; s < src.n_stages(); ++s) {
+        const int U = src.units(s);
+        if (U <= 0) continue;
+        const int u1 = cta_begin(U, n_cta, blockIdx.x + 1);
+        for (int u = cta_begin(U, n_cta, blockIdx.x); u < u1;) {
+            const Seg g = make_seg(src, s, u, u1);
+            u += g.jb - g.ja;
+            if (g.v.cb != cur_cb) {
+                const int h = ncb & 1;
+                if (ncb >= 2) wait_bar(sm, sm.cb_empty(h), ((ncb >> 1) - 1) & 1, status);
+                if (lane == 0) {
+                    const uint32_t bytes = 16u << g.v.log2K;
+                    mbar_arrive_expect_tx(sm.cb_full(h), bytes);
+                    bulk_g2s(sm.cbraw0 + h * sm.cbraw_bytes, g.v.cb, bytes, sm.cb_full(h));
+                }
+                cur_cb = g.v.cb;
+                ++ncb;
+            }
+            const int nc = n_chunks(g), G = g.v.d_in >> 7;
+            for (int c = 0; c < nc; ++c, ++t, ring_next(slot, ph, sm.slots)) {
+                if (throttled && t >= kStartChunks) {  // until the first window is gathered
+                    for (uint32_t i = 0; i < kWaitLimit && !*reinterpret_cast<volatile int*>(sm.misc + 10); ++i) {
+                        if (*sm.abort_flag()) break;
+                        __nanosleep(64);
+                    }
+                    throttled = false;
+                }
+                if (t >= sm.slots) wait_bar(sm, sm.empty(slot), ph ^ 1, status);
+                if (lane == 0) {
+                    const int2 cc = chunk_cols(g, c);
+                    const int ng = ((cc.y - 1) >> 4) - (cc.x >> 4) + 1;  // radius groups the chunk touches
+                    const uint32_t mb = (uint32_t)((cc.y - cc.x) * g.n_oct * 16), tb = (uint32_t)(ng * g.n_oct * 64);
+                    mbar_arrive_expect_tx(sm.full(slot), mb + tb);
+                    bulk_g2s_stream(sm.slot_addr(slot), g.v.main + main_word(g.v.R8, g.v.S, g.blk, cc.x, 0, 0), mb,
+                                    sm.full(slot), pol);
+                    bulk_g2s_stream(sm.slot_addr(slot) + kMainSlot,
+                                    g.v.meta + 2 * meta_entry(g.v.R8, G, g.blk, cc.x >> 4, 0, 0), tb, sm.full(slot), pol);
+                }
+            }
+        }
+    }
+    // the CTA may not exit while bulk copies are in flight
+    for (int k = max(0, t - sm.slots); k < t; ++k) wait_bar(sm, sm.full(k % sm.slots), (k / sm.slots) & 1, status);
+}
+
+// ------------------------------------------------------------------------
+// Activation gather (with the fused prologues)
+// ------------------------------------------------------------------------
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+__device__ __forceinline__ uint16_t ld16(const uint16_t* p, bool coherent) {
+    return coherent ? __ldcg(reinterpret_cast<const unsigned short*>(p)) : __ldg(reinterpret_cast<const unsigned short*>(p));
+}
+
+// Value of input channel c of batch row m after the stage's prologue (fp16 bits).
+template <class Src>
+__device__ __forceinline__ uint16_t prologue_value(const EngineStage& st, const JobView& v, int xr, int c, float inv,
+                                                   bool coh) {
+    switch (st.pro) {
+        case kProPlain:
+            return ld16(v.x + (size_t)xr * v.d_in + c, coh);
+        case kProRmsNorm: {
+            const float a = h2f(ld16(st.pa + (size_t)xr * st.pro_dim + c, coh));
+            return f2h(a * h2f(ld16(st.pg + c, false)) * inv);
+        }
+        case kProResidRmsNorm: {
+            const uint16_t r = f2h(h2f(ld16(st.pa + (size_t)xr * st.pro_dim + c, coh)) +
+                                   h2f(ld16(st.pb + (size_t)xr * st.pro_dim + c, coh)));
+            return f2h(h2f(r) * h2f(ld16(st.pg + c, false)) * inv);
+        }
+        case kProSiluMul: {
+            const float gt = h2f(ld16(st.pa + (size_t)xr * st.pro_dim + c, coh));
+            const float up = h2f(ld16(st.pb + (size_t)xr * st.pro_dim + c, coh));
+            return f2h(gt / (1.0f + expf(-gt)) * up);
+        }
+        default: {  // kProGqa: attention over one cached position returns the value row of the KV head
+            const int hd = st.gqa_hd, grp = st.gqa_grp;
+            const int src_c = (c / (hd * grp)) * hd + c % hd;
+            return ld16(st.pa + (size_t)xr * st.pro_dim + src_c, coh);
+        }
     }
 }
 
-// Per-role progress that persists across segment-table rounds.
-struct RoleState {
-    int t;      // chunk counter
-    int slot;   // ring slot of chunk t (t % slots, kept incrementally)
-    int ph;     // phase parity of that slot for chunk t ((t / slots) & 1)
-    int s;      // segment counter (codebook phases)
-    WinPos w;   // activation window placement
-    int cur_win;  // decode warps: the x window they hold (-1: none)
-};
-
-// ------------------------------------------------------------------------
-// Copy warp: bulk copies of codebooks and code chunks into the ring, issued
-// as far ahead as the ring allows (before and independent of the wait on the
-// preceding kernel: nothing it reads is written by that kernel).
-// ------------------------------------------------------------------------
+// 1 / sqrt(mean(v^2) + eps) of each batch row of the prologue's source vector
+// (RMSNorm), computed by the `nt` threads of a cooperative gather in a fixed
+// order (deterministic).  Only the first window of a stage needs it.
 template <int M>
-__device__ __forceinline__ void copy_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st,
-                                          bool first_round) {
-    const int lane = threadIdx.x & 31;
-    for (int si = 0; si < n_seg; ++si, ++st.s) {
-        const Seg& g = sm.segs[si];
-        const int s = st.s;
-        if (s >= 2) wait_bar(sm.cb_empty(s & 1), ((s >> 1) - 1) & 1, C);
-        const uint32_t cbb = (uint32_t)(16u << g.v.log2K);
-        if (lane == 0) {
-            mbar_arrive_expect_tx(sm.cb_full(s & 1), cbb);
-            bulk_g2s(sm.cbraw0 + (s & 1) * sm.cbraw_bytes, g.v.cb, cbb, sm.cb_full(s & 1));
+__device__ void rms_rows(const Smem& sm, const EngineStage& st, int tid, int nt, bool coh) {
+    float part[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) part[m] = 0.f;
+    for (int c = tid; c < st.pro_dim; c += nt) {
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            float a = h2f(ld16(st.pa + (size_t)m * st.pro_dim + c, coh));
+            if (st.pro == kProResidRmsNorm) a = h2f(f2h(a + h2f(ld16(st.pb + (size_t)m * st.pro_dim + c, coh))));
+            part[m] = fmaf(a, a, part[m]);
         }
-        // the first codebook goes first; then the first window's permutation
-        // entries (activation warp) ahead of the code chunks
-        if (first_round && si == 0) named_barrier(kBarPermIssued, 64);
-        const int n_oct = g.n_oct, R8 = g.v.R8, S = g.v.S, G = g.v.d_in >> 7, blk = g.blk;
-        for (int c = 0; c < g.n_chunks; ++c, ++st.t, ring_next(st.slot, st.ph, sm.slots)) {
-            const int k = st.slot;
-            if (st.t >= sm.slots) wait_bar(sm.empty(k), st.ph ^ 1, C);
-            if (lane == 0) {
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+        for (int o = 16; o; o >>= 1) part[m] += __shfl_xor_sync(0xffffffffu, part[m], o);
+    const int wid = tid >> 5;
+    if ((tid & 31) == 0)
+#pragma unroll
+        for (int m = 0; m < M; ++m) sm.red[wid * 8 + m] = part[m];
+    named_barrier(kBarGather, kGT);
+    if (tid < M) {
+        float t = 0.f;
+        for (int w = 0; w < nt / 32; ++w) t += sm.red[w * 8 + tid];
+        sm.inv_rms[tid] = rsqrtf(t / (float)st.pro_dim + st.eps);
+    }
+}
+
+// Gathers the window's x_perm for items e = tid, tid + nt, ... of (batch row,
+// position) and stores them (fp16, unscaled) into the window buffer; returns
+// the largest |x| bit pattern seen.
+template <int M, class Src>
+__device__ uint32_t gather_items(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid, int nt,
+                                 bool coh) {
+    const EngineStage& st = src.stage(s);
+    const int mrows = sm.misc[9];  // batch rows a window holds (<= M)
+    uint32_t mx = 0;
+    for (int e = tid; e < mrows * wlen; e += nt) {
+        const int m = e / wlen, p = e - m * wlen;
+        const uint32_t info = sm.posinfo[p];
+        const JobView v = src.job((int)(info >> 20));
+        const int j = (int)(info & 0xfffffu);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (m < v.Mk) {
+            const int xr = v.xrows ? v.xrows[m] : m;
+            const float inv = sm.inv_rms[m < 8 ? m : 0];
+            if (st.pro == kProPlain && !v.perm) {
+                const uint16_t* row = v.x + (size_t)xr * v.d_in + j * 8;
+                val = coh ? __ldcg(reinterpret_cast<const uint4*>(row)) : __ldg(reinterpret_cast<const uint4*>(row));
+            } else {
+                uint32_t h[8];
+                if (v.perm) {
+                    const uint4 pa = lds128(sm.perm0 + p * 32), pb = lds128(sm.perm0 + p * 32 + 16);
+                    const int cs[8] = {(int)pa.x, (int)pa.y, (int)pa.z, (int)pa.w, (int)pb.x, (int)pb.y, (int)pb.z, (int)pb.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) h[i] = prologue_value<Src>(st, v, xr, cs[i], inv, coh);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) h[i] = prologue_value<Src>(st, v, xr, j * 8 + i, inv, coh);
+                }
+                val = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+            }
+        }
+        sts128(xb + (uint32_t)(m * xw + p) * 16, val);
+        const uint32_t a = __vmaxu2(__vmaxu2(val.x & 0x7fff7fffu, val.y & 0x7fff7fffu),
+                                    __vmaxu2(val.z & 0x7fff7fffu, val.w & 0x7fff7fffu));
+        mx = max(mx, max(a & 0xffffu, a >> 16));
+    }
+    return mx;
+}
+
+// Power-of-two prescale of a window: k such that every |x| / 2^k <= 2^14, so
+// that no partial sum of a subvector's eight fp16 products (sum of |c_i| <= 2
+// per half2 lane, <= 2 sqrt 2 in all) can leave the fp16 range.
+__device__ __forceinline__ int window_shift(uint32_t maxbits) {
+    return maxbits <= 0x7400u ? 0 : maxbits <= 0x7800u ? 1 : 2;  // 2^14, 2^15, larger (<= 65504)
+}
+
+// Scales window items by 2^-k in place (only windows with very large |x|).
+template <int M>
+__device__ void rescale_items(const Smem& sm, int wlen, int xw, uint32_t xb, int k, int tid, int nt) {
+    const __half2 f = __float2half2_rn(k == 1 ? 0.5f : 0.25f);
+    for (int e = tid; e < sm.misc[9] * wlen; e += nt) {
+        const int m = e / wlen, p = e - m * wlen;
+        const uint32_t a = xb + (uint32_t)(m * xw + p) * 16;
+        uint4 v = lds128(a);
+        v.x = h22u(__hmul2(u2h2(v.x), f));
+        v.y = h22u(__hmul2(u2h2(v.y), f));
+        v.z = h22u(__hmul2(u2h2(v.z), f));
+        v.w = h22u(__hmul2(u2h2(v.w), f));
+        sts128(a, v);
+    }
+}
+
+// The cooperative part of a stage's first window, run by the gather warp and
+// the decode warps together (tid in [0, kGT)).
+template <int M, class Src>
+__device__ void coop_window(const Src& src, const Smem& sm, int s, int w, int xw, bool coh, int tid) {
+    const EngineStage& st = src.stage(s);
+    named_barrier(kBarGather, kGT);  // inputs ready, permutation entries landed, buffer free
+    if (st.pro == kProRmsNorm || st.pro == kProResidRmsNorm) {
+        rms_rows<M>(sm, st, tid, kGT, coh);
+        named_barrier(kBarGather, kGT);
+    }
+    const int wlen = sm.misc[8];
+    const uint32_t mx = gather_items<M>(src, sm, s, wlen, xw, sm.xwin(w), tid, kGT, coh);
+    atomicMax(reinterpret_cast<unsigned*>(sm.misc + 3), mx);
+    named_barrier(kBarGather, kGT);
+    const int k = window_shift((uint32_t)sm.misc[3]);
+    if (k) {
+        rescale_items<M>(sm, wlen, xw, sm.xwin(w), k, tid, kGT);
+    }
+    if (tid == 0) sm.misc[w & 1] = k;
+    named_barrier(kBarGather, kGT);
+}
+
+// Loads the permutation entries of the window's positions into the shared
+// buffer with plain loads (a bulk copy would queue behind the code chunks
+// already in the CTA's copy queue).  posperm holds each position's source.
+__device__ void load_perm(const Smem& sm, int wlen, int lane) {
+    __syncwarp();  // every lane's position entries are written
+    for (int q0 = 0; q0 < 2 * wlen; q0 += 32 * 8) {
+        uint4 v[8];
+        int dst[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int q = q0 + r * 32 + lane;
+            dst[r] = -1;
+            if (q < 2 * wlen) {
+                const int32_t* pm = sm.posperm[q >> 1];
+                if (pm) {
+                    v[r] = __ldg(reinterpret_cast<const uint4*>(pm + (q & 1) * 4));
+                    dst[r] = q;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            if (dst[r] >= 0) sts128(sm.perm0 + (uint32_t)dst[r] * 16, v[r]);
+    }
+    __syncwarp();
+}
+
+// Fills window `win` (wlen positions, recorded in posinfo) of stage s.
+template <int M, class Src>
+__device__ __noinline__ void fill_window(const Src& src, const Smem& sm, uint32_t* status, unsigned* sync, int s,
+                                         int win, int wlen, int xw, bool first, bool need_pdl) {
+    const int lane = threadIdx.x & 31;
+    const EngineStage& st = src.stage(s);
+    load_perm(sm, wlen, lane);  // static data: before any wait on earlier work
+    if (need_pdl) pdl_wait();        // inputs may come from the preceding kernel
+    if (first && st.wait) {
+        if (lane == 0) wait_count(sm, sync + kSyncStageDone + (s - 1), src.stage(s - 1).blocks, status);
+        __syncwarp();
+    }
+    if (win >= 2) wait_bar(sm, sm.x_empty(win & 1), ((win >> 1) - 1) & 1, status);
+    const bool coh = st.wait != 0;
+    if (lane == 0) {
+        sm.misc[8] = wlen;
+        sm.misc[3] = 0;
+    }
+    __syncwarp();
+    if (first) {
+        coop_window<M>(src, sm, s, win, xw, coh, kDT + lane);
+        if (lane == 0) *reinterpret_cast<volatile int*>(sm.misc + 10) = 1;  // release the copy warp
+    } else {
+        uint32_t mx = gather_items<M>(src, sm, s, wlen, xw, sm.xwin(win), lane, 32, coh);
+        for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const int k = window_shift(mx);
+        __syncwarp();
+        if (k) rescale_items<M>(sm, wlen, xw, sm.xwin(win), k, lane, 32);
+        if (lane == 0) sm.misc[win & 1] = k;
+        __syncwarp();
+    }
+    mbar_arrive(sm.x_full(win & 1));  // all 32 lanes, each after its own stores
+}
+
+template <int M, class Src>
+__device__ void gather_role(const Src& src, const Smem& sm, uint32_t* status, unsigned* sync, int n_cta, int xw,
+                            bool waited) {
+    const int lane = threadIdx.x & 31;
+    WinPos wp{0, 0};
+    for (int s = 0; s < src.n_stages(); ++s) {
+        const int U = src.units(s);
+        if (U <= 0) continue;
+        const int u0 = cta_begin(U, n_cta, blockIdx.x), u1 = cta_begin(U, n_cta, blockIdx.x + 1);
+        win_break(wp);
+        // walk the stage's chunks; a window is filled when the next chunk opens a new one (or at the end)
+        int wlen = 0, cur = -1;
+        bool first = true;
+        for (int u = u0; u < u1;) {
+            const Seg g = make_seg(src, s, u, u1);
+            u += g.jb - g.ja;
+            const int nc = n_chunks(g);
+            for (int c = 0; c < nc; ++c) {
                 const int2 cc = chunk_cols(g, c);
                 const int nj = cc.y - cc.x;
-                const uint32_t mb = (uint32_t)(nj * n_oct * 16), tb = (uint32_t)(n_oct * 64);
-                mbar_arrive_expect_tx(sm.full(k), mb + tb);
-                // the chunk's records: one contiguous range of the block; its group's meta entries
-                const uint64_t pol = l2_evict_first();
-                bulk_g2s_stream(sm.slot_addr(k), g.v.main + main_word(R8, S, blk, cc.x, 0, 0), mb, sm.full(k), pol);
-                bulk_g2s_stream(sm.slot_addr(k) + kMainSlot, g.v.meta + 2 * meta_entry(R8, G, blk, cc.x >> 4, 0, 0),
-                                tb, sm.full(k), pol);
-            }
-        }
-    }
-}
-
-// The CTA may not exit while bulk copies are in flight.
-template <int M>
-__device__ void copy_drain(const Common& C, const Smem<M>& sm, const RoleState& st) {
-    for (int t = max(0, st.t - sm.slots); t < st.t; ++t) wait_bar(sm.full(t % sm.slots), (t / sm.slots) & 1, C);
-}
-
-// ------------------------------------------------------------------------
-// Activation warp: x_perm[m][p] = x[m][perm[p]] for one window of columns
-// (Sec. 3.5 fuses this gather into the decode GEMV).  The permutation entries
-// are bulk-copied first -- for the first window before the wait on the
-// preceding kernel, since only x comes from that kernel -- so after the wait
-// the gather costs one round trip per window.
-// ------------------------------------------------------------------------
-// Gathers x_perm for window positions e = gi, gi + gn, ... of the (batch row,
-// position) pairs of a window of wlen positions into the window buffer xb.
-// All loads of a round are issued before any store.
-template <int M, int B>
-__device__ __forceinline__ void gather_x(const Smem<M>& sm, int wlen, uint32_t xb, int gi, int gn) {
-    constexpr int XW = Cfg<M>::kXW;
-    const int total = M * wlen;
-    for (int e0 = 0; e0 < total; e0 += B * gn) {
-        uint4 val[B];
-        uint32_t dst[B];
-#pragma unroll
-        for (int r = 0; r < B; ++r) {
-            const int e = e0 + r * gn + gi;
-            dst[r] = 0xffffffffu;
-            if (e < total) {
-                const int m = e / wlen, p = e - m * wlen;
-                const uint32_t info = sm.posinfo[p];
-                const Seg& g = sm.segs[info >> 24];
-                const int j = (int)(info & 0xffffffu);
-                if (m < g.v.Mk) {
-                    const int xr_idx = g.v.xrows ? row_at(g.v.xrows, m) : m;
-                    const unsigned short* xr =
-                        reinterpret_cast<const unsigned short*>(g.v.x) + (size_t)xr_idx * g.v.d_in;
-                    // x is read-only while this kernel runs and is first read here,
-                    // after the wait on the kernel that wrote it: the scattered
-                    // 2-byte reads go through L1, which holds the whole row.
-                    if (g.v.perm) {
-                        const uint32_t sp = sm.perm0 + p * 32;
-                        const uint4 pa = lds128(sp), pb = lds128(sp + 16);
-                        val[r].x = (uint32_t)__ldg(xr + pa.x) | ((uint32_t)__ldg(xr + pa.y) << 16);
-                        val[r].y = (uint32_t)__ldg(xr + pa.z) | ((uint32_t)__ldg(xr + pa.w) << 16);
-                        val[r].z = (uint32_t)__ldg(xr + pb.x) | ((uint32_t)__ldg(xr + pb.y) << 16);
-                        val[r].w = (uint32_t)__ldg(xr + pb.z) | ((uint32_t)__ldg(xr + pb.w) << 16);
-                    } else {
-                        val[r] = __ldg(reinterpret_cast<const uint4*>(xr + j * 8));
+                const int pos = win_place(wp, nj, xw);
+                if (wp.win != cur) {
+                    if (cur >= 0) {
+                        fill_window<M>(src, sm, status, sync, s, cur, wlen, xw, first, !waited);
+                        waited = true;
+                        first = false;
                     }
-                    dst[r] = xb + (m * XW + p) * 16;
+                    cur = wp.win;
+                    wlen = 0;
+                    __syncwarp();  // the filled window's positions are no longer read
                 }
+                if (lane < nj) {
+                    sm.posinfo[pos + lane] = ((uint32_t)g.v.id << 20) | (uint32_t)(cc.x + lane);
+                    sm.posperm[pos + lane] = g.v.perm ? g.v.perm + (size_t)(cc.x + lane) * 8 : nullptr;
+                }
+                wlen = pos + nj;
             }
         }
+        if (cur >= 0) {
+            fill_window<M>(src, sm, status, sync, s, cur, wlen, xw, first, !waited);
+            waited = true;
+        }
+    }
+    if (!waited) pdl_wait();
+}
+
+// ------------------------------------------------------------------------
+// Decode warps
+// ------------------------------------------------------------------------
+// (s (.) c) . x for one subvector: four half2 products with fp16 accumulation
+// (Fig. 6a), the two halves added in fp16, returned as fp32.
+__device__ __forceinline__ float sdot(uint4 c, uint4 x) {
+    __half2 h = __hmul2(u2h2(c.x), u2h2(x.x));
+    h = __hfma2(u2h2(c.y), u2h2(x.y), h);
+    h = __hfma2(u2h2(c.z), u2h2(x.z), h);
+    h = __hfma2(u2h2(c.w), u2h2(x.w), h);
+    return __half2float(__hadd(__low2half(h), __high2half(h)));
+}
+
+struct RowPair {
+    float mpA, dlA, mpB, dlB;   // r = mp + dl * (1 + q / 2^V)  (Eq. 2)
+    uint32_t auxA, auxB;        // component 6/7 signs of the group's 16 subvectors
+};
+
+// Decodes column t (position within the radius group) of both rows of a
+// record word w against the batch rows' x_perm values.  The shifts that line
+// sign bits up with the fp16 sign positions are integer multiplies by powers
+// of two held in registers (d.m*): they issue on the FMA pipe, which the
+// fp16 dot products leave room on, instead of the integer ALU pipe that the
+// masks and field extraction already load.
+template <int MK>
+__device__ __forceinline__ void decode_word(const VDec& d, uint32_t lane_off, uint32_t w, int t, const RowPair& rp,
+                                            const uint4 (&xv)[MK], float (&accA)[MK], float (&accB)[MK]) {
+    {   // row A: z at [7, 7 + log2K), q at [23 - V, 23); signs in slots 0..2 and aux
+        uint4 c = cw_load((w & d.zmask) | lane_off);
+        c.x ^= (w * d.m0) & 0x80008000u;
+        c.y ^= (w * d.m1) & 0x80008000u;
+        c.z ^= (w * d.m2) & 0x80008000u;
+        c.w ^= (rp.auxA << (15 - t)) & 0x80008000u;
+        const float r = fmaf(__uint_as_float((w & d.qmask) | 0x3F800000u), rp.dlA, rp.mpA);
 #pragma unroll
-        for (int r = 0; r < B; ++r)
-            if (dst[r] != 0xffffffffu) sts128(dst[r], val[r]);
+        for (int m = 0; m < MK; ++m) accA[m] = fmaf(r, sdot(c, xv[m]), accA[m]);
+    }
+    {   // row B: its fields sit 16 bits higher (z, from w >> 16) and lower (q, from w << 16);
+        // signs in slots 3..5 (slot 5 at bit 15) and aux
+        const uint32_t whi = __umulhi(w, d.m16), wlo = w * d.m16;
+        uint4 c = cw_load((whi & d.zmask) | lane_off);
+        c.x ^= (w * d.m3) & 0x80008000u;
+        c.y ^= (w * d.m4) & 0x80008000u;
+        c.z ^= w & 0x80008000u;
+        c.w ^= (rp.auxB << (15 - t)) & 0x80008000u;
+        const float r = fmaf(__uint_as_float((wlo & d.qmask) | 0x3F800000u), rp.dlB, rp.mpB);
+#pragma unroll
+        for (int m = 0; m < MK; ++m) accB[m] = fmaf(r, sdot(c, xv[m]), accB[m]);
     }
 }
 
-
-template <int M>
-__device__ __forceinline__ void fill_window(const Common& C, const Smem<M>& sm, int w, int si0, int c0, int nch, bool& waited) {
-    const int lane = threadIdx.x & 31;
-    fence_proxy_async_smem();  // earlier reads of the permutation buffer precede the copies below
-    int si = si0, c = c0, wlen = 0;
-    for (int k = 0; k < nch; ++k) {
-        const Seg& g = sm.segs[si];
-        const int2 cc = chunk_cols(g, c);
-        const int nj = cc.y - cc.x;
-        if (g.v.perm && lane == 0) {
-            mbar_expect_tx(sm.perm_full(), (uint32_t)(nj * 32));
-            bulk_g2s(sm.perm0 + wlen * 32, g.v.perm + cc.x * 8, (uint32_t)(nj * 32), sm.perm_full());
+// Decodes this thread's columns of one chunk (ring slot k) into accA/accB:
+// the thread's two rows, in radius group `ch` of the chunk.  xw0: shared
+// address of the chunk's first column in its window (batch row stride
+// xstride bytes); sc: 2^k of the window's prescale.
+template <int MK>
+__device__ __forceinline__ void decode_chunk(const Smem& sm, const Seg& g, const VDec& d, int k, int2 cc,
+                                             uint32_t xw0, uint32_t xstride, float sc, int warp, int lane,
+                                             float (&accA)[MK], float (&accB)[MK]) {
+    const int u = 32 * (warp & 3) + lane, o = u >> 2, wi = u & 3, part = warp >> 2;
+    const int gfirst = cc.x >> 4;
+    const int grp = ((cc.x >> 5) << 1) + part;           // this thread's radius group
+    const int lo = max(cc.x, grp << 4), hi = min(cc.y, (grp + 1) << 4);
+    if (o >= g.n_oct || lo >= hi) return;
+    const uint32_t base = sm.slot_addr(k);
+    RowPair rp;
+    {
+        const uint4 mt = lds128(base + kMainSlot + (uint32_t)(((grp - gfirst) * g.n_oct + o) * 64 + wi * 16));
+        const float2 a = __half22float2(u2h2(mt.y)), b = __half22float2(u2h2(mt.w));
+        rp.dlA = a.y * d.vscale * sc;
+        rp.mpA = a.x * sc - rp.dlA;
+        rp.dlB = b.y * d.vscale * sc;
+        rp.mpB = b.x * sc - rp.dlB;
+        rp.auxA = mt.x;
+        rp.auxB = mt.z;
+    }
+    const uint32_t lane_off = (uint32_t)(lane & 7) << 4;  // this lane's replica
+    const uint32_t rstride = (uint32_t)g.n_oct * 16;
+    const uint32_t wbase = base + (uint32_t)(o * 16 + wi * 4) + (uint32_t)(lo - cc.x) * rstride;
+    const uint32_t xbase = xw0 + (uint32_t)(lo - cc.x) * 16;
+    if (hi - lo == 16) {  // a whole radius group: fixed trip count, constant shifts
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const uint32_t w = lds32(wbase + (uint32_t)t * rstride);
+            uint4 xv[MK];
+#pragma unroll
+            for (int m = 0; m < MK; ++m) xv[m] = lds128(xbase + (uint32_t)m * xstride + (uint32_t)t * 16);
+            decode_word<MK>(d, lane_off, w, t, rp, xv, accA, accB);
         }
-        if (lane < nj) sm.posinfo[wlen + lane] = ((uint32_t)si << 24) | (uint32_t)(cc.x + lane);
-        wlen += nj;
-        if (++c == g.n_chunks) { c = 0; ++si; }
-    }
-    if (lane == 0) mbar_arrive(sm.perm_full());
-    // The first window's permutation entries go ahead of the code chunks in the
-    // copy queue: the copy warp starts once they are issued.
-    if (w == 0) named_barrier(kBarPermIssued, 64);
-    if (!waited) {
-        pdl_wait();  // x may be written by the preceding kernel
-        waited = true;
-    }
-    wait_bar(sm.perm_full(), w & 1, C);
-    if (w >= 2) wait_bar(sm.x_empty(w & 1), ((w >> 1) - 1) & 1, C);
-    __syncwarp();
-    if (w == 0) {  // the decode warps, idle until now, help with the first window
-        if (lane == 0) *sm.wlen0 = wlen;
-        named_barrier(kBarFirstWindow, 32 + Cfg<M>::kDecodeThreads);
-        gather_x<M, 2>(sm, wlen, sm.xwin(0), Cfg<M>::kDecodeThreads + lane, 32 + Cfg<M>::kDecodeThreads);
-        named_barrier(kBarFirstWindow, 32 + Cfg<M>::kDecodeThreads);
     } else {
-        gather_x<M, 8>(sm, wlen, sm.xwin(w), lane, 32);
-    }
-    mbar_arrive(sm.x_full(w & 1));  // all 32 lanes, each after its own stores
-}
-
-template <int M>
-__device__ __forceinline__ void act_warp(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st, bool& waited) {
-    win_break(st.w);
-    int pend = -1, si0 = 0, c0 = 0, nch = 0;
-    for (int si = 0; si < n_seg; ++si) {
-        const Seg& g = sm.segs[si];
-        for (int c = 0; c < g.n_chunks; ++c) {
-            const int2 cc = chunk_cols(g, c);
-            win_place(st.w, cc.y - cc.x, Cfg<M>::kXW);
-            if (st.w.win != pend) {
-                if (nch) fill_window<M>(C, sm, pend, si0, c0, nch, waited);
-                pend = st.w.win;
-                si0 = si;
-                c0 = c;
-                nch = 0;
-            }
-            ++nch;
-        }
-    }
-    if (nch) fill_window<M>(C, sm, pend, si0, c0, nch, waited);
-}
-
-// ------------------------------------------------------------------------
-// Decode warps.
-// ------------------------------------------------------------------------
-template <int M>
-__device__ __forceinline__ void decode_record(const VDec& d, uint4 rec, const uint32_t (&aux)[8], uint32_t sh_aux,
-                                              const float (&mup)[8], const float (&dlp)[8], uint32_t cbsel,
-                                              const uint4 (&xv)[M], float (&acc)[8][M]) {
-    const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const uint32_t wa = wv[u];
-        const uint32_t wb = rot16(wa);
-        {   // row A = 2u: z at [7, 7 + log2K), q at [23 - V, 23) of wa; signs in slots 0..2
-            uint4 c = lds128(cbsel + (wa & d.zmask));
-            c.x ^= (wa << d.sh0) & 0x80008000u;
-            c.y ^= (wa << d.sh1) & 0x80008000u;
-            c.z ^= (wa << d.sh2) & 0x80008000u;
-            c.w ^= (aux[2 * u] << sh_aux) & 0x80008000u;
-            const float r = fmaf(__uint_as_float((wa & d.qmask) | 0x3F800000u), dlp[2 * u], mup[2 * u]);
-#pragma unroll
-            for (int m = 0; m < M; ++m) acc[2 * u][m] = fmaf(r, signed_dot(c, xv[m]), acc[2 * u][m]);
-        }
-        {   // row B = 2u + 1: the same fields after a 16-bit rotation; signs in slots 3..5
-            uint4 c = lds128(cbsel + (wb & d.zmask));
-            c.x ^= (wa << d.sh3) & 0x80008000u;
-            c.y ^= (wa << d.sh4) & 0x80008000u;
-            c.z ^= wa & 0x80008000u;  // slot 5 sits at bit 15 for every split
-            c.w ^= (aux[2 * u + 1] << sh_aux) & 0x80008000u;
-            const float r = fmaf(__uint_as_float((wb & d.qmask) | 0x3F800000u), dlp[2 * u + 1], mup[2 * u + 1]);
-#pragma unroll
-            for (int m = 0; m < M; ++m)
-                acc[2 * u + 1][m] = fmaf(r, signed_dot(c, xv[m]), acc[2 * u + 1][m]);
-        }
-    }
-}
-
-// Decodes this warp's columns of one ring chunk (chunk c of segment g, in
-// ring slot k with phase parity ph): columns lw, lw + wpg, ... of the chunk,
-// against the x_perm window at xw, where the chunk's first column sits at
-// window position pos.
-template <int M, int MS>
-__device__ __forceinline__ void decode_chunk(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int k,
-                                             int ph, int c, uint32_t xw, int pos, int lw, int wpg, int lane,
-                                             float (&acc)[8][M]) {
-    constexpr int XW = Cfg<MS>::kXW;
-    const int2 cc = chunk_cols(g, c);
-    const int nj = cc.y - cc.x;
-    wait_bar(sm.full(k), ph, C);
-    const int n_oct = g.n_oct;
-    if (lw < nj && lane < n_oct) {
-        const uint32_t base = sm.slot_addr(k);
-        const uint32_t cbsel = sm.cb0 + ((uint32_t)(lane & 7) << 4);
-        uint32_t aux[8];
-        float mup[8], dlp[8];
-        {   // the group's grid and aux signs for this lane's 8 rows
-            uint4 q[4];
-            load_meta(base + kMainSlot + lane * 64, lane, q);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                aux[2 * e] = q[e].x;
-                aux[2 * e + 1] = q[e].z;
-                const float2 m0 = __half22float2(u2h2(q[e].y));
-                const float2 m1 = __half22float2(u2h2(q[e].w));
-                dlp[2 * e] = m0.y * d.vscale;
-                mup[2 * e] = m0.x - dlp[2 * e];
-                dlp[2 * e + 1] = m1.y * d.vscale;
-                mup[2 * e + 1] = m1.x - dlp[2 * e + 1];
-            }
-        }
-        auto column = [&](int i) {
-            const int j = cc.x + i;
-            const uint4 rec = lds128(base + (i * n_oct + lane) * 16);
-            uint4 xv[M];
-#pragma unroll
-            for (int m = 0; m < M; ++m) xv[m] = lds128(xw + (m * XW + pos + i) * 16);
-            decode_record<M>(d, rec, aux, (uint32_t)(15 - (j & 15)), mup, dlp, cbsel, xv, acc);
-        };
-        if constexpr (M <= 4) {  // two columns in flight where registers allow
 #pragma unroll 2
-            for (int i = lw; i < nj; i += wpg) column(i);
-        } else {
-#pragma unroll 1
-            for (int i = lw; i < nj; i += wpg) column(i);
+        for (int j = lo; j < hi; ++j) {
+            const uint32_t r = (uint32_t)(j - lo);
+            const uint32_t w = lds32(wbase + r * rstride);
+            uint4 xv[MK];
+#pragma unroll
+            for (int m = 0; m < MK; ++m) xv[m] = lds128(xbase + (uint32_t)m * xstride + r * 16);
+            decode_word<MK>(d, lane_off, w, j & 15, rp, xv, accA, accB);
         }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.empty(k));
 }
 
-// Decodes one ring chunk (chunk c of segment g, ring slot k, phase parity ph)
-// with one thread per row of the 256-row block: row 32 warp + lane, i.e. the
-// 8 lanes of a quarter warp hold the 8 rows of one octet.  Per row the grid
-// and aux signs are one 8-byte entry; per (row, column) the fields are the
-// row's half of one record word, and the codeword comes from the replica of
-// the row's position in its octet (no bank conflicts).  acc[m] accumulates the
-// row's output for batch row m.
-template <int M, int MS>
-__device__ __forceinline__ void decode_rows(const Smem<MS>& sm, const Common& C, const Seg& g, const VDec& d, int k,
-                                            int ph, int c, uint32_t xw, int pos, int warp, int lane, float (&acc)[M]) {
-    constexpr int XW = Cfg<MS>::kXW;
-    const int2 cc = chunk_cols(g, c);
-    const int nj = cc.y - cc.x;
-    wait_bar(sm.full(k), ph, C);
-    const int n_oct = g.n_oct;
-    const int o = (warp << 2) + (lane >> 3), tr = lane & 7;
-    if (o < n_oct) {
-        const uint32_t base = sm.slot_addr(k);
-        const uint2 e = lds64(base + kMainSlot + (uint32_t)(o * 8 + tr) * 8);
-        const float2 md = __half22float2(u2h2(e.y));
-        const float dl = md.y * d.vscale, mp = md.x - dl;
-        const uint32_t aux = e.x;
-        const bool odd = tr & 1;
-        const uint32_t s0 = odd ? d.sh3 : d.sh0, s1 = odd ? d.sh4 : d.sh1, s2 = odd ? d.sh5 : d.sh2;
-        const uint32_t cbsel = sm.cb0 + ((uint32_t)tr << 4);
-        const uint32_t wbase = base + (uint32_t)o * 16 + (uint32_t)(tr >> 1) * 4;
-        const uint32_t rstride = (uint32_t)n_oct * 16;
-        const uint32_t xbase = xw + (uint32_t)pos * 16;
-        // column i of the chunk; its sign bit 7 is aux bit (cc.x + i) % 16
-        auto column = [&](int i, uint32_t aux_shift) {
-            const uint32_t w = lds32(wbase + (uint32_t)i * rstride);
-            const uint32_t wf = odd ? rot16(w) : w;  // (z, q) field word of this row
-            uint4 cw = lds128(cbsel + (wf & d.zmask));
-            cw.x ^= (w << s0) & 0x80008000u;
-            cw.y ^= (w << s1) & 0x80008000u;
-            cw.z ^= (w << s2) & 0x80008000u;
-            cw.w ^= (aux << aux_shift) & 0x80008000u;
-            const float r = fmaf(__uint_as_float((wf & d.qmask) | 0x3F800000u), dl, mp);
+__device__ __forceinline__ void write_out(const EngineStage& st, const JobView& v, int m, int row, float tot) {
+    const int yr = v.yrows ? v.yrows[m] : m;
+    const uint16_t yb = f2h(tot);
+    v.y[(size_t)yr * v.d_out + row] = yb;
+    if (st.epi == kEpiResidual) {  // layer output: fp16(fp16(ea + eb) + y)
+        const size_t i = (size_t)yr * v.d_out + row;
+        const uint16_t r = f2h(h2f(__ldcg(reinterpret_cast<const unsigned short*>(st.ea + i))) +
+                               h2f(__ldcg(reinterpret_cast<const unsigned short*>(st.eb + i))));
+        st.eo[i] = f2h(h2f(r) + h2f(yb));
+    }
+}
+
+// Epilogue warp: writes (or combines) the outputs of the segments the decode
+// warps hand over through the stash ring, so that the decode warps never wait
+// on global-memory round trips.  Whole blocks are written directly.  Split
+// blocks: every contributor stores its partial sums and publishes them with
+// one acquire-release increment of the block's count; the contributor that
+// completes the count adds all partials in CTA order.  Blocks whose outputs
+// are final are added to the stage's completion count when a later stage of
+// the launch reads them.
+template <int M, class Src>
+__device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P) {
+    const int lane = threadIdx.x & 31;
+    constexpr int NS = Cfg<M>::kSlots;
+    int n = 0;  // segment counter (stash slot n % NS)
+    for (int s = 0; s < src.n_stages(); ++s) {
+        const int U = src.units(s);
+        if (U <= 0) continue;
+        const int u0 = cta_begin(U, P.n_cta, blockIdx.x), u1 = cta_begin(U, P.n_cta, blockIdx.x + 1);
+        const bool signal = s + 1 < src.n_stages() && src.stage(s + 1).wait;
+        unsigned done = 0;
+        for (int uu = u0; uu < u1; ++n) {
+            const int k = n % NS;
+            wait_bar(sm, sm.st_full(k), (n / NS) & 1, P.status);
+            const Pending& q = sm.pend[k];
+            const Seg& g = q.g;
+            uu += g.jb - g.ja;
+            const float* stk = sm.stash + (size_t)k * kParts * M * kBlockRows;
+            // the column parts of a row, added in part order
+            auto part_sum = [&](int m, int r) {
+                float t = 0.f;
 #pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const uint4 xv = lds128(xbase + (uint32_t)(m * XW + i) * 16);
-                acc[m] = fmaf(r, signed_dot(cw, xv), acc[m]);
-            }
-        };
-        if (nj == kChunkJ) {  // a whole radius group (cc.x % 16 == 0): fixed trip count, constant shifts
-            if constexpr (M == 1) {  // the whole chunk in one schedule (no spills at batch 1)
+                for (int pp = 0; pp < kParts; ++pp) t += stk[(pp * M + m) * kBlockRows + r];
+                return t;
+            };
+            const int mk = g.v.Mk;
+            if (g.full) {
 #pragma unroll
-                for (int i = 0; i < kChunkJ; ++i) column(i, (uint32_t)(15 - i));
+                for (int i = 0; i < 8; ++i) {
+                    const int r = lane + 32 * i, row = g.blk * kBlockRows + r;
+                    if (row < g.v.d_out)
+#pragma unroll
+                        for (int m = 0; m < M; ++m)
+                            if (m < mk) write_out(src.stage(s), g.v, m, row, part_sum(m, r));
+                }
+                ++done;
             } else {
-#pragma unroll 8
-                for (int i = 0; i < kChunkJ; ++i) column(i, (uint32_t)(15 - i));
-            }
-        } else {
-#pragma unroll 4
-            for (int i = 0; i < nj; ++i) column(i, (uint32_t)(15 - ((cc.x + i) & 15)));
-        }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.empty(k));
-}
-
-// Writes (or combines) the outputs of the pending segments tab[i0 .. i0 + n).
-// Split blocks: every contributor stores its partial sums, the CTA's writes are
-// published with one release atomic per block, and the contributor that sees
-// the count complete (acquire) adds all partials in CTA order.
-template <int M>
-__device__ void flush(const Common& C, const Smem<M>& sm, int i0, int n) {
-    constexpr int DT = Cfg<M>::kDecodeThreads;
-    const int tid = threadIdx.x;
-    const int cta = blockIdx.x;
-    const int l = tid & 31, r = tid >> 5;
-    const int row_local = l * 8 + r;
-    bool any_partial = false;
-    for (int i = 0; i < n; ++i) {
-        const Seg& g = sm.segs[i0 + i];
-        const int row = g.blk * kBlockRows + row_local;
-        const float* st = sm.stash + (size_t)i * M * kBlockRows;
-        if (g.full) {
-            if (tid < kBlockRows && row < g.v.d_out) {
+                float* part = P.partials + ((size_t)((s * P.n_cta + blockIdx.x) * 2 + (q.first ? 0 : 1)) * 8) * kBlockRows;
 #pragma unroll
-                for (int m = 0; m < M; ++m)
-                    if (m < g.v.Mk) {
-                        const int yr = g.v.yrows ? row_at(g.v.yrows, m) : m;
-                        g.v.y[(size_t)yr * g.v.d_out + row] = __half_as_ushort(__float2half_rn(st[m * kBlockRows + row_local]));
+                for (int i = 0; i < 8; ++i) {
+                    const int r = lane + 32 * i;
+#pragma unroll
+                    for (int m = 0; m < M; ++m)
+                        if (m < mk) part[m * kBlockRows + r] = part_sum(m, r);
+                }
+                const int b0 = g.v.unit0 + g.blk * g.v.S;
+                const int c_first = cta_of(U, P.n_cta, b0), c_last = cta_of(U, P.n_cta, b0 + g.v.S - 1);
+                unsigned* cnt = P.counters + src.stage(s).blk0 + g.v.blk0 + g.blk;
+                __syncwarp();  // the warp's partial stores precede the release below
+                int last = 0;
+                if (lane == 0) {
+                    const unsigned old = atom_add_acq_rel_gpu(cnt, 1u);
+                    last = old == (unsigned)(c_last - c_first);
+                    if (last) st_relaxed_gpu(cnt, 0u);  // restore for the next call
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {  // add the contributors' partials in CTA order, 8 rows per lane
+                    const int first_slot = (cta_begin(U, P.n_cta, c_first) >= b0) ? 0 : 1;
+                    float tot[8][M];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+#pragma unroll
+                        for (int m = 0; m < M; ++m) tot[i][m] = 0.f;
+                    constexpr int NF = M <= 2 ? 2 : 1;  // contributors whose loads are in flight at once
+                    for (int c0 = c_first; c0 <= c_last; c0 += NF) {
+                        float v[NF][8][M];
+#pragma unroll
+                        for (int kk = 0; kk < NF; ++kk) {
+                            const int c = c0 + kk;
+                            const int sp = (c == c_first) ? first_slot : 0;
+                            const float* src_p = P.partials + ((size_t)((s * P.n_cta + c) * 2 + sp) * 8) * kBlockRows + lane;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                                for (int m = 0; m < M; ++m)
+                                    v[kk][i][m] = (c <= c_last && m < mk) ? __ldcg(src_p + m * kBlockRows + 32 * i) : 0.f;
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < NF; ++kk)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                                for (int m = 0; m < M; ++m) tot[i][m] += v[kk][i][m];
                     }
-            }
-        } else {
-            any_partial = true;
-            float* part = C.partials + ((size_t)(cta * 2 + g.my_slot) * 8) * kBlockRows;
-            if (tid < kBlockRows)
 #pragma unroll
-                for (int m = 0; m < M; ++m)
-                    if (m < g.v.Mk) part[m * kBlockRows + row_local] = st[m * kBlockRows + row_local];
-        }
-    }
-    if (!any_partial) return;  // uniform across the decode threads
-    named_barrier(1, DT);      // every partial store of the CTA precedes the release below
-    if (tid < n) {
-        const Seg& g = sm.segs[i0 + tid];
-        int last = 0;
-        if (!g.full) {
-            const unsigned old = atom_add_acq_rel_gpu(g.counter, 1u);
-            last = (old == (unsigned)(g.c_last - g.c_first));
-            if (last) *reinterpret_cast<volatile unsigned*>(g.counter) = 0u;  // restore for the next call
-        }
-        sm.bcast[tid] = last;
-    }
-    named_barrier(1, DT);
-    for (int i = 0; i < n; ++i) {
-        const Seg& g = sm.segs[i0 + i];
-        if (!sm.bcast[i]) continue;
-        const int row = g.blk * kBlockRows + row_local;
-        if (tid < kBlockRows && row < g.v.d_out) {
-            const int c_first = g.c_first, c_last = g.c_last, first_slot = g.first_slot, mk = g.v.Mk;
-            float tot[M];
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = g.blk * kBlockRows + lane + 32 * i;
+                        if (row < g.v.d_out)
 #pragma unroll
-            for (int m = 0; m < M; ++m) tot[m] = 0.f;
-            constexpr int NF = (M <= 2) ? 16 : 8;  // contributors' loads in flight at once
-            for (int c0 = c_first; c0 <= c_last; c0 += NF) {
-                float v[NF][M];
-#pragma unroll
-                for (int k = 0; k < NF; ++k) {
-                    const int c = c0 + k;
-                    const int sp = (c == c_first) ? first_slot : 0;
-                    const float* src = C.partials + ((size_t)(c * 2 + sp) * 8) * kBlockRows + row_local;
-#pragma unroll
-                    for (int m = 0; m < M; ++m) v[k][m] = (c <= c_last && m < mk) ? __ldcg(src + m * kBlockRows) : 0.f;
+                            for (int m = 0; m < M; ++m)
+                                if (m < mk) write_out(src.stage(s), g.v, m, row, tot[i][m]);
+                    }
+                    ++done;
                 }
-#pragma unroll
-                for (int k = 0; k < NF; ++k)
-#pragma unroll
-                    for (int m = 0; m < M; ++m) tot[m] += v[k][m];
             }
-#pragma unroll
-            for (int m = 0; m < M; ++m)
-                if (m < g.v.Mk) {
-                    const int yr = g.v.yrows ? row_at(g.v.yrows, m) : m;
-                    g.v.y[(size_t)yr * g.v.d_out + row] = __half_as_ushort(__float2half_rn(tot[m]));
-                }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sm.st_empty(k));
+        }
+        if (signal && done) {
+            __syncwarp();  // the warp's output stores precede the release
+            if (lane == 0) red_add_release_gpu(P.sync + kSyncStageDone + s, done);
         }
     }
-    named_barrier(1, DT);  // bcast reuse
 }
 
-// Decodes one segment with compile-time batch MK (<= MS, the launch's stash
-// stride) and leaves its 256 x MS results in stash slot `slot`.
-template <int MK, int MS>
-__device__ __forceinline__ void segment_body_impl(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st,
-                                                  int slot) {
-    constexpr int DT = Cfg<MS>::kDecodeThreads;
-    static_assert(Cfg<MS>::kW * 32 == kBlockRows, "one decode thread per block row");
+// Decode state carried across segments and stages.
+struct DecState {
+    int t, slot, ph;      // chunk counter, its ring slot and phase parity
+    WinPos wp;
+    int cur_win;          // window the decode warps hold (-1: none)
+    bool first_win;       // the next window opened is a stage's first (cooperative gather)
+    float sc;             // 2^k of the held window's prescale
+};
+
+// Decodes one segment with compile-time batch MK (<= M, the window's batch
+// stride) into this thread's stash slot `si`.
+template <int MK, int M, class Src>
+__device__ __forceinline__ void seg_body(const Src& src, const Smem& sm, const EngineParams& P, int s, const Seg& g,
+                                         DecState& ds, int xw, int nseg, bool first_seg) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int u = 32 * (warp & 3) + lane, part = warp >> 2;
     const VDec d = vdec(g.v.log2K);
-    float acc[MK];
+    float accA[MK], accB[MK];
 #pragma unroll
-    for (int m = 0; m < MK; ++m) acc[m] = 0.f;
-    int t = st.t, k = st.slot, ph = st.ph, cur = st.cur_win;
-    WinPos w = st.w;
-    for (int c = 0; c < g.n_chunks; ++c, ++t, ring_next(k, ph, sm.slots)) {
+    for (int m = 0; m < MK; ++m) accA[m] = accB[m] = 0.f;
+    int t = ds.t, slot = ds.slot, ph = ds.ph, cur_win = ds.cur_win;
+    WinPos wp = ds.wp;
+    float sc = ds.sc;
+    const int nc = n_chunks(g);
+    for (int c = 0; c < nc; ++c, ++t, ring_next(slot, ph, sm.slots)) {
         const int2 cc = chunk_cols(g, c);
-        const int pos = win_place(w, cc.y - cc.x, Cfg<MS>::kXW);
-        if (w.win != cur) {  // release the previous x window, wait for this one
-            if (cur >= 0) {
+        const int pos = win_place(wp, cc.y - cc.x, xw);
+        if (wp.win != cur_win) {  // release the previous window, wait for this one
+            if (cur_win >= 0) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(sm.x_empty(cur & 1));
+                if (lane == 0) mbar_arrive(sm.x_empty(cur_win & 1));
             }
-            if (w.win == 0) {  // the first window is gathered together with the activation warp
-                pdl_wait();
-                named_barrier(kBarFirstWindow, 32 + DT);
-                gather_x<MS, 2>(sm, *sm.wlen0, sm.xwin(0), tid, 32 + DT);
-                named_barrier(kBarFirstWindow, 32 + DT);
-            } else {
-                wait_bar(sm.x_full(w.win & 1), (w.win >> 1) & 1, C);
+            if (ds.first_win) {
+                coop_window<M>(src, sm, s, wp.win, xw, src.stage(s).wait != 0, tid);
+                ds.first_win = false;
             }
-            cur = w.win;
+            wait_bar(sm, sm.x_full(wp.win & 1), (wp.win >> 1) & 1, P.status);
+            cur_win = wp.win;
+            const int k = sm.misc[cur_win & 1];
+            sc = k == 0 ? 1.f : (k == 1 ? 2.f : 4.f);
         }
-        decode_rows<MK, MS>(sm, C, g, d, k, ph, c, sm.xwin(w.win), pos, warp, lane, acc);
+        wait_bar(sm, sm.full(slot), ph, P.status);
+        decode_chunk<MK>(sm, g, d, slot, cc, sm.xwin(wp.win) + (uint32_t)pos * 16, (uint32_t)xw * 16, sc, warp, lane,
+                         accA, accB);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.empty(slot));
     }
-    st.t = t;
-    st.slot = k;
-    st.ph = ph;
-    st.cur_win = cur;
-    st.w = w;
-    // each thread owns one row: its sums go straight to the stash
-    const int row = 32 * warp + lane;
+    ds.t = t;
+    ds.slot = slot;
+    ds.ph = ph;
+    ds.cur_win = cur_win;
+    ds.wp = wp;
+    ds.sc = sc;
+    // hand this thread's two rows (this column half) to the epilogue warp
+    constexpr int NS = Cfg<M>::kSlots;
+    const int k = nseg % NS;
+    if (nseg >= NS) wait_bar(sm, sm.st_empty(k), ((nseg / NS) - 1) & 1, P.status);
+    float* st0 = sm.stash + ((size_t)(k * kParts + part) * M) * kBlockRows;
 #pragma unroll
-    for (int m = 0; m < MS; ++m) {
-        float v = 0.f;
-#pragma unroll
-        for (int mm = 0; mm < MK; ++mm)
-            if (mm == m) v = acc[mm];
-        sm.stash[((size_t)slot * MS + m) * kBlockRows + row] = v;
+    for (int m = 0; m < MK; ++m) {
+        st0[m * kBlockRows + 2 * u] = accA[m];
+        st0[m * kBlockRows + 2 * u + 1] = accB[m];
     }
-    named_barrier(1, DT);
+    if (tid == 0) {
+        sm.pend[k].g = g;
+        sm.pend[k].stage = s;
+        sm.pend[k].first = first_seg ? 1 : 0;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.st_full(k));
 }
 
-// The MoE kernel's segment body: lane <-> row octet, warps split each chunk's
-// columns within warp groups, and the warps' partial sums are reduced through
-// shared memory.  (Dense launches use segment_body_impl: one thread per row.)
-template <int MK, int MS>
-__device__ __forceinline__ void segment_body_octets(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st,
-                                                  int slot) {
-    constexpr int W = Cfg<MS>::kW, DT = Cfg<MS>::kDecodeThreads;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const VDec d = vdec(g.v.log2K);
-    float acc[8][MK];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int m = 0; m < MK; ++m) acc[r][m] = 0.f;
-    int t = st.t, k = st.slot, ph = st.ph, cur = st.cur_win;
-    WinPos w = st.w;
-    const int wpg = W / C.n_wg, grp = warp / wpg, lw = warp - grp * wpg;
-    for (int c = 0; c < g.n_chunks; ++c, ++t, ring_next(k, ph, sm.slots)) {
-        const int2 cc = chunk_cols(g, c);
-        const int pos = win_place(w, cc.y - cc.x, Cfg<MS>::kXW);
-        if (w.win != cur) {  // release the previous x window, wait for this one
-            if (cur >= 0) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sm.x_empty(cur & 1));
-            }
-            if (w.win == 0) {  // the first window is gathered together with the activation warp
-                pdl_wait();
-                named_barrier(kBarFirstWindow, 32 + DT);
-                gather_x<MS, 2>(sm, *sm.wlen0, sm.xwin(0), tid, 32 + DT);
-                named_barrier(kBarFirstWindow, 32 + DT);
-            } else {
-                wait_bar(sm.x_full(w.win & 1), (w.win >> 1) & 1, C);
-            }
-            cur = w.win;
-        }
-        if ((t & (C.n_wg - 1)) == grp) decode_chunk<MK, MS>(sm, C, g, d, k, ph, c, sm.xwin(w.win), pos, lw, wpg, lane, acc);
-    }
-    st.t = t;
-    st.slot = k;
-    st.ph = ph;
-    st.cur_win = cur;
-    st.w = w;
-    // reduce the warps' partial sums in a fixed order into the stash
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int m = 0; m < MK; ++m) sm.red[((warp * 8 + r) * MK + m) * 32 + lane] = acc[r][m];
-    named_barrier(1, DT);
-    if (tid < kBlockRows) {
-        const int l = tid & 31, r = tid >> 5;
-        for (int m = 0; m < MS; ++m) {
-            float sum = 0.f;
-            if (m < MK) {
-#pragma unroll
-                for (int w2 = 0; w2 < W; ++w2) sum += sm.red[((w2 * 8 + r) * MK + m) * 32 + l];
-            }
-            sm.stash[((size_t)slot * MS + m) * kBlockRows + l * 8 + r] = sum;
-        }
-    }
-    named_barrier(1, DT);
-}
-
-// Out-of-line instance for launches whose segments have different batch
-// sizes (the MoE kernel dispatches on each segment's).
-template <int MK, int MS>
-__device__ __noinline__ void segment_body(const Smem<MS>& sm, const Common& C, const Seg& g, RoleState& st, int slot) {
-    segment_body_octets<MK, MS>(sm, C, g, st, slot);
-}
-
-template <int MLO, int M>
-__device__ __forceinline__ void decode_warps(const Common& C, const Smem<M>& sm, int n_seg, RoleState& st) {
-    constexpr int DT = Cfg<M>::kDecodeThreads;
+template <int M, class Src>
+__device__ void decode_role(const Src& src, const Smem& sm, const EngineParams& P, int xw) {
     const int tid = threadIdx.x;
-    int npend = 0, i_pend = 0;
+    int ncb = 0, nseg = 0;
     const uint16_t* cur_cb = nullptr;
-    win_break(st.w);
-    for (int si = 0; si < n_seg; ++si, ++st.s) {
-        const Seg& g = sm.segs[si];
-        const int s = st.s;
-        wait_bar(sm.cb_full(s & 1), (s >> 1) & 1, C);
-        if (g.v.cb != cur_cb) {  // build the 8 bank-rotated replicas from the raw copy
-            if (cur_cb) named_barrier(1, DT);
-            const int K = 1 << g.v.log2K;
-            const uint32_t raw = sm.cbraw0 + (s & 1) * sm.cbraw_bytes;
-            for (int e = tid; e < K * 8; e += DT) sts128(sm.cb0 + e * 16, lds128(raw + (e >> 3) * 16));
-            named_barrier(1, DT);
-            cur_cb = g.v.cb;
-        }
-        if (tid == 0) mbar_arrive(sm.cb_empty(s & 1));
-        if constexpr (MLO == M) {
-            segment_body_impl<M, M>(sm, C, g, st, npend);
-        } else {
-            switch (g.v.Mk) {
-                case 1: segment_body<1, M>(sm, C, g, st, npend); break;
-                case 2: segment_body<2, M>(sm, C, g, st, npend); break;
-                case 3: segment_body<3, M>(sm, C, g, st, npend); break;
-                case 4: segment_body<4, M>(sm, C, g, st, npend); break;
-                case 5: segment_body<5, M>(sm, C, g, st, npend); break;
-                case 6: segment_body<6, M>(sm, C, g, st, npend); break;
-                case 7: segment_body<7, M>(sm, C, g, st, npend); break;
-                default: segment_body<8, M>(sm, C, g, st, npend); break;
+    DecState ds{0, 0, 0, {0, 0}, -1, false, 1.f};
+    for (int s = 0; s < src.n_stages(); ++s) {
+        const int U = src.units(s);
+        if (U <= 0) continue;
+        const int u0 = cta_begin(U, P.n_cta, blockIdx.x), u1 = cta_begin(U, P.n_cta, blockIdx.x + 1);
+        win_break(ds.wp);
+        ds.first_win = true;
+        bool first_seg = true;
+        for (int uu = u0; uu < u1; ++nseg) {
+            const Seg g = make_seg(src, s, uu, u1);
+            uu += g.jb - g.ja;
+            if (g.v.cb != cur_cb) {  // rebuild the 8 bank-rotated replicas from the raw copy
+                const int h = ncb & 1;
+                if (cur_cb) named_barrier(kBarDecode, kDT);
+                wait_bar(sm, sm.cb_full(h), (ncb >> 1) & 1, P.status);
+                const int K = 1 << g.v.log2K;
+                const uint32_t raw = sm.cbraw0 + h * sm.cbraw_bytes;
+                for (int e = tid; e < K * 8; e += kDT) sts128(sm.cb0 + e * 16, lds128(raw + (e >> 3) * 16));
+                named_barrier(kBarDecode, kDT);
+                if (tid == 0) mbar_arrive(sm.cb_empty(h));
+                cur_cb = g.v.cb;
+                ++ncb;
             }
+            if (Src::kVarBatch) {  // virtual experts carry 1..8 pairs
+                const int mk = g.v.Mk;
+                if (mk <= 1) seg_body<1, M>(src, sm, P, s, g, ds, xw, nseg, first_seg);
+                else if (mk <= 2) seg_body<(M < 2 ? M : 2), M>(src, sm, P, s, g, ds, xw, nseg, first_seg);
+                else if (mk <= 4) seg_body<(M < 4 ? M : 4), M>(src, sm, P, s, g, ds, xw, nseg, first_seg);
+                else seg_body<M, M>(src, sm, P, s, g, ds, xw, nseg, first_seg);
+            } else {
+                seg_body<M, M>(src, sm, P, s, g, ds, xw, nseg, first_seg);
+            }
+            first_seg = false;
         }
-        ++npend;
-        if (npend == kMaxSegs || si + 1 == n_seg) {
-            flush<M>(C, sm, i_pend, npend);
-            npend = 0;
-            i_pend = si + 1;
-        }
+    }
+    if (ds.cur_win >= 0) {
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(sm.x_empty(ds.cur_win & 1));
     }
 }
 
-template <int MLO, int M, class Problem>
-__device__ __forceinline__ void run(const Problem& P, const Common& C, uint8_t* smem_raw, bool plan_needs_wait) {
-    const Smem<M> sm = carve<M>(smem_raw, C.slots, C.kmax);
+template <int M, class Src>
+__device__ void run(const Src& src, const EngineParams& P, uint8_t* smem_raw, int xw, int mrows, bool waited) {
+    const Smem sm = carve<M>(smem_raw, P.slots, P.kmax);
     const int tid = threadIdx.x, warp = tid >> 5;
-    constexpr int W = Cfg<M>::kW;
     if (tid == 0) {
         for (int k = 0; k < kMaxSlots; ++k) {
-            mbar_init(sm.bars + k, 1);              // full: copy warp arrival + bytes
-            mbar_init(sm.bars + kMaxSlots + k, W / C.n_wg);  // empty: one arrival per warp of the chunk's group
+            mbar_init(sm.full(k), 1);
+            mbar_init(sm.empty(k), kDW);
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(sm.cb_full(h), 1);
             mbar_init(sm.cb_empty(h), 1);
             mbar_init(sm.x_full(h), 32);
-            mbar_init(sm.x_empty(h), W);
+            mbar_init(sm.x_empty(h), kDW);
         }
         mbar_init(sm.perm_full(), 1);
+        for (int k = 0; k < kStashSlots; ++k) {
+            mbar_init(sm.st_full(k), kDW);
+            mbar_init(sm.st_empty(k), 1);
+        }
         fence_mbar_init();
-        s_abort = 0;
+        for (int i = 0; i < 64; ++i) sm.misc[i] = 0;
+        sm.misc[9] = mrows;
+        for (int i = 0; i < 8; ++i) sm.inv_rms[i] = 1.f;
     }
-    pdl_launch_dependents();
-    if (plan_needs_wait) pdl_wait();  // the plan itself depends on preceding work
-    __shared__ long long s_next;
-    __shared__ int s_nseg;
-    const long long total = P.total();
-    const long long u0 = total > 0 ? P.cta_begin(blockIdx.x) : 0;
-    const long long u1 = total > 0 ? P.cta_begin(blockIdx.x + 1) : 0;
-    RoleState st{0, 0, 0, 0, {0, 0}, -1};
-    bool waited = plan_needs_wait;
-    for (long long u = u0; u < u1;) {
-        if (warp == 0) {  // lane 0 lays the segments out, then one lane per segment adds the split-K data
-            if ((tid & 31) == 0) s_nseg = build_segs(P, C, u, u1, u0, sm.segs, &s_next);
-            __syncwarp();
-            for (int i = tid & 31; i < s_nseg; i += 32) seg_split_info(P, C, sm.segs[i], u0);
-        }
-        __syncthreads();
-        const int n_seg = s_nseg;
-        if (warp == W) {
-            copy_warp<M>(C, sm, n_seg, st, u == u0);
-        } else if (warp == W + 1) {
-            act_warp<M>(C, sm, n_seg, st, waited);
-        } else {
-            decode_warps<MLO, M>(C, sm, n_seg, st);
-        }
-        u = s_next;
-        __syncthreads();  // the segment table is rebuilt for the next round
+    __syncthreads();
+    if (warp == kCopyWarp) {
+        copy_role(src, sm, P.status, P.n_cta);
+    } else if (warp == kGatherWarp) {
+        gather_role<M>(src, sm, P.status, P.sync, P.n_cta, xw, waited);
+    } else if (warp == kEpiWarp) {
+        epi_role<M>(src, sm, P);
+    } else {
+        decode_role<M>(src, sm, P, xw);
     }
-    if (warp == W) copy_drain<M>(C, sm, st);
-    if (warp == W + 1 && !waited) pdl_wait();
+    __syncthreads();
+    // the last CTA out restores the stage completion counts for the next call
+    if (tid == 0 && P.uses_sync) {
+        const unsigned old = atom_add_acq_rel_gpu(P.sync + kSyncExit, 1u);
+        if (old == (unsigned)(P.n_cta - 1)) {
+            for (int s = 0; s < kMaxStages; ++s) st_relaxed_gpu(P.sync + kSyncStageDone + s, 0u);
+            st_relaxed_gpu(P.sync + kSyncExit, 0u);
+        }
+    }
 }
 
 template <int M>
-__global__ void __launch_bounds__(Cfg<M>::kThreads, 1) gemv_kernel(const __grid_constant__ DenseParams p) {
+__global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_constant__ EngineParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ int s_cs[kMaxCta + 1];
-    __shared__ DenseMat s_ms[kMaxMats];
-    for (int i = threadIdx.x; i <= p.c.n_cta; i += blockDim.x) s_cs[i] = p.cta_start[i];
-    for (int i = threadIdx.x; i < p.n_mats; i += blockDim.x) s_ms[i] = p.mats[i];
-    __syncthreads();
-    const DenseProblem P{p, s_cs, s_ms};
-    run<M, M>(P, p.c, smem_raw, false);
+    pdl_launch_dependents();
+    const DenseSrc src{p};
+    run<M>(src, p, smem_raw, Cfg<M>::kXW, M, false);
 }
 
-// Virtual experts carry 1..8 pairs; each segment dispatches on its own count.
-__global__ void __launch_bounds__(Cfg<kMaxPairsPerVirtual>::kThreads, 1) moe_kernel(const __grid_constant__ MoeParams p) {
+// Virtual experts carry 1..8 pairs each; the kernel's batch stride is 8.
+__global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant__ MoeParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ MoeStage st;
+    __shared__ MoeStage ms;
+    pdl_launch_dependents();
     pdl_wait();  // the routing comes from the preceding kernel
+    const int upv = ((((p.d_out + 7) >> 3) + kOct - 1) / kOct) * (p.d_in >> 3);
     if (threadIdx.x == 0) {
-        const long long per = (long long)(((p.d_out + 7) / 8 + kOct - 1) / kOct) * (p.d_in >> 3);
-        st.total = (long long)__ldcg(&p.route->n_virtual) * per;
-        const long long u0 = (long long)blockIdx.x * st.total / p.c.n_cta;
-        const long long u1 = (long long)(blockIdx.x + 1) * st.total / p.c.n_cta;
-        st.vi0 = (int)(u0 / per);
-        st.nvi = u1 > u0 ? (int)min((long long)kMoeCache, (u1 - 1) / per - st.vi0 + 1) : 0;
+        ms.n_virtual = (int)__ldcg(reinterpret_cast<const unsigned*>(p.route));
+        ms.units = ms.n_virtual * upv;
+        const int u0 = cta_begin(ms.units, p.e.n_cta, blockIdx.x), u1 = cta_begin(ms.units, p.e.n_cta, blockIdx.x + 1);
+        ms.vi0 = u0 / upv;
+        const int need = u1 > u0 ? (u1 - 1) / upv - ms.vi0 + 1 : 0;
+        ms.nvi = min(kMoeCache, need);
+        ms.overflow = need > kMoeCache;
+        if (ms.overflow) flag(p.e.status, kDevUnsupported);
     }
     __syncthreads();
-    if ((int)threadIdx.x < st.nvi) {
-        const int vi = st.vi0 + threadIdx.x;
-        const int e = __ldcg(p.v_expert + vi);
-        st.v_expert[threadIdx.x] = e;
-        st.v_count[threadIdx.x] = __ldcg(p.v_count + vi);
-        st.emat[threadIdx.x] = p.experts[e];
+    if ((int)threadIdx.x < ms.nvi) {
+        const int vi = ms.vi0 + threadIdx.x;
+        ms.v_expert[threadIdx.x] = __ldcg(p.v_expert + vi);
+        ms.v_count[threadIdx.x] = __ldcg(p.v_count + vi);
     }
-    for (int i = threadIdx.x; i < st.nvi * kMaxPairsPerVirtual; i += blockDim.x) {
-        const size_t src = (size_t)st.vi0 * kMaxPairsPerVirtual + i;
-        st.v_xrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_xrows + src);
-        st.v_yrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_yrows + src);
+    for (int i = threadIdx.x; i < ms.nvi * kMaxPairsPerVirtual; i += blockDim.x) {
+        const size_t src_i = (size_t)ms.vi0 * kMaxPairsPerVirtual + i;
+        ms.v_xrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_xrows + src_i);
+        ms.v_yrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_yrows + src_i);
+    }
+    // the window holds the largest pair count of this CTA's virtual experts
+    __shared__ int s_m2;
+    if (threadIdx.x == 0) {
+        int mmax = 1;
+        for (int k = 0; k < ms.nvi; ++k) mmax = max(mmax, ms.v_count[k]);
+        int m2 = 1;
+        while (m2 < mmax) m2 <<= 1;
+        s_m2 = m2;
     }
     __syncthreads();
-    const MoeProblem P{p, st};
-    run<1, kMaxPairsPerVirtual>(P, p.c, smem_raw, true);
+    if (ms.overflow) return;  // more virtual experts than the staging holds (flagged above)
+    const MoeSrc src{p, ms};
+    run<kMaxPairsPerVirtual>(src, p.e, smem_raw, kXBufBytes / (16 * s_m2), s_m2, true);
 }
 
 // Groups the (pair -> expert) routing into virtual experts of at most 8 pairs,
 // in expert order and, within an expert, pair order (deterministic).
 __global__ void moe_route_kernel(const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs, int n_experts,
-                                 MoeRoute* route, int32_t* v_expert, int32_t* v_xrows, int32_t* v_yrows,
+                                 unsigned* route, int32_t* v_expert, int32_t* v_xrows, int32_t* v_yrows,
                                  int32_t* v_count, uint32_t* status) {
     pdl_wait();
     extern __shared__ int s_cnt[];  // [n_experts]
@@ -1087,7 +1132,7 @@ __global__ void moe_route_kernel(const int32_t* pair_expert, const int32_t* pair
             s_cnt[e] = nv;  // first virtual index of expert e
             nv += (c + kMaxPairsPerVirtual - 1) / kMaxPairsPerVirtual;
         }
-        route->n_virtual = nv;
+        *route = (unsigned)nv;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
@@ -1104,89 +1149,33 @@ __global__ void moe_route_kernel(const int32_t* pair_expert, const int32_t* pair
     pdl_launch_dependents();
 }
 
-int g_sm_count = 0;
-std::once_flag g_once;
-
-int sm_count() {
-    std::call_once(g_once, [] {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_sm_count, cudaDevAttrMultiProcessorCount, dev);
-        if (g_sm_count <= 0) g_sm_count = 148;
-    });
-    return g_sm_count;
-}
-
+// ------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------
 long long units_of(const sage_matrix& A) {
-    const int R8 = (A.d_out + 7) / 8;
-    return (long long)((R8 + kOct - 1) / kOct) * (A.d_in / 8);
+    const long long R8 = ((long long)A.d_out + 7) / 8;
+    return (R8 + kOct - 1) / kOct * (long long)(A.d_in / 8);
 }
-int blocks_of(const sage_matrix& A) { return ((A.d_out + 7) / 8 + kOct - 1) / kOct; }
+long long blocks_of(const sage_matrix& A) { return (((long long)A.d_out + 7) / 8 + kOct - 1) / kOct; }
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
-// CTA counts per matrix for a dense launch.  If giving every matrix its own
-// CTAs keeps the largest CTA within 6% of an even split of all units, each
-// matrix gets its own CTAs (one codebook per CTA, fewer segments); otherwise
-// the plan is plain stream-K over the flattened units (returns empty).
-std::vector<int> per_matrix_shares(const std::vector<long long>& units, int n_cta) {
-    long long total = 0;
-    for (long long u : units) total += u;
-    const int n_mat = (int)units.size();
-    if (n_mat == 1 || n_mat > n_cta) return {};
-    std::vector<int> share((size_t)n_mat);
-    int given = 0;
-    for (int k = 0; k < n_mat; ++k) {
-        share[k] = std::max(1, (int)((double)units[k] * n_cta / total));
-        given += share[k];
-    }
-    while (given < n_cta) {  // hand out the rest to the most loaded matrix
-        int best = 0;
-        for (int k = 1; k < n_mat; ++k)
-            if ((double)units[k] / share[k] > (double)units[best] / share[best]) best = k;
-        ++share[best];
-        ++given;
-    }
-    if (given > n_cta) return {};
-    double worst = 0;
-    for (int k = 0; k < n_mat; ++k) {
-        if (share[k] > units[k]) return {};
-        worst = std::max(worst, (double)units[k] / share[k]);
-    }
-    if (worst > 1.06 * (double)total / n_cta) return {};
-    return share;
-}
+// Dynamic shared memory per CTA: 227 KB less the static replicas (32 KB) and a
+// little static headroom.
+constexpr int kSmemBudget = 227 * 1024 - (int)sizeof(g_rep) - 1024;
 
-// Ring depth: as many chunk slots as fit next to the fixed shared memory (one
-// CTA per SM), at most one more than the widest CTA's chunk count.
-constexpr int kSmemBudget = 226 * 1024;  // 227 KB per CTA less static shared memory
-constexpr int kDenseStatic = (kMaxCta + 1) * 4 + kMaxMats * (int)sizeof(DenseMat);  // gemv_kernel's staged tables
 template <int M>
 int slots_for(long long max_units_per_cta, int kmax, int budget) {
     const long long chunks = (max_units_per_cta + kChunkJ - 1) / kChunkJ + 2;
     int n = (int)std::min<long long>(kMaxSlots, std::max<long long>(2, chunks));
-    while (n > 2 && Cfg<M>::smem(n, kmax) > budget) --n;
+    while (n > 2 && smem_bytes<M>(n, kmax) > budget) --n;
     return n;
 }
 
-// Decode warp groups: a chunk is decoded by one group, so that a warp handles
-// several columns per ring slot; each group needs two slots in flight.
-int wg_for(int slots) { return slots >= 8 ? 4 : slots >= 4 ? 2 : 1; }
-
-// Raises the kernel's dynamic shared memory limit when a launch needs more
-// than any earlier one (callers hold the launch mutex).
-template <class K>
-bool ensure_smem(K kernel, int bytes, int& configured) {
-    if (bytes <= configured) return true;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
-    configured = bytes;
-    return true;
-}
-
 template <class K, class Params>
-int launch_pdl(K kernel, const Params& p, int grid, int threads, int smem, sage_stream_t stream) {
+int launch_pdl(K kernel, const Params& p, int grid, int smem, sage_stream_t stream) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3((unsigned)threads);
+    cfg.blockDim = dim3((unsigned)kThreads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
@@ -1197,97 +1186,127 @@ int launch_pdl(K kernel, const Params& p, int grid, int threads, int smem, sage_
     return cudaLaunchKernelEx(&cfg, kernel, p) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
-
-template <int M>
-int launch_m(const GemvJob* jobs, int n, void* ws, sage_stream_t stream) {
-    static DenseParams p;  // large: keep off the stack
-    static std::mutex mu;
-    static int configured = 0;
-    std::lock_guard<std::mutex> lock(mu);
-    std::vector<long long> units((size_t)n);
-    long long unit = 0;
-    int blk = 0, kmax = 16;
-    for (int i = 0; i < n; ++i) {
-        const sage_matrix& A = jobs[i].A;
-        kmax = std::max(kmax, 1 << A.log2K);
-        DenseMat& d = p.mats[i];
-        d.main = A.main; d.meta = A.meta; d.cb = A.codebook; d.perm = A.perm;
-        d.x = jobs[i].x; d.y = jobs[i].y;
-        d.d_out = A.d_out; d.d_in = A.d_in; d.log2K = A.log2K;
-        d.unit0 = unit; d.blk0 = blk;
-        units[i] = units_of(A);
-        unit += units[i];
-        blk += blocks_of(A);
-    }
-    if (unit >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
-    const int n_cta = (int)std::max<long long>(1, std::min<long long>(std::min(sm_count(), kMaxCta), unit / 4));
-    const std::vector<int> share = per_matrix_shares(units, n_cta);
-    long long widest = 0;
-    p.per_matrix = share.empty() ? 0 : 1;
-    int cta = 0;
-    for (int i = 0; i < n; ++i) {
-        p.mats[i].units = units[i];
-        p.mats[i].cta0 = cta;
-        p.mats[i].ncta = share.empty() ? 0 : share[i];
-        cta += p.mats[i].ncta;
-        if (!share.empty()) widest = std::max(widest, (units[i] + share[i] - 1) / share[i]);
-    }
-    if (share.empty()) widest = (unit + n_cta - 1) / n_cta;
-    p.n_mats = n;
-    p.total_units = unit;
-    p.c.n_cta = n_cta;
-    for (int c = 0; c <= n_cta; ++c) {
-        long long b;
-        if (c == n_cta) {
-            b = unit;
-        } else if (share.empty()) {
-            b = (long long)c * unit / n_cta;
-        } else {
-            int k = 0;
-            while (k + 1 < n && p.mats[k + 1].cta0 <= c) ++k;
-            b = p.mats[k].unit0 + (long long)(c - p.mats[k].cta0) * p.mats[k].units / p.mats[k].ncta;
-        }
-        p.cta_start[c] = (int)b;
-    }
-    p.c.M = M;
-    p.c.slots = slots_for<M>(widest, kmax, kSmemBudget - kDenseStatic);
-    p.c.n_wg = 1;  // dense launches: every decode warp works on every chunk (one thread per block row)
-    p.c.kmax = kmax;
-    if (!ensure_smem(gemv_kernel<M>, Cfg<M>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    p.c.status = reinterpret_cast<uint32_t*>(w);
-    p.c.counters = reinterpret_cast<unsigned*>(w + kWsHeader);
-    p.c.partials = reinterpret_cast<float*>(w + kWsHeader + round256((size_t)blk * 4));
-    return launch_pdl(gemv_kernel<M>, p, n_cta, Cfg<M>::kThreads, Cfg<M>::smem(p.c.slots, kmax), stream);
+// Grid size of an engine launch: one CTA per SM, fewer when there is little work.
+int engine_ctas(long long max_stage_units) {
+    return (int)std::max<long long>(1, std::min<long long>(current_sm_count(), std::max<long long>(1, max_stage_units / 4)));
 }
 
 }  // namespace
 
+size_t engine_workspace_bytes(const EngineStageSpec* stages, int n_stages) {
+    long long blocks = 0, umax = 0;
+    for (int s = 0; s < n_stages; ++s) {
+        long long u = 0;
+        for (int i = 0; i < stages[s].n_jobs; ++i) {
+            blocks += blocks_of(stages[s].jobs[i].A);
+            u += units_of(stages[s].jobs[i].A);
+        }
+        umax = std::max(umax, u);
+    }
+    const int n_cta = engine_ctas(umax);
+    return kWsHeader + round256((size_t)blocks * 4) + (size_t)n_stages * n_cta * 2 * 8 * kBlockRows * sizeof(float);
+}
+
+template <int M>
+static int launch_engine_m(const EngineStageSpec* stages, int n_stages, void* ws, sage_stream_t stream) {
+    static EngineParams p;  // large: keep off the stack
+    static std::mutex mu;
+    static SmemLimit limit;
+    std::lock_guard<std::mutex> lock(mu);
+    p = EngineParams{};
+    int nj = 0, kmax = 16;
+    long long blk_total = 0, umax = 0;
+    bool uses_sync = false;
+    for (int s = 0; s < n_stages; ++s) {
+        const EngineStageSpec& ss = stages[s];
+        EngineStage& st = p.st[s];
+        st = ss.stage;
+        st.job0 = nj;
+        st.n_jobs = ss.n_jobs;
+        st.blk0 = (int)blk_total;
+        long long unit = 0, blk = 0;
+        for (int i = 0; i < ss.n_jobs; ++i) {
+            const sage_matrix& A = ss.jobs[i].A;
+            EngineJob& d = p.jobs[nj++];
+            d.main = A.main; d.meta = A.meta; d.cb = A.codebook; d.perm = A.perm;
+            d.x = ss.jobs[i].x; d.y = ss.jobs[i].y;
+            d.d_out = A.d_out; d.d_in = A.d_in; d.log2K = A.log2K;
+            d.unit0 = (int)unit;
+            d.blk0 = (int)blk;
+            kmax = std::max(kmax, 1 << A.log2K);
+            unit += units_of(A);
+            blk += blocks_of(A);
+        }
+        if (unit >= (1ll << 31) / 2) return SAGE_ERR_UNSUPPORTED;
+        st.units = (int)unit;
+        st.blocks = (int)blk;
+        blk_total += blk;
+        umax = std::max(umax, unit);
+        if (s > 0 && st.wait) uses_sync = true;
+    }
+    const int n_cta = engine_ctas(umax);
+    long long widest = 0;
+    for (int s = 0; s < n_stages; ++s) widest += (p.st[s].units + n_cta - 1) / n_cta;
+    p.n_stages = n_stages;
+    p.n_cta = n_cta;
+    p.M = M;
+    p.kmax = kmax;
+    p.slots = slots_for<M>(widest, kmax, kSmemBudget);
+    p.uses_sync = uses_sync ? 1 : 0;
+    const int smem = smem_bytes<M>(p.slots, kmax);
+    if (smem > kSmemBudget) return SAGE_ERR_UNSUPPORTED;
+    if (!limit.ensure(engine_kernel<M>, smem)) return SAGE_ERR_CUDA;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.status = reinterpret_cast<uint32_t*>(w);
+    p.sync = reinterpret_cast<unsigned*>(w);
+    p.counters = reinterpret_cast<unsigned*>(w + kWsHeader);
+    p.partials = reinterpret_cast<float*>(w + kWsHeader + round256((size_t)blk_total * 4));
+    return launch_pdl(engine_kernel<M>, p, n_cta, smem, stream);
+}
+
+int launch_engine(const EngineStageSpec* stages, int n_stages, int M, void* ws, size_t ws_bytes, sage_stream_t stream) {
+    if (n_stages < 1 || n_stages > kMaxStages) return SAGE_ERR_UNSUPPORTED;
+    int nj = 0;
+    for (int s = 0; s < n_stages; ++s) nj += stages[s].n_jobs;
+    if (nj > kMaxJobs) return SAGE_ERR_UNSUPPORTED;
+    if (ws_bytes < engine_workspace_bytes(stages, n_stages)) return SAGE_ERR_WORKSPACE;
+    switch (M) {
+        case 1: return launch_engine_m<1>(stages, n_stages, ws, stream);
+        case 2: return launch_engine_m<2>(stages, n_stages, ws, stream);
+        case 3: return launch_engine_m<3>(stages, n_stages, ws, stream);
+        case 4: return launch_engine_m<4>(stages, n_stages, ws, stream);
+        case 5: return launch_engine_m<5>(stages, n_stages, ws, stream);
+        case 6: return launch_engine_m<6>(stages, n_stages, ws, stream);
+        case 7: return launch_engine_m<7>(stages, n_stages, ws, stream);
+        case 8: return launch_engine_m<8>(stages, n_stages, ws, stream);
+        default: return SAGE_ERR_UNSUPPORTED;
+    }
+}
+
+// One stage of plain GEMVs (sage_gemv, sage_gemv_grouped).
 size_t gemv_workspace_bytes(const sage_matrix* mats, int n, int M) {
     (void)M;
-    long long units = 0;
-    int blk = 0;
-    for (int i = 0; i < n; ++i) { units += units_of(mats[i]); blk += blocks_of(mats[i]); }
-    const int n_cta = (int)std::max<long long>(1, std::min<long long>(sm_count(), units / 4));
-    return kWsHeader + round256((size_t)blk * 4) + (size_t)n_cta * 2 * 8 * kBlockRows * sizeof(float);
+    std::vector<EngineJobSpec> jobs((size_t)n);
+    for (int i = 0; i < n; ++i) jobs[i].A = mats[i];
+    EngineStageSpec st{};
+    st.jobs = jobs.data();
+    st.n_jobs = n;
+    return engine_workspace_bytes(&st, 1);
 }
 
 int launch_gemv(const GemvJob* jobs, int n, int M, void* ws, size_t ws_bytes, sage_stream_t stream) {
-    if (n > kMaxMats) return SAGE_ERR_UNSUPPORTED;
-    std::vector<sage_matrix> mats((size_t)n);
-    for (int i = 0; i < n; ++i) mats[i] = jobs[i].A;
-    if (ws_bytes < gemv_workspace_bytes(mats.data(), n, M)) return SAGE_ERR_WORKSPACE;
-    switch (M) {
-        case 1: return launch_m<1>(jobs, n, ws, stream);
-        case 2: return launch_m<2>(jobs, n, ws, stream);
-        case 3: return launch_m<3>(jobs, n, ws, stream);
-        case 4: return launch_m<4>(jobs, n, ws, stream);
-        case 5: return launch_m<5>(jobs, n, ws, stream);
-        case 6: return launch_m<6>(jobs, n, ws, stream);
-        case 7: return launch_m<7>(jobs, n, ws, stream);
-        case 8: return launch_m<8>(jobs, n, ws, stream);
-        default: return SAGE_ERR_UNSUPPORTED;
+    std::vector<EngineJobSpec> js((size_t)n);
+    for (int i = 0; i < n; ++i) {
+        js[i].A = jobs[i].A;
+        js[i].x = jobs[i].x;
+        js[i].y = jobs[i].y;
     }
+    EngineStageSpec st{};
+    st.jobs = js.data();
+    st.n_jobs = n;
+    st.stage.pro = kProPlain;
+    st.stage.epi = kEpiPlain;
+    return launch_engine(&st, 1, M, ws, ws_bytes, stream);
 }
 
 // MoE workspace: header | route | v_expert | v_xrows | v_yrows | v_count | counters | partials
@@ -1313,39 +1332,47 @@ MoeWs moe_ws_layout(int n_pairs, int d_out, int n_cta) {
 
 size_t moe_workspace_bytes(const sage_matrix* experts, int n_experts, int n_pairs) {
     (void)n_experts;
-    return moe_ws_layout(std::max(1, n_pairs), experts[0].d_out, sm_count()).total;
+    return moe_ws_layout(std::max(1, n_pairs), experts[0].d_out, current_sm_count()).total;
 }
 
 int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_expert, const int32_t* pair_xrow,
                int n_pairs, const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream) {
     constexpr int MV = kMaxPairsPerVirtual;
     if (n_experts > kMaxExperts) return SAGE_ERR_UNSUPPORTED;
-    const int n_cta = sm_count();
+    const int n_cta = current_sm_count();
     const MoeWs L = moe_ws_layout(n_pairs, experts[0].d_out, n_cta);
     if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
     static MoeParams p;
     static std::mutex mu;
-    static int configured = 0;
+    static SmemLimit limit;
     std::lock_guard<std::mutex> lock(mu);
-    p.c.n_cta = n_cta;
-    p.c.M = 0;
+    p = MoeParams{};
     int kmax = 16;
     for (int e = 0; e < n_experts; ++e) kmax = std::max(kmax, 1 << experts[e].log2K);
-    p.c.kmax = kmax;
-    p.c.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget - (int)sizeof(MoeStage));
-    p.c.n_wg = wg_for(p.c.slots);
-    if (!ensure_smem(moe_kernel, Cfg<MV>::smem(p.c.slots, kmax), configured)) return SAGE_ERR_CUDA;
-    p.c.status = reinterpret_cast<uint32_t*>(w);
-    p.c.counters = reinterpret_cast<unsigned*>(w + L.counters);
-    p.c.partials = reinterpret_cast<float*>(w + L.partials);
+    p.e.n_stages = 1;
+    p.e.n_cta = n_cta;
+    p.e.M = MV;
+    p.e.kmax = kmax;
+    p.e.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget - (int)sizeof(MoeStage));
+    p.e.uses_sync = 0;
+    const int smem = smem_bytes<MV>(p.e.slots, kmax);
+    if (smem > kSmemBudget - (int)sizeof(MoeStage)) return SAGE_ERR_UNSUPPORTED;
+    if (!limit.ensure(moe_kernel, smem)) return SAGE_ERR_CUDA;
+    p.e.status = reinterpret_cast<uint32_t*>(w);
+    p.e.sync = reinterpret_cast<unsigned*>(w);
+    p.e.counters = reinterpret_cast<unsigned*>(w + L.counters);
+    p.e.partials = reinterpret_cast<float*>(w + L.partials);
+    p.st.pro = kProPlain;
+    p.st.epi = kEpiPlain;
+    p.st.blk0 = 0;
     p.n_experts = n_experts;
     p.d_out = experts[0].d_out;
     p.d_in = experts[0].d_in;
     p.n_pairs = n_pairs;
     p.x = x;
     p.y = y;
-    p.route = reinterpret_cast<const MoeRoute*>(w + L.route);
+    p.route = reinterpret_cast<const unsigned*>(w + L.route);
     p.v_expert = reinterpret_cast<const int32_t*>(w + L.v_expert);
     p.v_xrows = reinterpret_cast<const int32_t*>(w + L.v_xrows);
     p.v_yrows = reinterpret_cast<const int32_t*>(w + L.v_yrows);
@@ -1369,12 +1396,12 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, moe_route_kernel, pair_expert, pair_xrow, n_pairs, n_experts,
-                               reinterpret_cast<MoeRoute*>(w + L.route), reinterpret_cast<int32_t*>(w + L.v_expert),
+                               reinterpret_cast<unsigned*>(w + L.route), reinterpret_cast<int32_t*>(w + L.v_expert),
                                reinterpret_cast<int32_t*>(w + L.v_xrows), reinterpret_cast<int32_t*>(w + L.v_yrows),
-                               reinterpret_cast<int32_t*>(w + L.v_count), p.c.status) != cudaSuccess)
+                               reinterpret_cast<int32_t*>(w + L.v_count), p.e.status) != cudaSuccess)
             return SAGE_ERR_CUDA;
     }
-    return launch_pdl(moe_kernel, p, n_cta, Cfg<MV>::kThreads, Cfg<MV>::smem(p.c.slots, kmax), stream);
+    return launch_pdl(moe_kernel, p, n_cta, smem, stream);
 }
 
 }  // namespace sage

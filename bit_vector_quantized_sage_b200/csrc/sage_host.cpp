@@ -40,6 +40,25 @@ struct PlaneIndex {
     size_t meta_word(int g, int t) const { return meta0 + (((size_t)g * nB + ob) * 8 + t) * 2; }
 };
 
+int current_device() {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+int current_sm_count() {
+    static std::mutex mu;
+    static int count[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (count[dev] <= 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        count[dev] = n;
+    }
+    return count[dev];
+}
+
 int check_matrix(const sage_matrix* A) {
     if (!A) return SAGE_ERR_INVALID_ARGUMENT;
     if (A->d_out < 1 || A->d_in < 1) return SAGE_ERR_INVALID_ARGUMENT;

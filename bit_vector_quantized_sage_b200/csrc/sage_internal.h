@@ -1,8 +1,11 @@
 // Internal declarations shared by the host and device translation units of libsage.
 #pragma once
 
+#include <cuda_runtime.h>
+
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/sage.h"
 
@@ -21,6 +24,32 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Validates one matrix descriptor; returns SAGE_OK or the error.
 int check_matrix(const sage_matrix* A);
+
+// Per-device facts, looked up with the device current at the time of the call.
+constexpr int kMaxDevices = 64;
+int current_device();        // -1 when no device can be queried
+int current_sm_count();      // SM count of the current device (cached per device)
+
+// Raises a kernel's dynamic shared-memory limit on the current device when a
+// launch needs more than any earlier launch on that device did.
+class SmemLimit {
+  public:
+    template <class K>
+    bool ensure(K kernel, int bytes) {
+        const int dev = current_device();
+        if (dev < 0 || dev >= kMaxDevices) return false;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (bytes <= done_[dev]) return true;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return false;
+        done_[dev] = bytes;
+        return true;
+    }
+
+  private:
+    std::mutex mu_;
+    int done_[kMaxDevices] = {};
+};
 
 // Kernel launchers (sage_gemv.cu / sage_hooks.cu / sage_gemm_sm100.cu).
 struct GemvJob {

@@ -222,6 +222,55 @@ int sage_moe_gemv(const sage_matrix* experts, int n_experts,
                   const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs,
                   const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Fused decoder layer.  The packed projections of one transformer decoder
+ * layer run as ONE launch of four dependent stages, with the operations
+ * between them fused into the activation gather of the next stage (Sec. 3.5:
+ * the ESG permutation is fused with the preceding normalisation or
+ * activation) and into the output writes:
+ *   x1  = fp16(h * attn_norm / sqrt(mean(h^2) + eps))             RMSNorm
+ *   q, k, v = W_q x1, W_k x1, W_v x1                             stage 1
+ *   a   = attention over the single cached position: query head i reads the
+ *         value row of key/value head i / (n_heads / n_kv_heads)
+ *   o   = W_o a                                                   stage 2
+ *   r   = fp16(h + o);  x3 = fp16(r * mlp_norm / sqrt(mean(r^2) + eps))
+ *   gate, up = W_gate x3, W_up x3                                stage 3
+ *   m   = fp16(silu(gate) * up),  silu(t) = t / (1 + e^-t)
+ *   down = W_down m;   h_out = fp16(r + down)                    stage 4
+ * A stage starts decoding as soon as the stage it reads is complete on the
+ * whole device (a completion count in the workspace), not at a kernel
+ * boundary; the packed planes of later stages stream in meanwhile.  Every
+ * projection has the numerics of sage_gemv.  The attention is the first
+ * position of a sequence, which needs no key/value cache and no rotary
+ * embedding; the rest of a longer sequence's attention is outside libsage.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    sage_matrix q, k, v, o, gate, up, down;   /* packed projections */
+    const uint16_t* attn_norm;   /* fp16 [hidden] RMSNorm weight before q|k|v (device) */
+    const uint16_t* mlp_norm;    /* fp16 [hidden] RMSNorm weight before gate|up (device) */
+    int32_t n_heads, n_kv_heads, head_dim;
+    float eps;
+} sage_decoder_layer;
+
+typedef struct {   /* device outputs, fp16 [M][...] (all written) */
+    uint16_t *q, *k, *v, *o, *gate, *up, *down, *h_out;
+} sage_decoder_outputs;
+
+/* Workspace bytes of sage_decoder_layer_forward (zero-filled once before first
+ * use, as for the other compute calls).  Errors: INVALID_ARGUMENT, UNSUPPORTED
+ * (shapes that do not form a decoder layer, see sage_decoder_layer_forward). */
+int sage_decoder_layer_workspace_size(const sage_decoder_layer* L, int M, size_t* bytes);
+
+/* One decoder layer at batch M (1..8) on input rows h (fp16 [M][hidden], device).
+ * Shapes: hidden = d_in of q, k, v, gate, up = d_out of o and down;
+ * q.d_out = o.d_in = n_heads * head_dim; k.d_out = v.d_out = n_kv_heads *
+ * head_dim (n_heads a multiple of n_kv_heads); gate.d_out = up.d_out =
+ * down.d_in.  Errors: INVALID_ARGUMENT (null pointer, eps < 0), UNSUPPORTED
+ * (shapes, M), MISALIGNED, WORKSPACE, CUDA; device-side timeouts as for
+ * sage_gemv (sage_query_status). */
+int sage_decoder_layer_forward(const sage_decoder_layer* L, const uint16_t* h, int M,
+                               const sage_decoder_outputs* out, void* ws, size_t ws_bytes, sage_stream_t stream);
+
 /* Test hook: fp16 reconstruction W[d_out][d_in] (storage column order),
  * computed by the same device decode as the kernels (Eq. 1-2). */
 int sage_dequant(const sage_matrix* A, uint16_t* W, sage_stream_t stream);

@@ -37,7 +37,9 @@ def lib():
     global _lib
     with _lock:
         if _lib is None:
-            L = C.CDLL(build())
+            # SAGE_ORACLE_LIB loads another build of sage_oracle.c (the mutation
+            # check points it at a deliberately broken copy in a temp directory)
+            L = C.CDLL(os.environ.get("SAGE_ORACLE_LIB") or build())
             P = C.c_void_p
             i32, u16, f64, i64, sz = C.c_int, C.c_uint16, C.c_double, C.c_int64, C.c_size_t
             L.oracle_half_to_double.argtypes = [u16]
@@ -70,6 +72,14 @@ def lib():
             L.oracle_encode.restype = i32
             L.oracle_bpw.argtypes = [i32, i32, i32, i32, i32, i32, f64]
             L.oracle_bpw.restype = f64
+            L.oracle_rmsnorm.argtypes = [i32, i32, P, P, f64, P]
+            L.oracle_rmsnorm.restype = None
+            L.oracle_add.argtypes = [sz, P, P, P]
+            L.oracle_add.restype = None
+            L.oracle_silu_mul.argtypes = [sz, P, P, P]
+            L.oracle_silu_mul.restype = None
+            L.oracle_attend_one_position.argtypes = [i32, i32, i32, i32, P, P]
+            L.oracle_attend_one_position.restype = None
             _lib = L
     return _lib
 
@@ -235,3 +245,37 @@ def encode(inp):
 
 def bpw(v: int, B: int, G: int, bg: int, K: int, bc: int, N: float) -> float:
     return float(lib().oracle_bpw(v, B, G, bg, K, bc, float(N)))
+
+
+# ---------------------------------------------------------------------------
+# Decoder-layer operations around the packed projections (fp16 bits in / out)
+# ---------------------------------------------------------------------------
+
+def rmsnorm(x16: np.ndarray, g16: np.ndarray, eps: float) -> np.ndarray:
+    """fp16(x * g / sqrt(mean(x^2) + eps)) per row of x ([M][d] fp16 bits)."""
+    x = _c(np.atleast_2d(x16), np.uint16)
+    g = _c(g16, np.uint16)
+    out = np.zeros_like(x)
+    lib().oracle_rmsnorm(x.shape[0], x.shape[1], _p(x), _p(g), float(eps), _p(out))
+    return out
+
+
+def add(a16: np.ndarray, b16: np.ndarray) -> np.ndarray:
+    a, b = _c(a16, np.uint16), _c(b16, np.uint16)
+    out = np.zeros_like(a)
+    lib().oracle_add(a.size, _p(a), _p(b), _p(out))
+    return out
+
+
+def silu_mul(gate16: np.ndarray, up16: np.ndarray) -> np.ndarray:
+    g, u = _c(gate16, np.uint16), _c(up16, np.uint16)
+    out = np.zeros_like(g)
+    lib().oracle_silu_mul(g.size, _p(g), _p(u), _p(out))
+    return out
+
+
+def attend_one_position(v16: np.ndarray, n_heads: int, n_kv: int, hd: int) -> np.ndarray:
+    v = _c(np.atleast_2d(v16), np.uint16)
+    out = np.zeros((v.shape[0], n_heads * hd), np.uint16)
+    lib().oracle_attend_one_position(v.shape[0], n_heads, n_kv, hd, _p(v), _p(out))
+    return out

@@ -430,3 +430,53 @@ int oracle_encode(int d_out, int d_in, int log2K, const double* W, const double*
 double oracle_bpw(int v, int B, int G, int bg, int K, int bc, double N) {
     return (double)B / v + 2.0 * bg / G + (double)K * v * bc / N;
 }
+
+/* ------------------------------------------------------------------ */
+/* The operations either side of the packed GEMVs in a decoder layer  */
+/* (Sec. 3.5: the ESG permutation is fused with the preceding          */
+/* normalisation or activation).  fp16 in, fp64 arithmetic, fp16 out   */
+/* (the activations a layer stores between its projections).           */
+/* ------------------------------------------------------------------ */
+
+/* RMSNorm of each of the M rows of x [M][d] with weight g [d]:
+ *   out = fp16( x * g / sqrt(mean(x^2) + eps) ). */
+void oracle_rmsnorm(int M, int d, const uint16_t* x, const uint16_t* g, double eps, uint16_t* out) {
+    for (int m = 0; m < M; ++m) {
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) {
+            const double v = oracle_half_to_double(x[(size_t)m * d + c]);
+            ss += v * v;
+        }
+        const double inv = 1.0 / sqrt(ss / (double)d + eps);
+        for (int c = 0; c < d; ++c) {
+            const double v = oracle_half_to_double(x[(size_t)m * d + c]);
+            out[(size_t)m * d + c] = oracle_double_to_half(v * oracle_half_to_double(g[c]) * inv);
+        }
+    }
+}
+
+/* Elementwise fp16 sum (the residual stream): out = fp16(a + b). */
+void oracle_add(size_t n, const uint16_t* a, const uint16_t* b, uint16_t* out) {
+    for (size_t i = 0; i < n; ++i)
+        out[i] = oracle_double_to_half(oracle_half_to_double(a[i]) + oracle_half_to_double(b[i]));
+}
+
+/* SwiGLU activation: out = fp16( silu(gate) * up ), silu(t) = t / (1 + e^-t). */
+void oracle_silu_mul(size_t n, const uint16_t* gate, const uint16_t* up, uint16_t* out) {
+    for (size_t i = 0; i < n; ++i) {
+        const double t = oracle_half_to_double(gate[i]);
+        out[i] = oracle_double_to_half(t / (1.0 + exp(-t)) * oracle_half_to_double(up[i]));
+    }
+}
+
+/* Attention over a single cached position (the first token of a sequence):
+ * the softmax over one key is 1, so query head h returns the value vector of
+ * its key/value head h / (n_heads / n_kv) (grouped-query attention).
+ * v: [M][n_kv * hd]; out: [M][n_heads * hd]. */
+void oracle_attend_one_position(int M, int n_heads, int n_kv, int hd, const uint16_t* v, uint16_t* out) {
+    const int grp = n_heads / n_kv;
+    for (int m = 0; m < M; ++m)
+        for (int h = 0; h < n_heads; ++h)
+            for (int e = 0; e < hd; ++e)
+                out[((size_t)m * n_heads + h) * hd + e] = v[((size_t)m * n_kv + h / grp) * hd + e];
+}

@@ -168,6 +168,42 @@ def config1(M: int = 1, replica: int = 0) -> LayerSpec:
     return LayerSpec(mats, energies, xs)
 
 
+# Attention geometry of the Qwen3-4B-shaped layer: 32 query heads and 8
+# key/value heads of dimension 128 (q 4096 = 32 x 128, k / v 1024 = 8 x 128).
+QWEN3_4B_HEADS = (32, 8, 128)
+
+
+@dataclass
+class DecoderInputs:
+    h: np.ndarray          # fp16 bits (M, hidden): the layer's input rows
+    attn_norm: np.ndarray  # fp16 bits (hidden,)
+    mlp_norm: np.ndarray   # fp16 bits (hidden,)
+    eps: float
+
+
+def decoder_inputs(config: int, M: int, hidden: int, replica: int = 0) -> DecoderInputs:
+    """Inputs of a decoder layer around its projections: h ~ N(0, 1) and RMSNorm
+    weights ~ U(0.5, 1.5), all fp16; eps = 1e-6."""
+    g = rng(config, 300, replica)
+    return DecoderInputs(f16_bits(g.standard_normal((M, hidden))), f16_bits(g.uniform(0.5, 1.5, hidden)),
+                         f16_bits(g.uniform(0.5, 1.5, hidden)), 1e-6)
+
+
+def small_layer(seed: int, hidden: int = 256, heads=(4, 2, 64), inter: int = 512) -> LayerSpec:
+    """A small decoder layer with the Qwen3 structure (for fast parity tests):
+    each projection draws its split from the five 18-bit splits."""
+    nh, nkv, hd = heads
+    shapes = (("q", nh * hd, hidden), ("k", nkv * hd, hidden), ("v", nkv * hd, hidden), ("o", hidden, nh * hd),
+              ("gate", inter, hidden), ("up", inter, hidden), ("down", hidden, inter))
+    g = np.random.default_rng(seed)
+    mats, energies = [], {}
+    for name, d_out, d_in in shapes:
+        K, _V = SPLITS[int(g.integers(0, len(SPLITS)))]
+        mats.append(random_fields(g, d_out, d_in, int(K).bit_length() - 1, name=name))
+        energies[name] = lognormal_energies(g, d_in, 1.5)
+    return LayerSpec(mats, energies, {})
+
+
 @dataclass
 class EncoderInputs:
     W: np.ndarray            # fp64 (d_out, d_in), original channel order

@@ -490,3 +490,151 @@ def test_kmeans_channel_without_weight_gets_zero_component():
     cb = oracle.kmeans(P, Wt, K, init, 2)
     assert np.all(cb[:, 3] == 0.0)
     assert np.allclose(np.linalg.norm(cb, axis=1), 1.0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# The encoder's composition, hand-worked: Eq. 5 -> Eq. 4 -> Eq. 6 -> Eq. 14 -> Eq. 2
+# ---------------------------------------------------------------------------
+
+# Row 1 of the hand example: 16 unit directions exactly representable in fp16.
+# k = 0..7 are the one-hot vectors e_k; k = 8..15 are half-vectors h_S = 1_S / 2
+# over the listed four positions (norm 1, entries 0.5).
+_HALVES = [(0, 1, 2, 3), (4, 5, 6, 7), (0, 1, 4, 5), (2, 3, 6, 7),
+           (0, 2, 4, 6), (1, 3, 5, 7), (0, 1, 6, 7), (2, 3, 4, 5)]
+
+
+def _direction(k):
+    c = np.zeros(8)
+    if k < 8:
+        c[k] = 1.0
+    else:
+        c[list(_HALVES[k - 8])] = 0.5
+    return c
+
+
+def test_encode_composition_hand_worked():
+    """A 2 x 128 layer encoded with K = 16 (V = 6), gamma = 1 and no k-means
+    update (iters = 0, so the codebook is the directions of the initial
+    samples), built so that every step has a closed form:
+
+    * Eq. 5 (ESG): energies 3 for channels 0..31 and 1 for the rest are already
+      sorted, so tier t holds channels 16t .. 16t + 15 and storage position
+      8j + t holds channel 16t + j.
+    * Eq. 4: every subvector has energies (3, 3, 1, 1, 1, 1, 1, 1) across its
+      positions; gamma = 1, mean 1.5, so omega = (2, 2, 2/3, ..., 2/3).
+    * Row 1 holds the 16 codeword directions, each scaled by 0.5 + n/16; it is
+      the k-means sample and its subvector k initialises codeword k.
+    * Eq. 6: a subvector parallel to codeword k scores sum(omega p^2) there and
+      strictly less at every other codeword (weighted Cauchy-Schwarz), and its
+      optimal radius is its length.  Row 0's subvector 1, p = (1, 1, 1/2, 1/2,
+      0, 0, 0, 0), is parallel to no codeword: h_0123 scores
+      (7/3)^2 / (4/3) = 49/12 (next best 3, at h_0145 and h_0167) with the
+      weighted radius (7/3) / (4/3) = 7/4; the unweighted fit would be 3/2.
+    * Eq. 14: row 0's radii span [1/2, 7/4], so mu = 1/2 and
+      delta = (5/4) / 63 = 0.0198412..., stored in fp16 as 1300 / 65536
+      (0x2514); row 1's span [1/2, 1/2 + 63/16] gives delta = 1/16 exactly.
+    * Eq. 2 with the stored grid: row 0's subvector 2 has radius 1.1249, i.e.
+      31.5027 fp16 steps (q = 32) but 31.4950 unrounded steps (31); the other
+      radii are exact multiples of the stored step, or the ends of the group.
+    """
+    d_out, d_in, S = 2, 128, 16
+    energies = np.where(np.arange(d_in) < 32, 3.0, 1.0)
+    step16 = 1300.0 / 65536.0  # fp16 of 1.25 / 63
+    # row 0: (codeword, radius) per subvector; subvector 1 is the non-parallel one
+    row0 = [(3, 0.5), (None, None), (5, 1.1249), (10, 1.0), (0, 1.5)]
+    fill_k = [1, 2, 4, 6, 7, 9, 11, 12, 13, 14, 15]
+    fill_n = [3, 7, 12, 18, 22, 37, 41, 47, 55, 60, 62]
+    row0 += [(k, 0.5 + n * step16) for k, n in zip(fill_k, fill_n)]
+    n1 = [0, 5, 10, 15, 20, 25, 30, 35, 40, 45, 50, 55, 60, 62, 1, 63]
+    P = np.zeros((d_out, S, 8))
+    for t, (k, r) in enumerate(row0):
+        P[0, t] = r * _direction(k) if k is not None else [1, 1, 0.5, 0.5, 0, 0, 0, 0]
+    for k in range(S):
+        P[1, k] = (0.5 + n1[k] / 16.0) * _direction(k)
+    neg = np.zeros((d_out, S, 8), bool)
+    for o in range(d_out):
+        for j in range(S):
+            for i in range(8):
+                neg[o, j, i] = (o + j + i) % 2 == 1 and P[o, j, i] > 0
+    W = np.zeros((d_out, d_in))
+    for j in range(S):
+        for i in range(8):
+            W[:, 16 * i + j] = np.where(neg[:, j, i], -P[:, j, i], P[:, j, i])
+    inp = synth.EncoderInputs(W, energies, np.arange(16, 32, dtype=np.int64), np.arange(16, dtype=np.int64),
+                              1.0, 0, 4)
+    out = oracle.encode(inp)
+
+    assert np.array_equal(out["perm"], np.array([16 * t + j for j in range(S) for t in range(8)]))
+    cb = out["codebook"].view(np.float16).astype(np.float64)
+    assert np.array_equal(cb, np.stack([_direction(k) for k in range(16)]))
+    assert out["idx"][0].tolist() == [3, 8, 5, 10, 0] + fill_k
+    assert out["idx"][1].tolist() == list(range(16))
+    assert out["mu"].tolist() == [[0x3800], [0x3800]]          # 1/2, both rows
+    assert out["delta"].tolist() == [[0x2514], [0x2C00]]       # 1300/65536 and 1/16
+    assert out["q"][0].tolist() == [0, 63, 32, 25, 50] + fill_n
+    assert out["q"][1].tolist() == n1
+    signs = (neg * (1 << np.arange(8))).sum(-1)
+    assert np.array_equal(out["signs"], signs)
+
+
+# ---------------------------------------------------------------------------
+# Decoder-layer operations either side of the projections (Sec. 3.5 fuses the
+# permutation with them): RMSNorm, residual add, SiLU * up, one-position attention
+# ---------------------------------------------------------------------------
+
+def _h(a):
+    return np.asarray(a, np.float16).view(np.uint16)
+
+
+def test_rmsnorm_constant_vector_and_scale_invariance():
+    """RMSNorm of a constant vector c (eps = 0) is sign(c) * g exactly; scaling
+    x by a power of two changes nothing; a hand-worked pair: x = (3, 4) has
+    rms sqrt(12.5), so the outputs are 3 / sqrt(12.5) and 4 / sqrt(12.5)."""
+    g = _h(np.linspace(-2, 3, 64))
+    for c in (1.5, -0.25, 1000.0):
+        out = oracle.rmsnorm(_h(np.full((1, 64), c)), g, 0.0)
+        assert np.array_equal(out[0], _h(np.sign(c) * np.asarray(g.view(np.float16), np.float64)))
+    x = _h(np.random.default_rng(3).standard_normal((2, 64)))
+    x4 = _h(x.view(np.float16).astype(np.float64) * 4)
+    assert np.array_equal(oracle.rmsnorm(x, g, 0.0), oracle.rmsnorm(x4, g, 0.0))
+    out = oracle.rmsnorm(_h([[3.0, 4.0]]), _h([1.0, 1.0]), 0.0)
+    assert np.array_equal(out[0], _h([3 / np.sqrt(12.5), 4 / np.sqrt(12.5)]))
+    # eps enters under the root: x = (1, 1), eps = 3 -> 1 / 2
+    assert np.array_equal(oracle.rmsnorm(_h([[1.0, 1.0]]), _h([1.0, 1.0]), 3.0)[0], _h([0.5, 0.5]))
+
+
+def test_residual_add_matches_fp16_addition():
+    g = np.random.default_rng(4)
+    a = g.uniform(-8, 8, 1000).astype(np.float16)
+    b = g.uniform(-8, 8, 1000).astype(np.float16)
+    # operands within a few binades: their exact sum is an fp32 number, so
+    # NumPy's fp16 addition (fp32 sum, one rounding) is the correctly rounded sum
+    assert np.array_equal(oracle.add(a.view(np.uint16), b.view(np.uint16)), (a + b).view(np.uint16))
+
+
+def test_silu_mul_closed_forms():
+    """silu(0) = 0; silu(t) - silu(-t) = t (its odd part is t / 2); silu(ln 3)
+    = (3/4) ln 3; silu(t) -> t for large t; the product is with `up`."""
+    one = _h([1.0])
+    assert oracle.silu_mul(_h([0.0]), one)[0] == 0
+    ts = np.linspace(-6, 6, 97)
+    pos = oracle.silu_mul(_h(ts), _h(np.ones_like(ts))).view(np.float16).astype(np.float64)
+    neg = oracle.silu_mul(_h(-ts), _h(np.ones_like(ts))).view(np.float16).astype(np.float64)
+    t16 = _h(ts).view(np.float16).astype(np.float64)
+    assert np.all(np.abs((pos - neg) - t16) <= 2.0 ** -9 * np.maximum(1.0, np.abs(t16)))
+    t = np.log(3.0)
+    assert oracle.silu_mul(_h([t]), one)[0] == _h([0.75 * float(np.float16(t))])[0] or \
+        abs(float(oracle.silu_mul(_h([t]), one).view(np.float16)[0]) - 0.75 * t) <= 2.0 ** -11
+    assert oracle.silu_mul(_h([20.0]), _h([0.5]))[0] == _h([10.0])[0]
+    assert oracle.silu_mul(_h([-2.0]), _h([-3.0]))[0] == _h([-2.0 / (1 + np.exp(2.0)) * -3.0])[0]
+
+
+def test_attention_over_one_position_returns_the_kv_value_rows():
+    """With a single cached key the softmax weight is 1: query head h reads the
+    value row of key/value head h // (n_heads / n_kv)."""
+    g = np.random.default_rng(5)
+    n_heads, n_kv, hd = 8, 2, 16
+    v = _h(g.standard_normal((3, n_kv * hd)))
+    out = oracle.attend_one_position(v, n_heads, n_kv, hd)
+    ref = np.repeat(v.reshape(3, n_kv, hd), n_heads // n_kv, axis=1).reshape(3, n_heads * hd)
+    assert np.array_equal(out, ref)
