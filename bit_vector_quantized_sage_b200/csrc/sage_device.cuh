@@ -35,6 +35,31 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
+// Shared-memory loads the compiler may reorder among themselves (no
+// `volatile`, no memory clobber).  They must only be used with addresses that
+// derive from an order_token() taken after the wait that makes the data
+// valid, so that no load can be hoisted above that wait, and their results
+// must be consumed (see keep()) before the buffer is released.
+__device__ __forceinline__ uint4 lds128_r(uint32_t addr) {
+    uint4 v;
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32_r(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+// A zero the compiler cannot see through, produced in program order after the
+// preceding waits (it is a volatile statement with a memory clobber).
+__device__ __forceinline__ uint32_t order_token() {
+    uint32_t t;
+    asm volatile("mov.u32 %0, 0;" : "=r"(t)::"memory");
+    return t;
+}
+// Forces v to be computed before the next volatile statement (e.g. a buffer release).
+__device__ __forceinline__ void keep(float v) { asm volatile("" ::"f"(v)); }
+
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)

@@ -80,12 +80,10 @@ constexpr int kMaxPairsPerVirtual = 8;
 // op on the record word plus the load's immediate offset.
 __shared__ __align__(1024) uint4 g_rep[256 * 8];
 
-// Codeword at byte offset `off` of the replicas (z * 128 + r * 16).  A plain
-// C++ load, so the array's shared-memory address becomes the instruction's
-// immediate offset.
-__device__ __forceinline__ uint4 cw_load(uint32_t off) {
-    return *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(g_rep) + off);
-}
+// Codeword at byte offset `off` of the replicas (z * 128 + r * 16): an
+// explicit shared-memory load (short scoreboard) whose base is the array's
+// link-time shared address, which the assembler can fold into the load.
+__device__ __forceinline__ uint4 cw_load(uint32_t base, uint32_t off) { return lds128_r(base + off); }
 
 template <int M>
 struct Cfg {
@@ -221,6 +219,8 @@ struct Pending {
     int first;   // the CTA's first segment of the stage (split-K slot 0)
 };
 static_assert(sizeof(Pending) <= 192, "pending-segment table entry outgrew its shared memory");
+static_assert(sizeof(JobView) <= 112, "job cache entry outgrew its shared memory");
+static_assert(sizeof(EngineStage) <= 128, "stage copy outgrew its shared memory");
 
 // ------------------------------------------------------------------------
 // Shared memory
@@ -233,16 +233,18 @@ struct Smem {
     uint32_t xbuf0;     // two activation windows
     uint32_t perm0;     // the window's permutation entries (8 int32 per column)
     int slots;
-    uint32_t* posinfo;  // per window position: job << 20 | column j
+    uint32_t* posinfo;  // per window position: job slot << 20 | column j
     const int32_t** posperm;  // per window position: its 8 permutation entries (null: identity)
     float* stash;       // [slot][column part][M][256] decode sums awaiting the epilogue
     float* red;         // [kGT / 32][8] cooperative reductions
     uint64_t* bars;
     int* misc;          // [0..1] window shift k per buffer, [2] abort flag, [3] window max |x| bits,
-                        // [8] window length, [9] batch rows per window, [10] first window gathered,
+                        // [8] window length, [9] batch rows per window, [10] stages whose first window is gathered,
                         // [16..24) flush flags
     float* inv_rms;     // [8] per batch row
     struct Pending* pend;  // segments awaiting their flush (written by decode thread 0)
+    EngineStage* stc;   // the stage being gathered (copied from the parameters by the gather warp)
+    JobView* jc;        // jobs of the stage's windows, by window job slot (see posinfo)
     __device__ uint32_t slot_addr(int k) const { return ring0 + (uint32_t)k * kSlot; }
     __device__ uint64_t* full(int k) const { return bars + k; }
     __device__ uint64_t* empty(int k) const { return bars + kMaxSlots + k; }
@@ -259,11 +261,13 @@ struct Smem {
 constexpr int kBars = 2 * kMaxSlots + 9 + 2 * kStashSlots;
 
 constexpr int kPendBytes = kStashSlots * 192;  // pending-segment table (sizeof(Pending) <= 192)
+constexpr int kJobCache = 64;                    // job slots of a stage (jobs of one CTA range)
+constexpr int kJcBytes = kJobCache * 112 + 128;  // job cache (sizeof(JobView) <= 112) + stage copy
 
 template <int M>
 constexpr int fixed_smem() {
     return 2 * kXBufBytes + kPermBuf + kMaxXW * 4 + kMaxXW * 8 + Cfg<M>::kStash + (kGT / 32) * 8 * 4 + kBars * 8 +
-           64 * 4 + 8 * 4 + kPendBytes;
+           64 * 4 + 8 * 4 + kPendBytes + kJcBytes;
 }
 // Dynamic shared memory of a launch: raw codebooks + ring + fixed buffers.
 template <int M>
@@ -289,7 +293,9 @@ __device__ Smem carve(uint8_t* base, int slots, int kmax) {
     s.bars = reinterpret_cast<uint64_t*>(p); p += kBars * 8;
     s.misc = reinterpret_cast<int*>(p); p += 64 * 4;
     s.inv_rms = reinterpret_cast<float*>(p); p += 8 * 4;
-    s.pend = reinterpret_cast<Pending*>(p);
+    s.pend = reinterpret_cast<Pending*>(p); p += kPendBytes;
+    s.stc = reinterpret_cast<EngineStage*>(p); p += 128;
+    s.jc = reinterpret_cast<JobView*>(p);  // kJobCache entries of 112 bytes
     return s;
 }
 
@@ -346,22 +352,24 @@ __device__ __forceinline__ void win_break(WinPos& w) {
 // ------------------------------------------------------------------------
 // Copy warp
 // ------------------------------------------------------------------------
-// Chunks requested before the launch's first activation window is gathered:
-// the permutation entries, x and the kernel parameters must not queue behind
-// the CTA's whole share of the packed planes.
+// Chunks of a stage requested before the stage's first activation window is
+// gathered: the gather's small, latency-critical loads (permutation entries,
+// inputs, norm weights, the kernel parameters) must not queue in the memory
+// system behind the CTA's whole share of the packed planes.  After the
+// gather, HBM delivers chunks faster than the decode consumes them.
 constexpr int kStartChunks = 2;
 
 template <class Src>
 __device__ void copy_role(const Src& src, const Smem& sm, uint32_t* status, int n_cta) {
     const int lane = threadIdx.x & 31;
     int t = 0, slot = 0, ph = 0, ncb = 0;
-    bool throttled = true;
     const uint16_t* cur_cb = nullptr;
     const uint64_t pol = l2_evict_first();
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
         if (U <= 0) continue;
         const int u1 = cta_begin(U, n_cta, blockIdx.x + 1);
+        int ts = 0;  // chunks of this stage issued so far
         for (int u = cta_begin(U, n_cta, blockIdx.x); u < u1;) {
             const Seg g = make_seg(src, s, u, u1);
             u += g.jb - g.ja;
@@ -377,13 +385,12 @@ __device__ void copy_role(const Src& src, const Smem& sm, uint32_t* status, int 
                 ++ncb;
             }
             const int nc = n_chunks(g), G = g.v.d_in >> 7;
-            for (int c = 0; c < nc; ++c, ++t, ring_next(slot, ph, sm.slots)) {
-                if (throttled && t >= kStartChunks) {  // until the first window is gathered
-                    for (uint32_t i = 0; i < kWaitLimit && !*reinterpret_cast<volatile int*>(sm.misc + 10); ++i) {
+            for (int c = 0; c < nc; ++c, ++t, ++ts, ring_next(slot, ph, sm.slots)) {
+                if (ts == kStartChunks) {  // until the stage's first window is gathered
+                    for (uint32_t i = 0; i < kWaitLimit && *reinterpret_cast<volatile int*>(sm.misc + 10) <= s; ++i) {
                         if (*sm.abort_flag()) break;
                         __nanosleep(64);
                     }
-                    throttled = false;
                 }
                 if (t >= sm.slots) wait_bar(sm, sm.empty(slot), ph ^ 1, status);
                 if (lane == 0) {
@@ -409,37 +416,61 @@ __device__ void copy_role(const Src& src, const Smem& sm, uint32_t* status, int 
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 __device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
 
-__device__ __forceinline__ uint16_t ld16(const uint16_t* p, bool coherent) {
-    return coherent ? __ldcg(reinterpret_cast<const unsigned short*>(p)) : __ldg(reinterpret_cast<const unsigned short*>(p));
+// Activation loads of the gather: through L2 (data written by an earlier stage
+// of the same launch is not in any L1).  The flag is kept for the call sites.
+__device__ __forceinline__ uint16_t ld16(const uint16_t* p, bool) {
+    return __ldcg(reinterpret_cast<const unsigned short*>(p));
 }
 
-// Value of input channel c of batch row m after the stage's prologue (fp16 bits).
-template <class Src>
-__device__ __forceinline__ uint16_t prologue_value(const EngineStage& st, const JobView& v, int xr, int c, float inv,
-                                                   bool coh) {
-    switch (st.pro) {
-        case kProPlain:
-            return ld16(v.x + (size_t)xr * v.d_in + c, coh);
-        case kProRmsNorm: {
-            const float a = h2f(ld16(st.pa + (size_t)xr * st.pro_dim + c, coh));
-            return f2h(a * h2f(ld16(st.pg + c, false)) * inv);
+// The stage's prologue applied to the 8 input channels cs[] of batch row xr
+// (fp16 bits out).  All operand loads are issued before any is used, so one
+// item costs one round trip to L2.
+template <int PRO>
+__device__ __forceinline__ uint4 prologue8(const EngineStage& st, const JobView& v, int xr, const int (&cs)[8],
+                                           float inv, bool coh) {
+    uint32_t h[8];
+    if (PRO == kProPlain || PRO == kProGqa) {
+        const uint16_t* base = PRO == kProPlain ? v.x + (size_t)xr * v.d_in : st.pa + (size_t)xr * st.pro_dim;
+        uint16_t a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = PRO == kProPlain ? cs[i] : (cs[i] / (st.gqa_hd * st.gqa_grp)) * st.gqa_hd + cs[i] % st.gqa_hd;
+            a[i] = ld16(base + c, coh);
         }
-        case kProResidRmsNorm: {
-            const uint16_t r = f2h(h2f(ld16(st.pa + (size_t)xr * st.pro_dim + c, coh)) +
-                                   h2f(ld16(st.pb + (size_t)xr * st.pro_dim + c, coh)));
-            return f2h(h2f(r) * h2f(ld16(st.pg + c, false)) * inv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = a[i];
+    } else if (PRO == kProRmsNorm || PRO == kProResidRmsNorm) {
+        const uint16_t* ra = st.pa + (size_t)xr * st.pro_dim;
+        const uint16_t* rb = st.pb + (size_t)xr * st.pro_dim;
+        uint16_t a[8], b[8], g[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a[i] = ld16(ra + cs[i], coh);
+            if (PRO == kProResidRmsNorm) b[i] = ld16(rb + cs[i], coh);
+            g[i] = ld16(st.pg + cs[i], false);
         }
-        case kProSiluMul: {
-            const float gt = h2f(ld16(st.pa + (size_t)xr * st.pro_dim + c, coh));
-            const float up = h2f(ld16(st.pb + (size_t)xr * st.pro_dim + c, coh));
-            return f2h(gt / (1.0f + expf(-gt)) * up);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float x = h2f(a[i]);
+            if (PRO == kProResidRmsNorm) x = h2f(f2h(x + h2f(b[i])));  // the residual stream is fp16
+            h[i] = f2h(x * h2f(g[i]) * inv);
         }
-        default: {  // kProGqa: attention over one cached position returns the value row of the KV head
-            const int hd = st.gqa_hd, grp = st.gqa_grp;
-            const int src_c = (c / (hd * grp)) * hd + c % hd;
-            return ld16(st.pa + (size_t)xr * st.pro_dim + src_c, coh);
+    } else {  // kProSiluMul
+        const uint16_t* ra = st.pa + (size_t)xr * st.pro_dim;
+        const uint16_t* rb = st.pb + (size_t)xr * st.pro_dim;
+        uint16_t a[8], b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a[i] = ld16(ra + cs[i], coh);
+            b[i] = ld16(rb + cs[i], coh);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float gt = h2f(a[i]);
+            h[i] = f2h(gt / (1.0f + expf(-gt)) * h2f(b[i]));
         }
     }
+    return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
 }
 
 // 1 / sqrt(mean(v^2) + eps) of each batch row of the prologue's source vector
@@ -450,12 +481,24 @@ __device__ void rms_rows(const Smem& sm, const EngineStage& st, int tid, int nt,
     float part[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) part[m] = 0.f;
-    for (int c = tid; c < st.pro_dim; c += nt) {
+    constexpr int B = 8;  // loads in flight per thread and row
+    for (int c0 = tid; c0 < st.pro_dim; c0 += B * nt) {
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            float a = h2f(ld16(st.pa + (size_t)m * st.pro_dim + c, coh));
-            if (st.pro == kProResidRmsNorm) a = h2f(f2h(a + h2f(ld16(st.pb + (size_t)m * st.pro_dim + c, coh))));
-            part[m] = fmaf(a, a, part[m]);
+            uint16_t a[B], b[B];
+#pragma unroll
+            for (int r = 0; r < B; ++r) {
+                const int c = c0 + r * nt;
+                a[r] = c < st.pro_dim ? ld16(st.pa + (size_t)m * st.pro_dim + c, coh) : (uint16_t)0;
+                b[r] = (st.pro == kProResidRmsNorm && c < st.pro_dim) ? ld16(st.pb + (size_t)m * st.pro_dim + c, coh)
+                                                                      : (uint16_t)0;
+            }
+#pragma unroll
+            for (int r = 0; r < B; ++r) {
+                float x = h2f(a[r]);
+                if (st.pro == kProResidRmsNorm) x = h2f(f2h(x + h2f(b[r])));
+                part[m] = fmaf(x, x, part[m]);
+            }
         }
     }
 #pragma unroll
@@ -476,36 +519,34 @@ __device__ void rms_rows(const Smem& sm, const EngineStage& st, int tid, int nt,
 // Gathers the window's x_perm for items e = tid, tid + nt, ... of (batch row,
 // position) and stores them (fp16, unscaled) into the window buffer; returns
 // the largest |x| bit pattern seen.
-template <int M, class Src>
-__device__ uint32_t gather_items(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid, int nt,
-                                 bool coh) {
-    const EngineStage& st = src.stage(s);
+template <int M, int PRO, class Src>
+__device__ uint32_t gather_items_k(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid,
+                                   int nt, bool coh) {
+    const EngineStage& st = *sm.stc;
     const int mrows = sm.misc[9];  // batch rows a window holds (<= M)
     uint32_t mx = 0;
     for (int e = tid; e < mrows * wlen; e += nt) {
         const int m = e / wlen, p = e - m * wlen;
         const uint32_t info = sm.posinfo[p];
-        const JobView v = src.job((int)(info >> 20));
+        const JobView& v = sm.jc[info >> 20];
         const int j = (int)(info & 0xfffffu);
         uint4 val = make_uint4(0, 0, 0, 0);
         if (m < v.Mk) {
             const int xr = v.xrows ? v.xrows[m] : m;
-            const float inv = sm.inv_rms[m < 8 ? m : 0];
-            if (st.pro == kProPlain && !v.perm) {
+            if (PRO == kProPlain && !v.perm) {
                 const uint16_t* row = v.x + (size_t)xr * v.d_in + j * 8;
-                val = coh ? __ldcg(reinterpret_cast<const uint4*>(row)) : __ldg(reinterpret_cast<const uint4*>(row));
+                val = __ldcg(reinterpret_cast<const uint4*>(row));
             } else {
-                uint32_t h[8];
+                int cs[8];
                 if (v.perm) {
                     const uint4 pa = lds128(sm.perm0 + p * 32), pb = lds128(sm.perm0 + p * 32 + 16);
-                    const int cs[8] = {(int)pa.x, (int)pa.y, (int)pa.z, (int)pa.w, (int)pb.x, (int)pb.y, (int)pb.z, (int)pb.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) h[i] = prologue_value<Src>(st, v, xr, cs[i], inv, coh);
+                    cs[0] = (int)pa.x; cs[1] = (int)pa.y; cs[2] = (int)pa.z; cs[3] = (int)pa.w;
+                    cs[4] = (int)pb.x; cs[5] = (int)pb.y; cs[6] = (int)pb.z; cs[7] = (int)pb.w;
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) h[i] = prologue_value<Src>(st, v, xr, j * 8 + i, inv, coh);
+                    for (int i = 0; i < 8; ++i) cs[i] = j * 8 + i;
                 }
-                val = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+                val = prologue8<PRO>(st, v, xr, cs, sm.inv_rms[m < 8 ? m : 0], coh);
             }
         }
         sts128(xb + (uint32_t)(m * xw + p) * 16, val);
@@ -514,6 +555,18 @@ __device__ uint32_t gather_items(const Src& src, const Smem& sm, int s, int wlen
         mx = max(mx, max(a & 0xffffu, a >> 16));
     }
     return mx;
+}
+
+template <int M, class Src>
+__device__ uint32_t gather_items(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid, int nt,
+                                 bool coh) {
+    switch (sm.stc->pro) {  // uniform: one specialised loop per prologue
+        case kProRmsNorm: return gather_items_k<M, kProRmsNorm>(src, sm, s, wlen, xw, xb, tid, nt, coh);
+        case kProResidRmsNorm: return gather_items_k<M, kProResidRmsNorm>(src, sm, s, wlen, xw, xb, tid, nt, coh);
+        case kProSiluMul: return gather_items_k<M, kProSiluMul>(src, sm, s, wlen, xw, xb, tid, nt, coh);
+        case kProGqa: return gather_items_k<M, kProGqa>(src, sm, s, wlen, xw, xb, tid, nt, coh);
+        default: return gather_items_k<M, kProPlain>(src, sm, s, wlen, xw, xb, tid, nt, coh);
+    }
 }
 
 // Power-of-two prescale of a window: k such that every |x| / 2^k <= 2^14, so
@@ -543,7 +596,7 @@ __device__ void rescale_items(const Smem& sm, int wlen, int xw, uint32_t xb, int
 // the decode warps together (tid in [0, kGT)).
 template <int M, class Src>
 __device__ void coop_window(const Src& src, const Smem& sm, int s, int w, int xw, bool coh, int tid) {
-    const EngineStage& st = src.stage(s);
+    const EngineStage& st = *sm.stc;
     named_barrier(kBarGather, kGT);  // inputs ready, permutation entries landed, buffer free
     if (st.pro == kProRmsNorm || st.pro == kProResidRmsNorm) {
         rms_rows<M>(sm, st, tid, kGT, coh);
@@ -590,7 +643,7 @@ __device__ void load_perm(const Smem& sm, int wlen, int lane) {
 
 // Fills window `win` (wlen positions, recorded in posinfo) of stage s.
 template <int M, class Src>
-__device__ __noinline__ void fill_window(const Src& src, const Smem& sm, uint32_t* status, unsigned* sync, int s,
+__device__ __forceinline__ void fill_window(const Src& src, const Smem& sm, uint32_t* status, unsigned* sync, int s,
                                          int win, int wlen, int xw, bool first, bool need_pdl) {
     const int lane = threadIdx.x & 31;
     const EngineStage& st = src.stage(s);
@@ -609,7 +662,7 @@ __device__ __noinline__ void fill_window(const Src& src, const Smem& sm, uint32_
     __syncwarp();
     if (first) {
         coop_window<M>(src, sm, s, win, xw, coh, kDT + lane);
-        if (lane == 0) *reinterpret_cast<volatile int*>(sm.misc + 10) = 1;  // release the copy warp
+        if (lane == 0) *reinterpret_cast<volatile int*>(sm.misc + 10) = s + 1;  // release the copy warp
     } else {
         uint32_t mx = gather_items<M>(src, sm, s, wlen, xw, sm.xwin(win), lane, 32, coh);
         for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -632,12 +685,22 @@ __device__ void gather_role(const Src& src, const Smem& sm, uint32_t* status, un
         if (U <= 0) continue;
         const int u0 = cta_begin(U, n_cta, blockIdx.x), u1 = cta_begin(U, n_cta, blockIdx.x + 1);
         win_break(wp);
+        if (u0 < u1) {  // the stage's descriptor, for this warp and the cooperative gather
+            __syncwarp();
+            if (lane == 0) *sm.stc = src.stage(s);
+            __syncwarp();
+        }
         // walk the stage's chunks; a window is filled when the next chunk opens a new one (or at the end)
-        int wlen = 0, cur = -1;
+        int wlen = 0, cur = -1, base = -1, last_id = -1;
         bool first = true;
         for (int u = u0; u < u1;) {
             const Seg g = make_seg(src, s, u, u1);
             u += g.jb - g.ja;
+            if (base < 0) base = g.v.id;
+            if (g.v.id != last_id) {  // cache the job's view: the gather reads it from shared memory
+                if (lane == 0) sm.jc[g.v.id - base] = g.v;
+                last_id = g.v.id;
+            }
             const int nc = n_chunks(g);
             for (int c = 0; c < nc; ++c) {
                 const int2 cc = chunk_cols(g, c);
@@ -654,7 +717,7 @@ __device__ void gather_role(const Src& src, const Smem& sm, uint32_t* status, un
                     __syncwarp();  // the filled window's positions are no longer read
                 }
                 if (lane < nj) {
-                    sm.posinfo[pos + lane] = ((uint32_t)g.v.id << 20) | (uint32_t)(cc.x + lane);
+                    sm.posinfo[pos + lane] = ((uint32_t)(g.v.id - base) << 20) | (uint32_t)(cc.x + lane);
                     sm.posperm[pos + lane] = g.v.perm ? g.v.perm + (size_t)(cc.x + lane) * 8 : nullptr;
                 }
                 wlen = pos + nj;
@@ -693,10 +756,11 @@ struct RowPair {
 // fp16 dot products leave room on, instead of the integer ALU pipe that the
 // masks and field extraction already load.
 template <int MK>
-__device__ __forceinline__ void decode_word(const VDec& d, uint32_t lane_off, uint32_t w, int t, const RowPair& rp,
+__device__ __forceinline__ void decode_word(const VDec& d, uint32_t rep, uint32_t lane_off, uint32_t w, int t,
+                                            const RowPair& rp,
                                             const uint4 (&xv)[MK], float (&accA)[MK], float (&accB)[MK]) {
     {   // row A: z at [7, 7 + log2K), q at [23 - V, 23); signs in slots 0..2 and aux
-        uint4 c = cw_load((w & d.zmask) | lane_off);
+        uint4 c = cw_load(rep, (w & d.zmask) | lane_off);
         c.x ^= (w * d.m0) & 0x80008000u;
         c.y ^= (w * d.m1) & 0x80008000u;
         c.z ^= (w * d.m2) & 0x80008000u;
@@ -708,7 +772,7 @@ __device__ __forceinline__ void decode_word(const VDec& d, uint32_t lane_off, ui
     {   // row B: its fields sit 16 bits higher (z, from w >> 16) and lower (q, from w << 16);
         // signs in slots 3..5 (slot 5 at bit 15) and aux
         const uint32_t whi = __umulhi(w, d.m16), wlo = w * d.m16;
-        uint4 c = cw_load((whi & d.zmask) | lane_off);
+        uint4 c = cw_load(rep, (whi & d.zmask) | lane_off);
         c.x ^= (w * d.m3) & 0x80008000u;
         c.y ^= (w * d.m4) & 0x80008000u;
         c.z ^= w & 0x80008000u;
@@ -732,10 +796,14 @@ __device__ __forceinline__ void decode_chunk(const Smem& sm, const Seg& g, const
     const int grp = ((cc.x >> 5) << 1) + part;           // this thread's radius group
     const int lo = max(cc.x, grp << 4), hi = min(cc.y, (grp + 1) << 4);
     if (o >= g.n_oct || lo >= hi) return;
-    const uint32_t base = sm.slot_addr(k);
+    // every load below derives its address from a token taken after the
+    // caller's waits on this chunk and its activation window
+    const uint32_t tok = order_token();
+    const uint32_t base = sm.slot_addr(k) + tok;
+    const uint32_t rep = static_cast<uint32_t>(__cvta_generic_to_shared(g_rep)) + tok;
     RowPair rp;
     {
-        const uint4 mt = lds128(base + kMainSlot + (uint32_t)(((grp - gfirst) * g.n_oct + o) * 64 + wi * 16));
+        const uint4 mt = lds128_r(base + kMainSlot + (uint32_t)(((grp - gfirst) * g.n_oct + o) * 64 + wi * 16));
         const float2 a = __half22float2(u2h2(mt.y)), b = __half22float2(u2h2(mt.w));
         rp.dlA = a.y * d.vscale * sc;
         rp.mpA = a.x * sc - rp.dlA;
@@ -747,26 +815,32 @@ __device__ __forceinline__ void decode_chunk(const Smem& sm, const Seg& g, const
     const uint32_t lane_off = (uint32_t)(lane & 7) << 4;  // this lane's replica
     const uint32_t rstride = (uint32_t)g.n_oct * 16;
     const uint32_t wbase = base + (uint32_t)(o * 16 + wi * 4) + (uint32_t)(lo - cc.x) * rstride;
-    const uint32_t xbase = xw0 + (uint32_t)(lo - cc.x) * 16;
+    const uint32_t xbase = xw0 + tok + (uint32_t)(lo - cc.x) * 16;
     if (hi - lo == 16) {  // a whole radius group: fixed trip count, constant shifts
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-            const uint32_t w = lds32(wbase + (uint32_t)t * rstride);
+            const uint32_t w = lds32_r(wbase + (uint32_t)t * rstride);
             uint4 xv[MK];
 #pragma unroll
-            for (int m = 0; m < MK; ++m) xv[m] = lds128(xbase + (uint32_t)m * xstride + (uint32_t)t * 16);
-            decode_word<MK>(d, lane_off, w, t, rp, xv, accA, accB);
+            for (int m = 0; m < MK; ++m) xv[m] = lds128_r(xbase + (uint32_t)m * xstride + (uint32_t)t * 16);
+            decode_word<MK>(d, rep, lane_off, w, t, rp, xv, accA, accB);
         }
     } else {
 #pragma unroll 2
         for (int j = lo; j < hi; ++j) {
             const uint32_t r = (uint32_t)(j - lo);
-            const uint32_t w = lds32(wbase + r * rstride);
+            const uint32_t w = lds32_r(wbase + r * rstride);
             uint4 xv[MK];
 #pragma unroll
-            for (int m = 0; m < MK; ++m) xv[m] = lds128(xbase + (uint32_t)m * xstride + r * 16);
-            decode_word<MK>(d, lane_off, w, j & 15, rp, xv, accA, accB);
+            for (int m = 0; m < MK; ++m) xv[m] = lds128_r(xbase + (uint32_t)m * xstride + r * 16);
+            decode_word<MK>(d, rep, lane_off, w, j & 15, rp, xv, accA, accB);
         }
+    }
+    // the chunk's sums exist before the caller releases the ring slot
+#pragma unroll
+    for (int m = 0; m < MK; ++m) {
+        keep(accA[m]);
+        keep(accB[m]);
     }
 }
 
