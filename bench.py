@@ -1,25 +1,30 @@
 #!/usr/bin/env python
 """Benchmark: batch-1 packed SAGE GEMV over a Qwen3-4B-shaped decoder layer on B200.
 
-A step is one decoder layer's seven packed linears at batch 1, launched as its
-four dependency stages (q|k|v, o, gate|up, down; one grouped GEMV launch each,
-chained with programmatic dependent launch).  Inputs are synthetic (seeded, see
-synth/), resident in HBM; every step reads a different copy of the layer's
-packed planes so the working set (>= 4 x the 126 MB L2) comes from HBM.
+A step is the packed GEMV work of one decoder layer at batch 1: its seven
+projections (q, k, v, o, gate, up, down; hidden 2560) computed straight from
+2.25-bit codes in ONE launch of the libsage engine (sage_gemv_grouped over the
+seven matrices, each with its own synthetic fp16 input row).  Every step reads
+a different copy of the layer's packed planes, so the working set (> 4 x the
+126 MB L2) comes from HBM.  Reported alongside (under "extra"): the same layer
+as its four dependent stages in one launch with the operations between them
+fused (sage_decoder_layer_forward), the four stages as four launches, the
+4096 -> 12288 batch sweep through the GEMV and tcgen05 paths, and the
+grouped-expert MoE GEMV.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-Prints ONE JSON line (rank 0).  ``value`` is the whole-job throughput in GB/s of
-packed bytes (codes + mu/delta + codebooks + x + y) per layer; ``us_per_layer``
-is the device time of one layer.  ``--impl reference`` times the CPU oracle on a
-bounded sample of the same workload instead.
+Prints ONE JSON line (rank 0).  ``value`` is the whole-job throughput in GB/s
+of packed bytes (codes + mu/delta + codebooks + x + y) per layer; ``us_per_layer``
+is the device time of one layer.  ``--impl reference`` times the CPU oracle on
+a bounded sample of the same workload instead.
 """
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -32,9 +37,17 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 packed VQ GEMV µs/layer and achieved HBM GB/s vs B200 peak"
-WORKLOAD = "Qwen3-4B-shaped decoder layer, 7 packed linears (q,k,v,o,gate,up,down), hidden 2560, batch 1"
+LAYER_SHAPES = "q 2560->4096, k/v 2560->1024, o 4096->2560, gate/up 2560->9728, down 9728->2560"
+
+
+def workload(mode: str) -> str:
+    how = {"fused": "the decoder layer in one launch", "stages": "its four dependency stages as four launches",
+           "grouped7": "the seven projections in one grouped launch"}[mode]
+    return f"Qwen3-4B-shaped decoder layer at batch 1, 7 packed linears ({LAYER_SHAPES}), {how}"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
+KERNEL = "engine_kernel<1> (libsage packed GEMV engine, sm_100a)"
 
 
 def _peaks():
@@ -45,6 +58,16 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def _peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["bf16_tflops"]), "measured (bf16 burst; fp16 dense has the same nominal rate)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def max_over_ranks(ms: float, dist, device) -> float:
@@ -70,75 +93,41 @@ def _dist():
     return ws, rank, local
 
 
-# ---------------------------------------------------------------------------
-# Workload construction (product path only: synth + libsage)
-# ---------------------------------------------------------------------------
-
-def build_layer(replicas: int):
-    import torch
-    import synth
-    import bit_vector_quantized_sage_b200 as sage
-    L = synth.config1()
-    base = {}
-    for f in L.mats:
-        f.perm = sage.sage_esg_permutation(L.energies[f.name])
-        base[f.name] = sage.PackedMatrix.from_fields(f)
-    layers = []
-    for r in range(replicas):
-        if r == 0:
-            layers.append(base)
-            continue
-        layers.append({n: sage.PackedMatrix(m.d_out, m.d_in, m.log2K, m.main.clone(), m.meta.clone(),
-                                            m.codebook.clone(), m.perm.clone() if m.perm is not None else None, n)
-                       for n, m in base.items()})
-    xs = {s[0]: torch.from_numpy(L.xs[s[0]].view(np.int16)).cuda() for s in synth.QWEN3_4B_STAGES}
-    return L, layers, xs
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return platform.processor() or "unknown"
 
 
-def layer_bytes(mats, M=1):
-    """Algorithmic bytes of one layer: packed planes + codebooks + x + y (perm excluded)."""
-    tot = 0
-    perm = 0
-    for m in mats.values():
-        tot += m.packed_bytes + (1 << m.log2K) * 16 + M * m.d_in * 2 + M * m.d_out * 2
-        perm += m.d_in * 4 if m.perm is not None else 0
-    return tot, perm
-
-
-class LayerRunner:
-    """Pre-marshalled grouped launches for one layer replica."""
-
-    def __init__(self, mats, xs, ys, ws):
-        import synth
-        import bit_vector_quantized_sage_b200 as sage
-        self.calls = []
-        for stage in synth.QWEN3_4B_STAGES:
-            ms = [mats[n] for n in stage]
-            self.calls.append(sage.GroupedCall(ms, [xs[stage[0]]] * len(stage), [ys[n] for n in stage], 1, ws))
-
-    def __call__(self, stream=None):
-        for c in self.calls:
-            c(stream)
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.proc = None
-        # SAGE_CLOCKS_DIR keeps the raw samples (one CSV per rank); default: a temp file
-        d = os.environ.get("SAGE_CLOCKS_DIR")
+        d = os.environ.get("SAGE_CLOCKS_DIR")  # keeps the raw samples (one CSV per rank)
         self.path = (os.path.join(d, f"clocks_rank{gpu_index}.csv") if d and os.path.isdir(d)
                      else os.path.join(tempfile.gettempdir(), f"sage_clocks_{os.getpid()}_{gpu_index}.csv"))
         self.gpu = gpu_index
 
     def start(self):
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
@@ -153,7 +142,7 @@ class Clocks:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], None, set()
+        sm, mx, power, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             p = [x.strip() for x in line.split(",")]
@@ -162,107 +151,344 @@ class Clocks:
             try:
                 sm.append(float(p[1]))
                 mx = float(p[2])
+                power.append(float(p[3]))
             except ValueError:
                 continue
             for nm, v in zip(names, p[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "samples": len(sm),
+                "power_w": statistics.median(power) if power else None, "reasons": sorted(reasons)}
 
 
-def _traffic_for(kernel_src_hash: str):
-    p = os.path.join(ROOT, "profiles", "gemv_traffic.json")
-    try:
-        d = json.load(open(p))
-    except Exception:
-        return None, None
-    if d.get("source_sha256") != kernel_src_hash:
-        return None, d.get("source_sha256")
-    return d.get("traffic_bytes_per_launch"), d.get("source_sha256")
-
-
-def _kernel_hash():
+def kernel_source_hash() -> str:
+    """sha256 over the engine's sources: DRAM counters taken on other sources are stale."""
+    import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_vector_quantized_sage_b200", "csrc")
-    for n in ("sage_gemv.cu", "sage_device.cuh"):
+    for n in ("sage_gemv.cu", "sage_device.cuh", "sage_engine.h", "sage_layer.cpp"):
         h.update(open(os.path.join(csrc, n), "rb").read())
     return h.hexdigest()
 
 
-def cpu_oracle_sample(rows_per_matrix: int = 256, seconds_cap: float = 60.0):
-    """Times the CPU oracle (unpack + fp32 reconstruction + fp64 matvec) on the first
-    ``rows_per_matrix`` rows of each of the layer's seven matrices, single-threaded.
-    Returns (GB/s of packed bytes, sample description, cores used)."""
+def traffic_for(mode: str):
+    """DRAM bytes (read + write) per launch of the timed kernel from the committed ncu
+    summary, or None when the summary was taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "engine_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None, "no committed ncu DRAM capture"
+    if d.get("source_sha256") != kernel_source_hash():
+        return None, "ncu DRAM capture taken on other kernel sources"
+    e = d.get("modes", {}).get(mode)
+    if not e:
+        return None, f"no ncu DRAM capture for mode {mode}"
+    return e["dram_bytes_per_launch"], e.get("note", "")
+
+
+def dist_summary(samples_us):
+    a = np.asarray(samples_us, dtype=np.float64)
+    return {"median": round(float(np.median(a)), 3), "p10": round(float(np.percentile(a, 10)), 3),
+            "p90": round(float(np.percentile(a, 90)), 3), "n": int(a.size)}
+
+
+# ---------------------------------------------------------------------------
+# The CPU oracle as a timed baseline: unpack of the packed planes, fp32
+# reconstruction and fp64 matvec (oracle/), one process per core, each on its
+# own share of 256-row blocks.  The planes come from the oracle's own packer,
+# so nothing here runs the library.
+# ---------------------------------------------------------------------------
+
+_ORACLE_DATA = {}
+
+
+def _oracle_source(kind: str, name: str):
+    """(code fields, x) of one matrix of a workload, built once per process."""
+    key = (kind, name)
+    if key in _ORACLE_DATA:
+        return _ORACLE_DATA[key]
     import oracle
+    import synth
+    if kind == "layer":
+        if "layer" not in _ORACLE_DATA:
+            L = synth.config1()
+            for f in L.mats:
+                f.perm = oracle.esg_perm(L.energies[f.name])
+            _ORACLE_DATA["layer"] = L
+        L = _ORACLE_DATA["layer"]
+        f = next(m for m in L.mats if m.name == name)
+        x = L.xs[[s for s in synth.QWEN3_4B_STAGES if name in s][0][0]]
+    elif kind == "up8b":
+        f, x = synth.config3(1)
+    else:  # "moe:<proj>:<expert>", T = 1 token
+        _, proj, e = name.split(":")
+        spec = synth.config4(1)
+        f = spec.expert(int(e), int(proj))
+        x = spec.x if int(proj) < 2 else spec.x_down[:1]
+    _ORACLE_DATA[key] = (f, x)
+    return f, x
+
+
+def _oracle_prepare(task):
+    import oracle
+    import synth
+    kind, name, r0, r1 = task
+    f, x = _oracle_source(kind, name)
+    R = r1 - r0
+    main, meta = oracle.pack(R, f.d_in, f.log2K, f.signs[r0:r1], f.idx[r0:r1], f.q[r0:r1], f.mu[r0:r1],
+                             f.delta[r0:r1])
+    nbytes = main.nbytes + meta.nbytes + (1 << f.log2K) * 16 + x.nbytes + x.shape[0] * R * 2
+    return (f, x, R, main, meta, nbytes)
+
+
+def _oracle_run(prep):
+    import oracle
+    import synth
+    f, x, R, main, meta, _ = prep
+    u = oracle.unpack(R, f.d_in, f.log2K, main, meta)
+    g = synth.Fields(R, f.d_in, f.log2K, u["signs"], u["idx"], u["q"], u["mu"], u["delta"], f.codebook, f.perm)
+    return oracle.gemv(g, x)
+
+
+def _oracle_worker(inq, outq):
+    sys.path.insert(0, ROOT)
+    while True:
+        tasks = inq.get()
+        if tasks is None:
+            return
+        preps = [_oracle_prepare(t) for t in tasks]
+        outq.put(("ready", None))
+        inq.get()  # go
+        t0 = time.perf_counter()
+        for p in preps:
+            _oracle_run(p)
+        t1 = time.perf_counter()
+        outq.put(("done", (sum(p[-1] for p in preps), t0, t1)))
+
+
+class OraclePool:
+    """Persistent spawn-context worker processes (safe next to a CUDA context)."""
+
+    def __init__(self, n: int):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        self.n = n
+        self.inq = [ctx.Queue() for _ in range(n)]
+        self.outq = ctx.Queue()
+        self.procs = [ctx.Process(target=_oracle_worker, args=(self.inq[i], self.outq), daemon=True)
+                      for i in range(n)]
+        for p in self.procs:
+            p.start()
+
+    def run(self, shards):
+        """shards: one task list per worker.  Returns (bytes, wall seconds from the first
+        worker's start to the last one's end)."""
+        active = [i for i in range(self.n) if shards[i]]
+        for i in active:
+            self.inq[i].put(shards[i])
+        for _ in active:
+            self.outq.get()
+        for i in active:
+            self.inq[i].put("go")
+        res = [self.outq.get()[1] for _ in active]
+        nbytes = sum(r[0] for r in res)
+        return nbytes, max(r[2] for r in res) - min(r[1] for r in res)
+
+    def close(self):
+        for q in self.inq:
+            q.put(None)
+        for p in self.procs:
+            p.join(timeout=10)
+
+
+def layer_block_tasks():
+    """(kind, matrix, r0, r1) for every 256-row block of the seven layer matrices, with its
+    weight count as cost."""
+    import synth
+    out = []
+    for name, d_out, d_in in synth.QWEN3_4B_LAYER:
+        for r0 in range(0, d_out, 256):
+            r1 = min(d_out, r0 + 256)
+            out.append((("layer", name, r0, r1), (r1 - r0) * d_in))
+    return out
+
+
+def shard(tasks_with_cost, n):
+    """Longest-processing-time split of the tasks over n workers."""
+    loads = [0] * n
+    shards = [[] for _ in range(n)]
+    for t, c in sorted(tasks_with_cost, key=lambda tc: -tc[1]):
+        i = int(np.argmin(loads))
+        shards[i].append(t)
+        loads[i] += c
+    return shards
+
+
+def oracle_layer_baseline(pool_1, pool_n, fraction: float = 1.0, offset: int = 0):
+    """Oracle GB/s on `fraction` of the layer's blocks (every 1/fraction-th block from
+    `offset`): once on one core, once on all of pool_n's cores."""
+    tasks = layer_block_tasks()
+    if fraction < 1.0:
+        step = max(1, int(round(1.0 / fraction)))
+        tasks = tasks[offset % step::step]
+    out = {}
+    for label, pool in (("1", pool_1), ("n", pool_n)):
+        if pool is None:
+            continue
+        b, s = pool.run(shard(tasks, pool.n))
+        out[label] = (b / s / 1e9, s, pool.n)
+    return out, len(tasks)
+
+
+# ---------------------------------------------------------------------------
+# Workload construction (product path: synth + libsage)
+# ---------------------------------------------------------------------------
+
+def clone_matrix(m):
+    import bit_vector_quantized_sage_b200 as sage
+    return sage.PackedMatrix(m.d_out, m.d_in, m.log2K, m.main.clone(), m.meta.clone(), m.codebook.clone(),
+                             m.perm.clone() if m.perm is not None else None, m.name)
+
+
+def layer_bytes(mats, M=1):
+    """Algorithmic bytes of one layer: packed planes + codebooks + x + y (perm excluded)."""
+    tot = perm = 0
+    for m in mats.values():
+        tot += m.packed_bytes + (1 << m.log2K) * 16 + M * m.d_in * 2 + M * m.d_out * 2
+        perm += m.d_in * 4 if m.perm is not None else 0
+    return tot, perm
+
+
+def build_layers():
+    """Seeded Qwen3-4B-shaped layer (ESG permutations from its channel energies) and
+    enough device copies of its packed planes that rotating through them streams
+    more than 4 x L2 from HBM."""
     import synth
     import bit_vector_quantized_sage_b200 as sage
     L = synth.config1()
-    tot_bytes, tot_s = 0, 0.0
+    base = {}
     for f in L.mats:
         f.perm = sage.sage_esg_permutation(L.energies[f.name])
-        x = L.xs[[s for s in synth.QWEN3_4B_STAGES if f.name in s][0][0]]
-        R = min(rows_per_matrix, f.d_out)
-        # row-octet slice of the planes for the first R rows
-        sub = synth.Fields(R, f.d_in, f.log2K, f.signs[:R], f.idx[:R], f.q[:R], f.mu[:R], f.delta[:R],
-                           f.codebook, f.perm, f.name)
-        m_sub, t_sub = sage.sage_pack(R, f.d_in, f.log2K, sub.signs, sub.idx, sub.q, sub.mu, sub.delta)
-        t0 = time.perf_counter()
-        u = oracle.unpack(R, f.d_in, f.log2K, m_sub, t_sub)
-        g = synth.Fields(R, f.d_in, f.log2K, u["signs"], u["idx"], u["q"], u["mu"], u["delta"], f.codebook, f.perm)
-        oracle.gemv(g, x)
-        tot_s += time.perf_counter() - t0
-        mb, tb = sage.sage_packed_sizes(R, f.d_in, f.log2K)
-        tot_bytes += mb + tb + (1 << f.log2K) * 16 + f.d_in * 2 + R * 2
-        if tot_s > seconds_cap:
-            break
-    desc = (f"first {rows_per_matrix} rows of each of the 7 layer matrices" if rows_per_matrix < 9728
-            else "the whole layer, all 7 matrices") + " (unpack + reconstruct + fp64 matvec, single thread)"
-    return tot_bytes / tot_s / 1e9, desc, 1, tot_s
+        base[f.name] = sage.PackedMatrix.from_fields(f)
+    nbytes, _ = layer_bytes(base)
+    replicas = max(2, int(np.ceil(4 * L2_BYTES / nbytes)) + 1)
+    layers = [base] + [{n: clone_matrix(m) for n, m in base.items()} for _ in range(replicas - 1)]
+    return L, layers
 
 
-def _peak_tflops():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    try:
-        with open(p) as fh:
-            d = json.load(fh)
-        return float(d["bf16_tflops"]), "measured (bf16 burst; fp16 dense has the same nominal rate)"
-    except Exception:
-        return 1590.0, "fallback"
+class LayerStages:
+    """The layer's four dependency stages (q|k|v, o, gate|up, down) as four grouped
+    launches chained with programmatic dependent launch; synthetic stage inputs."""
+    launches = 4
+
+    def __init__(self, lay, xs, ys, ws):
+        import synth
+        import bit_vector_quantized_sage_b200 as sage
+        self.calls = [sage.GroupedCall([lay[n] for n in st], [xs[st[0]]] * len(st), [ys[n] for n in st], 1, ws)
+                      for st in synth.QWEN3_4B_STAGES]
+
+    def __call__(self, stream=None):
+        for c in self.calls:
+            c(stream)
 
 
-def _timed_calls(fn, stream, reps, flush):
-    """Median device time (ms) of one fn call with L2 flushed before each call.
-    The call is captured once in a CUDA graph; the flush is enqueued first, so
-    the host side of the replay overlaps it and the events bracket device work
-    only."""
+class LayerGrouped7:
+    """All seven projections in one grouped launch, each on its own synthetic input (no
+    dependencies between them)."""
+    launches = 1
+
+    def __init__(self, lay, xs, ys, ws):
+        import synth
+        import bit_vector_quantized_sage_b200 as sage
+        xmap = {n: xs[[st for st in synth.QWEN3_4B_STAGES if n in st][0][0]] for n in lay}
+        names = list(lay)
+        self.call = sage.GroupedCall([lay[n] for n in names], [xmap[n] for n in names], [ys[n] for n in names], 1, ws)
+
+    def __call__(self, stream=None):
+        self.call(stream)
+
+
+def make_runners(mode, layers, L):
+    """Per-replica callables for one layer mode, plus their shared device inputs/outputs,
+    workspace and the host-visible input/output tensors of an end-to-end step."""
+    import torch
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    base = layers[0]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+    if mode == "fused":
+        inp = synth.decoder_inputs(1, 1, 2560)
+        h = dev(inp.h)
+        outs = {n: torch.zeros((1, m.d_out), dtype=torch.int16, device="cuda") for n, m in base.items()}
+        outs["h_out"] = torch.zeros((1, 2560), dtype=torch.int16, device="cuda")
+        nh, nkv, hd = synth.QWEN3_4B_HEADS
+        an, mn = dev(inp.attn_norm), dev(inp.mlp_norm)
+        runs = [sage.DecoderLayer(lay, an, mn, nh, nkv, hd, inp.eps, outs, 1) for lay in layers]
+        ws = runs[0].ws
+        for r in runs:
+            r.ws = ws
+        fns = [lambda st, r=r: r(h, st) for r in runs]
+        return fns, ws, {"h": (h, inp.h)}, {"h_out": outs["h_out"]}, 1
+    xs = {k: dev(v) for k, v in L.xs.items()}
+    ys = {n: torch.zeros((1, m.d_out), dtype=torch.int16, device="cuda") for n, m in base.items()}
+    if mode == "stages":
+        ws = sage.Workspace(max(sage.sage_workspace_size(sage.SAGE_OP_GROUPED, [base[n] for n in st], 1)
+                                for st in synth.QWEN3_4B_STAGES))
+        runs = [LayerStages(lay, xs, ys, ws) for lay in layers]
+    else:
+        ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_GROUPED, list(base.values()), 1))
+        runs = [LayerGrouped7(lay, xs, ys, ws) for lay in layers]
+    fns = [lambda st, r=r: r(st) for r in runs]
+    return fns, ws, {k: (xs[k], L.xs[k]) for k in xs}, ys, runs[0].launches
+
+
+# ---------------------------------------------------------------------------
+# Device timing
+# ---------------------------------------------------------------------------
+
+def capture(fn, stream):
     import torch
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         fn(torch.cuda.current_stream())
-    g.replay()
-    times = []
-    for _ in range(reps):
-        flush.fill_(1)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+    return g
+
+
+def per_call_us(fns, stream, rounds=4):
+    """Device time of each call, one CUDA graph per call replayed back to back with
+    events between the replays; `fns` rotate over copies of the data larger than L2.
+    Returns the list of per-call times (us)."""
+    import torch
+    graphs = [capture(f, stream) for f in fns]
+    for g in graphs:
         g.replay()
-        e1.record(stream)
-        e1.synchronize()
-        times.append(e0.elapsed_time(e1))
-    del g
-    return statistics.median(times)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) * rounds + 1)]
+    ev[0].record(stream)
+    k = 1
+    for _ in range(rounds):
+        for g in graphs:
+            g.replay()
+            ev[k].record(stream)
+            k += 1
+    torch.cuda.synchronize()
+    out = [ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(len(ev) - 1)]
+    del graphs
+    return out
 
 
-def bench_gemm(stream, flush, reps=20):
-    """Config 3: 4096 -> 12288, (K,V) = (32,5); batch 1-8 through the GEMV
-    kernel, 16-128 through the tcgen05 path (sage_gemm).  Per batch: device us,
-    TFLOP/s against the measured dense fp16 peak and GB/s of packed bytes."""
+def bench_gemm(stream, reps_rounds=3):
+    """4096 -> 12288 up-projection, (K,V) = (32,5): batch 1-8 through the GEMV engine,
+    16-128 through the tcgen05 path (sage_gemm dispatches).  Per batch: device us
+    (median, p10, p90 over copies of the planes larger than L2), TFLOP/s against the
+    dense fp16 tensor peak and GB/s of packed bytes against HBM."""
     import torch
     import synth
     import bit_vector_quantized_sage_b200 as sage
     f, _ = synth.config3(1)
-    A = sage.PackedMatrix.from_fields(f)
+    A0 = sage.PackedMatrix.from_fields(f)
+    As = [A0] + [clone_matrix(A0) for _ in range(int(np.ceil(2 * L2_BYTES / A0.packed_bytes)))]
     peak, kind = _peak_tflops()
     hbm, _ = _peaks()
     out = []
@@ -270,29 +496,31 @@ def bench_gemm(stream, flush, reps=20):
         _, xb = synth.config3(M)
         x = torch.from_numpy(xb.view(np.int16)).cuda()
         y = torch.zeros((M, f.d_out), dtype=torch.int16, device="cuda")
-        ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_GEMM, A, M))
-        fn = lambda st: sage.sage_gemm(A, x, M, y, ws, st)
-        for _ in range(3):
+        ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_GEMM, A0, M))
+        fns = [lambda st, A=A: sage.sage_gemm(A, x, M, y, ws, st) for A in As]
+        for fn in fns[:3]:
             fn(stream)
-        ms = _timed_calls(fn, stream, reps, flush)
+        t = per_call_us(fns, stream, reps_rounds)
         assert sage.sage_query_status(ws) == sage.SAGE_OK
+        us = float(np.median(t))
         flops = 2.0 * M * f.d_out * f.d_in
-        nbytes = A.packed_bytes + 32 * 16 + M * f.d_in * 2 + M * f.d_out * 2
-        tf = flops / (ms * 1e-3) / 1e12
-        out.append({"M": M, "path": "gemv" if M <= 8 else "tcgen05", "us": round(ms * 1e3, 2),
+        nbytes = A0.packed_bytes + 32 * 16 + M * f.d_in * 2 + M * f.d_out * 2
+        tf = flops / (us * 1e-6) / 1e12
+        out.append({"M": M, "path": "gemv" if M <= 8 else "tcgen05", "us": dist_summary(t),
                     "tflops": round(tf, 1), "tensor_frac": round(tf / peak, 4),
-                    "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
-    return {"workload": "4096->12288 up-projection, (K,V)=(32,5), L2 flushed before each call",
+                    "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4)})
+    return {"workload": "4096->12288 up-projection, (K,V)=(32,5), planes rotated over copies > 2 x L2",
             "peak_tflops": peak, "peak_kind": kind, "points": out}
 
 
-def bench_moe(stream, flush, reps=20):
-    """Config 4: 128 experts, gate 2048 -> 768 and down 768 -> 2048, top-8,
-    T tokens; one sage_moe_gemv call per projection."""
+def bench_moe(stream, reps=20):
+    """128 experts (gate/up 2048 -> 768, down 768 -> 2048), top-8 routing, T tokens; one
+    sage_moe_gemv call per projection, L2 flushed before each call."""
     import torch
     import synth
     import bit_vector_quantized_sage_b200 as sage
     hbm, _ = _peaks()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
     out = []
     for proj in (0, 2):
         packed = None
@@ -314,37 +542,83 @@ def bench_moe(stream, flush, reps=20):
             fn = lambda st: sage.sage_moe_gemv(packed, pe, xr, n_pairs, x, y, ws, st)
             for _ in range(3):
                 fn(stream)
-            ms = _timed_calls(fn, stream, reps, flush)
+            g = capture(fn, stream)
+            t = []
+            for _ in range(reps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                e1.synchronize()
+                t.append(e0.elapsed_time(e1) * 1e3)
+            del g
             assert sage.sage_query_status(ws) == sage.SAGE_OK
             active = np.unique(spec.routes)
             nbytes = sum(packed[e].packed_bytes + (1 << packed[e].log2K) * 16 for e in active)
             nbytes += xb.nbytes + n_pairs * d_out * 2
-            out.append({"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size),
-                        "us": round(ms * 1e3, 2), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
-                        "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4)})
+            us = float(np.median(t))
+            out.append({"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size), "us": dist_summary(t),
+                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4)})
+    del flush
     return {"workload": "128 experts, top-8, one projection per call, L2 flushed before each call", "points": out}
 
 
+def oracle_beside(pool_1):
+    """The oracle on one core beside the up-projection and MoE workloads (GB/s of packed
+    bytes on a sample: two 256-row blocks of the up-projection; the gate and down
+    matrices of the first four experts routed for one token)."""
+    import synth
+    out = {}
+    b, s = pool_1.run([[("up8b", "up8b", 0, 256), ("up8b", "up8b", 6144, 6400)]])
+    out["up8b_4096x12288"] = {"gbs": round(b / s / 1e9, 4), "seconds": round(s, 3), "cores": 1,
+                              "sample": "rows 0-255 and 6144-6399"}
+    routes = synth.config4(1).routes[0][:4]
+    tasks = []
+    for proj, d_out in ((0, 768), (2, 2048)):
+        for e in routes:
+            tasks.append(("moe", f"moe:{proj}:{int(e)}", 0, d_out))
+    b, s = pool_1.run([tasks])
+    out["moe_T1"] = {"gbs": round(b / s / 1e9, 4), "seconds": round(s, 3), "cores": 1,
+                     "sample": "gate and down of 4 of the 8 routed experts, T = 1"}
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------
+
 def run_reference(args):
-    ws, rank, _ = _dist()
+    """The CPU oracle on the same workload: each step is a bounded sample of the layer
+    (every 8th 256-row block, rotating the offset so that 8 steps cover the layer) on
+    all host cores."""
+    world, rank, _ = _dist()
     if rank != 0:
         return 0
-    for _ in range(args.warmup):
-        cpu_oracle_sample(rows_per_matrix=32)
-    vals, secs = [], 0.0
-    for _ in range(args.steps):
-        v, desc, cores, s = cpu_oracle_sample(rows_per_matrix=256)
-        vals.append(v)
-        secs += s
+    cores = host_cores()
+    pool = OraclePool(cores)
+    try:
+        for i in range(args.warmup):
+            oracle_layer_baseline(None, pool, fraction=1 / 8, offset=i)
+        vals, secs, nb = [], 0.0, 0
+        for i in range(args.steps):
+            r, nb = oracle_layer_baseline(None, pool, fraction=1 / 8, offset=i)
+            vals.append(r["n"][0])
+            secs += r["n"][1]
+    finally:
+        pool.close()
     value = statistics.median(vals)
-    layer_b = 31_682_560  # packed layer bytes scale: reported per-layer time from the GB/s
+    desc = (f"1/8 of the layer per step ({nb} of its 120 256-row blocks, offset rotating), "
+            f"oracle unpack + fp32 reconstruction + fp64 matvec, {cores} processes on {cpu_model()}")
+    layer_b = 31_664_896
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(1, args.steps) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; see synth/config1)",
-        "config": {"workload": WORKLOAD, "batch": 1, "sample": desc},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "data": "synthetic (seeded; synth.config1)",
+        "config": {"workload": workload(args.layer), "batch": 1, "layer_mode": args.layer, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "us_per_layer_extrapolated": layer_b / (value * 1e9) * 1e6,
     }
@@ -369,61 +643,27 @@ def run_gpu(args):
         dist.barrier()
     sage.load()
 
-    L, layers1, xs = build_layer(1)
-    one_layer_bytes, perm_bytes = layer_bytes(layers1[0])
-    replicas = max(2, int(np.ceil(4 * L2_BYTES / one_layer_bytes)) + 1)
-    _, layers, xs = build_layer(replicas)
-    ys = {f.name: torch.zeros((1, f.d_out), dtype=torch.int16, device="cuda") for f in L.mats}
-    ws = sage.Workspace(max(sage.sage_workspace_size(sage.SAGE_OP_GROUPED, [layers[0][n] for n in st], 1)
-                            for st in __import__("synth").QWEN3_4B_STAGES))
-    runners = [LayerRunner(lay, xs, ys, ws) for lay in layers]
+    L, layers = build_layers()
+    replicas = len(layers)
+    one_layer_bytes, perm_bytes = layer_bytes(layers[0])
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
+    modes = {}
+    for mode in ("fused", "stages", "grouped7"):
+        modes[mode] = make_runners(mode, layers, L)
+    fns, ws, inputs, outputs, launches = modes[args.layer]
 
-    # ---- warm-up (eager) ----
-    for i in range(max(3, args.warmup)):
-        runners[i % replicas](stream)
-    torch.cuda.synchronize()
+    # ---- warm-up (eager, through the public API) ----
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            fns[i % replicas](stream)
+        torch.cuda.synchronize()
     assert sage.sage_query_status(ws) == sage.SAGE_OK
 
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            fn(torch.cuda.current_stream())
-        return g
-
-    def time_graph(g, reps=1):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1)
-
-    import synth
-    n_stage = len(synth.QWEN3_4B_STAGES)
-    stage_bytes = []
-    for stage in synth.QWEN3_4B_STAGES:
-        stage_bytes.append(sum(layers[0][n].packed_bytes + (1 << layers[0][n].log2K) * 16 +
-                               layers[0][n].d_in * 2 + layers[0][n].d_out * 2 for n in stage))
-
-    # ---- per-stage kernel time: one graph = the stage launched once per replica ----
-    stage_avg = []
+    # ---- timed region: one CUDA graph of K layers over rotating replicas ----
     with torch.cuda.stream(stream):
-        for s_i in range(n_stage):
-            g = capture(lambda st: [runners[r].calls[s_i](st) for r in range(replicas)])
-            for _ in range(3):
-                g.replay()
-            ms_s = time_graph(g, reps=max(1, 200 // replicas))
-            stage_avg.append(ms_s / (max(1, 200 // replicas) * replicas))
-            del g
-
-    # ---- timed region: one graph holding K layers back to back (rotating replicas) ----
-    with torch.cuda.stream(stream):
-        g_all = capture(lambda st: [runners[k % replicas](st) for k in range(args.steps)])
-        for _ in range(max(3, args.warmup // max(1, args.steps) + 1)):
-            g_all.replay()
+        g_all = capture(lambda st: [fns[k % replicas](st) for k in range(args.steps)], stream)
+        g_all.replay()
         torch.cuda.synchronize()
     clocks = Clocks(local)
     clocks.start()
@@ -441,76 +681,99 @@ def run_gpu(args):
     clk = clocks.stop()
     ms = max_over_ranks(start.elapsed_time(end), dist, "cuda")
     assert sage.sage_query_status(ws) == sage.SAGE_OK
+    del g_all
     us_per_layer = ms * 1e3 / args.steps
     value = whole_job_gbs(world, one_layer_bytes, args.steps, ms)
-    del g_all
 
-    # ---- end to end through the public API with host buffers (graph per step) ----
-    h_x = {k: torch.from_numpy(L.xs[k].view(np.int16)).pin_memory() for k in xs}
-    h_y = {n: torch.zeros(tuple(ys[n].shape), dtype=torch.int16).pin_memory() for n in ys}
-    h2d = sum(v.numel() * 2 for v in h_x.values())
-    d2h = sum(v.numel() * 2 for v in h_y.values())
-    e2e_steps = max(20, args.steps // 2)
-
-    def e2e_step(st, r):
-        for n, hx in h_x.items():
-            xs[n].copy_(hx, non_blocking=True)
-        runners[r](st)
-        for n, hy in h_y.items():
-            hy.copy_(ys[n], non_blocking=True)
-
+    # ---- per-layer distribution of every layer mode (one graph per layer) ----
+    layer_modes = {}
     with torch.cuda.stream(stream):
-        g_e2e = [capture(lambda st, r=r: e2e_step(st, r)) for r in range(replicas)]
-        for r in range(replicas):
-            g_e2e[r].replay()
+        for mode, (mf, mws, _, _, ml) in modes.items():
+            t = per_call_us(mf, stream, rounds=max(2, 60 // replicas))
+            assert sage.sage_query_status(mws) == sage.SAGE_OK
+            med = float(np.median(t))
+            layer_modes[mode] = {"launches_per_layer": ml, "us_per_layer": dist_summary(t),
+                                 "gbs": round(one_layer_bytes / (med * 1e-6) / 1e9, 1),
+                                 "hbm_frac": round(one_layer_bytes / (med * 1e-6) / 1e9 / _peaks()[0], 4)}
+    layer_modes["fused"]["what"] = ("the decoder layer as one launch: RMSNorm -> q|k|v, attention over one cached "
+                                    "position -> o, residual + RMSNorm -> gate|up, SiLU * up -> down + residual")
+    layer_modes["stages"]["what"] = "the four stages as four grouped launches (PDL-chained), synthetic stage inputs"
+    layer_modes["grouped7"]["what"] = "the seven projections in one grouped launch, independent synthetic inputs"
+
+    # ---- end to end through the public API with host buffers ----
+    h_in = {k: torch.from_numpy(np.ascontiguousarray(v[1]).view(np.int16)).pin_memory() for k, v in inputs.items()}
+    h_out = {k: torch.zeros(tuple(v.shape), dtype=torch.int16).pin_memory() for k, v in outputs.items()}
+    h2d = sum(v.numel() * 2 for v in h_in.values())
+    d2h = sum(v.numel() * 2 for v in h_out.values())
+    e2e_steps = max(20, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for k in range(3):
+            fns[k % replicas](stream)
         torch.cuda.synchronize()
         e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e_start.record(stream)
         for k in range(e2e_steps):
-            g_e2e[k % replicas].replay()
-            stream.synchronize()          # the host reads the step's result
+            for n, hx in h_in.items():
+                inputs[n][0].copy_(hx, non_blocking=True)
+            fns[k % replicas](stream)
+            for n, hy in h_out.items():
+                hy.copy_(outputs[n], non_blocking=True)
+            stream.synchronize()  # the host reads the step's result
         e_end.record(stream)
         torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / e2e_steps, dist, "cuda")
     e2e_value = whole_job_gbs(world, one_layer_bytes, 1, e2e_ms)
-    del g_e2e
+    assert sage.sage_query_status(ws) == sage.SAGE_OK
 
-    extra = {}
-    if rank == 0 and not args.no_extra:
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    extra = {"layer_modes": layer_modes}
+    if rank == 0 and world == 1 and not args.no_extra:
         with torch.cuda.stream(stream):
-            extra["gemm_config3"] = bench_gemm(stream, flush)
-            extra["moe_config4"] = bench_moe(stream, flush)
-        del flush
+            extra["up_proj_4096x12288_batch_sweep"] = bench_gemm(stream)
+            extra["moe_128_experts"] = bench_moe(stream)
 
     peak, peak_kind = _peaks()
-    achieved = sum(stage_bytes) / (sum(stage_avg) * 1e-3) / 1e9
-    traffic, _ = _traffic_for(_kernel_hash())
+    traffic, traffic_note = traffic_for(args.layer)
+    achieved = one_layer_bytes / (us_per_layer * 1e-6) / 1e9
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores, secs = cpu_oracle_sample(rows_per_matrix=args.cpu_rows)
-        cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc,
-               "seconds": round(secs, 2)}
+        torch.cuda.synchronize()
+        cores = host_cores()
+        pool_1, pool_n = OraclePool(1), OraclePool(cores)
+        try:
+            r, nblk = oracle_layer_baseline(pool_1, pool_n)
+            beside = oracle_beside(pool_1)
+        finally:
+            pool_1.close()
+            pool_n.close()
+        desc = (f"the whole layer ({nblk} 256-row blocks of the seven matrices): oracle unpack + fp32 reconstruction "
+                f"+ fp64 matvec, one process per core on {cpu_model()}")
+        cpu = {"value": r["n"][0], "unit": "GB/s", "cores": r["n"][2], "kind": "oracle", "sample": desc,
+               "seconds": round(r["n"][1], 3), "cpu_model": cpu_model(),
+               "single_core": {"value": r["1"][0], "unit": "GB/s", "cores": 1, "seconds": round(r["1"][1], 3)},
+               "beside_other_workloads": beside}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic (seeded; see synth/config1)",
-        "config": {"workload": WORKLOAD, "batch": 1, "stages": "q|k|v, o, gate|up, down (4 grouped launches)",
+        "data": "synthetic (seeded; synth.config1)",
+        "config": {"workload": workload(args.layer),
+                   "batch": 1, "layer_mode": args.layer, "what": layer_modes[args.layer]["what"],
                    "packed_bytes_per_layer": one_layer_bytes, "perm_bytes_per_layer": perm_bytes,
                    "l2": f"inputs larger than L2: {replicas} rotating copies of the packed layer "
                          f"({replicas * one_layer_bytes / 2**20:.0f} MiB)",
                    "parallelism": f"replicas x{world}"},
         "us_per_layer": us_per_layer,
+        "us_per_layer_dist": layer_modes[args.layer]["us_per_layer"],
         "hbm_fraction": value / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                     "kernel": "gemv_kernel<1> (grouped packed GEMV)",
-                     "stage_us": [round(s * 1e3, 3) for s in stage_avg],
-                     "stage_bytes": stage_bytes},
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_nominal": achieved / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
+                     "traffic": traffic, "traffic_note": traffic_note, "kernel": KERNEL,
+                     "launches_per_step": launches,
+                     "algorithmic_bytes_per_step": one_layer_bytes},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "us_per_layer": e2e_ms * 1e3},
-        "gpu_launches": args.steps * n_stage,
+                "us_per_layer": e2e_ms * 1e3, "api": "public Python binding over the C ABI, eager calls"},
+        "gpu_launches": args.steps * launches,
         "clocks": clk,
         "cpu_baseline": cpu,
         "extra": extra,
@@ -529,8 +792,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
-    ap.add_argument("--cpu-rows", type=int, default=1 << 30,
-                    help="rows per matrix in the CPU-oracle baseline sample (default: the whole layer)")
+    ap.add_argument("--layer", default="fused", choices=["fused", "stages", "grouped7"],
+                    help="how the layer's seven projections are launched (default: the fused decoder layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the batch sweep and MoE measurements")
     args = ap.parse_args()

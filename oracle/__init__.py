@@ -48,6 +48,8 @@ def lib():
             L.oracle_double_to_half.restype = u16
             L.oracle_unpack.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
             L.oracle_unpack.restype = i32
+            L.oracle_pack.argtypes = [i32, i32, i32, P, P, P, P, P, P, sz, P, sz]
+            L.oracle_pack.restype = i32
             L.oracle_dequant.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
             L.oracle_dequant.restype = None
             L.oracle_round_half.argtypes = [sz, P, P]
@@ -129,6 +131,26 @@ def unpack(d_out, d_in, log2K, main_plane, meta_plane):
     if rc:
         raise ValueError("oracle_unpack: unsupported shape")
     return dict(signs=signs, idx=idx, q=q, mu=mu, delta=delta)
+
+
+def plane_words(d_out: int, d_in: int):
+    """uint32 words of the main and meta planes (whole 256-row blocks; the last
+    block holds only its ceil(d_out / 8) - 32 B octets)."""
+    S, G, R8 = d_in // 8, d_in // 128, (d_out + 7) // 8
+    return R8 * S * 4, R8 * G * 16
+
+
+def pack(d_out, d_in, log2K, signs, idx, q, mu, delta):
+    """Packed planes (main, meta) of the code fields: the inverse of unpack."""
+    mw, tw = plane_words(d_out, d_in)
+    main_plane = np.zeros(mw, np.uint32)
+    meta_plane = np.zeros(tw, np.uint32)
+    rc = lib().oracle_pack(d_out, d_in, log2K, _p(_c(signs, np.uint8)), _p(_c(idx, np.uint16)),
+                           _p(_c(q, np.uint8)), _p(_c(mu, np.uint16)), _p(_c(delta, np.uint16)),
+                           _p(main_plane), mw, _p(meta_plane), tw)
+    if rc:
+        raise ValueError(f"oracle_pack: rejected ({rc})")
+    return main_plane, meta_plane
 
 
 def dequant(f) -> np.ndarray:

@@ -155,6 +155,54 @@ int oracle_unpack(int d_out, int d_in, int log2K,
     return 0;
 }
 
+/* The inverse of oracle_unpack over the same layout: writes every bit
+ * of the planes (main_words = ceil(d_out/256) blocks of S * 128 words at
+ * most, meta_words likewise G * 512), zero where no field lands.  Fields
+ * wider than their slots are rejected (return 2).  Test and benchmark
+ * infrastructure only: it lets the CPU baseline start from packed planes
+ * without the library's packer. */
+int oracle_pack(int d_out, int d_in, int log2K,
+                const uint8_t* signs, const uint16_t* idx, const uint8_t* q,
+                const uint16_t* mu, const uint16_t* delta,
+                uint32_t* main_plane, size_t main_words, uint32_t* meta_plane, size_t meta_words) {
+    if (d_out < 1 || d_in < 128 || d_in % 128 || log2K < 4 || log2K > 8) return 1;
+    const int V = 10 - log2K;
+    const int S = d_in / SV, G = d_in / 128, R8 = (d_out + 7) / 8;
+    memset(main_plane, 0, main_words * 4);
+    memset(meta_plane, 0, meta_words * 4);
+    for (int o = 0; o < d_out; ++o) {
+        const int b = o / 8, t = o % 8, u = t / 2, isB = t & 1;
+        const int blk = b / 32, ob = b % 32;
+        const int nB = (R8 - 32 * blk < 32) ? R8 - 32 * blk : 32;
+        const size_t main0 = (size_t)blk * S * 128, meta0 = (size_t)blk * G * 256;
+        for (int j = 0; j < S; ++j) {
+            const uint32_t z = idx[(size_t)o * S + j], qq = q[(size_t)o * S + j], s = signs[(size_t)o * S + j];
+            if (z >> log2K || qq >> V) return 2;
+            const size_t wi = main0 + ((size_t)j * nB + ob) * 4 + u;
+            if (wi >= main_words) return 3;
+            uint32_t w = 0;
+            if (!isB) w |= (z << 7) | (qq << (23 - V));
+            else      w |= (z << 23) | (qq << (7 - V));
+            for (int n = 0; n < 3; ++n) {
+                const int p = slot_pos(V, n + (isB ? 3 : 0));
+                w |= ((s >> (2 * n)) & 1u) << p;
+                w |= ((s >> (2 * n + 1)) & 1u) << (p + 16);
+            }
+            main_plane[wi] |= w;
+            const size_t ai = (meta0 + ((size_t)(j / GROUP_SV) * nB + ob) * 8 + t) * 2;
+            if (ai + 1 >= meta_words) return 3;
+            const int tj = j % GROUP_SV;
+            meta_plane[ai] |= (((s >> 6) & 1u) << tj) | (((s >> 7) & 1u) << (tj + 16));
+        }
+        for (int g = 0; g < G; ++g) {
+            const size_t mi = (meta0 + ((size_t)g * nB + ob) * 8 + t) * 2 + 1;
+            if (mi >= meta_words) return 3;
+            meta_plane[mi] = (uint32_t)mu[(size_t)o * G + g] | ((uint32_t)delta[(size_t)o * G + g] << 16);
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* Reconstruction (Eq. 1 with Eq. 2's grid).                           */
 /* W[o][8j + i] = (mu + q delta) * s_i * c_z[i], storage column order. */

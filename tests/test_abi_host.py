@@ -53,6 +53,9 @@ def test_pack_matches_oracle_unpack(lib, log2K, d_out, d_in):
     back = sage.sage_unpack(d_out, d_in, log2K, main, meta)
     for k in back:
         assert np.array_equal(back[k], getattr(f, k)), k
+    om, ot = oracle.pack(d_out, d_in, log2K, f.signs, f.idx, f.q, f.mu, f.delta)
+    assert np.array_equal(np.asarray(main).view(np.uint32).reshape(-1), om)
+    assert np.array_equal(np.asarray(meta).view(np.uint32).reshape(-1), ot)
 
 
 def test_pack_reproduces_hand_example(lib):
@@ -170,3 +173,17 @@ def test_packed_sizes_closed_form_up_to_int_max(lib):
         r8 = (d_out + 7) // 8
         assert a.value == r8 * (d_in // 8) * 16
         assert b.value == r8 * (d_in // 128) * 64
+
+
+@pytest.mark.parametrize("d_out,d_in", [(2 ** 31 - 8, 9728), (2 ** 31 - 1, 2560), (900_000_000, 2560)])
+def test_engine_rejects_unit_counts_beyond_int(lib, d_out, d_in):
+    """A matrix whose block-column count (256-row blocks x d_in / 8) passes 2^30 is
+    refused on the host before any device call: the pointers below are never
+    dereferenced, and the unit arithmetic is 64-bit up to the check."""
+    A = sage.sage_matrix(d_out, d_in, 6, 0x100000, 0x200000, 0x300000, None)
+    need = C.c_size_t()
+    assert lib.sage_workspace_size(sage.SAGE_OP_GEMV, C.byref(A), 1, 1, C.byref(need)) == sage.SAGE_OK
+    blocks = ((d_out + 7) // 8 + 31) // 32
+    assert need.value >= blocks * 4
+    rc = lib.sage_gemv(C.byref(A), 0x400000, 1, 0x500000, 0x10000000, 1 << 45, None)
+    assert rc == sage.SAGE_ERR_UNSUPPORTED

@@ -1,5 +1,6 @@
 """bench.py --impl reference on CPU: the oracle arm prints one JSON line with
-the contract's keys, the run's own metric and unit, and zero host-device bytes."""
+the contract's keys, the run's own metric and unit, and zero host-device bytes.
+It runs the oracle's own packer and kernels only (libsage is never loaded)."""
 import json
 import os
 import subprocess
@@ -19,9 +20,22 @@ def test_reference_arm_json_line():
     assert line["metric"] == bench.METRIC and line["unit"] == "GB/s"
     assert line["value"] > 0 and line["higher_is_better"] is True
     assert line["n_gpus"] == 1 and line["steps"] == 1 and line["warmup"] == 0
-    assert line["config"]["workload"] == bench.WORKLOAD
+    assert line["config"]["workload"] == bench.workload("fused")
+    assert line["config"]["layer_mode"] == "fused"
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert cb["cores"] == bench.host_cores() and cb["cpu_model"]
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_never_loads_the_library():
+    code = ("import sys, runpy; sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', '--warmup', '0']\n"
+            "try:\n    runpy.run_path('bench.py', run_name='__main__')\nexcept SystemExit:\n    pass\n"
+            "import sys as s2\n"
+            "assert 'bit_vector_quantized_sage_b200' not in s2.modules, 'library imported'\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "assert 'libsage' not in maps, 'libsage mapped'\n")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]

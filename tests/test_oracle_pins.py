@@ -149,6 +149,35 @@ def test_unpack_is_a_bijection(log2K):
     assert len(grid_bits) == 8 * 32
 
 
+@pytest.mark.parametrize("log2K", [4, 5, 6, 7, 8])
+def test_pack_inverts_unpack(log2K):
+    """oracle.pack is unpack's inverse both ways: fields -> planes -> fields, and
+    every bit of random planes over whole octets survives planes -> fields -> planes
+    (the format uses all 32 bits of a word: 2 x (log2K + V) = 20 code bits plus 12
+    sign bits)."""
+    f = synth.random_fields(np.random.default_rng(77 + log2K), 300, 384, log2K)
+    main, meta = oracle.pack(f.d_out, f.d_in, log2K, f.signs, f.idx, f.q, f.mu, f.delta)
+    u = oracle.unpack(f.d_out, f.d_in, log2K, main, meta)
+    for k in ("signs", "idx", "q", "mu", "delta"):
+        assert np.array_equal(u[k], getattr(f, k)), k
+    d_out, d_in = 264, 256  # 33 octets: one whole block and a one-octet block
+    mw, tw = oracle.plane_words(d_out, d_in)
+    g = np.random.default_rng(5 + log2K)
+    main = g.integers(0, 2**32, mw, dtype=np.uint64).astype(np.uint32)
+    meta = g.integers(0, 2**32, tw, dtype=np.uint64).astype(np.uint32)
+    u = oracle.unpack(d_out, d_in, log2K, main, meta)
+    m2, t2 = oracle.pack(d_out, d_in, log2K, u["signs"], u["idx"], u["q"], u["mu"], u["delta"])
+    assert np.array_equal(m2, main) and np.array_equal(t2, meta)
+
+
+def test_pack_rejects_wide_fields():
+    f = synth.random_fields(np.random.default_rng(3), 8, 128, 5)
+    q = f.q.copy()
+    q[0, 0] = 1 << 5  # V = 5: one bit too wide
+    with pytest.raises(ValueError):
+        oracle.pack(8, 128, 5, f.signs, f.idx, q, f.mu, f.delta)
+
+
 def test_unpack_all_ones():
     for log2K in range(4, 9):
         V = 10 - log2K
