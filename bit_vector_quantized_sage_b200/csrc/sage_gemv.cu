@@ -11,8 +11,8 @@
 //    are flattened (matrix, block, j) and cut into one contiguous range per
 //    CTA of a persistent grid (one CTA per SM); every stage is spread over
 //    every CTA.
-//  * The copy warp bulk-copies (1-D TMA) codebooks and, chunk by chunk (16
-//    columns = one radius group), the code records and grid/aux meta into a
+//  * The copy warp bulk-copies (1-D TMA) codebooks and, chunk by chunk (32
+//    columns = two radius groups), the code records and grid/aux meta into a
 //    ring of shared-memory slots.  It runs ahead across segments and stages:
 //    the packed planes never depend on earlier work, so the next stage's codes
 //    stream in while the current stage finishes.
@@ -28,12 +28,9 @@
 //    address is one logic op on the word (format v2), the codeword one
 //    conflict-free 128-bit load from the replica of the thread's lane position
 //    (8 bank-rotated replicas of the codebook), the signs are XORed into the
-//    fp16 sign bits, four half2 products with fp16 accumulation form
-//    (s (.) c) . x (Fig. 6a), and r = mu + q delta (Eq. 2) scales it once, in
-//    fp32, into the row's fp32 accumulator.
-//  * Overflow guard for the fp16 local sums: each window's largest |x| decides
-//    a power-of-two prescale (x / 2^k, k <= 2) that keeps every partial sum of
-//    a subvector finite; the radius carries 2^k back.  Powers of two are exact.
+//    fp16 sign bits, eight fp16 x fp16 products summed in fp32 (mixed-precision
+//    FMA; Fig. 6a sums them in fp16) form (s (.) c) . x, and r = mu + q delta
+//    (Eq. 2) scales it once, in fp32, into the row's fp32 accumulator.
 //  * Rows whose columns are split between CTAs are combined deterministically:
 //    partial sums go to the workspace and the last CTA to finish a block adds
 //    them in CTA order.  A block whose final outputs are written bumps its
@@ -65,7 +62,8 @@ constexpr int kDW = 8;                          // decode warps: 4 row quarters 
 constexpr int kParts = kDW / 4;                 // column parts of a chunk (one radius group each)
 constexpr int kDT = kDW * 32;                   // decode threads
 constexpr int kGT = kDT + 32;                   // threads of a cooperative gather
-constexpr int kThreads = kDT + 96;              // + copy, gather and epilogue warps
+constexpr int kEpiWarps = 2;                    // epilogue warps (segments dealt out alternately)
+constexpr int kThreads = kDT + 32 * (2 + kEpiWarps);  // + copy, gather and epilogue warps
 constexpr int kCopyWarp = kDW, kGatherWarp = kDW + 1, kEpiWarp = kDW + 2;
 constexpr int kStashSlots = 4;                  // segments between the decode and epilogue warps (at most)
 constexpr int kBarDecode = 1, kBarGather = 2;   // named barriers (0 is __syncthreads)
@@ -238,8 +236,7 @@ struct Smem {
     float* stash;       // [slot][column part][M][256] decode sums awaiting the epilogue
     float* red;         // [kGT / 32][8] cooperative reductions
     uint64_t* bars;
-    int* misc;          // [0..1] window shift k per buffer, [2] abort flag, [3] window max |x| bits,
-                        // [8] window length, [9] batch rows per window, [10] stages whose first window is gathered,
+    int* misc;          // [2] abort flag, [8] window length, [9] batch rows per window, [10] stages whose first window is gathered,
                         // [16..24) flush flags
     float* inv_rms;     // [8] per batch row
     struct Pending* pend;  // segments awaiting their flush (written by decode thread 0)
@@ -517,14 +514,12 @@ __device__ void rms_rows(const Smem& sm, const EngineStage& st, int tid, int nt,
 }
 
 // Gathers the window's x_perm for items e = tid, tid + nt, ... of (batch row,
-// position) and stores them (fp16, unscaled) into the window buffer; returns
-// the largest |x| bit pattern seen.
+// position) and stores them (fp16) into the window buffer.
 template <int M, int PRO, class Src>
-__device__ uint32_t gather_items_k(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid,
+__device__ void gather_items_k(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid,
                                    int nt, bool coh) {
     const EngineStage& st = *sm.stc;
     const int mrows = sm.misc[9];  // batch rows a window holds (<= M)
-    uint32_t mx = 0;
     for (int e = tid; e < mrows * wlen; e += nt) {
         const int m = e / wlen, p = e - m * wlen;
         const uint32_t info = sm.posinfo[p];
@@ -550,45 +545,18 @@ __device__ uint32_t gather_items_k(const Src& src, const Smem& sm, int s, int wl
             }
         }
         sts128(xb + (uint32_t)(m * xw + p) * 16, val);
-        const uint32_t a = __vmaxu2(__vmaxu2(val.x & 0x7fff7fffu, val.y & 0x7fff7fffu),
-                                    __vmaxu2(val.z & 0x7fff7fffu, val.w & 0x7fff7fffu));
-        mx = max(mx, max(a & 0xffffu, a >> 16));
     }
-    return mx;
 }
 
 template <int M, class Src>
-__device__ uint32_t gather_items(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid, int nt,
-                                 bool coh) {
+__device__ void gather_items(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid, int nt,
+                             bool coh) {
     switch (sm.stc->pro) {  // uniform: one specialised loop per prologue
-        case kProRmsNorm: return gather_items_k<M, kProRmsNorm>(src, sm, s, wlen, xw, xb, tid, nt, coh);
-        case kProResidRmsNorm: return gather_items_k<M, kProResidRmsNorm>(src, sm, s, wlen, xw, xb, tid, nt, coh);
-        case kProSiluMul: return gather_items_k<M, kProSiluMul>(src, sm, s, wlen, xw, xb, tid, nt, coh);
-        case kProGqa: return gather_items_k<M, kProGqa>(src, sm, s, wlen, xw, xb, tid, nt, coh);
-        default: return gather_items_k<M, kProPlain>(src, sm, s, wlen, xw, xb, tid, nt, coh);
-    }
-}
-
-// Power-of-two prescale of a window: k such that every |x| / 2^k <= 2^14, so
-// that no partial sum of a subvector's eight fp16 products (sum of |c_i| <= 2
-// per half2 lane, <= 2 sqrt 2 in all) can leave the fp16 range.
-__device__ __forceinline__ int window_shift(uint32_t maxbits) {
-    return maxbits <= 0x7400u ? 0 : maxbits <= 0x7800u ? 1 : 2;  // 2^14, 2^15, larger (<= 65504)
-}
-
-// Scales window items by 2^-k in place (only windows with very large |x|).
-template <int M>
-__device__ void rescale_items(const Smem& sm, int wlen, int xw, uint32_t xb, int k, int tid, int nt) {
-    const __half2 f = __float2half2_rn(k == 1 ? 0.5f : 0.25f);
-    for (int e = tid; e < sm.misc[9] * wlen; e += nt) {
-        const int m = e / wlen, p = e - m * wlen;
-        const uint32_t a = xb + (uint32_t)(m * xw + p) * 16;
-        uint4 v = lds128(a);
-        v.x = h22u(__hmul2(u2h2(v.x), f));
-        v.y = h22u(__hmul2(u2h2(v.y), f));
-        v.z = h22u(__hmul2(u2h2(v.z), f));
-        v.w = h22u(__hmul2(u2h2(v.w), f));
-        sts128(a, v);
+        case kProRmsNorm: gather_items_k<M, kProRmsNorm>(src, sm, s, wlen, xw, xb, tid, nt, coh); return;
+        case kProResidRmsNorm: gather_items_k<M, kProResidRmsNorm>(src, sm, s, wlen, xw, xb, tid, nt, coh); return;
+        case kProSiluMul: gather_items_k<M, kProSiluMul>(src, sm, s, wlen, xw, xb, tid, nt, coh); return;
+        case kProGqa: gather_items_k<M, kProGqa>(src, sm, s, wlen, xw, xb, tid, nt, coh); return;
+        default: gather_items_k<M, kProPlain>(src, sm, s, wlen, xw, xb, tid, nt, coh); return;
     }
 }
 
@@ -603,14 +571,7 @@ __device__ void coop_window(const Src& src, const Smem& sm, int s, int w, int xw
         named_barrier(kBarGather, kGT);
     }
     const int wlen = sm.misc[8];
-    const uint32_t mx = gather_items<M>(src, sm, s, wlen, xw, sm.xwin(w), tid, kGT, coh);
-    atomicMax(reinterpret_cast<unsigned*>(sm.misc + 3), mx);
-    named_barrier(kBarGather, kGT);
-    const int k = window_shift((uint32_t)sm.misc[3]);
-    if (k) {
-        rescale_items<M>(sm, wlen, xw, sm.xwin(w), k, tid, kGT);
-    }
-    if (tid == 0) sm.misc[w & 1] = k;
+    gather_items<M>(src, sm, s, wlen, xw, sm.xwin(w), tid, kGT, coh);
     named_barrier(kBarGather, kGT);
 }
 
@@ -655,22 +616,13 @@ __device__ __forceinline__ void fill_window(const Src& src, const Smem& sm, uint
     }
     if (win >= 2) wait_bar(sm, sm.x_empty(win & 1), ((win >> 1) - 1) & 1, status);
     const bool coh = st.wait != 0;
-    if (lane == 0) {
-        sm.misc[8] = wlen;
-        sm.misc[3] = 0;
-    }
+    if (lane == 0) sm.misc[8] = wlen;
     __syncwarp();
     if (first) {
         coop_window<M>(src, sm, s, win, xw, coh, kDT + lane);
         if (lane == 0) *reinterpret_cast<volatile int*>(sm.misc + 10) = s + 1;  // release the copy warp
     } else {
-        uint32_t mx = gather_items<M>(src, sm, s, wlen, xw, sm.xwin(win), lane, 32, coh);
-        for (int o = 16; o; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const int k = window_shift(mx);
-        __syncwarp();
-        if (k) rescale_items<M>(sm, wlen, xw, sm.xwin(win), k, lane, 32);
-        if (lane == 0) sm.misc[win & 1] = k;
-        __syncwarp();
+        gather_items<M>(src, sm, s, wlen, xw, sm.xwin(win), lane, 32, coh);
     }
     mbar_arrive(sm.x_full(win & 1));  // all 32 lanes, each after its own stores
 }
@@ -734,14 +686,35 @@ __device__ void gather_role(const Src& src, const Smem& sm, uint32_t* status, un
 // ------------------------------------------------------------------------
 // Decode warps
 // ------------------------------------------------------------------------
-// (s (.) c) . x for one subvector: four half2 products with fp16 accumulation
-// (Fig. 6a), the two halves added in fp16, returned as fp32.
+// (s (.) c) . x for one subvector: the eight fp16 x fp16 products, exact in
+// fp32, summed in fp32 by mixed-precision FMAs (fp16 operands, fp32
+// accumulator).  The paper's kernel (Fig. 6a) sums them in fp16 instead; an
+// fp16 partial sum rounds at 2^-11 of its own size, which a subvector that
+// dominates its output row turns into more than 1e-3 of sum |w||x|.
 __device__ __forceinline__ float sdot(uint4 c, uint4 x) {
-    __half2 h = __hmul2(u2h2(c.x), u2h2(x.x));
-    h = __hfma2(u2h2(c.y), u2h2(x.y), h);
-    h = __hfma2(u2h2(c.z), u2h2(x.z), h);
-    h = __hfma2(u2h2(c.w), u2h2(x.w), h);
-    return __half2float(__hadd(__low2half(h), __high2half(h)));
+    float d;
+    asm("{\n\t"
+        ".reg .f16 c0, c1, c2, c3, c4, c5, c6, c7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
+        "mov.b32 {c0, c1}, %1;\n\t"
+        "mov.b32 {c2, c3}, %2;\n\t"
+        "mov.b32 {c4, c5}, %3;\n\t"
+        "mov.b32 {c6, c7}, %4;\n\t"
+        "mov.b32 {x0, x1}, %5;\n\t"
+        "mov.b32 {x2, x3}, %6;\n\t"
+        "mov.b32 {x4, x5}, %7;\n\t"
+        "mov.b32 {x6, x7}, %8;\n\t"
+        "fma.rn.f32.f16 %0, c0, x0, 0f00000000;\n\t"
+        "fma.rn.f32.f16 %0, c1, x1, %0;\n\t"
+        "fma.rn.f32.f16 %0, c2, x2, %0;\n\t"
+        "fma.rn.f32.f16 %0, c3, x3, %0;\n\t"
+        "fma.rn.f32.f16 %0, c4, x4, %0;\n\t"
+        "fma.rn.f32.f16 %0, c5, x5, %0;\n\t"
+        "fma.rn.f32.f16 %0, c6, x6, %0;\n\t"
+        "fma.rn.f32.f16 %0, c7, x7, %0;\n\t"
+        "}"
+        : "=&f"(d)
+        : "r"(c.x), "r"(c.y), "r"(c.z), "r"(c.w), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w));
+    return d;
 }
 
 struct RowPair {
@@ -786,10 +759,10 @@ __device__ __forceinline__ void decode_word(const VDec& d, uint32_t rep, uint32_
 // Decodes this thread's columns of one chunk (ring slot k) into accA/accB:
 // the thread's two rows, in radius group `ch` of the chunk.  xw0: shared
 // address of the chunk's first column in its window (batch row stride
-// xstride bytes); sc: 2^k of the window's prescale.
+// xstride bytes).
 template <int MK>
 __device__ __forceinline__ void decode_chunk(const Smem& sm, const Seg& g, const VDec& d, int k, int2 cc,
-                                             uint32_t xw0, uint32_t xstride, float sc, int warp, int lane,
+                                             uint32_t xw0, uint32_t xstride, int warp, int lane,
                                              float (&accA)[MK], float (&accB)[MK]) {
     const int u = 32 * (warp & 3) + lane, o = u >> 2, wi = u & 3, part = warp >> 2;
     const int gfirst = cc.x >> 4;
@@ -805,10 +778,10 @@ __device__ __forceinline__ void decode_chunk(const Smem& sm, const Seg& g, const
     {
         const uint4 mt = lds128_r(base + kMainSlot + (uint32_t)(((grp - gfirst) * g.n_oct + o) * 64 + wi * 16));
         const float2 a = __half22float2(u2h2(mt.y)), b = __half22float2(u2h2(mt.w));
-        rp.dlA = a.y * d.vscale * sc;
-        rp.mpA = a.x * sc - rp.dlA;
-        rp.dlB = b.y * d.vscale * sc;
-        rp.mpB = b.x * sc - rp.dlB;
+        rp.dlA = a.y * d.vscale;
+        rp.mpA = a.x - rp.dlA;
+        rp.dlB = b.y * d.vscale;
+        rp.mpB = b.x - rp.dlB;
         rp.auxA = mt.x;
         rp.auxB = mt.z;
     }
@@ -856,18 +829,23 @@ __device__ __forceinline__ void write_out(const EngineStage& st, const JobView& 
     }
 }
 
-// Epilogue warp: writes (or combines) the outputs of the segments the decode
+// Epilogue warps: write (or combine) the outputs of the segments the decode
 // warps hand over through the stash ring, so that the decode warps never wait
-// on global-memory round trips.  Whole blocks are written directly.  Split
+// on global-memory round trips; two warps take alternate segments, so one
+// segment's round trips overlap the next one's.  Whole blocks are written directly.  Split
 // blocks: every contributor stores its partial sums and publishes them with
 // one acquire-release increment of the block's count; the contributor that
 // completes the count adds all partials in CTA order.  Blocks whose outputs
 // are final are added to the stage's completion count when a later stage of
 // the launch reads them.
 template <int M, class Src>
-__device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P) {
+__device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P, int e) {
     const int lane = threadIdx.x & 31;
     constexpr int NS = Cfg<M>::kSlots;
+    // segment n goes to epilogue warp n % NE, so that a warp owns stash slots
+    // k = e, e + NE, ... and waits on their phases in order
+    constexpr int NE = NS % kEpiWarps == 0 ? kEpiWarps : 1;
+    if (e >= NE) return;
     int n = 0;  // segment counter (stash slot n % NS)
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
@@ -876,6 +854,11 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P) 
         const bool signal = s + 1 < src.n_stages() && src.stage(s + 1).wait;
         unsigned done = 0;
         for (int uu = u0; uu < u1; ++n) {
+            if (n % NE != e) {  // another epilogue warp's segment
+                const Seg g = make_seg(src, s, uu, u1);
+                uu += g.jb - g.ja;
+                continue;
+            }
             const int k = n % NS;
             wait_bar(sm, sm.st_full(k), (n / NS) & 1, P.status);
             const Pending& q = sm.pend[k];
@@ -927,7 +910,8 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P) 
                     for (int i = 0; i < 8; ++i)
 #pragma unroll
                         for (int m = 0; m < M; ++m) tot[i][m] = 0.f;
-                    constexpr int NF = M <= 2 ? 2 : 1;  // contributors whose loads are in flight at once
+                    // contributors whose loads are in flight at once (8 x M x NF values per lane)
+                    constexpr int NF = M == 1 ? 8 : M == 2 ? 4 : M <= 4 ? 2 : 1;
                     for (int c0 = c_first; c0 <= c_last; c0 += NF) {
                         float v[NF][8][M];
 #pragma unroll
@@ -975,7 +959,6 @@ struct DecState {
     WinPos wp;
     int cur_win;          // window the decode warps hold (-1: none)
     bool first_win;       // the next window opened is a stage's first (cooperative gather)
-    float sc;             // 2^k of the held window's prescale
 };
 
 // Decodes one segment with compile-time batch MK (<= M, the window's batch
@@ -991,7 +974,6 @@ __device__ __forceinline__ void seg_body(const Src& src, const Smem& sm, const E
     for (int m = 0; m < MK; ++m) accA[m] = accB[m] = 0.f;
     int t = ds.t, slot = ds.slot, ph = ds.ph, cur_win = ds.cur_win;
     WinPos wp = ds.wp;
-    float sc = ds.sc;
     const int nc = n_chunks(g);
     for (int c = 0; c < nc; ++c, ++t, ring_next(slot, ph, sm.slots)) {
         const int2 cc = chunk_cols(g, c);
@@ -1007,11 +989,9 @@ __device__ __forceinline__ void seg_body(const Src& src, const Smem& sm, const E
             }
             wait_bar(sm, sm.x_full(wp.win & 1), (wp.win >> 1) & 1, P.status);
             cur_win = wp.win;
-            const int k = sm.misc[cur_win & 1];
-            sc = k == 0 ? 1.f : (k == 1 ? 2.f : 4.f);
         }
         wait_bar(sm, sm.full(slot), ph, P.status);
-        decode_chunk<MK>(sm, g, d, slot, cc, sm.xwin(wp.win) + (uint32_t)pos * 16, (uint32_t)xw * 16, sc, warp, lane,
+        decode_chunk<MK>(sm, g, d, slot, cc, sm.xwin(wp.win) + (uint32_t)pos * 16, (uint32_t)xw * 16, warp, lane,
                          accA, accB);
         __syncwarp();
         if (lane == 0) mbar_arrive(sm.empty(slot));
@@ -1021,7 +1001,6 @@ __device__ __forceinline__ void seg_body(const Src& src, const Smem& sm, const E
     ds.ph = ph;
     ds.cur_win = cur_win;
     ds.wp = wp;
-    ds.sc = sc;
     // hand this thread's two rows (this column half) to the epilogue warp
     constexpr int NS = Cfg<M>::kSlots;
     const int k = nseg % NS;
@@ -1046,7 +1025,7 @@ __device__ void decode_role(const Src& src, const Smem& sm, const EngineParams& 
     const int tid = threadIdx.x;
     int ncb = 0, nseg = 0;
     const uint16_t* cur_cb = nullptr;
-    DecState ds{0, 0, 0, {0, 0}, -1, false, 1.f};
+    DecState ds{0, 0, 0, {0, 0}, -1, false};
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
         if (U <= 0) continue;
@@ -1117,8 +1096,8 @@ __device__ void run(const Src& src, const EngineParams& P, uint8_t* smem_raw, in
         copy_role(src, sm, P.status, P.n_cta);
     } else if (warp == kGatherWarp) {
         gather_role<M>(src, sm, P.status, P.sync, P.n_cta, xw, waited);
-    } else if (warp == kEpiWarp) {
-        epi_role<M>(src, sm, P);
+    } else if (warp >= kEpiWarp) {
+        epi_role<M>(src, sm, P, warp - kEpiWarp);
     } else {
         decode_role<M>(src, sm, P, xw);
     }

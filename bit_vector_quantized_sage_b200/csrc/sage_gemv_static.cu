@@ -6,6 +6,7 @@
 // call.  The entry point itself allocates nothing: it calls no cudaMalloc or
 // cudaFree, no allocating library and no torch, and it runs the same kernel as
 // sage_gemv with the array below standing in for the workspace.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -27,21 +28,58 @@ __device__ __align__(256) uint8_t g_gemv_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+    unsigned long long ctx_id;  // context the address belongs to (0: unknown)
+    void* ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of g_gemv_scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// Unique id of the calling thread's current context (cuCtxGetId), or 0 when
+// the driver does not provide it.  The driver calls are reached through the
+// runtime's entry-point query, so nothing links against libcuda.  Called with
+// g_mu held.
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static bool queried = false;
+    if (!queried) {
+        queried = true;
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(f);
+    }
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (get_current && get_id && get_current(&c) == CUDA_SUCCESS && c && get_id(c, &id) == CUDA_SUCCESS) return id;
+    return 0;
+}
+
+// Device address of g_gemv_scratch in the current context, looked up with
+// that context current and cached per device together with the context's id:
+// a new context on the device (after cudaDeviceReset, say) reloads the
+// library's device code, and the address is looked up again.
 int scratch_for_current_device(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    ScratchEntry& e = g_scratch[dev];
+    const unsigned long long id = current_context_id();
+    if (!e.ptr || id == 0 || id != e.ctx_id) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_gemv_scratch) != cudaSuccess || !p) return SAGE_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
+        e.ptr = p;
+        e.ctx_id = current_context_id();  // the lookup made the context current if it was not yet
     }
-    *out = g_scratch_ptr[dev];
+    *out = e.ptr;
     return SAGE_OK;
 }
 

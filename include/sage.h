@@ -177,16 +177,21 @@ int sage_gemv(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y,
  *     sums on a 148-SM GPU; the rest holds one 4-byte counter per 256 output
  *     rows, so any d_out up to about 400,000 rows fits.  Larger shapes return
  *     SAGE_ERR_WORKSPACE before anything is launched.
- *   - The first call on each device looks up the array's device address with
- *     that device current; make that first call outside any CUDA stream
- *     capture.
+ *   - The first call in each CUDA context (per device, and again after the
+ *     context is replaced, e.g. by cudaDeviceReset) looks up the array's
+ *     device address in that context; make that first call outside any CUDA
+ *     stream capture.
  *   - Calls on one device share the scratch: they must not overlap.  Two calls
  *     in flight at once (different streams, or different host threads without
  *     ordering) race on it and give wrong results.
  *   - The status word and counters in the scratch start at zero and every
  *     completed call leaves them at zero.  A bounded device wait that gives up
- *     (SAGE_ERR_TIMEOUT under sage_gemv) is not reported by this entry point:
- *     use sage_gemv with a workspace where that report is needed.
+ *     (SAGE_ERR_TIMEOUT under sage_gemv; only a GPU stalled for seconds causes
+ *     one) is not reported by this entry point, and it may leave split-K
+ *     counters non-zero, after which later calls in the same context compute
+ *     wrong sums until the context is replaced.  Use sage_gemv with a
+ *     workspace where that report, or recovery by zeroing the workspace,
+ *     is needed.
  * Errors: as sage_gemv, with WORKSPACE meaning "shape beyond the 4 MiB
  * scratch". */
 int sage_gemv_static(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y, sage_stream_t stream);

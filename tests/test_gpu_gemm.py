@@ -59,6 +59,51 @@ def test_gemm_deterministic_and_status_clean():
     assert np.array_equal(host_u16(y), y1)
 
 
+@pytest.mark.parametrize("M,entry", [(1, "gemv"), (2, "gemv"), (4, "gemv"), (8, "gemv"), (16, "gemm"), (128, "gemm")])
+def test_config3_full_rows(M, entry):
+    """The 4096 -> 12288 up-projection at full size, every output row against the
+    oracle: batch 1-8 through the GEMV engine, 16 and 128 through the tcgen05 path."""
+    f, x = synth.config3(M)
+    y, _, _ = gemv(f, x, entry=entry)
+    y_ref, B = oracle.gemv(f, x)
+    assert_within_bound(y, y_ref, B, f"config3 M={M} ({entry})")
+
+
+def test_config3_back_to_back_replicas():
+    """The launch form the benchmark times: a CUDA graph of the GEMV over copies of the
+    planes back to back (programmatic dependent launch between them, one workspace).
+    Each copy's output, captured in its own buffer, is bit-identical to an eager call."""
+    import torch
+    f, xb = synth.config3(1)
+    A0 = sage.PackedMatrix.from_fields(f)
+    As = [A0] + [sage.PackedMatrix(A0.d_out, A0.d_in, A0.log2K, A0.main.clone(), A0.meta.clone(),
+                                   A0.codebook.clone(), None, "copy") for _ in range(3)]
+    x = dev_u16(xb)
+    ys = [torch.zeros((1, f.d_out), dtype=torch.int16, device="cuda") for _ in As]
+    ws = workspace_for(sage.SAGE_OP_GEMV, A0, 1)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        for A, y in zip(As, ys):
+            sage.sage_gemv(A, x, 1, y, ws, s)
+        s.synchronize()
+        eager = [host_u16(y) for y in ys]
+        for y in ys:
+            y.zero_()
+        with torch.cuda.graph(g, stream=s):
+            for A, y in zip(As, ys):
+                sage.sage_gemv(A, x, 1, y, ws, torch.cuda.current_stream())
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    assert sage.sage_query_status(ws) == sage.SAGE_OK
+    for y, e in zip(ys, eager):
+        assert np.array_equal(host_u16(y), e)
+    y_ref, B = oracle.gemv(f, xb)
+    assert_within_bound(eager[-1], y_ref, B, "config3 last copy")
+    del g
+
+
 @pytest.mark.parametrize("M", [16, 32, 64, 128])
 def test_config3_sampled_rows(M):
     """Qwen3-8B-shaped up-projection 4096 -> 12288, (K,V) = (32,5), at full size;

@@ -54,6 +54,41 @@ def test_batches(M):
     assert_within_bound(y, y_ref, B, f"M={M}")
 
 
+def _heavy_inputs(kind, g, M, d_in, perm):
+    """Heavy-tailed activations: N(0,1) scaled by sqrt of LogNormal(0, 1.5) channel
+    energies (the energy model the ESG permutation is built from); a few channels at
+    1e3..1e4; or one storage subvector whose four low-lane components (0, 2, 4, 6;
+    one half2 accumulator) sit near 2^15, so that the power-of-two window prescale
+    must act for the fp16 partial sums to stay finite."""
+    x = g.standard_normal((M, d_in))
+    if kind == "energy":
+        x *= np.sqrt(synth.lognormal_energies(g, d_in, 1.5))[None, :]
+    elif kind == "outliers":
+        for m in range(M):
+            c = g.choice(d_in, 6, replace=False)
+            x[m, c] = g.choice([-1.0, 1.0], 6) * g.uniform(1e3, 1e4, 6)
+    else:
+        sv = 37
+        for m in range(M):
+            for i in (0, 2, 4, 6):
+                x[m, perm[8 * sv + i]] = (1.0 if i % 4 == 0 else -1.0) * (29000.0 + 500.0 * i)
+    return synth.f16_bits(x)
+
+
+@pytest.mark.parametrize("kind", ["energy", "outliers", "near_2p15"])
+@pytest.mark.parametrize("log2K", [4, 6, 8])
+@pytest.mark.parametrize("M,entry", [(1, "gemv"), (3, "gemv"), (16, "gemm")])
+def test_heavy_tailed_activations(kind, log2K, M, entry):
+    g = np.random.default_rng(1000 * ("energy", "outliers", "near_2p15").index(kind) + 10 * log2K + M)
+    f = synth.random_fields(g, 520, 2560, log2K)
+    f.perm = g.permutation(2560).astype(np.int32)
+    x = _heavy_inputs(kind, g, M, 2560, f.perm)
+    y, _, _ = gemv(f, x, entry=entry)
+    assert np.isfinite(f16_to_f64(y)).all()
+    y_ref, B = oracle.gemv(f, x)
+    assert_within_bound(y, y_ref, B, f"{kind} K=2^{log2K} M={M} {entry}")
+
+
 def test_deterministic_and_status_clean():
     f = _fields(5, 3000, 2560, 6)
     x = synth.activations(np.random.default_rng(5), 2, 2560)

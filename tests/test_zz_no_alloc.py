@@ -28,12 +28,27 @@ def test_static_rejects_shapes_beyond_its_scratch(lib):
     assert lib.sage_gemv_static(C.byref(A), 0x400002, 1, 0x500000, None) == sage.SAGE_ERR_MISALIGNED
 
 
+def _split_ways(d_out, d_in, sms):
+    """CTAs sharing the widest 256-row block under the engine's launch geometry:
+    one CTA per SM (at most a quarter as many CTAs as block columns), the block
+    columns of the launch split evenly over them."""
+    units = ((d_out + 7) // 8 + 31) // 32 * (d_in // 8)
+    n_cta = max(1, min(sms, units // 4))
+    per_block = d_in // 8
+    return min(n_cta, -(-per_block * n_cta // units) + 1)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("d_out,d_in,log2K,M", [(256, 512, 6, 1), (3000, 2560, 5, 1), (1500, 4096, 7, 4)])
+@pytest.mark.parametrize("d_out,d_in,log2K,M", [(256, 512, 6, 1), (3000, 2560, 5, 1), (1500, 4096, 7, 4),
+                                                (64, 9728, 6, 1), (200, 9728, 8, 2)])
 def test_static_matches_workspace_entry_twice(lib, d_out, d_in, log2K, M):
     """Two calls in a row (the second relies on the first leaving the scratch's
-    counters at zero) give the bits of sage_gemv, within the oracle's bound."""
+    counters at zero) give the bits of sage_gemv, within the oracle's bound.  Every
+    case splits a block over several CTAs, so the split-K counters and partial sums
+    in the scratch are exercised (the last two over the whole GPU)."""
     import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert _split_ways(d_out, d_in, sms) >= 2
     g = np.random.default_rng(d_out + M)
     f = synth.random_fields(g, d_out, d_in, log2K)
     f.perm = g.permutation(d_in).astype(np.int32)
