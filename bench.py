@@ -455,33 +455,31 @@ def capture(fn, stream):
     return g
 
 
-def per_call_us(fns, stream, rounds=4):
-    """Device time of each call, one CUDA graph per call replayed back to back with
-    events between the replays; `fns` rotate over copies of the data larger than L2.
-    Returns the list of per-call times (us)."""
+def per_call_us(fns, stream, rounds=12):
+    """Device time per call: one CUDA graph holds the calls back to back (they rotate
+    over copies of the data larger than L2, chained by programmatic dependent launch
+    as a stream of layers is), replayed `rounds` times with events around each
+    replay.  Returns one per-call average per replay (us)."""
     import torch
-    graphs = [capture(f, stream) for f in fns]
-    for g in graphs:
+    g = capture(lambda st: [f(st) for f in fns], stream)
+    for _ in range(2):
         g.replay()
     torch.cuda.synchronize()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) * rounds + 1)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(rounds + 1)]
     ev[0].record(stream)
-    k = 1
-    for _ in range(rounds):
-        for g in graphs:
-            g.replay()
-            ev[k].record(stream)
-            k += 1
+    for k in range(rounds):
+        g.replay()
+        ev[k + 1].record(stream)
     torch.cuda.synchronize()
-    out = [ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(len(ev) - 1)]
-    del graphs
+    out = [ev[i].elapsed_time(ev[i + 1]) * 1e3 / len(fns) for i in range(rounds)]
+    del g
     return out
 
 
-def bench_gemm(stream, reps_rounds=3):
+def bench_gemm(stream):
     """4096 -> 12288 up-projection, (K,V) = (32,5): batch 1-8 through the GEMV engine,
     16-128 through the tcgen05 path (sage_gemm dispatches).  Per batch: device us
-    (median, p10, p90 over copies of the planes larger than L2), TFLOP/s against the
+    (median, p10, p90 over replays of the copies of the planes), TFLOP/s against the
     dense fp16 tensor peak and GB/s of packed bytes against HBM."""
     import torch
     import synth
@@ -500,7 +498,7 @@ def bench_gemm(stream, reps_rounds=3):
         fns = [lambda st, A=A: sage.sage_gemm(A, x, M, y, ws, st) for A in As]
         for fn in fns[:3]:
             fn(stream)
-        t = per_call_us(fns, stream, reps_rounds)
+        t = per_call_us(fns, stream)
         assert sage.sage_query_status(ws) == sage.SAGE_OK
         us = float(np.median(t))
         flops = 2.0 * M * f.d_out * f.d_in
@@ -515,12 +513,15 @@ def bench_gemm(stream, reps_rounds=3):
 
 def bench_moe(stream, reps=20):
     """128 experts (gate/up 2048 -> 768, down 768 -> 2048), top-8 routing, T tokens; one
-    sage_moe_gemv call per projection, L2 flushed before each call."""
+    sage_moe_gemv call per projection, L2 flushed before each call by reading a buffer
+    twice its size (a read leaves clean lines: a write-based flush would leave the call
+    to write back ~126 MB of dirty lines)."""
     import torch
     import synth
     import bit_vector_quantized_sage_b200 as sage
     hbm, _ = _peaks()
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    sink = torch.empty((), dtype=torch.float32, device="cuda")
     out = []
     for proj in (0, 2):
         packed = None
@@ -545,7 +546,7 @@ def bench_moe(stream, reps=20):
             g = capture(fn, stream)
             t = []
             for _ in range(reps):
-                flush.fill_(1)
+                sink = flush.sum()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 g.replay()
@@ -561,7 +562,8 @@ def bench_moe(stream, reps=20):
             out.append({"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size), "us": dist_summary(t),
                         "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4)})
     del flush
-    return {"workload": "128 experts, top-8, one projection per call, L2 flushed before each call", "points": out}
+    return {"workload": "128 experts, top-8, one projection per call (routing + grouped GEMV), L2 flushed "
+                        "(read) before each call", "points": out}
 
 
 def oracle_beside(pool_1):
@@ -689,12 +691,14 @@ def run_gpu(args):
     layer_modes = {}
     with torch.cuda.stream(stream):
         for mode, (mf, mws, _, _, ml) in modes.items():
-            t = per_call_us(mf, stream, rounds=max(2, 60 // replicas))
+            t = per_call_us(mf, stream)
             assert sage.sage_query_status(mws) == sage.SAGE_OK
             med = float(np.median(t))
             layer_modes[mode] = {"launches_per_layer": ml, "us_per_layer": dist_summary(t),
                                  "gbs": round(one_layer_bytes / (med * 1e-6) / 1e9, 1),
                                  "hbm_frac": round(one_layer_bytes / (med * 1e-6) / 1e9 / _peaks()[0], 4)}
+    for m in layer_modes.values():
+        m["timing"] = "per layer: one CUDA graph over the rotating copies, median/p10/p90 over 12 replays"
     layer_modes["fused"]["what"] = ("the decoder layer as one launch: RMSNorm -> q|k|v, attention over one cached "
                                     "position -> o, residual + RMSNorm -> gate|up, SiLU * up -> down + residual")
     layer_modes["stages"]["what"] = "the four stages as four grouped launches (PDL-chained), synthetic stage inputs"

@@ -87,11 +87,8 @@ struct MoeParams {
     int n_experts, d_out, d_in, n_pairs;
     const uint16_t* x;
     uint16_t* y;
-    const unsigned* route;      // ws: number of virtual experts
-    const int32_t* v_expert;    // ws [n_pairs]
-    const int32_t* v_xrows;     // ws [n_pairs][8]
-    const int32_t* v_yrows;     // ws [n_pairs][8]
-    const int32_t* v_count;     // ws [n_pairs]
+    const int32_t* pair_expert;  // [n_pairs]
+    const int32_t* pair_xrow;    // [n_pairs]
     EngineExpert experts[kMaxExperts];
 };
 

@@ -208,12 +208,13 @@ __host__ __device__ inline int gemm_smem_bytes(int K, int n_pad, int a_slots, in
 // Rebuilds one subvector of one row (Eq. 1-2), rounded to fp16: w is the
 // record word holding the row, odd selects the row's half of it (rows 2u and
 // 2u + 1 share word u), s0..s2 are the row's sign-slot shifts, and the aux
-// signs come from the row's group word at bit `col`.
+// signs come from the row's group word at bit `col`.  The codeword load may be
+// reordered by the compiler (cbsel carries the caller's order token).
 __device__ __forceinline__ uint4 decode_sv(const VDec& d, uint32_t w, bool odd, uint32_t s0, uint32_t s1,
                                            uint32_t s2, uint32_t aux, uint32_t sh_aux, float mp, float dl,
                                            uint32_t cbsel) {
     const uint32_t wf = odd ? rot16(w) : w;  // (z, q) field word of this row
-    uint4 c = lds128(cbsel + (wf & d.zmask));
+    uint4 c = lds128_r(cbsel + (wf & d.zmask));
     c.x ^= (w << s0) & 0x80008000u;
     c.y ^= (w << s1) & 0x80008000u;
     c.z ^= (w << s2) & 0x80008000u;
@@ -354,18 +355,25 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
                 const int s = 2 * t + h;
                 // the A buffer of slab s was last read by the MMAs of slab s - NA
                 if (s >= NA) gwait(sm.mma_done(s - NA, NB), ((s - NA) / NB) & 1, p.status);
+                // The four subvectors' shared loads are independent: non-volatile
+                // loads whose addresses carry a token taken after the waits above
+                // (chunk resident, slab buffer free) let them overlap; the stores,
+                // which consume every result, stay in order before the arrival.
+                const uint32_t tok = order_token();
                 const uint32_t a_slab = sm.a0 + (uint32_t)(s % NA) * kASlab + a_row;
+                uint4 v[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int wc = 4 * cw + i;          // slab column
-                    const int jl = h * kGSlabJ + wc;    // chunk column
-                    uint4 v = make_uint4(0, 0, 0, 0);
+                    const int jl = h * kGSlabJ + 4 * cw + i;  // chunk column
+                    v[i] = make_uint4(0, 0, 0, 0);
                     if (active) {
-                        const uint32_t w = lds32(slot + (uint32_t)(jl * n_oct + o) * 16 + (uint32_t)(tr >> 1) * 4);
-                        v = decode_sv(d, w, odd, s0, s1, s2, aux, (uint32_t)(15 - jl), mp, dl, cbsel);
+                        const uint32_t w =
+                            lds32_r(slot + tok + (uint32_t)(jl * n_oct + o) * 16 + (uint32_t)(tr >> 1) * 4);
+                        v[i] = decode_sv(d, w, odd, s0, s1, s2, aux, (uint32_t)(15 - jl), mp, dl, cbsel + tok);
                     }
-                    sts128(a_slab + (uint32_t)wc * 128, v);
                 }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sts128(a_slab + (uint32_t)(4 * cw + i) * 128, v[i]);
                 fence_proxy_async_smem();  // the generic-proxy writes above are read by the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sm.a_full(s, NA));

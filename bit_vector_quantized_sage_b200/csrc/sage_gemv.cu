@@ -130,9 +130,9 @@ struct DenseSrc {
     }
 };
 
-// The MoE routing result this CTA needs (virtual-expert ids, pair counts and
-// row lists of the virtual experts its range touches) is staged in shared
-// memory once, after the routing kernel.
+// The MoE routing this CTA needs (virtual-expert ids, pair counts and row
+// lists of the virtual experts its range touches), built in shared memory by
+// the CTA at the start of the MoE kernel.
 struct MoeStage {
     int n_virtual, units, vi0, nvi, overflow;
     int v_expert[kMoeCache];
@@ -413,10 +413,18 @@ __device__ void copy_role(const Src& src, const Smem& sm, uint32_t* status, int 
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 __device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
 
-// Activation loads of the gather: through L2 (data written by an earlier stage
-// of the same launch is not in any L1).  The flag is kept for the call sites.
+// Activation loads of the gather, cached in L1.  Every CTA reads the same few
+// KB of sources (an activation row, a norm weight vector, an earlier stage's
+// outputs) as scattered 2-byte loads; through L2 alone each one is its own
+// L2 request, and all CTAs' requests fall on the same few dozen lines, which
+// serialises them at the L2 slices (microseconds per window).  Through L1 a
+// CTA asks L2 for each line once.  Staleness: no CTA reads a source before
+// it is final -- earlier kernels' outputs after the wait on them
+// (griddepcontrol.wait), earlier stages' outputs after the acquire of the
+// stage's completion count, which the other gathering warps follow through
+// a CTA barrier -- and an acquire at GPU scope invalidates the SM's L1.
 __device__ __forceinline__ uint16_t ld16(const uint16_t* p, bool) {
-    return __ldcg(reinterpret_cast<const unsigned short*>(p));
+    return __ldca(reinterpret_cast<const unsigned short*>(p));
 }
 
 // The stage's prologue applied to the 8 input channels cs[] of batch row xr
@@ -530,7 +538,7 @@ __device__ void gather_items_k(const Src& src, const Smem& sm, int s, int wlen, 
             const int xr = v.xrows ? v.xrows[m] : m;
             if (PRO == kProPlain && !v.perm) {
                 const uint16_t* row = v.x + (size_t)xr * v.d_in + j * 8;
-                val = __ldcg(reinterpret_cast<const uint4*>(row));
+                val = __ldca(reinterpret_cast<const uint4*>(row));
             } else {
                 int cs[8];
                 if (v.perm) {
@@ -828,6 +836,15 @@ __device__ __forceinline__ void write_out(const EngineStage& st, const JobView& 
         st.eo[i] = f2h(h2f(r) + h2f(yb));
     }
 }
+// The same with fp16(ea + eb) loaded ahead (rsum: its fp16 bits).
+__device__ __forceinline__ void write_out_pre(const EngineStage& st, const JobView& v, int m, int row, float tot,
+                                              uint16_t rsum) {
+    const int yr = v.yrows ? v.yrows[m] : m;
+    const uint16_t yb = f2h(tot);
+    const size_t i = (size_t)yr * v.d_out + row;
+    v.y[i] = yb;
+    st.eo[i] = f2h(h2f(rsum) + h2f(yb));
+}
 
 // Epilogue warps: write (or combine) the outputs of the segments the decode
 // warps hand over through the stash ring, so that the decode warps never wait
@@ -873,6 +890,27 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P, 
                 return t;
             };
             const int mk = g.v.Mk;
+            // residual epilogue at batch <= 2: fp16(ea + eb) of this lane's rows is
+            // loaded before the split-K round trips, off the critical path
+            constexpr int RM = M <= 2 ? M : 1;
+            const bool pre = M <= 2 && src.stage(s).epi == kEpiResidual;
+            uint16_t rsum[8][RM];
+            if (pre) {
+                const EngineStage& es = src.stage(s);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int m = 0; m < RM; ++m) {
+                        const int row = g.blk * kBlockRows + lane + 32 * i;
+                        rsum[i][m] = 0;
+                        if (row < g.v.d_out && m < mk) {
+                            const int yr = g.v.yrows ? g.v.yrows[m] : m;
+                            const size_t e = (size_t)yr * g.v.d_out + row;
+                            rsum[i][m] = f2h(h2f(__ldcg(reinterpret_cast<const unsigned short*>(es.ea + e))) +
+                                             h2f(__ldcg(reinterpret_cast<const unsigned short*>(es.eb + e))));
+                        }
+                    }
+            }
             if (g.full) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -880,7 +918,10 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P, 
                     if (row < g.v.d_out)
 #pragma unroll
                         for (int m = 0; m < M; ++m)
-                            if (m < mk) write_out(src.stage(s), g.v, m, row, part_sum(m, r));
+                            if (m < mk) {
+                                if (pre) write_out_pre(src.stage(s), g.v, m, row, part_sum(m, r), rsum[i][m < RM ? m : 0]);
+                                else write_out(src.stage(s), g.v, m, row, part_sum(m, r));
+                            }
                 }
                 ++done;
             } else {
@@ -938,7 +979,10 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P, 
                         if (row < g.v.d_out)
 #pragma unroll
                             for (int m = 0; m < M; ++m)
-                                if (m < mk) write_out(src.stage(s), g.v, m, row, tot[i][m]);
+                                if (m < mk) {
+                                    if (pre) write_out_pre(src.stage(s), g.v, m, row, tot[i][m], rsum[i][m < RM ? m : 0]);
+                                    else write_out(src.stage(s), g.v, m, row, tot[i][m]);
+                                }
                     }
                     ++done;
                 }
@@ -1121,14 +1165,49 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
 }
 
 // Virtual experts carry 1..8 pairs each; the kernel's batch stride is 8.
+// Grouped-expert GEMV.  Every CTA groups the (token, slot) pairs by expert
+// itself -- in expert order and, within an expert, in pair order, into virtual
+// experts of at most 8 pairs -- and keeps the virtual experts that its unit
+// range covers; all CTAs derive the same grouping from the same pairs
+// (deterministic), and no routing kernel or routing round trip precedes the
+// decode.
 __global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant__ MoeParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ MoeStage ms;
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_first[kMaxExperts + 1];  // first virtual expert of expert e; [n_experts]: their number
+    __shared__ int s_m2;
+    constexpr int MV = kMaxPairsPerVirtual;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, n_e = p.n_experts;
     pdl_launch_dependents();
-    pdl_wait();  // the routing comes from the preceding kernel
+    pdl_wait();  // the pairs and x come from the preceding kernel
+    for (int e = tid; e < n_e; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    for (int q = tid; q < p.n_pairs; q += blockDim.x) {
+        const int e = __ldca(p.pair_expert + q);
+        if (e >= 0 && e < n_e) atomicAdd(&s_cnt[e], 1);
+        else if (blockIdx.x == 0) flag(p.e.status, kDevUnsupported);  // that pair's output is not written
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the virtual-expert counts, 32 experts at a time
+        int carry = 0;
+        for (int e0 = 0; e0 < n_e; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < n_e ? (s_cnt[e] + MV - 1) / MV : 0;
+            int incl = v;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (e < n_e) s_first[e] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_first[n_e] = carry;
+    }
+    __syncthreads();
     const int upv = ((((p.d_out + 7) >> 3) + kOct - 1) / kOct) * (p.d_in >> 3);
-    if (threadIdx.x == 0) {
-        ms.n_virtual = (int)__ldcg(reinterpret_cast<const unsigned*>(p.route));
+    if (tid == 0) {
+        ms.n_virtual = s_first[n_e];
         ms.units = ms.n_virtual * upv;
         const int u0 = cta_begin(ms.units, p.e.n_cta, blockIdx.x), u1 = cta_begin(ms.units, p.e.n_cta, blockIdx.x + 1);
         ms.vi0 = u0 / upv;
@@ -1138,19 +1217,35 @@ __global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant_
         if (ms.overflow) flag(p.e.status, kDevUnsupported);
     }
     __syncthreads();
-    if ((int)threadIdx.x < ms.nvi) {
-        const int vi = ms.vi0 + threadIdx.x;
-        ms.v_expert[threadIdx.x] = __ldcg(p.v_expert + vi);
-        ms.v_count[threadIdx.x] = __ldcg(p.v_count + vi);
+    // the pairs of the CTA's virtual experts: one warp per expert whose virtual
+    // experts meet [vi0, vi0 + nvi), ranking its pairs by a ballot over the pair list
+    const int v0 = ms.vi0, v1 = ms.vi0 + ms.nvi;
+    for (int e = warp; e < n_e; e += kThreads / 32) {
+        const int f0 = s_first[e], f1 = s_first[e + 1];
+        if (f1 <= v0 || f0 >= v1) continue;
+        int k = 0;  // pairs of expert e before this round
+        for (int q0 = 0; q0 < p.n_pairs; q0 += 32) {
+            const int q = q0 + lane;
+            const bool hit = q < p.n_pairs && __ldca(p.pair_expert + q) == e;
+            const unsigned b = __ballot_sync(0xffffffffu, hit);
+            if (hit) {
+                const int kk = k + __popc(b & ((1u << lane) - 1u));
+                const int vi = f0 + kk / MV;
+                if (vi >= v0 && vi < v1) {
+                    ms.v_xrows[vi - v0][kk % MV] = __ldca(p.pair_xrow + q);
+                    ms.v_yrows[vi - v0][kk % MV] = q;
+                }
+            }
+            k += __popc(b);
+        }
+        for (int vi = max(f0, v0) + lane; vi < min(f1, v1); vi += 32) {
+            ms.v_expert[vi - v0] = e;
+            ms.v_count[vi - v0] = min(MV, s_cnt[e] - (vi - f0) * MV);
+        }
     }
-    for (int i = threadIdx.x; i < ms.nvi * kMaxPairsPerVirtual; i += blockDim.x) {
-        const size_t src_i = (size_t)ms.vi0 * kMaxPairsPerVirtual + i;
-        ms.v_xrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_xrows + src_i);
-        ms.v_yrows[i / kMaxPairsPerVirtual][i % kMaxPairsPerVirtual] = __ldcg(p.v_yrows + src_i);
-    }
+    __syncthreads();
     // the window holds the largest pair count of this CTA's virtual experts
-    __shared__ int s_m2;
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         int mmax = 1;
         for (int k = 0; k < ms.nvi; ++k) mmax = max(mmax, ms.v_count[k]);
         int m2 = 1;
@@ -1161,45 +1256,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant_
     if (ms.overflow) return;  // more virtual experts than the staging holds (flagged above)
     const MoeSrc src{p, ms};
     run<kMaxPairsPerVirtual>(src, p.e, smem_raw, kXBufBytes / (16 * s_m2), s_m2, true);
-}
-
-// Groups the (pair -> expert) routing into virtual experts of at most 8 pairs,
-// in expert order and, within an expert, pair order (deterministic).
-__global__ void moe_route_kernel(const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs, int n_experts,
-                                 unsigned* route, int32_t* v_expert, int32_t* v_xrows, int32_t* v_yrows,
-                                 int32_t* v_count, uint32_t* status) {
-    pdl_wait();
-    extern __shared__ int s_cnt[];  // [n_experts]
-    for (int e = threadIdx.x; e < n_experts; e += blockDim.x) s_cnt[e] = 0;
-    __syncthreads();
-    for (int q = threadIdx.x; q < n_pairs; q += blockDim.x) {
-        const int e = pair_expert[q];
-        if (e >= 0 && e < n_experts) atomicAdd(&s_cnt[e], 1);
-        else atomicOr(status, kDevUnsupported);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int nv = 0;
-        for (int e = 0; e < n_experts; ++e) {
-            const int c = s_cnt[e];
-            s_cnt[e] = nv;  // first virtual index of expert e
-            nv += (c + kMaxPairsPerVirtual - 1) / kMaxPairsPerVirtual;
-        }
-        *route = (unsigned)nv;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < n_experts; e += blockDim.x) {
-        int vi = s_cnt[e], k = 0;
-        for (int q = 0; q < n_pairs; ++q) {
-            if (pair_expert[q] != e) continue;
-            if (k == kMaxPairsPerVirtual) { ++vi; k = 0; }
-            v_expert[vi] = e;
-            v_xrows[(size_t)vi * kMaxPairsPerVirtual + k] = pair_xrow[q];
-            v_yrows[(size_t)vi * kMaxPairsPerVirtual + k] = q;
-            v_count[vi] = ++k;
-        }
-    }
-    pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------------
@@ -1362,19 +1418,14 @@ int launch_gemv(const GemvJob* jobs, int n, int M, void* ws, size_t ws_bytes, sa
     return launch_engine(&st, 1, M, ws, ws_bytes, stream);
 }
 
-// MoE workspace: header | route | v_expert | v_xrows | v_yrows | v_count | counters | partials
+// MoE workspace: header | split-K counters | partials
 namespace {
 struct MoeWs {
-    size_t route, v_expert, v_xrows, v_yrows, v_count, counters, partials, total;
+    size_t counters, partials, total;
 };
 MoeWs moe_ws_layout(int n_pairs, int d_out, int n_cta) {
     MoeWs L;
     size_t o = kWsHeader;
-    L.route = o; o += 256;
-    L.v_expert = o; o += round256((size_t)n_pairs * 4);
-    L.v_xrows = o; o += round256((size_t)n_pairs * kMaxPairsPerVirtual * 4);
-    L.v_yrows = o; o += round256((size_t)n_pairs * kMaxPairsPerVirtual * 4);
-    L.v_count = o; o += round256((size_t)n_pairs * 4);
     const int nblk = ((d_out + 7) / 8 + kOct - 1) / kOct;
     L.counters = o; o += round256((size_t)n_pairs * nblk * 4);
     L.partials = o; o += (size_t)n_cta * 2 * 8 * kBlockRows * sizeof(float);
@@ -1391,6 +1442,7 @@ size_t moe_workspace_bytes(const sage_matrix* experts, int n_experts, int n_pair
 int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_expert, const int32_t* pair_xrow,
                int n_pairs, const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream) {
     constexpr int MV = kMaxPairsPerVirtual;
+    constexpr int kMoeStatic = (int)(sizeof(MoeStage) + (2 * kMaxExperts + 2) * sizeof(int));
     if (n_experts > kMaxExperts) return SAGE_ERR_UNSUPPORTED;
     const int n_cta = current_sm_count();
     const MoeWs L = moe_ws_layout(n_pairs, experts[0].d_out, n_cta);
@@ -1407,10 +1459,10 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
     p.e.n_cta = n_cta;
     p.e.M = MV;
     p.e.kmax = kmax;
-    p.e.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget - (int)sizeof(MoeStage));
+    p.e.slots = slots_for<MV>(1 << 30, kmax, kSmemBudget - kMoeStatic);
     p.e.uses_sync = 0;
     const int smem = smem_bytes<MV>(p.e.slots, kmax);
-    if (smem > kSmemBudget - (int)sizeof(MoeStage)) return SAGE_ERR_UNSUPPORTED;
+    if (smem > kSmemBudget - kMoeStatic) return SAGE_ERR_UNSUPPORTED;
     if (!limit.ensure(moe_kernel, smem)) return SAGE_ERR_CUDA;
     p.e.status = reinterpret_cast<uint32_t*>(w);
     p.e.sync = reinterpret_cast<unsigned*>(w);
@@ -1425,34 +1477,14 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
     p.n_pairs = n_pairs;
     p.x = x;
     p.y = y;
-    p.route = reinterpret_cast<const unsigned*>(w + L.route);
-    p.v_expert = reinterpret_cast<const int32_t*>(w + L.v_expert);
-    p.v_xrows = reinterpret_cast<const int32_t*>(w + L.v_xrows);
-    p.v_yrows = reinterpret_cast<const int32_t*>(w + L.v_yrows);
-    p.v_count = reinterpret_cast<const int32_t*>(w + L.v_count);
+    p.pair_expert = pair_expert;
+    p.pair_xrow = pair_xrow;
     for (int e = 0; e < n_experts; ++e) {
         p.experts[e].main = experts[e].main;
         p.experts[e].meta = experts[e].meta;
         p.experts[e].cb = experts[e].codebook;
         p.experts[e].perm = experts[e].perm;
         p.experts[e].log2K = experts[e].log2K;
-    }
-    {
-        cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3(1);
-        cfg.blockDim = dim3(256);
-        cfg.dynamicSmemBytes = (size_t)n_experts * sizeof(int);
-        cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, moe_route_kernel, pair_expert, pair_xrow, n_pairs, n_experts,
-                               reinterpret_cast<unsigned*>(w + L.route), reinterpret_cast<int32_t*>(w + L.v_expert),
-                               reinterpret_cast<int32_t*>(w + L.v_xrows), reinterpret_cast<int32_t*>(w + L.v_yrows),
-                               reinterpret_cast<int32_t*>(w + L.v_count), p.e.status) != cudaSuccess)
-            return SAGE_ERR_CUDA;
     }
     return launch_pdl(moe_kernel, p, n_cta, smem, stream);
 }

@@ -57,6 +57,15 @@ PLANTS = {
                              "            for (int i = 0; i < SV; ++i) acc[z[s] * SV + i] += Wt[(size_t)s * SV + 0] * p[i] / nn;"),
     "kmeans_empty_cluster_reset": ("            if (nn <= 0.0) continue;\n            nn = sqrt(nn);\n            for (int i = 0; i < SV; ++i) cb[k * SV + i] = acc[k * SV + i] / nn;",
                                    "            if (nn <= 0.0) { for (int i = 0; i < SV; ++i) cb[k * SV + i] = 0.0; continue; }\n            nn = sqrt(nn);\n            for (int i = 0; i < SV; ++i) cb[k * SV + i] = acc[k * SV + i] / nn;"),
+    "pack_q_one_bit_low": ("            if (!isB) w |= (z << 7) | (qq << (23 - V));", "            if (!isB) w |= (z << 7) | (qq << (22 - V));"),
+    "pack_aux_pair_swapped": ("            meta_plane[ai] |= (((s >> 6) & 1u) << tj) | (((s >> 7) & 1u) << (tj + 16));",
+                              "            meta_plane[ai] |= (((s >> 7) & 1u) << tj) | (((s >> 6) & 1u) << (tj + 16));"),
+    "rmsnorm_no_eps": ("        const double inv = 1.0 / sqrt(ss / (double)d + eps);", "        const double inv = 1.0 / sqrt(ss / (double)d);"),
+    "rmsnorm_sum_not_mean": ("        const double inv = 1.0 / sqrt(ss / (double)d + eps);", "        const double inv = 1.0 / sqrt(ss + eps);"),
+    "silu_sign": ("        out[i] = oracle_double_to_half(t / (1.0 + exp(-t)) * oracle_half_to_double(up[i]));",
+                  "        out[i] = oracle_double_to_half(t / (1.0 + exp(t)) * oracle_half_to_double(up[i]));"),
+    "attend_head_map": ("                out[((size_t)m * n_heads + h) * hd + e] = v[((size_t)m * n_kv + h / grp) * hd + e];",
+                        "                out[((size_t)m * n_heads + h) * hd + e] = v[((size_t)m * n_kv + h % n_kv) * hd + e];"),
     "encode_grid_unweighted_radius": _UNWEIGHTED,
     "encode_quantize_unrounded_grid": _UNROUNDED,
 }

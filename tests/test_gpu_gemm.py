@@ -113,3 +113,28 @@ def test_config3_sampled_rows(M):
     for r0, r1 in ((0, 40), (250, 262), (6140, 6160), (12230, 12288)):
         y_ref, B = oracle.gemv(f, x, rows=(r0, r1))
         assert_within_bound(y[:, r0:r1], y_ref[:, r0:r1], B[:, r0:r1], f"config3 M={M} rows {r0}:{r1}")
+
+
+@pytest.mark.parametrize("log2K", [4, 6, 8])
+def test_gemm_reconstruction_within_one_ulp(log2K):
+    """The tensor-core path's own fp16 W_hat tiles, read back through one-hot
+    inputs: batch row m selects original channel c_m, so y[m] is column
+    pi^-1(c_m) of the tile-reconstructed W_hat times 1.0 summed in fp32 with
+    zeros -- exactly its fp16 value.  Every such column is within 1 fp16 ulp
+    of the oracle's W_hat rounded to fp16 (the bar for reconstructed
+    weights), across all 256-row blocks and two radius groups."""
+    g = np.random.default_rng(300 + log2K)
+    d_out, d_in, M = 520, 256, 32
+    f = synth.random_fields(g, d_out, d_in, log2K)
+    f.perm = g.permutation(d_in).astype(np.int32)
+    chans = g.choice(d_in, M, replace=False)
+    x = np.zeros((M, d_in))
+    x[np.arange(M), chans] = 1.0
+    y, _, _ = gemv(f, synth.f16_bits(x), entry="gemm")
+    ref16 = oracle.round_half(oracle.dequant(f))  # [d_out][storage position]
+    pos = np.array([int(np.nonzero(f.perm == c)[0][0]) for c in chans])
+    got = y.astype(np.int32)                      # [M][d_out]
+    ref = ref16[:, pos].T.astype(np.int32)
+    same_sign = ((got ^ ref) & 0x8000) == 0
+    dist = np.where(same_sign, np.abs(got - ref), np.abs((got & 0x7FFF) + (ref & 0x7FFF)))
+    assert dist.max() <= 1, (log2K, int(dist.max()))
