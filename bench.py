@@ -513,15 +513,17 @@ def bench_gemm(stream):
 
 def bench_moe(stream, reps=20):
     """128 experts (gate/up 2048 -> 768, down 768 -> 2048), top-8 routing, T tokens; one
-    sage_moe_gemv call per projection, L2 flushed before each call by reading a buffer
-    twice its size (a read leaves clean lines: a write-based flush would leave the call
-    to write back ~126 MB of dirty lines)."""
+    sage_moe_gemv call per projection.  Two timings per point:
+      - `us`: calls back to back over four copies of the expert set (252 MB > L2), one
+        CUDA graph, as a stream of MoE layers runs (median/p10/p90 over 12 replays);
+      - `us_cold`: a single call after L2 is flushed by reading a buffer twice its size
+        (a read leaves clean lines: a write-based flush would leave the call to write
+        back ~126 MB of dirty lines), launch latency included."""
     import torch
     import synth
     import bit_vector_quantized_sage_b200 as sage
     hbm, _ = _peaks()
     flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
-    sink = torch.empty((), dtype=torch.float32, device="cuda")
     out = []
     for proj in (0, 2):
         packed = None
@@ -529,6 +531,7 @@ def bench_moe(stream, reps=20):
             spec = synth.config4(T)
             if packed is None:
                 packed = [sage.PackedMatrix.from_fields(spec.expert(e, proj)) for e in range(synth.MOE_EXPERTS)]
+                sets = [packed] + [[clone_matrix(m) for m in packed] for _ in range(3)]
             n_pairs = T * synth.MOE_TOPK
             pe = torch.from_numpy(spec.routes.reshape(-1).astype(np.int32)).cuda()
             if proj < 2:
@@ -540,11 +543,12 @@ def bench_moe(stream, reps=20):
             d_out = synth.MOE_PROJ[proj][1]
             y = torch.zeros((n_pairs, d_out), dtype=torch.int16, device="cuda")
             ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_MOE, packed, n_pairs))
-            fn = lambda st: sage.sage_moe_gemv(packed, pe, xr, n_pairs, x, y, ws, st)
-            for _ in range(3):
+            fns = [lambda st, E=E: sage.sage_moe_gemv(E, pe, xr, n_pairs, x, y, ws, st) for E in sets]
+            for fn in fns:
                 fn(stream)
-            g = capture(fn, stream)
-            t = []
+            t = per_call_us(fns, stream)
+            g = capture(fns[0], stream)
+            tc = []
             for _ in range(reps):
                 sink = flush.sum()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -552,18 +556,20 @@ def bench_moe(stream, reps=20):
                 g.replay()
                 e1.record(stream)
                 e1.synchronize()
-                t.append(e0.elapsed_time(e1) * 1e3)
-            del g
+                tc.append(e0.elapsed_time(e1) * 1e3)
+            del g, sink
             assert sage.sage_query_status(ws) == sage.SAGE_OK
             active = np.unique(spec.routes)
             nbytes = sum(packed[e].packed_bytes + (1 << packed[e].log2K) * 16 for e in active)
             nbytes += xb.nbytes + n_pairs * d_out * 2
             us = float(np.median(t))
             out.append({"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size), "us": dist_summary(t),
-                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4)})
+                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
+                        "us_cold": dist_summary(tc)})
+        del sets
     del flush
-    return {"workload": "128 experts, top-8, one projection per call (routing + grouped GEMV), L2 flushed "
-                        "(read) before each call", "points": out}
+    return {"workload": "128 experts, top-8, one projection per call (in-kernel routing + grouped GEMV)",
+            "points": out}
 
 
 def oracle_beside(pool_1):

@@ -35,7 +35,7 @@ using namespace dev;
 namespace {
 
 constexpr int kGW = 16;                       // decode warps: two per (slab column, record half)
-constexpr int kGThreads = (kGW + 2) * 32;     // + copy warp + MMA warp
+constexpr int kGThreads = (kGW + 3) * 32;     // + code copy warp + MMA warp + x_perm copy warp
 constexpr int kGDecodeThreads = kGW * 32;
 constexpr int kGOct = 32;                     // row octets per block
 constexpr int kGChunkJ = 16;                  // subvector columns per chunk (one radius group)
@@ -292,14 +292,21 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
                 bulk_g2s(dst, p.main + main_word(R8, S, blk, g * kGChunkJ, 0, 0), mb, sm.code_full(t));
                 bulk_g2s(dst + kGChunkJ * kGOct * 16, p.meta + 2 * meta_entry(R8, G, blk, g, 0, 0), tb,
                          sm.code_full(t));
-                for (int h = 0; h < 2; ++h) {
-                    const int s = 2 * t + h;
-                    if (s >= NB) gwait(sm.mma_done(s, NB), ((s / NB) - 1) & 1, p.status);
-                    mbar_arrive_expect_tx(sm.b_full(s, NB), sm.b_bytes);
-                    bulk_g2s(sm.b0 + (uint32_t)(s % NB) * sm.b_bytes, p.xt + (size_t)(2 * g + h) * p.n_pad * 8,
-                             sm.b_bytes, sm.b_full(s, NB));
-                }
             }
+        }
+    } else if (warp == kGW + 2) {
+        // ---------------- x_perm copy warp ----------------
+        // Its own warp, so that a slab's wait for its buffer (the MMAs of slab
+        // s - NB) never holds back the code copies, and the reverse.
+        if (lane == 0) {
+            for (int s = 0; s < n_slab; ++s) {
+                if (s >= NB) gwait(sm.mma_done(s, NB), ((s / NB) - 1) & 1, p.status);
+                mbar_arrive_expect_tx(sm.b_full(s, NB), sm.b_bytes);
+                bulk_g2s(sm.b0 + (uint32_t)(s % NB) * sm.b_bytes, p.xt + (size_t)(2 * g0 + s) * p.n_pad * 8,
+                         sm.b_bytes, sm.b_full(s, NB));
+            }
+            // no exit while copies are in flight: the MMAs of the last slabs consumed them
+            for (int s = max(0, n_slab - NB); s < n_slab; ++s) gwait(sm.b_full(s, NB), (s / NB) & 1, p.status);
         }
     } else if (warp == kGW + 1) {
         // ---------------- MMA warp: one thread issues the tensor-core work ----------------
@@ -336,6 +343,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
         const int cw = warp >> 3;
         const bool odd = tr & 1;
         const bool active = o < n_oct;
+        const int oc = active ? o : 0;  // a row octet that exists: inactive rows decode it and store zeros
         const uint32_t cbsel = sm.cb0 + ((uint32_t)tr << 4);
         const uint32_t s0 = odd ? d.sh3 : d.sh0, s1 = odd ? d.sh4 : d.sh1, s2 = odd ? d.sh5 : d.sh2;
         const uint32_t a_row = (uint32_t)(r >> 7) * kAHalf + (uint32_t)((r & 127) >> 3) * kASbo + (uint32_t)tr * 16;
@@ -361,16 +369,15 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
                 // which consume every result, stay in order before the arrival.
                 const uint32_t tok = order_token();
                 const uint32_t a_slab = sm.a0 + (uint32_t)(s % NA) * kASlab + a_row;
+                // No branch around each subvector: the four decodes form one
+                // straight-line block whose loads and arithmetic interleave.
                 uint4 v[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int jl = h * kGSlabJ + 4 * cw + i;  // chunk column
-                    v[i] = make_uint4(0, 0, 0, 0);
-                    if (active) {
-                        const uint32_t w =
-                            lds32_r(slot + tok + (uint32_t)(jl * n_oct + o) * 16 + (uint32_t)(tr >> 1) * 4);
-                        v[i] = decode_sv(d, w, odd, s0, s1, s2, aux, (uint32_t)(15 - jl), mp, dl, cbsel + tok);
-                    }
+                    const uint32_t w = lds32_r(slot + tok + (uint32_t)(jl * n_oct + oc) * 16 + (uint32_t)(tr >> 1) * 4);
+                    v[i] = decode_sv(d, w, odd, s0, s1, s2, aux, (uint32_t)(15 - jl), mp, dl, cbsel + tok);
+                    if (!active) v[i] = make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) sts128(a_slab + (uint32_t)(4 * cw + i) * 128, v[i]);

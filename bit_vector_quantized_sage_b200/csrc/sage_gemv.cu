@@ -71,6 +71,7 @@ constexpr int kXBufBytes = 8192;                // one activation window buffer
 constexpr int kMaxXW = 512;                     // window columns at batch 1
 constexpr int kPermBuf = kMaxXW * 32;           // the window's permutation entries
 constexpr int kMoeCache = 32;                   // virtual experts staged per CTA
+constexpr int kMaxMoeCtas = 256;                // CTAs of a MoE launch (one per SM)
 constexpr int kMaxPairsPerVirtual = 8;
 
 // Codebook replicas: codeword z of replica r at byte z*128 + r*16.  Static
@@ -86,7 +87,7 @@ __device__ __forceinline__ uint4 cw_load(uint32_t base, uint32_t off) { return l
 template <int M>
 struct Cfg {
     static constexpr int kXW = kXBufBytes / (16 * M);    // window columns
-    static constexpr int kSlots = M <= 2 ? kStashSlots : M <= 4 ? 2 : 1;  // stash ring depth
+    static constexpr int kSlots = M <= 2 ? kStashSlots : 2;  // stash ring depth
     static constexpr int kStash = kSlots * kParts * M * kBlockRows * 4;  // [slot][column part][m][row]
 };
 
@@ -107,12 +108,37 @@ struct JobView {
     int unit0, d_out, d_in, log2K, S, R8, blk0, Mk, id;
 };
 
+// Balanced split of `units` over n_cta CTAs: the first units % n_cta CTAs
+// take one unit more.  32-bit arithmetic only.
+__device__ __forceinline__ int cta_begin(int units, int n_cta, int c) {
+    const int q = units / n_cta, r = units - q * n_cta;
+    return q * c + min(c, r);
+}
+// The CTA whose range [cta_begin(c), cta_begin(c + 1)) holds unit u.
+__device__ __forceinline__ int cta_of(int units, int n_cta, int u) {
+    const int q = units / n_cta, r = units - q * n_cta;
+    const int big = (q + 1) * r;  // units held by the CTAs that take q + 1
+    return u < big ? u / (q + 1) : r + (u - big) / q;
+}
+
+// The same over a 64-bit total (the MoE cost space).
+__device__ __forceinline__ long long cta_begin64(long long total, int n_cta, int c) {
+    const long long q = total / n_cta, r = total - q * n_cta;
+    return q * c + min((long long)c, r);
+}
+
 struct DenseSrc {
     static constexpr bool kVarBatch = false;
     const EngineParams& p;
     __device__ int n_stages() const { return p.n_stages; }
     __device__ const EngineStage& stage(int s) const { return p.st[s]; }
     __device__ int units(int s) const { return p.st[s].units; }
+    // first unit of CTA c (c = n_cta: the end) and the CTA holding unit u
+    __device__ int cta_u0(int s, int n_cta, int c) const { return cta_begin(p.st[s].units, n_cta, c); }
+    __device__ int owner(int s, int n_cta, int u) const { return cta_of(p.st[s].units, n_cta, u); }
+    // every CTA of a dense launch holds units (at least 4 per CTA)
+    __device__ bool cta_nonempty(int, int, int) const { return true; }
+    __device__ int contributors(int, int, int c_first, int c_last) const { return c_last - c_first + 1; }
     __device__ JobView job_at(int s, int u) const {
         const EngineStage& st = p.st[s];
         int k = st.job0;
@@ -130,11 +156,20 @@ struct DenseSrc {
     }
 };
 
+// Decode batch width of a virtual expert with n pairs (1, 2, 4 or 8): the
+// cost weight of its units in the MoE split.
+__host__ __device__ constexpr int moe_weight(int n) { return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : 8; }
+
 // The MoE routing this CTA needs (virtual-expert ids, pair counts and row
 // lists of the virtual experts its range touches), built in shared memory by
 // the CTA at the start of the MoE kernel.
 struct MoeStage {
-    int n_virtual, units, vi0, nvi, overflow;
+    int n_virtual, units, vi0, nvi, overflow, n_e, upv;
+    long long cost_total;
+    int cnt[kMaxExperts];             // pairs per expert
+    int first[kMaxExperts + 1];       // first virtual expert of each expert; [n_e]: their number
+    long long cost[kMaxExperts + 1];  // first cost unit of each expert (exclusive prefix)
+    int bound[kMaxMoeCtas + 1];       // first unit of each CTA (cost-balanced); [n_cta]: the end
     int v_expert[kMoeCache];
     int v_count[kMoeCache];
     int v_xrows[kMoeCache][kMaxPairsPerVirtual];
@@ -148,7 +183,54 @@ struct MoeSrc {
     __device__ int n_stages() const { return 1; }
     __device__ const EngineStage& stage(int) const { return p.st; }
     __device__ int units(int) const { return ms.units; }
-    __device__ int upv() const { return ((((p.d_out + 7) >> 3) + kOct - 1) / kOct) * (p.d_in >> 3); }
+    __device__ int upv() const { return ms.upv; }
+    // CTA ranges are balanced over decode cost, not units: a unit of a virtual
+    // expert with n pairs costs moe_weight(n), the batch width its segments
+    // decode with (the decode time per column grows about linearly with it).
+    __device__ int cta_u0(int, int, int c) const { return ms.bound[c]; }
+    // The unit where CTA c's share of the cost starts (64-bit divisions: built
+    // once per launch into ms.bound, one CTA index per thread).
+    __device__ int cost_bound(int n_cta, int c) const {
+        const long long cp = cta_begin64(ms.cost_total, n_cta, c);
+        if (cp >= ms.cost_total) return ms.units;
+        int lo = 0, hi = ms.n_e - 1;  // the expert whose cost range holds cp
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (ms.cost[mid] <= cp) lo = mid; else hi = mid - 1;
+        }
+        const int e = lo, c_e = ms.cnt[e], full = c_e / kMaxPairsPerVirtual;
+        long long r = cp - ms.cost[e];
+        const long long full_cost = (long long)ms.upv * kMaxPairsPerVirtual;
+        int k, w;
+        if (r < full * full_cost) {
+            k = (int)(r / full_cost);
+            r -= k * full_cost;
+            w = kMaxPairsPerVirtual;
+        } else {
+            k = full;
+            r -= full * full_cost;
+            w = moe_weight(c_e - full * kMaxPairsPerVirtual);
+        }
+        // the first unit whose cost starts at or after cp
+        return (ms.first[e] + k) * ms.upv + (int)((r + w - 1) / w);
+    }
+    // A cost-balanced split can leave a CTA without units (a unit of an
+    // 8-pair virtual expert outweighs a CTA's share when there is little
+    // work); such CTAs take no part in any block.
+    __device__ bool cta_nonempty(int, int, int c) const { return ms.bound[c] < ms.bound[c + 1]; }
+    __device__ int contributors(int s, int n_cta, int c_first, int c_last) const {
+        int n = 0;
+        for (int c = c_first; c <= c_last; ++c) n += cta_nonempty(s, n_cta, c) ? 1 : 0;
+        return n;
+    }
+    __device__ int owner(int, int n_cta, int u) const {  // the last CTA whose range starts at or before u
+        int lo = 0, hi = n_cta - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (ms.bound[mid] <= u) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    }
     __device__ JobView job_at(int, int u) const { return job(u / upv()); }
     __device__ JobView job(int vi) const {
         const int k = vi - ms.vi0;  // always staged: a CTA only touches its own range
@@ -166,19 +248,6 @@ struct MoeSrc {
         return v;
     }
 };
-
-// Balanced split of `units` over n_cta CTAs: the first units % n_cta CTAs
-// take one unit more.  32-bit arithmetic only.
-__device__ __forceinline__ int cta_begin(int units, int n_cta, int c) {
-    const int q = units / n_cta, r = units - q * n_cta;
-    return q * c + min(c, r);
-}
-// The CTA whose range [cta_begin(c), cta_begin(c + 1)) holds unit u.
-__device__ __forceinline__ int cta_of(int units, int n_cta, int u) {
-    const int q = units / n_cta, r = units - q * n_cta;
-    const int big = (q + 1) * r;  // units held by the CTAs that take q + 1
-    return u < big ? u / (q + 1) : r + (u - big) / q;
-}
 
 // A segment: one job, one 256-row block, columns [ja, jb) of a CTA's range.
 struct Seg {
@@ -365,9 +434,9 @@ __device__ void copy_role(const Src& src, const Smem& sm, uint32_t* status, int 
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
         if (U <= 0) continue;
-        const int u1 = cta_begin(U, n_cta, blockIdx.x + 1);
+        const int u1 = src.cta_u0(s, n_cta, blockIdx.x + 1);
         int ts = 0;  // chunks of this stage issued so far
-        for (int u = cta_begin(U, n_cta, blockIdx.x); u < u1;) {
+        for (int u = src.cta_u0(s, n_cta, blockIdx.x); u < u1;) {
             const Seg g = make_seg(src, s, u, u1);
             u += g.jb - g.ja;
             if (g.v.cb != cur_cb) {
@@ -523,9 +592,67 @@ __device__ void rms_rows(const Smem& sm, const EngineStage& st, int tid, int nt,
 
 // Gathers the window's x_perm for items e = tid, tid + nt, ... of (batch row,
 // position) and stores them (fp16) into the window buffer.
+//
+// Plain inputs: a thread takes kGatherBatch items per round and issues all
+// their loads before it uses any, so a round costs one memory round trip,
+// not one per item (a window of 8 batch rows has 16 items per lane of a lone
+// gather warp).  The fused prologues gather a stage's first window with all
+// 288 gathering threads (one item each, typically) and keep one item per
+// round: their wider operand sets would not fit the registers left.
+constexpr int kGatherBatch = 2;
+
+template <int M, class Src>
+__device__ void gather_plain(const Src& src, const Smem& sm, int wlen, int xw, uint32_t xb, int tid, int nt) {
+    constexpr int U = kGatherBatch;
+    const int total = sm.misc[9] * wlen;  // batch rows a window holds (<= M) x positions
+    for (int e0 = tid; e0 < total; e0 += U * nt) {
+        uint32_t r[U][8];  // direct rows: r[u][0..3]; permuted: eight fp16 values
+        uint32_t dst[U];
+        bool zero[U], direct[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = e0 + u * nt;
+            const bool live = e < total;
+            const int ee = live ? e : e0;  // an item that exists: its loads are harmless
+            const int m = ee / wlen, p = ee - m * wlen;
+            const uint32_t info = sm.posinfo[p];
+            const JobView& v = sm.jc[info >> 20];
+            const int j = (int)(info & 0xfffffu);
+            dst[u] = live ? xb + (uint32_t)(m * xw + p) * 16 : 0xffffffffu;
+            zero[u] = m >= v.Mk;  // rows past a virtual expert's pairs
+            const int xr = zero[u] ? 0 : (v.xrows ? v.xrows[m] : m);
+            const uint16_t* row = v.x + (size_t)xr * v.d_in;
+            direct[u] = !v.perm;
+            if (direct[u]) {
+                const uint4 q = __ldca(reinterpret_cast<const uint4*>(row + j * 8));
+                r[u][0] = q.x; r[u][1] = q.y; r[u][2] = q.z; r[u][3] = q.w;
+            } else {
+                const uint4 pa = lds128(sm.perm0 + p * 32), pb = lds128(sm.perm0 + p * 32 + 16);
+                r[u][0] = ld16(row + (int)pa.x, true); r[u][1] = ld16(row + (int)pa.y, true);
+                r[u][2] = ld16(row + (int)pa.z, true); r[u][3] = ld16(row + (int)pa.w, true);
+                r[u][4] = ld16(row + (int)pb.x, true); r[u][5] = ld16(row + (int)pb.y, true);
+                r[u][6] = ld16(row + (int)pb.z, true); r[u][7] = ld16(row + (int)pb.w, true);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (dst[u] == 0xffffffffu) continue;
+            uint4 val = direct[u] ? make_uint4(r[u][0], r[u][1], r[u][2], r[u][3])
+                                  : make_uint4(r[u][0] | (r[u][1] << 16), r[u][2] | (r[u][3] << 16),
+                                               r[u][4] | (r[u][5] << 16), r[u][6] | (r[u][7] << 16));
+            if (zero[u]) val = make_uint4(0, 0, 0, 0);
+            sts128(dst[u], val);
+        }
+    }
+}
+
 template <int M, int PRO, class Src>
 __device__ void gather_items_k(const Src& src, const Smem& sm, int s, int wlen, int xw, uint32_t xb, int tid,
-                                   int nt, bool coh) {
+                               int nt, bool coh) {
+    if (PRO == kProPlain) {
+        gather_plain<M>(src, sm, wlen, xw, xb, tid, nt);
+        return;
+    }
     const EngineStage& st = *sm.stc;
     const int mrows = sm.misc[9];  // batch rows a window holds (<= M)
     for (int e = tid; e < mrows * wlen; e += nt) {
@@ -643,7 +770,7 @@ __device__ void gather_role(const Src& src, const Smem& sm, uint32_t* status, un
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
         if (U <= 0) continue;
-        const int u0 = cta_begin(U, n_cta, blockIdx.x), u1 = cta_begin(U, n_cta, blockIdx.x + 1);
+        const int u0 = src.cta_u0(s, n_cta, blockIdx.x), u1 = src.cta_u0(s, n_cta, blockIdx.x + 1);
         win_break(wp);
         if (u0 < u1) {  // the stage's descriptor, for this warp and the cooperative gather
             __syncwarp();
@@ -846,6 +973,54 @@ __device__ __forceinline__ void write_out_pre(const EngineStage& st, const JobVi
     st.eo[i] = f2h(h2f(rsum) + h2f(yb));
 }
 
+// The split-K combine of one block by its last contributor: every
+// contributor's fp32 partials added in CTA order (8 rows per lane, MKC batch
+// rows, 8 / MKC contributors' loads in flight at once), then the outputs.
+template <int MKC, int M, class Src>
+__device__ __forceinline__ void combine_block(const Src& src, const EngineParams& P, int s, const Seg& g, int c_first,
+                                              int c_last, int first_slot, int mk, int lane, bool pre,
+                                              const uint16_t (&rsum)[8][M <= 2 ? M : 1]) {
+    constexpr int NF = 8 / MKC;
+    constexpr int RM = M <= 2 ? M : 1;
+    float tot[8][MKC];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int m = 0; m < MKC; ++m) tot[i][m] = 0.f;
+    for (int c0 = c_first; c0 <= c_last; c0 += NF) {
+        float v[NF][8][MKC];
+#pragma unroll
+        for (int kk = 0; kk < NF; ++kk) {
+            const int c = c0 + kk;
+            const int sp = (c == c_first) ? first_slot : 0;
+            const bool has = c <= c_last && src.cta_nonempty(s, P.n_cta, c);
+            const float* src_p = P.partials + ((size_t)((s * P.n_cta + c) * 2 + sp) * 8) * kBlockRows + lane;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int m = 0; m < MKC; ++m)
+                    v[kk][i][m] = (has && m < mk) ? __ldcg(src_p + m * kBlockRows + 32 * i) : 0.f;
+        }
+#pragma unroll
+        for (int kk = 0; kk < NF; ++kk)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int m = 0; m < MKC; ++m) tot[i][m] += v[kk][i][m];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int row = g.blk * kBlockRows + lane + 32 * i;
+        if (row < g.v.d_out)
+#pragma unroll
+            for (int m = 0; m < MKC; ++m)
+                if (m < mk) {
+                    if (pre) write_out_pre(src.stage(s), g.v, m, row, tot[i][m], rsum[i][m < RM ? m : 0]);
+                    else write_out(src.stage(s), g.v, m, row, tot[i][m]);
+                }
+    }
+}
+
 // Epilogue warps: write (or combine) the outputs of the segments the decode
 // warps hand over through the stash ring, so that the decode warps never wait
 // on global-memory round trips; two warps take alternate segments, so one
@@ -867,7 +1042,7 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P, 
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
         if (U <= 0) continue;
-        const int u0 = cta_begin(U, P.n_cta, blockIdx.x), u1 = cta_begin(U, P.n_cta, blockIdx.x + 1);
+        const int u0 = src.cta_u0(s, P.n_cta, blockIdx.x), u1 = src.cta_u0(s, P.n_cta, blockIdx.x + 1);
         const bool signal = s + 1 < src.n_stages() && src.stage(s + 1).wait;
         unsigned done = 0;
         for (int uu = u0; uu < u1; ++n) {
@@ -934,56 +1109,29 @@ __device__ void epi_role(const Src& src, const Smem& sm, const EngineParams& P, 
                         if (m < mk) part[m * kBlockRows + r] = part_sum(m, r);
                 }
                 const int b0 = g.v.unit0 + g.blk * g.v.S;
-                const int c_first = cta_of(U, P.n_cta, b0), c_last = cta_of(U, P.n_cta, b0 + g.v.S - 1);
+                const int c_first = src.owner(s, P.n_cta, b0), c_last = src.owner(s, P.n_cta, b0 + g.v.S - 1);
                 unsigned* cnt = P.counters + src.stage(s).blk0 + g.v.blk0 + g.blk;
                 __syncwarp();  // the warp's partial stores precede the release below
                 int last = 0;
                 if (lane == 0) {
                     const unsigned old = atom_add_acq_rel_gpu(cnt, 1u);
-                    last = old == (unsigned)(c_last - c_first);
+                    last = old == (unsigned)(src.contributors(s, P.n_cta, c_first, c_last) - 1);
                     if (last) st_relaxed_gpu(cnt, 0u);  // restore for the next call
                 }
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {  // add the contributors' partials in CTA order, 8 rows per lane
-                    const int first_slot = (cta_begin(U, P.n_cta, c_first) >= b0) ? 0 : 1;
-                    float tot[8][M];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int m = 0; m < M; ++m) tot[i][m] = 0.f;
-                    // contributors whose loads are in flight at once (8 x M x NF values per lane)
-                    constexpr int NF = M == 1 ? 8 : M == 2 ? 4 : M <= 4 ? 2 : 1;
-                    for (int c0 = c_first; c0 <= c_last; c0 += NF) {
-                        float v[NF][8][M];
-#pragma unroll
-                        for (int kk = 0; kk < NF; ++kk) {
-                            const int c = c0 + kk;
-                            const int sp = (c == c_first) ? first_slot : 0;
-                            const float* src_p = P.partials + ((size_t)((s * P.n_cta + c) * 2 + sp) * 8) * kBlockRows + lane;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                                for (int m = 0; m < M; ++m)
-                                    v[kk][i][m] = (c <= c_last && m < mk) ? __ldcg(src_p + m * kBlockRows + 32 * i) : 0.f;
-                        }
-#pragma unroll
-                        for (int kk = 0; kk < NF; ++kk)
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                                for (int m = 0; m < M; ++m) tot[i][m] += v[kk][i][m];
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int row = g.blk * kBlockRows + lane + 32 * i;
-                        if (row < g.v.d_out)
-#pragma unroll
-                            for (int m = 0; m < M; ++m)
-                                if (m < mk) {
-                                    if (pre) write_out_pre(src.stage(s), g.v, m, row, tot[i][m], rsum[i][m < RM ? m : 0]);
-                                    else write_out(src.stage(s), g.v, m, row, tot[i][m]);
-                                }
-                    }
+                    const int first_slot = (src.cta_u0(s, P.n_cta, c_first) >= b0) ? 0 : 1;
+                    // batch width of the combine: the segment's own row count (MoE virtual
+                    // experts carry 1..8 pairs), so that narrow segments keep more
+                    // contributors' loads in flight
+                    if (mk <= 1)
+                        combine_block<1, M>(src, P, s, g, c_first, c_last, first_slot, mk, lane, pre, rsum);
+                    else if (mk <= 2)
+                        combine_block<(M < 2 ? M : 2), M>(src, P, s, g, c_first, c_last, first_slot, mk, lane, pre, rsum);
+                    else if (mk <= 4)
+                        combine_block<(M < 4 ? M : 4), M>(src, P, s, g, c_first, c_last, first_slot, mk, lane, pre, rsum);
+                    else
+                        combine_block<M, M>(src, P, s, g, c_first, c_last, first_slot, mk, lane, pre, rsum);
                     ++done;
                 }
             }
@@ -1002,7 +1150,6 @@ struct DecState {
     int t, slot, ph;      // chunk counter, its ring slot and phase parity
     WinPos wp;
     int cur_win;          // window the decode warps hold (-1: none)
-    bool first_win;       // the next window opened is a stage's first (cooperative gather)
 };
 
 // Decodes one segment with compile-time batch MK (<= M, the window's batch
@@ -1026,10 +1173,6 @@ __device__ __forceinline__ void seg_body(const Src& src, const Smem& sm, const E
             if (cur_win >= 0) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sm.x_empty(cur_win & 1));
-            }
-            if (ds.first_win) {
-                coop_window<M>(src, sm, s, wp.win, xw, src.stage(s).wait != 0, tid);
-                ds.first_win = false;
             }
             wait_bar(sm, sm.x_full(wp.win & 1), (wp.win >> 1) & 1, P.status);
             cur_win = wp.win;
@@ -1069,13 +1212,22 @@ __device__ void decode_role(const Src& src, const Smem& sm, const EngineParams& 
     const int tid = threadIdx.x;
     int ncb = 0, nseg = 0;
     const uint16_t* cur_cb = nullptr;
-    DecState ds{0, 0, 0, {0, 0}, -1, false};
+    DecState ds{0, 0, 0, {0, 0}, -1};
     for (int s = 0; s < src.n_stages(); ++s) {
         const int U = src.units(s);
         if (U <= 0) continue;
-        const int u0 = cta_begin(U, P.n_cta, blockIdx.x), u1 = cta_begin(U, P.n_cta, blockIdx.x + 1);
+        const int u0 = src.cta_u0(s, P.n_cta, blockIdx.x), u1 = src.cta_u0(s, P.n_cta, blockIdx.x + 1);
         win_break(ds.wp);
-        ds.first_win = true;
+        if (u0 < u1) {
+            // the stage's first window, gathered together with the gather warp
+            // here, where no decode state is live
+            if (ds.cur_win >= 0) {
+                __syncwarp();
+                if ((tid & 31) == 0) mbar_arrive(sm.x_empty(ds.cur_win & 1));
+                ds.cur_win = -1;
+            }
+            coop_window<M>(src, sm, s, ds.wp.win, xw, src.stage(s).wait != 0, tid);
+        }
         bool first_seg = true;
         for (int uu = u0; uu < u1; ++nseg) {
             const Seg g = make_seg(src, s, uu, u1);
@@ -1174,9 +1326,9 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(const __grid_consta
 __global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant__ MoeParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ MoeStage ms;
-    __shared__ int s_cnt[kMaxExperts];
-    __shared__ int s_first[kMaxExperts + 1];  // first virtual expert of expert e; [n_experts]: their number
     __shared__ int s_m2;
+    int* const s_cnt = ms.cnt;
+    int* const s_first = ms.first;
     constexpr int MV = kMaxPairsPerVirtual;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, n_e = p.n_experts;
     pdl_launch_dependents();
@@ -1189,27 +1341,48 @@ __global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant_
         else if (blockIdx.x == 0) flag(p.e.status, kDevUnsupported);  // that pair's output is not written
     }
     __syncthreads();
-    if (warp == 0) {  // exclusive scan of the virtual-expert counts, 32 experts at a time
+    const int upv = ((((p.d_out + 7) >> 3) + kOct - 1) / kOct) * (p.d_in >> 3);
+    if (warp == 0) {  // exclusive scans of the virtual-expert counts and costs, 32 experts at a time
         int carry = 0;
+        long long ccarry = 0;
         for (int e0 = 0; e0 < n_e; e0 += 32) {
             const int e = e0 + lane;
-            const int v = e < n_e ? (s_cnt[e] + MV - 1) / MV : 0;
+            const int c = e < n_e ? s_cnt[e] : 0, full = c / MV, tail = c - full * MV;
+            const int v = full + (tail > 0 ? 1 : 0);
+            const long long w = (long long)upv * (full * MV + (tail > 0 ? moe_weight(tail) : 0));
             int incl = v;
+            long long wincl = w;
             for (int o = 1; o < 32; o <<= 1) {
                 const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
+                const long long tw = __shfl_up_sync(0xffffffffu, wincl, o);
+                if (lane >= o) {
+                    incl += t;
+                    wincl += tw;
+                }
             }
-            if (e < n_e) s_first[e] = carry + incl - v;
+            if (e < n_e) {
+                s_first[e] = carry + incl - v;
+                ms.cost[e] = ccarry + wincl - w;
+            }
             carry += __shfl_sync(0xffffffffu, incl, 31);
+            ccarry += __shfl_sync(0xffffffffu, wincl, 31);
         }
-        if (lane == 0) s_first[n_e] = carry;
+        if (lane == 0) {
+            s_first[n_e] = carry;
+            ms.cost[n_e] = ccarry;
+            ms.cost_total = ccarry;
+            ms.n_e = n_e;
+            ms.upv = upv;
+            ms.n_virtual = carry;
+            ms.units = carry * upv;
+        }
     }
     __syncthreads();
-    const int upv = ((((p.d_out + 7) >> 3) + kOct - 1) / kOct) * (p.d_in >> 3);
+    const MoeSrc src{p, ms};
+    for (int c = tid; c <= p.e.n_cta; c += blockDim.x) ms.bound[c] = src.cost_bound(p.e.n_cta, c);
+    __syncthreads();
     if (tid == 0) {
-        ms.n_virtual = s_first[n_e];
-        ms.units = ms.n_virtual * upv;
-        const int u0 = cta_begin(ms.units, p.e.n_cta, blockIdx.x), u1 = cta_begin(ms.units, p.e.n_cta, blockIdx.x + 1);
+        const int u0 = src.cta_u0(0, p.e.n_cta, blockIdx.x), u1 = src.cta_u0(0, p.e.n_cta, blockIdx.x + 1);
         ms.vi0 = u0 / upv;
         const int need = u1 > u0 ? (u1 - 1) / upv - ms.vi0 + 1 : 0;
         ms.nvi = min(kMoeCache, need);
@@ -1254,7 +1427,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_kernel(const __grid_constant_
     }
     __syncthreads();
     if (ms.overflow) return;  // more virtual experts than the staging holds (flagged above)
-    const MoeSrc src{p, ms};
     run<kMaxPairsPerVirtual>(src, p.e, smem_raw, kXBufBytes / (16 * s_m2), s_m2, true);
 }
 
@@ -1442,9 +1614,9 @@ size_t moe_workspace_bytes(const sage_matrix* experts, int n_experts, int n_pair
 int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_expert, const int32_t* pair_xrow,
                int n_pairs, const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream) {
     constexpr int MV = kMaxPairsPerVirtual;
-    constexpr int kMoeStatic = (int)(sizeof(MoeStage) + (2 * kMaxExperts + 2) * sizeof(int));
+    constexpr int kMoeStatic = (int)(sizeof(MoeStage) + 16);
     if (n_experts > kMaxExperts) return SAGE_ERR_UNSUPPORTED;
-    const int n_cta = current_sm_count();
+    const int n_cta = std::min(current_sm_count(), kMaxMoeCtas);
     const MoeWs L = moe_ws_layout(n_pairs, experts[0].d_out, n_cta);
     if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
