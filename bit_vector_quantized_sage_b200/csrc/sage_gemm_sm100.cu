@@ -35,7 +35,7 @@ using namespace dev;
 namespace {
 
 constexpr int kGW = 16;                       // decode warps: two per (slab column, record half)
-constexpr int kGThreads = (kGW + 3) * 32;     // + code copy warp + MMA warp + x_perm copy warp
+constexpr int kGThreads = (kGW + 4) * 32;     // + code copy warp, two MMA warps, x_perm copy warp
 constexpr int kGDecodeThreads = kGW * 32;
 constexpr int kGOct = 32;                     // row octets per block
 constexpr int kGChunkJ = 16;                  // subvector columns per chunk (one radius group)
@@ -197,6 +197,10 @@ struct GemmSmem {
     __device__ uint64_t* b_full(int s, int nb) const { return bars + 2 * kGCodeSlots + 1 + (s % nb); }
     __device__ uint64_t* mma_done(int s, int nb) const { return bars + 2 * kGCodeSlots + 1 + 8 + (s % nb); }
     __device__ uint64_t* a_full(int s, int na) const { return bars + 2 * kGCodeSlots + 1 + 16 + (s % na); }
+    // the same by ring slot (the loops carry slot and phase instead of dividing)
+    __device__ uint64_t* b_full_at(int k) const { return bars + 2 * kGCodeSlots + 1 + k; }
+    __device__ uint64_t* mma_done_at(int k) const { return bars + 2 * kGCodeSlots + 1 + 8 + k; }
+    __device__ uint64_t* a_full_at(int k) const { return bars + 2 * kGCodeSlots + 1 + 16 + k; }
 };
 
 constexpr int kMaxASlots = 4;
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
         mbar_init(sm.cb_full(), 1);
         for (int k = 0; k < 8; ++k) {
             mbar_init(sm.bars + 2 * kGCodeSlots + 1 + k, 1);      // b_full
-            mbar_init(sm.bars + 2 * kGCodeSlots + 1 + 8 + k, 1);  // mma_done (tcgen05.commit)
+            mbar_init(sm.bars + 2 * kGCodeSlots + 1 + 8 + k, 2);  // mma_done: a commit from each MMA warp
         }
         for (int k = 0; k < kMaxASlots; ++k) mbar_init(sm.a_full(k, kMaxASlots), kGW);  // one arrival per decode warp
         fence_mbar_init();
@@ -299,34 +303,44 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
         // Its own warp, so that a slab's wait for its buffer (the MMAs of slab
         // s - NB) never holds back the code copies, and the reverse.
         if (lane == 0) {
+            int bs = 0, bph = 0;  // slab s's buffer slot and the parity of its fill
             for (int s = 0; s < n_slab; ++s) {
-                if (s >= NB) gwait(sm.mma_done(s, NB), ((s / NB) - 1) & 1, p.status);
-                mbar_arrive_expect_tx(sm.b_full(s, NB), sm.b_bytes);
-                bulk_g2s(sm.b0 + (uint32_t)(s % NB) * sm.b_bytes, p.xt + (size_t)(2 * g0 + s) * p.n_pad * 8,
-                         sm.b_bytes, sm.b_full(s, NB));
+                if (s >= NB) gwait(sm.mma_done_at(bs), bph ^ 1, p.status);  // the MMAs of slab s - NB
+                mbar_arrive_expect_tx(sm.b_full_at(bs), sm.b_bytes);
+                bulk_g2s(sm.b0 + (uint32_t)bs * sm.b_bytes, p.xt + (size_t)(2 * g0 + s) * p.n_pad * 8, sm.b_bytes,
+                         sm.b_full_at(bs));
+                if (++bs == NB) { bs = 0; bph ^= 1; }
             }
             // no exit while copies are in flight: the MMAs of the last slabs consumed them
             for (int s = max(0, n_slab - NB); s < n_slab; ++s) gwait(sm.b_full(s, NB), (s / NB) & 1, p.status);
         }
-    } else if (warp == kGW + 1) {
-        // ---------------- MMA warp: one thread issues the tensor-core work ----------------
+    } else if (warp == kGW + 1 || warp == kGW + 3) {
+        // ---------------- MMA warps: one thread each issues the tensor-core work ----------------
+        // of one 128-row half of the block (its own accumulator); the two warps
+        // sit on different schedulers and issue in parallel.
+        const int hf = warp == kGW + 1 ? 0 : 1;
         if (lane == 0) {
+            // This thread shares its scheduler with four busy decode warps, so
+            // its loop is kept short: ring slots and phases are carried, not
+            // divided out, and the operand descriptors are the slab base
+            // descriptor plus the tile's offset in 16-byte units (the address
+            // field cannot carry: shared addresses stay below 2^18).
             const uint32_t idesc = idesc_f16(p.n_pad);
+            const uint64_t a_desc0 = smem_desc(sm.a0, 128, kASbo), b_desc0 = smem_desc(sm.b0, 128, kBSbo);
+            int as = 0, aph = 0, bs = 0, bph = 0;
             for (int s = 0; s < n_slab; ++s) {
-                gwait(sm.a_full(s, NA), (s / NA) & 1, p.status);
-                gwait(sm.b_full(s, NB), (s / NB) & 1, p.status);
+                gwait(sm.a_full_at(as), aph, p.status);
+                gwait(sm.b_full_at(bs), bph, p.status);
                 tc_fence_after();
-                const uint32_t a_base = sm.a0 + (uint32_t)(s % NA) * kASlab;
-                const uint32_t b_base = sm.b0 + (uint32_t)(s % NB) * sm.b_bytes;
+                const uint64_t ad = a_desc0 + (uint64_t)((uint32_t)as * (kASlab >> 4));
+                const uint64_t bd = b_desc0 + (uint64_t)((uint32_t)bs * (sm.b_bytes >> 4));
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = smem_desc(b_base + kk * 256, 128, kBSbo);
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf)
-                        mma_f16(taddr + (uint32_t)(hf * p.n_alloc), smem_desc(a_base + hf * kAHalf + kk * 256, 128, kASbo),
-                                bd, idesc, (s > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(sm.mma_done(s, NB));
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_f16(taddr + (uint32_t)(hf * p.n_alloc), ad + (uint64_t)((hf * kAHalf + kk * 256) >> 4),
+                            bd + (uint64_t)((kk * 256) >> 4), idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(sm.mma_done_at(bs));
+                if (++as == NA) { as = 0; aph ^= 1; }
+                if (++bs == NB) { bs = 0; bph ^= 1; }
             }
         }
     } else {
@@ -347,6 +361,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
         const uint32_t cbsel = sm.cb0 + ((uint32_t)tr << 4);
         const uint32_t s0 = odd ? d.sh3 : d.sh0, s1 = odd ? d.sh4 : d.sh1, s2 = odd ? d.sh5 : d.sh2;
         const uint32_t a_row = (uint32_t)(r >> 7) * kAHalf + (uint32_t)((r & 127) >> 3) * kASbo + (uint32_t)tr * 16;
+        int as = 0;                  // slab s's A slot (s mod NA)
+        int ms = 0, mph = 0;         // slab s - NA's mma_done slot and parity (over NB)
         for (int t = 0; t < n_chunk; ++t) {
             gwait(sm.code_full(t), (t / kGCodeSlots) & 1, p.status);
             const uint32_t slot = sm.code0 + (uint32_t)(t % kGCodeSlots) * kGCodeSlot;
@@ -362,13 +378,16 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
             for (int h = 0; h < 2; ++h) {
                 const int s = 2 * t + h;
                 // the A buffer of slab s was last read by the MMAs of slab s - NA
-                if (s >= NA) gwait(sm.mma_done(s - NA, NB), ((s - NA) / NB) & 1, p.status);
+                if (s >= NA) {
+                    gwait(sm.mma_done_at(ms), mph, p.status);
+                    if (++ms == NB) { ms = 0; mph ^= 1; }
+                }
                 // The four subvectors' shared loads are independent: non-volatile
                 // loads whose addresses carry a token taken after the waits above
                 // (chunk resident, slab buffer free) let them overlap; the stores,
                 // which consume every result, stay in order before the arrival.
                 const uint32_t tok = order_token();
-                const uint32_t a_slab = sm.a0 + (uint32_t)(s % NA) * kASlab + a_row;
+                const uint32_t a_slab = sm.a0 + (uint32_t)as * kASlab + a_row;
                 // No branch around each subvector: the four decodes form one
                 // straight-line block whose loads and arithmetic interleave.
                 uint4 v[4];
@@ -383,7 +402,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_kernel(const __grid_constan
                 for (int i = 0; i < 4; ++i) sts128(a_slab + (uint32_t)(4 * cw + i) * 128, v[i]);
                 fence_proxy_async_smem();  // the generic-proxy writes above are read by the tensor core
                 __syncwarp();
-                if (lane == 0) mbar_arrive(sm.a_full(s, NA));
+                if (lane == 0) mbar_arrive(sm.a_full_at(as));
+                if (++as == NA) as = 0;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.code_empty(t));
