@@ -82,6 +82,14 @@ def lib():
             L.oracle_silu_mul.restype = None
             L.oracle_attend_one_position.argtypes = [i32, i32, i32, i32, P, P]
             L.oracle_attend_one_position.restype = None
+            L.oracle_qdq_angle.argtypes = [f64]
+            L.oracle_qdq_angle.restype = f64
+            L.oracle_softplus.argtypes = [f64]
+            L.oracle_softplus.restype = f64
+            L.oracle_codebook_from_angles.argtypes = [i32, P, P]
+            L.oracle_codebook_from_angles.restype = None
+            L.oracle_qdq_forward.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
+            L.oracle_qdq_forward.restype = i32
             _lib = L
     return _lib
 
@@ -301,3 +309,40 @@ def attend_one_position(v16: np.ndarray, n_heads: int, n_kv: int, hd: int) -> np
     out = np.zeros((v.shape[0], n_heads * hd), np.uint16)
     lib().oracle_attend_one_position(v.shape[0], n_heads, n_kv, hd, _p(v), _p(out))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Continuous-parameter decode (blockwise optimisation forward; Sec. 3.4,
+# App. A.6, Eqs. 12-14 and Eq. 2)
+# ---------------------------------------------------------------------------
+
+def qdq_angle(alpha: float) -> float:
+    """Eq. 13: theta = eps + (pi/2 - 2 eps) sigmoid(alpha), eps = 1e-4."""
+    return lib().oracle_qdq_angle(float(alpha))
+
+
+def softplus(rho: float) -> float:
+    return lib().oracle_softplus(float(rho))
+
+
+def codebook_from_angles(alpha) -> np.ndarray:
+    """Eq. 12: unit nonnegative codewords [K][8] from angle logits [K][7] (fp32 in)."""
+    alpha = _c(alpha, np.float32)
+    K = alpha.shape[0]
+    cb = np.zeros((K, 8), np.float64)
+    lib().oracle_codebook_from_angles(K, _p(alpha), _p(cb))
+    return cb
+
+
+def qdq_forward(d_out, d_in, log2K, alpha, rho, signs, idx):
+    """The forward pass: W [d_out][d_in] (fp64), q [d_out][d_in/8] and the
+    unrounded grid positions t = (r~ - mu) / delta [d_out][d_in/8]."""
+    S = d_in // 8
+    W = np.zeros((d_out, d_in), np.float64)
+    q = np.zeros((d_out, S), np.uint8)
+    t = np.zeros((d_out, S), np.float64)
+    rc = lib().oracle_qdq_forward(d_out, d_in, log2K, _p(_c(alpha, np.float32)), _p(_c(rho, np.float32)),
+                                  _p(_c(signs, np.uint8)), _p(_c(idx, np.uint16)), _p(W), _p(q), _p(t))
+    if rc:
+        raise ValueError("oracle_qdq_forward: unsupported shape")
+    return W, q, t

@@ -66,6 +66,16 @@ PLANTS = {
                   "        out[i] = oracle_double_to_half(t / (1.0 + exp(t)) * oracle_half_to_double(up[i]));"),
     "attend_head_map": ("                out[((size_t)m * n_heads + h) * hd + e] = v[((size_t)m * n_kv + h / grp) * hd + e];",
                         "                out[((size_t)m * n_heads + h) * hd + e] = v[((size_t)m * n_kv + h % n_kv) * hd + e];"),
+    "qdq_angle_no_eps": ("    return QDQ_EPS + (QDQ_HALF_PI - 2.0 * QDQ_EPS) / (1.0 + exp(-alpha));",
+                         "    return QDQ_HALF_PI / (1.0 + exp(-alpha));"),
+    "qdq_sine_product_off_by_one": ("            cb[(size_t)k * SV + i] = s * cos(t);\n            s *= sin(t);",
+                                    "            s *= sin(t);\n            cb[(size_t)k * SV + i] = s * cos(t);"),
+    "softplus_negative_branch": ("    return rho > 0.0 ? rho + log1p(exp(-rho)) : log1p(exp(rho));",
+                                 "    return rho > 0.0 ? rho + log1p(exp(-rho)) : log1p(exp(-rho));"),
+    "qdq_grid_step_2V": ("            const double delta = (hi - lo) / (double)((1 << V) - 1);",
+                         "            const double delta = (hi - lo) / (double)(1 << V);"),
+    "qdq_sign_component_reversed": ("                    W[(size_t)o * d_in + (size_t)j * SV + i] = (((s >> i) & 1) ? -rh : rh) * c[i];",
+                                    "                    W[(size_t)o * d_in + (size_t)j * SV + i] = (((s >> (SV - 1 - i)) & 1) ? -rh : rh) * c[i];"),
     "encode_grid_unweighted_radius": _UNWEIGHTED,
     "encode_quantize_unrounded_grid": _UNROUNDED,
 }

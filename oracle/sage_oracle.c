@@ -528,3 +528,88 @@ void oracle_attend_one_position(int M, int n_heads, int n_kv, int hd, const uint
             for (int e = 0; e < hd; ++e)
                 out[((size_t)m * n_heads + h) * hd + e] = v[((size_t)m * n_kv + h / grp) * hd + e];
 }
+
+/* ------------------------------------------------------------------ */
+/* Continuous-parameter decode for blockwise optimisation (Sec. 3.4,   */
+/* App. A.6; Eqs. 12-14 and Eq. 2): the forward pass that blockwise    */
+/* training evaluates, with the discrete assignments (signs, codeword  */
+/* indices) kept and the codebook and radii continuous.                */
+/* ------------------------------------------------------------------ */
+
+#define QDQ_EPS 1e-4
+#define QDQ_HALF_PI 1.57079632679489661923  /* pi / 2 */
+
+/* Eq. 13: theta = eps + (pi/2 - 2 eps) * sigmoid(alpha). */
+double oracle_qdq_angle(double alpha) {
+    return QDQ_EPS + (QDQ_HALF_PI - 2.0 * QDQ_EPS) / (1.0 + exp(-alpha));
+}
+
+/* Eq. 12: the unit codeword of v - 1 = 7 hyperspherical angles,
+ *   c_1 = cos t_1,  c_j = sin t_1 ... sin t_{j-1} cos t_j (j = 2..7),
+ *   c_8 = sin t_1 ... sin t_7;
+ * every angle lies in (0, pi/2), so every component is positive.
+ * alpha: [K][7] logits; cb: [K][8]. */
+void oracle_codebook_from_angles(int K, const float* alpha, double* cb) {
+    for (int k = 0; k < K; ++k) {
+        double s = 1.0;
+        for (int i = 0; i < SV - 1; ++i) {
+            const double t = oracle_qdq_angle((double)alpha[(size_t)k * (SV - 1) + i]);
+            cb[(size_t)k * SV + i] = s * cos(t);
+            s *= sin(t);
+        }
+        cb[(size_t)k * SV + SV - 1] = s;
+    }
+}
+
+/* r~ = softplus(rho) = log(1 + e^rho). */
+double oracle_softplus(double rho) {
+    return rho > 0.0 ? rho + log1p(exp(-rho)) : log1p(exp(rho));
+}
+
+/* The forward pass: per row group of 16 subvectors the grid spans the
+ * continuous radii (Eq. 14: mu = min r~, delta = (max r~ - min r~) /
+ * (2^V - 1), in full precision: the grid is recomputed from the current
+ * radii each step); q = clamp(floor((r~ - mu) / delta + 0.5), 0, 2^V - 1)
+ * (Eq. 2; delta = 0 gives q = 0, so a group of equal radii reconstructs
+ * their common value); r^ = mu + q delta; W[o][8j + i] = r^ s_i c_{z,i}
+ * (Eq. 1), storage column order.  t_out (optional): (r~ - mu) / delta of
+ * every subvector (0 where delta = 0), for checking rounding ties.
+ * Returns 1 for an unsupported shape. */
+int oracle_qdq_forward(int d_out, int d_in, int log2K, const float* alpha, const float* rho,
+                       const uint8_t* signs, const uint16_t* idx, double* W, uint8_t* q, double* t_out) {
+    if (d_out < 1 || d_in < 128 || d_in % 128 || log2K < 4 || log2K > 8) return 1;
+    const int K = 1 << log2K, V = 10 - log2K, S = d_in / SV, G = d_in / 128;
+    double* cb = (double*)malloc(sizeof(double) * (size_t)K * SV);
+    if (!cb) return 2;
+    oracle_codebook_from_angles(K, alpha, cb);
+    for (int o = 0; o < d_out; ++o) {
+        for (int g = 0; g < G; ++g) {
+            double r[GROUP_SV], lo = 0.0, hi = 0.0;
+            for (int t = 0; t < GROUP_SV; ++t) {
+                r[t] = oracle_softplus((double)rho[(size_t)o * S + g * GROUP_SV + t]);
+                if (t == 0 || r[t] < lo) lo = r[t];
+                if (t == 0 || r[t] > hi) hi = r[t];
+            }
+            const double delta = (hi - lo) / (double)((1 << V) - 1);
+            for (int t = 0; t < GROUP_SV; ++t) {
+                const int j = g * GROUP_SV + t;
+                double tt = 0.0, qq = 0.0;
+                if (delta > 0.0) {
+                    tt = (r[t] - lo) / delta;
+                    qq = floor(tt + 0.5);
+                    if (qq < 0.0) qq = 0.0;
+                    if (qq > (double)((1 << V) - 1)) qq = (double)((1 << V) - 1);
+                }
+                if (q) q[(size_t)o * S + j] = (uint8_t)qq;
+                if (t_out) t_out[(size_t)o * S + j] = tt;
+                const double rh = lo + qq * delta;
+                const uint8_t s = signs[(size_t)o * S + j];
+                const double* c = cb + (size_t)idx[(size_t)o * S + j] * SV;
+                for (int i = 0; i < SV; ++i)
+                    W[(size_t)o * d_in + (size_t)j * SV + i] = (((s >> i) & 1) ? -rh : rh) * c[i];
+            }
+        }
+    }
+    free(cb);
+    return 0;
+}

@@ -268,3 +268,32 @@ def config4(T: int) -> MoESpec:
     x = activations(gt, T, 2048)
     x_down = activations(gt, T * MOE_TOPK, 768)
     return MoESpec(T, routes, x, x_down, splits)
+
+
+@dataclass
+class QdqInputs:
+    """Training state of one matrix for the continuous-parameter decode: codebook
+    angle logits [K][7], radius logits [d_out][d_in/8] (r~ = softplus(rho)) and
+    the retained discrete assignments (signs, codeword indices)."""
+    d_out: int
+    d_in: int
+    log2K: int
+    alpha: np.ndarray
+    rho: np.ndarray
+    signs: np.ndarray
+    idx: np.ndarray
+
+
+def qdq_inputs(seed: int, d_out: int, d_in: int, log2K: int) -> QdqInputs:
+    """alpha ~ N(0, 1); rho ~ N(-2, 0.5), so that softplus(rho) ~ 0.13 with a
+    spread, about the radius of an 8-weight subvector of N(0, 0.02^2) weights
+    (0.02 x sqrt(8) = 0.057) to a few times it; Bernoulli(1/2) signs; uniform
+    codeword indices."""
+    g = rng(5, seed)
+    S = d_in // 8
+    K = 1 << log2K
+    return QdqInputs(d_out, d_in, log2K,
+                     g.standard_normal((K, 7)).astype(np.float32),
+                     (g.standard_normal((d_out, S)) * 0.5 - 2.0).astype(np.float32),
+                     g.integers(0, 256, (d_out, S), dtype=np.uint8),
+                     g.integers(0, K, (d_out, S)).astype(np.uint16))

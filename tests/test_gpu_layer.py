@@ -98,3 +98,60 @@ def test_qwen3_4b_layer_fused():
     spec = synth.config1()
     fields, inp, got, *_ = _run_layer(spec, synth.QWEN3_4B_HEADS, 1, config=1)
     _check_layer(fields, inp, got, synth.QWEN3_4B_HEADS)
+
+
+@pytest.mark.gpu
+def test_qwen3_4b_two_layers_chained_in_a_graph():
+    """The launch form the benchmark times, with a real dependency between
+    layers: two Qwen3-4B-shaped fused layers in one CUDA graph, the second
+    reading the first's h_out (programmatic dependent launch between them, one
+    workspace).  Every output is bit-identical to eager calls, and the second
+    layer is held to the bound against the oracle on the first layer's GPU
+    output."""
+    import types
+    import torch
+    heads = synth.QWEN3_4B_HEADS
+    nh, nkv, hd = heads
+    layers, fields_by_layer = [], []
+    inp = synth.decoder_inputs(1, 1, 2560)
+    ws = None
+    outs_all = []
+    for replica in (0, 1):
+        spec = synth.config1(1, replica)
+        mats, fields = {}, {}
+        for f in spec.mats:
+            f.perm = sage.sage_esg_permutation(spec.energies[f.name])
+            fields[f.name] = f
+            mats[f.name] = sage.PackedMatrix.from_fields(f)
+        outs = {n: torch.zeros((1, fields[n].d_out), dtype=torch.int16, device="cuda") for n in NAMES}
+        outs["h_out"] = torch.zeros((1, 2560), dtype=torch.int16, device="cuda")
+        lay = sage.DecoderLayer(mats, dev_u16(inp.attn_norm), dev_u16(inp.mlp_norm), nh, nkv, hd, inp.eps, outs, 1, ws)
+        ws = lay.ws
+        layers.append(lay)
+        fields_by_layer.append(fields)
+        outs_all.append(outs)
+    h0 = dev_u16(inp.h)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        layers[0](h0, s)
+        layers[1](outs_all[0]["h_out"], s)
+        s.synchronize()
+        eager = [{n: host_u16(t) for n, t in o.items()} for o in outs_all]
+        for o in outs_all:
+            for t in o.values():
+                t.zero_()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            layers[0](h0, torch.cuda.current_stream())
+            layers[1](outs_all[0]["h_out"], torch.cuda.current_stream())
+        for _ in range(2):
+            g.replay()
+    torch.cuda.synchronize()
+    assert sage.sage_query_status(ws) == sage.SAGE_OK
+    for o, e in zip(outs_all, eager):
+        for n, t in o.items():
+            assert np.array_equal(host_u16(t), e[n]), n
+    _check_layer(fields_by_layer[0], inp, eager[0], heads)
+    inp1 = types.SimpleNamespace(h=eager[0]["h_out"], attn_norm=inp.attn_norm, mlp_norm=inp.mlp_norm, eps=inp.eps)
+    _check_layer(fields_by_layer[1], inp1, eager[1], heads)
+    del g

@@ -667,3 +667,84 @@ def test_attention_over_one_position_returns_the_kv_value_rows():
     out = oracle.attend_one_position(v, n_heads, n_kv, hd)
     ref = np.repeat(v.reshape(3, n_kv, hd), n_heads // n_kv, axis=1).reshape(3, n_heads * hd)
     assert np.array_equal(out, ref)
+
+
+# ---------------------------------------------------------------------------
+# Continuous-parameter decode (Sec. 3.4, App. A.6, Eqs. 12-14, Eq. 2)
+# ---------------------------------------------------------------------------
+
+def test_codeword_angles_closed_form_at_zero_logits():
+    """alpha = 0 puts every angle at exactly pi/4 (Eq. 13), so Eq. 12 gives
+    c_j = 2^(-j/2) for j = 1..7 and c_8 = 2^(-7/2)."""
+    cb = oracle.codebook_from_angles(np.zeros((1, 7), np.float32))[0]
+    exp = np.array([2.0 ** (-j / 2) for j in range(1, 8)] + [2.0 ** -3.5])
+    assert np.allclose(cb, exp, rtol=0, atol=1e-15)
+
+
+def test_codeword_angles_unit_nonnegative_and_saturation():
+    """Every codeword is a nonnegative unit vector (the map's purpose).  Saturated
+    logits reach the boundaries kept eps = 1e-4 away: alpha -> -inf gives every
+    angle eps, so c = (cos eps, sin eps cos eps, ...); alpha -> +inf gives
+    pi/2 - eps, so the last component -> 1 and c_1 = sin eps."""
+    a = np.random.default_rng(3).standard_normal((64, 7)).astype(np.float32) * 3
+    cb = oracle.codebook_from_angles(a)
+    assert (cb > 0).all()
+    assert np.allclose(np.linalg.norm(cb, axis=1), 1.0, rtol=0, atol=1e-14)
+    eps = 1e-4
+    lo = oracle.codebook_from_angles(np.full((1, 7), -60.0, np.float32))[0]
+    assert np.isclose(lo[0], np.cos(eps), rtol=1e-12) and np.isclose(lo[1], np.sin(eps) * np.cos(eps), rtol=1e-9)
+    hi = oracle.codebook_from_angles(np.full((1, 7), 60.0, np.float32))[0]
+    assert np.isclose(hi[0], np.sin(eps), rtol=1e-9) and np.isclose(hi[7], np.cos(eps) ** 7, rtol=1e-9)
+
+
+def test_softplus_closed_forms():
+    assert oracle.softplus(0.0) == np.log(2.0)
+    assert np.isclose(oracle.softplus(40.0), 40.0, rtol=0, atol=1e-15)
+    assert np.isclose(oracle.softplus(-40.0), np.exp(-40.0), rtol=1e-12, atol=0)
+    assert np.isclose(oracle.softplus(1.0), np.log1p(np.e), rtol=1e-15)
+
+
+def _qdq(seed=0, d_out=5, d_in=256, log2K=5):
+    f = synth.qdq_inputs(seed, d_out, d_in, log2K)
+    return f, oracle.qdq_forward(d_out, d_in, log2K, f.alpha, f.rho, f.signs, f.idx)
+
+
+@pytest.mark.parametrize("log2K", [4, 6, 8])
+def test_qdq_grid_invariants(log2K):
+    """Per row group of 16 subvectors (Eq. 14, Eq. 2): the smallest fitted
+    radius sits on code 0 and the largest on the top code 2^V - 1; every
+    reconstructed radius is within half a grid step of its fitted radius; and
+    the subvector norm |w^| is the reconstructed radius (unit codewords)."""
+    f, (W, q, t) = _qdq(seed=log2K, log2K=log2K)
+    V = 10 - log2K
+    r = np.array([[oracle.softplus(v) for v in row] for row in f.rho.astype(np.float64)])
+    S = f.d_in // 8
+    for o in range(f.d_out):
+        for g in range(f.d_in // 128):
+            sl = slice(16 * g, 16 * g + 16)
+            rr, qq = r[o, sl], q[o, sl].astype(int)
+            assert qq[np.argmin(rr)] == 0 and qq[np.argmax(rr)] == (1 << V) - 1
+            mu, delta = rr.min(), (rr.max() - rr.min()) / ((1 << V) - 1)
+            rhat = mu + qq * delta
+            assert np.all(np.abs(rhat - rr) <= delta / 2 + 1e-15)
+            norms = np.linalg.norm(W[o].reshape(S, 8)[sl], axis=1)
+            assert np.allclose(norms, rhat, rtol=1e-13, atol=0)
+
+
+def test_qdq_equal_radii_and_signs():
+    """A group whose radii coincide reconstructs their common value (delta = 0,
+    q = 0); flipping one sign bit negates exactly that component."""
+    f = synth.qdq_inputs(11, 2, 128, 6)
+    f.rho[0, :] = -1.25
+    W, q, _ = oracle.qdq_forward(2, 128, 6, f.alpha, f.rho, f.signs, f.idx)
+    assert (q[0] == 0).all()
+    cb = oracle.codebook_from_angles(f.alpha)
+    r0 = oracle.softplus(-1.25)
+    for j in range(16):
+        s = np.where((f.signs[0, j] >> np.arange(8)) & 1, -1.0, 1.0)
+        assert np.allclose(W[0, 8 * j:8 * j + 8], r0 * s * cb[f.idx[0, j]], rtol=1e-15, atol=0)
+    s2 = f.signs.copy()
+    s2[1, 3] ^= 1 << 5
+    W2, _, _ = oracle.qdq_forward(2, 128, 6, f.alpha, f.rho, s2, f.idx)
+    d = W2 != W
+    assert d.sum() == 1 and d[1, 8 * 3 + 5] and W2[1, 29] == -W[1, 29]
