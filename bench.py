@@ -572,6 +572,33 @@ def bench_moe(stream, reps=20):
             "points": out}
 
 
+def bench_qdq(stream):
+    """The continuous-parameter decode (blockwise optimisation forward) of a
+    4096 x 4096 matrix at (K, V) = (64, 4): per subvector it reads rho, the
+    sign byte and the index (7 B) and writes 8 fp32 weights and the radius code
+    (33 B).  HBM-bound on those writes."""
+    import torch
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    f = synth.qdq_inputs(7, 4096, 4096, 6)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    alpha, rho, signs, idx = dev(f.alpha), dev(f.rho), dev(f.signs), dev(f.idx.view(np.int16))
+    Ws = [torch.empty((4096, 4096), dtype=torch.float32, device="cuda") for _ in range(3)]
+    q = torch.empty((4096, 512), dtype=torch.uint8, device="cuda")
+    fns = [lambda st, W=W: sage.sage_qdq_forward(4096, 4096, 6, alpha, rho, signs, idx, W, q, None, st) for W in Ws]
+    for fn in fns:
+        fn(stream)
+    t = per_call_us(fns, stream)
+    us = float(np.median(t))
+    nsv = 4096 * 512
+    nbytes = nsv * (4 + 1 + 2) + nsv * (32 + 1) + 64 * 7 * 4
+    hbm, _ = _peaks()
+    del Ws
+    return {"workload": "continuous-parameter decode (QDQ forward), 4096 x 4096, (K,V)=(64,4), fp32 W out",
+            "us": dist_summary(t), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+            "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4), "bytes_per_call": nbytes}
+
+
 def oracle_beside(pool_1):
     """The oracle on one core beside the up-projection and MoE workloads (GB/s of packed
     bytes on a sample: two 256-row blocks of the up-projection; the gate and down
@@ -740,6 +767,7 @@ def run_gpu(args):
         with torch.cuda.stream(stream):
             extra["up_proj_4096x12288_batch_sweep"] = bench_gemm(stream)
             extra["moe_128_experts"] = bench_moe(stream)
+            extra["qdq_forward_4096x4096"] = bench_qdq(stream)
 
     peak, peak_kind = _peaks()
     traffic, traffic_note = traffic_for(args.layer)

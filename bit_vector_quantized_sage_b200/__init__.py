@@ -36,6 +36,7 @@ EXPORTS = (
     "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
     "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
+    "sage_qdq_forward",
 )
 
 
@@ -97,6 +98,7 @@ def load(path: str = LIB_PATH):
         "sage_decoder_layer_workspace_size": ([C.POINTER(sage_decoder_layer), I, C.POINTER(SZ)], I),
         "sage_decoder_layer_forward": ([C.POINTER(sage_decoder_layer), P, I, C.POINTER(sage_decoder_outputs), P, SZ,
                                         P], I),
+        "sage_qdq_forward": ([I, I, I, P, P, P, P, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -314,6 +316,17 @@ def sage_moe_gemv(experts: Sequence[PackedMatrix], pair_expert, pair_xrow, n_pai
     arr = _mat_array(experts)
     _check("sage_moe_gemv", load().sage_moe_gemv(arr, len(experts), _ptr(pair_expert), _ptr(pair_xrow), n_pairs,
                                                  _ptr(x), _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def sage_qdq_forward(d_out: int, d_in: int, log2K: int, alpha, rho, signs, idx, W, q=None, codebook=None,
+                     stream=None):
+    """Continuous-parameter decode (blockwise optimisation forward): device
+    tensors alpha fp32 [K][7], rho fp32 [d_out][d_in/8], signs u8, idx int16/u16
+    [d_out][d_in/8]; W fp32 [d_out][d_in] out; q u8 and codebook fp32 [K][8]
+    optional outputs."""
+    _check("sage_qdq_forward", load().sage_qdq_forward(d_out, d_in, log2K, _ptr(alpha), _ptr(rho), _ptr(signs),
+                                                       _ptr(idx), _ptr(W), _ptr(q), _ptr(codebook),
+                                                       _stream(stream)))
 
 
 def sage_dequant(A: PackedMatrix, W, stream=None):

@@ -276,6 +276,36 @@ int sage_decoder_layer_workspace_size(const sage_decoder_layer* L, int M, size_t
 int sage_decoder_layer_forward(const sage_decoder_layer* L, const uint16_t* h, int M,
                                const sage_decoder_outputs* out, void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Continuous-parameter decode for blockwise optimisation: the forward pass
+ * of Sec. 3.4 and App. A.6.  Blockwise training keeps the discrete
+ * assignments (signs, codeword indices) and trains the codebook and the
+ * radii as continuous parameters:
+ *   - codeword k from 7 hyperspherical angles (Eq. 12):
+ *       c_1 = cos t_1, c_j = sin t_1 ... sin t_(j-1) cos t_j (j = 2..7),
+ *       c_8 = sin t_1 ... sin t_7, with t_i = eps + (pi/2 - 2 eps) *
+ *       sigmoid(alpha_ki), eps = 1e-4 (Eq. 13): unit and positive;
+ *   - radius r~ = softplus(rho);
+ *   - per row group of 16 subvectors the grid is recomputed from the current
+ *     radii, mu = min r~, delta = (max r~ - min r~) / (2^V - 1) (Eq. 14),
+ *     q = clamp(floor((r~ - mu) / delta + 0.5), 0, 2^V - 1) (Eq. 2; delta = 0
+ *     gives q = 0: a group of equal radii reconstructs their common value);
+ *   - W[o][8j + i] = (mu + q delta) s_i c_{z,i} (Eq. 1), storage column order.
+ * The straight-through estimator of the backward pass is the caller's: this is
+ * the forward only.  fp32 arithmetic throughout (the pages fix no precision
+ * for training).
+ *   alpha: device fp32 [K][7], K = 2^log2K (V = 10 - log2K);
+ *   rho: device fp32 [d_out][d_in/8]; signs: device u8 [d_out][d_in/8] (bit
+ *   i: component i negative); idx: device u16 [d_out][d_in/8];
+ *   W: device fp32 [d_out][d_in], 16-byte aligned (output);
+ *   q: device u8 [d_out][d_in/8] radius codes, or null;
+ *   codebook: device fp32 [K][8] unit codewords, or null.
+ * Errors: INVALID_ARGUMENT (null alpha, rho, signs, idx or W), UNSUPPORTED
+ * (d_in % 128, log2K outside 4..8), MISALIGNED (W), CUDA. */
+int sage_qdq_forward(int d_out, int d_in, int log2K, const float* alpha, const float* rho,
+                     const uint8_t* signs, const uint16_t* idx, float* W, uint8_t* q, float* codebook,
+                     sage_stream_t stream);
+
 /* Test hook: fp16 reconstruction W[d_out][d_in] (storage column order),
  * computed by the same device decode as the kernels (Eq. 1-2). */
 int sage_dequant(const sage_matrix* A, uint16_t* W, sage_stream_t stream);

@@ -187,3 +187,14 @@ def test_engine_rejects_unit_counts_beyond_int(lib, d_out, d_in):
     assert need.value >= blocks * 4
     rc = lib.sage_gemv(C.byref(A), 0x400000, 1, 0x500000, 0x10000000, 1 << 45, None)
     assert rc == sage.SAGE_ERR_UNSUPPORTED
+
+
+def test_qdq_forward_argument_errors(lib):
+    """Refused on the host before any launch (the pointers are never dereferenced)."""
+    a, r, s, i, w = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    assert lib.sage_qdq_forward(8, 128, 6, None, r, s, i, w, None, None, None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_qdq_forward(8, 128, 6, a, r, s, i, None, None, None, None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_qdq_forward(8, 100, 6, a, r, s, i, w, None, None, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_qdq_forward(8, 128, 3, a, r, s, i, w, None, None, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_qdq_forward(0, 128, 6, a, r, s, i, w, None, None, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_qdq_forward(8, 128, 6, a, r, s, i, w + 4, None, None, None) == sage.SAGE_ERR_MISALIGNED
