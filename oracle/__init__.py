@@ -90,6 +90,8 @@ def lib():
             L.oracle_codebook_from_angles.restype = None
             L.oracle_qdq_forward.argtypes = [i32, i32, i32, P, P, P, P, P, P, P]
             L.oracle_qdq_forward.restype = i32
+            L.oracle_abs_error.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P, P]
+            L.oracle_abs_error.restype = f64
             _lib = L
     return _lib
 
@@ -346,3 +348,27 @@ def qdq_forward(d_out, d_in, log2K, alpha, rho, signs, idx):
     if rc:
         raise ValueError("oracle_qdq_forward: unsupported shape")
     return W, q, t
+
+
+# ---------------------------------------------------------------------------
+# Adaptive bit splitting (Sec. 3.3, Eqs. 7-9)
+# ---------------------------------------------------------------------------
+
+def abs_error(f, W: np.ndarray, energy: np.ndarray) -> float:
+    """Eq. 8 for fields f against original weights W [d_out][d_in] (original channel
+    order) with channel energies e [d_in]."""
+    pp = _c(f.perm, np.int32) if f.perm is not None else None
+    e = lib().oracle_abs_error(f.d_out, f.d_in, f.log2K, _p(_c(f.signs, np.uint8)), _p(_c(f.idx, np.uint16)),
+                               _p(_c(f.q, np.uint8)), _p(_c(f.mu, np.uint16)), _p(_c(f.delta, np.uint16)),
+                               _p(_c(f.codebook, np.uint16)), _p(pp) if pp is not None else None,
+                               _p(_c(W, np.float64)), _p(_c(energy, np.float64)))
+    if e < 0:
+        raise ValueError("oracle_abs_error: unsupported shape or zero denominator")
+    return e
+
+
+def abs_select(candidates, W: np.ndarray, energy: np.ndarray):
+    """Eq. 9: the candidate encoding (one per (K, V) split) with the smallest Eq. 8
+    error; ties go to the earlier candidate.  Returns (index, errors)."""
+    errs = [abs_error(f, W, energy) for f in candidates]
+    return int(np.argmin(errs)), errs

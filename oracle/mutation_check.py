@@ -76,6 +76,10 @@ PLANTS = {
                          "            const double delta = (hi - lo) / (double)(1 << V);"),
     "qdq_sign_component_reversed": ("                    W[(size_t)o * d_in + (size_t)j * SV + i] = (((s >> i) & 1) ? -rh : rh) * c[i];",
                                     "                    W[(size_t)o * d_in + (size_t)j * SV + i] = (((s >> (SV - 1 - i)) & 1) ? -rh : rh) * c[i];"),
+    "abs_perm_direction": ("            const int c = perm ? perm[p] : p;\n            const double w = W[(size_t)o * d_in + c], d = w - Wh[(size_t)o * d_in + p];",
+                           "            const int c = perm ? perm[p] : p;\n            const double w = W[(size_t)o * d_in + p], d = w - Wh[(size_t)o * d_in + p];"),
+    "abs_energy_storage_order": ("            num += energy[c] * d * d;", "            num += energy[p] * d * d;"),
+    "abs_denominator_unweighted": ("            den += energy[c] * w * w;", "            den += w * w;"),
     "encode_grid_unweighted_radius": _UNWEIGHTED,
     "encode_quantize_unrounded_grid": _UNROUNDED,
 }

@@ -613,3 +613,33 @@ int oracle_qdq_forward(int d_out, int d_in, int log2K, const float* alpha, const
     free(cb);
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Adaptive bit splitting (Sec. 3.3, Eqs. 7-9).                        */
+/* ------------------------------------------------------------------ */
+
+/* Eq. 8: the energy-weighted relative reconstruction error of one encoded
+ * matrix in ORIGINAL channel order,
+ *   E = sum_c e_c ||W_:,c - W^_:,c||^2 / sum_c e_c ||W_:,c||^2,
+ * with W^ rebuilt from the fields (oracle_dequant, storage column order:
+ * storage column p holds original channel perm[p]; perm null = identity).
+ * W: [d_out][d_in] fp64, original column order; energy: [d_in].  Returns -1
+ * for an unsupported shape or a zero denominator. */
+double oracle_abs_error(int d_out, int d_in, int log2K, const uint8_t* signs, const uint16_t* idx,
+                        const uint8_t* q, const uint16_t* mu, const uint16_t* delta, const uint16_t* codebook,
+                        const int32_t* perm, const double* W, const double* energy) {
+    if (d_out < 1 || d_in < 128 || d_in % 128 || log2K < 4 || log2K > 8) return -1.0;
+    double* Wh = (double*)malloc(sizeof(double) * (size_t)d_out * d_in);
+    if (!Wh) return -1.0;
+    oracle_dequant(d_out, d_in, log2K, signs, idx, q, mu, delta, codebook, Wh);
+    double num = 0.0, den = 0.0;
+    for (int o = 0; o < d_out; ++o)
+        for (int p = 0; p < d_in; ++p) {
+            const int c = perm ? perm[p] : p;
+            const double w = W[(size_t)o * d_in + c], d = w - Wh[(size_t)o * d_in + p];
+            num += energy[c] * d * d;
+            den += energy[c] * w * w;
+        }
+    free(Wh);
+    return den > 0.0 ? num / den : -1.0;
+}

@@ -748,3 +748,60 @@ def test_qdq_equal_radii_and_signs():
     W2, _, _ = oracle.qdq_forward(2, 128, 6, f.alpha, f.rho, s2, f.idx)
     d = W2 != W
     assert d.sum() == 1 and d[1, 8 * 3 + 5] and W2[1, 29] == -W[1, 29]
+
+
+# ---------------------------------------------------------------------------
+# Adaptive bit splitting (Sec. 3.3, Eqs. 7-9)
+# ---------------------------------------------------------------------------
+
+def _abs_case(seed=0, d_out=24, d_in=256, log2K=5):
+    g = np.random.default_rng(seed)
+    f = synth.random_fields(g, d_out, d_in, log2K)
+    f.perm = g.permutation(d_in).astype(np.int32)
+    W = g.standard_normal((d_out, d_in)) * 0.1
+    e = synth.lognormal_energies(g, d_in, 1.5)
+    return f, W, e
+
+
+def test_abs_error_exact_and_empty_reconstructions():
+    """Eq. 8 is 0 when W is exactly the reconstruction (moved back to original
+    channel order through the permutation) and 1 when the reconstruction is
+    zero (all mu = delta = 0)."""
+    f, _, e = _abs_case(1)
+    Wh = oracle.dequant(f)                      # storage column order
+    W = np.zeros_like(Wh)
+    W[:, f.perm] = Wh                           # storage column p -> original channel perm[p]
+    assert oracle.abs_error(f, W, e) == 0.0
+    z = synth.Fields(f.d_out, f.d_in, f.log2K, f.signs, f.idx, f.q, np.zeros_like(f.mu), np.zeros_like(f.delta),
+                     f.codebook, f.perm)
+    assert oracle.abs_error(z, W + 0.5, e) == 1.0
+
+
+def test_abs_error_single_channel_and_scale_invariance():
+    """With all energy on one original channel c, Eq. 8 is that column's
+    relative error, where W^'s column for c is storage column perm^-1(c); and it
+    does not change when every energy is scaled by one constant."""
+    f, W, e = _abs_case(2)
+    Wh = oracle.dequant(f)
+    c = 77
+    p = int(np.nonzero(f.perm == c)[0][0])
+    one = np.zeros(f.d_in)
+    one[c] = 3.0
+    exp = np.sum((W[:, c] - Wh[:, p]) ** 2) / np.sum(W[:, c] ** 2)
+    assert np.isclose(oracle.abs_error(f, W, one), exp, rtol=1e-13)
+    assert np.isclose(oracle.abs_error(f, W, e * 7.25), oracle.abs_error(f, W, e), rtol=1e-13)
+
+
+def test_abs_select_picks_the_smallest_error():
+    """Eq. 9 over candidate encodings of the same W: the exact encoding wins (E = 0);
+    among equal errors the earlier candidate is kept."""
+    f, _, e = _abs_case(3)
+    Wh = oracle.dequant(f)
+    W = np.zeros_like(Wh)
+    W[:, f.perm] = Wh
+    g1, _, _ = _abs_case(4)
+    g2, _, _ = _abs_case(5)
+    best, errs = oracle.abs_select([g1, f, g2], W, e)
+    assert best == 1 and errs[1] == 0.0 and min(errs[0], errs[2]) > 0
+    best, errs = oracle.abs_select([g1, g1, f, f], W, e)
+    assert best == 2 and errs[0] == errs[1]
