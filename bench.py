@@ -599,6 +599,43 @@ def bench_qdq(stream):
             "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4), "bytes_per_call": nbytes}
 
 
+def bench_abs(stream, reps=10):
+    """Adaptive bit splitting on the weight-derived 4096 x 4096 layer: Eq. 8 of
+    each of the five split encodings (the library's CPU encoder, outside the
+    timing) against W, and the Eq. 9 choice.  Per candidate the score reads the
+    packed planes, the permutation, W (fp32, 64 MB) and the energies."""
+    import torch
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    packed = []
+    for log2K in (4, 5, 6, 7, 8):
+        inp, _ = synth.config2(d_out=4096, d_in=4096, n_samples=65536, iters=10, log2K=log2K)
+        r = sage.sage_encode(inp.W, inp.energies, log2K, inp.gamma, inp.sample, inp.init, inp.iters)
+        f = synth.Fields(4096, 4096, log2K, r["signs"], r["idx"], r["q"], r["mu"], r["delta"], r["codebook"],
+                         r["perm"], f"K=2^{log2K}")
+        packed.append(sage.PackedMatrix.from_fields(f))
+    W = torch.from_numpy(inp.W.astype(np.float32)).cuda()
+    e = torch.from_numpy(inp.energies.astype(np.float32)).cuda()
+    ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_ABS, packed[0], 1))
+    best, errs = sage.sage_abs_select(packed, W, e, ws, stream)
+    t = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        sage.sage_abs_select(packed, W, e, ws, stream)
+        e1.record(stream)
+        e1.synchronize()
+        t.append(e0.elapsed_time(e1) * 1e3 / 5)
+    us = float(np.median(t))
+    nbytes = packed[0].packed_bytes + 4096 * 4 + 4096 * 4096 * 4 + 4096 * 4
+    hbm, _ = _peaks()
+    return {"workload": "Eq. 8 score of the five split encodings of the weight-derived 4096 x 4096 layer, Eq. 9 choice",
+            "best_log2K": 4 + best, "errors": [round(x, 6) for x in errs],
+            "us_per_candidate": dist_summary(t), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+            "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
+            "note": "synchronous calls (each adds its CTAs' partial sums on the host)"}
+
+
 def oracle_beside(pool_1):
     """The oracle on one core beside the up-projection and MoE workloads (GB/s of packed
     bytes on a sample: two 256-row blocks of the up-projection; the gate and down
@@ -768,6 +805,7 @@ def run_gpu(args):
             extra["up_proj_4096x12288_batch_sweep"] = bench_gemm(stream)
             extra["moe_128_experts"] = bench_moe(stream)
             extra["qdq_forward_4096x4096"] = bench_qdq(stream)
+            extra["abs_select_4096x4096"] = bench_abs(stream)
 
     peak, peak_kind = _peaks()
     traffic, traffic_note = traffic_for(args.layer)

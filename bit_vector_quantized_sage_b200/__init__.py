@@ -28,7 +28,7 @@ SAGE_ERR_WORKSPACE = 4
 SAGE_ERR_CUDA = 5
 SAGE_ERR_TIMEOUT = 6
 
-SAGE_OP_GEMV, SAGE_OP_GEMM, SAGE_OP_MOE, SAGE_OP_GROUPED = 0, 1, 2, 3
+SAGE_OP_GEMV, SAGE_OP_GEMM, SAGE_OP_MOE, SAGE_OP_GROUPED, SAGE_OP_ABS = 0, 1, 2, 3, 4
 
 # Every extern "C" symbol declared in include/sage.h.
 EXPORTS = (
@@ -36,7 +36,7 @@ EXPORTS = (
     "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
     "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
-    "sage_qdq_forward",
+    "sage_qdq_forward", "sage_abs_error", "sage_abs_select",
 )
 
 
@@ -99,6 +99,8 @@ def load(path: str = LIB_PATH):
         "sage_decoder_layer_forward": ([C.POINTER(sage_decoder_layer), P, I, C.POINTER(sage_decoder_outputs), P, SZ,
                                         P], I),
         "sage_qdq_forward": ([I, I, I, P, P, P, P, P, P, P, P], I),
+        "sage_abs_error": ([MP, P, P, P, SZ, C.POINTER(C.c_double), P], I),
+        "sage_abs_select": ([MP, I, P, P, P, SZ, C.POINTER(I), P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -316,6 +318,26 @@ def sage_moe_gemv(experts: Sequence[PackedMatrix], pair_expert, pair_xrow, n_pai
     arr = _mat_array(experts)
     _check("sage_moe_gemv", load().sage_moe_gemv(arr, len(experts), _ptr(pair_expert), _ptr(pair_xrow), n_pairs,
                                                  _ptr(x), _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def sage_abs_error(A: PackedMatrix, W, energy, ws: Workspace, stream=None) -> float:
+    """Eq. 8 of packed matrix A against W (device fp32 [d_out][d_in], original
+    channel order) with device fp32 channel energies (synchronous)."""
+    d = A.desc()
+    e = C.c_double()
+    _check("sage_abs_error", load().sage_abs_error(C.byref(d), _ptr(W), _ptr(energy), ws.ptr, ws.nbytes, C.byref(e),
+                                                   _stream(stream)))
+    return e.value
+
+
+def sage_abs_select(cands: Sequence[PackedMatrix], W, energy, ws: Workspace, stream=None):
+    """Eq. 9 over candidate encodings of the same W: (index of the best, errors)."""
+    arr = _mat_array(cands)
+    best = C.c_int()
+    errs = (C.c_double * len(cands))()
+    _check("sage_abs_select", load().sage_abs_select(arr, len(cands), _ptr(W), _ptr(energy), ws.ptr, ws.nbytes,
+                                                     C.byref(best), errs, _stream(stream)))
+    return best.value, list(errs)
 
 
 def sage_qdq_forward(d_out: int, d_in: int, log2K: int, alpha, rho, signs, idx, W, q=None, codebook=None,

@@ -99,7 +99,7 @@ typedef struct {
 } sage_matrix;
 
 /* Operation selector for sage_workspace_size(). */
-enum { SAGE_OP_GEMV = 0, SAGE_OP_GEMM = 1, SAGE_OP_MOE = 2, SAGE_OP_GROUPED = 3 };
+enum { SAGE_OP_GEMV = 0, SAGE_OP_GEMM = 1, SAGE_OP_MOE = 2, SAGE_OP_GROUPED = 3, SAGE_OP_ABS = 4 };
 
 /* Human-readable name of a status code (static storage). */
 const char* sage_status_string(int status);
@@ -275,6 +275,31 @@ int sage_decoder_layer_workspace_size(const sage_decoder_layer* L, int M, size_t
  * sage_gemv (sage_query_status). */
 int sage_decoder_layer_forward(const sage_decoder_layer* L, const uint16_t* h, int M,
                                const sage_decoder_outputs* out, void* ws, size_t ws_bytes, sage_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Adaptive bit splitting (Sec. 3.3, Eqs. 7-9).  Each matrix chooses its
+ * (K, V) split among the 18-bit candidates by the energy-weighted relative
+ * reconstruction error in ORIGINAL channel order (Eq. 8),
+ *   E = sum_c e_c ||W_:,c - W^_:,c||^2 / sum_c e_c ||W_:,c||^2,
+ * where W^ is rebuilt from the packed codes (storage column p holds original
+ * channel perm[p]; no perm = identity) with r^ = mu + q delta in fp32 and the
+ * signed fp16 codeword, and sums are in fp64.
+ *   sage_abs_error: E of packed matrix A against W (device fp32
+ *     [d_out][d_in], original column order, 16-byte aligned) with channel
+ *     energies `energy` (device fp32 [d_in]); *err is a HOST double.
+ *     Synchronous: it waits for the stream and adds the CTAs' partial sums on
+ *     the host in a fixed order (deterministic).  ws: device workspace of
+ *     sage_workspace_size(SAGE_OP_ABS, ...) bytes.
+ *   sage_abs_select: Eq. 9, the index of the candidate encoding with the
+ *     smallest E (ties: the earlier candidate); cands: host array of n packed
+ *     encodings of the same W (one per split); errs: host double [n] or null.
+ * The encodings themselves come from sage_encode, one call per split.
+ * Errors: INVALID_ARGUMENT (null pointers, zero-energy W), UNSUPPORTED
+ * (candidates of different shapes), MISALIGNED, WORKSPACE, CUDA. */
+int sage_abs_error(const sage_matrix* A, const float* W, const float* energy, void* ws, size_t ws_bytes,
+                   double* err, sage_stream_t stream);
+int sage_abs_select(const sage_matrix* cands, int n, const float* W, const float* energy, void* ws,
+                    size_t ws_bytes, int* best, double* errs, sage_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Continuous-parameter decode for blockwise optimisation: the forward pass

@@ -198,3 +198,20 @@ def test_qdq_forward_argument_errors(lib):
     assert lib.sage_qdq_forward(8, 128, 3, a, r, s, i, w, None, None, None) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_qdq_forward(0, 128, 6, a, r, s, i, w, None, None, None) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_qdq_forward(8, 128, 6, a, r, s, i, w + 4, None, None, None) == sage.SAGE_ERR_MISALIGNED
+
+
+def test_abs_argument_errors(lib):
+    """Refused on the host before any launch (the pointers are never dereferenced)."""
+    A = sage.sage_matrix(64, 256, 6, 0x100000, 0x200000, 0x300000, None)
+    e = C.c_double()
+    need = C.c_size_t()
+    assert lib.sage_workspace_size(sage.SAGE_OP_ABS, C.byref(A), 1, 1, C.byref(need)) == sage.SAGE_OK
+    assert need.value >= 256 + 16
+    ws = 0x10000000
+    assert lib.sage_abs_error(C.byref(A), None, 0x500000, ws, need.value, C.byref(e), None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_abs_error(C.byref(A), 0x400000, 0x500000, None, need.value, C.byref(e), None) == sage.SAGE_ERR_WORKSPACE
+    assert lib.sage_abs_error(C.byref(A), 0x400004, 0x500000, ws, need.value, C.byref(e), None) == sage.SAGE_ERR_MISALIGNED
+    assert lib.sage_abs_error(C.byref(A), 0x400000, 0x500000, ws, 16, C.byref(e), None) == sage.SAGE_ERR_WORKSPACE
+    B = (sage.sage_matrix * 2)(A, sage.sage_matrix(64, 512, 6, 0x100000, 0x200000, 0x300000, None))
+    best = C.c_int()
+    assert lib.sage_abs_select(B, 2, 0x400000, 0x500000, ws, need.value, C.byref(best), None, None) == sage.SAGE_ERR_UNSUPPORTED
