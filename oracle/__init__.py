@@ -92,6 +92,8 @@ def lib():
             L.oracle_qdq_forward.restype = i32
             L.oracle_abs_error.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P, P]
             L.oracle_abs_error.restype = f64
+            L.oracle_encode_rows.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P, P]
+            L.oracle_encode_rows.restype = None
             _lib = L
     return _lib
 
@@ -372,3 +374,28 @@ def abs_select(candidates, W: np.ndarray, energy: np.ndarray):
     error; ties go to the earlier candidate.  Returns (index, errors)."""
     errs = [abs_error(f, W, energy) for f in candidates]
     return int(np.argmin(errs)), errs
+
+
+def omega_columns(energy: np.ndarray, perm: np.ndarray, gamma: float) -> np.ndarray:
+    """Eq. 4 weights per storage column: omega of subvector group j (storage
+    columns 8j .. 8j + 7, original channels perm[8j + i])."""
+    e = _c(energy, np.float64)
+    perm = np.asarray(perm)
+    out = np.zeros(e.size, np.float64)
+    for j in range(e.size // 8):
+        out[8 * j:8 * j + 8] = omega(e[perm[8 * j:8 * j + 8]], gamma)
+    return out
+
+
+def encode_rows(W: np.ndarray, perm: np.ndarray, omega_cols: np.ndarray, codebook: np.ndarray, log2K: int):
+    """The encoder's per-row part for a given stored codebook (fp16 bits [K][8]):
+    signs, Eq. 6 indices, Eq. 14 grid (fp16 bits), Eq. 2 codes."""
+    W = _c(W, np.float64)
+    d_out, d_in = W.shape
+    S, G = d_in // 8, d_in // 128
+    out = dict(signs=np.zeros((d_out, S), np.uint8), idx=np.zeros((d_out, S), np.uint16),
+               q=np.zeros((d_out, S), np.uint8), mu=np.zeros((d_out, G), np.uint16),
+               delta=np.zeros((d_out, G), np.uint16))
+    lib().oracle_encode_rows(d_out, d_in, log2K, _p(W), _p(_c(perm, np.int32)), _p(_c(omega_cols, np.float64)),
+                             _p(_c(codebook, np.uint16)), *[_p(out[k]) for k in ("signs", "idx", "q", "mu", "delta")])
+    return out

@@ -420,6 +420,40 @@ void oracle_kmeans(int n, const double* P, const double* Wt, int K, const int64_
  * codebook, Eq. 14 grid per group (fp16) and Eq. 2 radius codes.
  * W is d_out x d_in in original channel order; sample holds subvector ids
  * o * (d_in/8) + j; init holds positions into sample. */
+/* The per-row part of the encoder for a given stored codebook: signs, the
+ * Eq. 6 assignment of every subvector (storage column order through perm,
+ * omega per storage column), the Eq. 14 grid of every group of 16 and the
+ * Eq. 2 radius codes.  codebook: fp16 [K][8] as stored. */
+void oracle_encode_rows(int d_out, int d_in, int log2K, const double* W, const int32_t* perm,
+                        const double* omega, const uint16_t* codebook,
+                        uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu, uint16_t* delta) {
+    const int K = 1 << log2K, V = 10 - log2K, S = d_in / SV, G = d_in / 128;
+    double* cb = (double*)malloc(sizeof(double) * (size_t)K * SV);
+    for (int k = 0; k < K * SV; ++k) cb[k] = oracle_half_to_double(codebook[k]);
+    double rs[GROUP_SV];
+    for (int o = 0; o < d_out; ++o) {
+        for (int g = 0; g < G; ++g) {
+            for (int t = 0; t < GROUP_SV; ++t) {
+                const int j = g * GROUP_SV + t;
+                double p8[SV];
+                uint8_t s = 0;
+                for (int i = 0; i < SV; ++i) {
+                    const double w = W[(size_t)o * d_in + perm[j * SV + i]];
+                    p8[i] = fabs(w);
+                    if (w < 0.0) s |= (uint8_t)(1u << i);
+                }
+                signs[(size_t)o * S + j] = s;
+                idx[(size_t)o * S + j] = (uint16_t)oracle_assign(p8, omega + (size_t)j * SV, cb, K, &rs[t]);
+            }
+            oracle_grid(rs, V, &mu[(size_t)o * G + g], &delta[(size_t)o * G + g]);
+            for (int t = 0; t < GROUP_SV; ++t)
+                q[(size_t)o * S + g * GROUP_SV + t] =
+                    (uint8_t)oracle_quantize(rs[t], mu[(size_t)o * G + g], delta[(size_t)o * G + g], V);
+        }
+    }
+    free(cb);
+}
+
 int oracle_encode(int d_out, int d_in, int log2K, const double* W, const double* energy,
                   double gamma, int n_samples, const int64_t* sample, const int64_t* init, int iters,
                   int32_t* perm, uint16_t* codebook,
@@ -449,28 +483,8 @@ int oracle_encode(int d_out, int d_in, int log2K, const double* W, const double*
         codebook[k] = oracle_double_to_half(cb[k]);
         cb[k] = oracle_half_to_double(codebook[k]);
     }
-    double* rs = (double*)malloc(sizeof(double) * GROUP_SV);
-    for (int o = 0; o < d_out; ++o) {
-        for (int g = 0; g < G; ++g) {
-            for (int t = 0; t < GROUP_SV; ++t) {
-                const int j = g * GROUP_SV + t;
-                double p8[SV];
-                uint8_t s = 0;
-                for (int i = 0; i < SV; ++i) {
-                    const double w = W[(size_t)o * d_in + perm[j * SV + i]];
-                    p8[i] = fabs(w);
-                    if (w < 0.0) s |= (uint8_t)(1u << i);
-                }
-                signs[(size_t)o * S + j] = s;
-                idx[(size_t)o * S + j] = (uint16_t)oracle_assign(p8, omega + (size_t)j * SV, cb, K, &rs[t]);
-            }
-            oracle_grid(rs, V, &mu[(size_t)o * G + g], &delta[(size_t)o * G + g]);
-            for (int t = 0; t < GROUP_SV; ++t)
-                q[(size_t)o * S + g * GROUP_SV + t] =
-                    (uint8_t)oracle_quantize(rs[t], mu[(size_t)o * G + g], delta[(size_t)o * G + g], V);
-        }
-    }
-    free(omega); free(P); free(Wt); free(cb); free(rs);
+    oracle_encode_rows(d_out, d_in, log2K, W, perm, omega, codebook, signs, idx, q, mu, delta);
+    free(omega); free(P); free(Wt); free(cb);
     return 0;
 }
 

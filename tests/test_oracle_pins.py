@@ -805,3 +805,16 @@ def test_abs_select_picks_the_smallest_error():
     assert best == 1 and errs[1] == 0.0 and min(errs[0], errs[2]) > 0
     best, errs = oracle.abs_select([g1, g1, f, f], W, e)
     assert best == 2 and errs[0] == errs[1]
+
+
+def test_encode_rows_is_the_encoders_row_part():
+    """The per-row stage on its own (Eq. 6, Eq. 14, Eq. 2 for a given stored
+    codebook) reproduces the full encoder's fields exactly when given the
+    encoder's permutation, codebook and Eq. 4 weights."""
+    for log2K in (4, 6, 8):
+        inp, _ = synth.config2(d_out=96, d_in=256, n_samples=2048, iters=3, log2K=log2K)
+        ref = oracle.encode(inp)
+        om = oracle.omega_columns(inp.energies, ref["perm"], inp.gamma)
+        rows = oracle.encode_rows(inp.W, ref["perm"], om, ref["codebook"], log2K)
+        for k in rows:
+            assert np.array_equal(rows[k], ref[k]), (log2K, k)
