@@ -636,6 +636,37 @@ def bench_abs(stream, reps=10):
             "note": "synchronous calls (each adds its CTAs' partial sums on the host)"}
 
 
+def bench_encode_rows(stream, reps=10):
+    """The encoder's per-row stage (Eq. 6 over K codewords in fp64, Eq. 14, Eq. 2)
+    on the weight-derived 4096 x 4096 layer at (K, V) = (64, 4), with the CPU
+    encoder's codebook and permutation; the oracle's same stage on one host core
+    beside it."""
+    import torch
+    import oracle
+    import synth
+    import bit_vector_quantized_sage_b200 as sage
+    inp, _ = synth.config2()
+    r = sage.sage_encode(inp.W, inp.energies, inp.log2K, inp.gamma, inp.sample, inp.init, inp.iters)
+    om = oracle.omega_columns(inp.energies, r["perm"], inp.gamma)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    W, perm, omd, cb = dev(inp.W), dev(r["perm"].astype(np.int32)), dev(om), dev(r["codebook"].view(np.int16))
+    S, G = 512, 32
+    outs = [torch.empty((4096, S), dtype=torch.uint8, device="cuda"), torch.empty((4096, S), dtype=torch.int16, device="cuda"),
+            torch.empty((4096, S), dtype=torch.uint8, device="cuda"), torch.empty((4096, G), dtype=torch.int16, device="cuda"),
+            torch.empty((4096, G), dtype=torch.int16, device="cuda")]
+    fn = lambda st: sage.sage_encode_rows(4096, 4096, inp.log2K, W, perm, omd, cb, *outs, st)
+    fn(stream)
+    t = per_call_us([fn], stream)
+    t0 = time.perf_counter()
+    oracle.encode_rows(inp.W[:256], r["perm"], om, r["codebook"], inp.log2K)
+    cpu_s = (time.perf_counter() - t0) * 16  # 256 of 4096 rows
+    us = float(np.median(t))
+    return {"workload": "encoder row stage (Eq. 6 over 64 codewords in fp64, Eq. 14, Eq. 2), 4096 x 4096",
+            "us": dist_summary(t), "subvectors_per_s": round(4096 * 512 / (us * 1e-6) / 1e9, 3),
+            "unit": "G subvectors/s", "oracle_one_core_s_extrapolated": round(cpu_s, 3),
+            "oracle_sample": "rows 0-255, scaled by 16"}
+
+
 def oracle_beside(pool_1):
     """The oracle on one core beside the up-projection and MoE workloads (GB/s of packed
     bytes on a sample: two 256-row blocks of the up-projection; the gate and down
@@ -806,6 +837,7 @@ def run_gpu(args):
             extra["moe_128_experts"] = bench_moe(stream)
             extra["qdq_forward_4096x4096"] = bench_qdq(stream)
             extra["abs_select_4096x4096"] = bench_abs(stream)
+            extra["encode_rows_4096x4096"] = bench_encode_rows(stream)
 
     peak, peak_kind = _peaks()
     traffic, traffic_note = traffic_for(args.layer)

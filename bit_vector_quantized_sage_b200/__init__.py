@@ -36,7 +36,7 @@ EXPORTS = (
     "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
     "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
-    "sage_qdq_forward", "sage_abs_error", "sage_abs_select",
+    "sage_qdq_forward", "sage_abs_error", "sage_abs_select", "sage_encode_rows",
 )
 
 
@@ -101,6 +101,7 @@ def load(path: str = LIB_PATH):
         "sage_qdq_forward": ([I, I, I, P, P, P, P, P, P, P, P], I),
         "sage_abs_error": ([MP, P, P, P, SZ, C.POINTER(C.c_double), P], I),
         "sage_abs_select": ([MP, I, P, P, P, SZ, C.POINTER(I), P, P], I),
+        "sage_encode_rows": ([I, I, I, P, P, P, P, P, P, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -318,6 +319,16 @@ def sage_moe_gemv(experts: Sequence[PackedMatrix], pair_expert, pair_xrow, n_pai
     arr = _mat_array(experts)
     _check("sage_moe_gemv", load().sage_moe_gemv(arr, len(experts), _ptr(pair_expert), _ptr(pair_xrow), n_pairs,
                                                  _ptr(x), _ptr(y), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def sage_encode_rows(d_out: int, d_in: int, log2K: int, W, perm, omega, codebook, signs, idx, q, mu, delta,
+                     stream=None):
+    """The encoder's per-row stage on the GPU (device tensors: W fp64, perm int32, omega
+    fp64 per storage column, codebook fp16 bits; outputs signs u8, idx int16/u16,
+    q u8, mu/delta fp16 bits)."""
+    _check("sage_encode_rows", load().sage_encode_rows(d_out, d_in, log2K, _ptr(W), _ptr(perm), _ptr(omega),
+                                                       _ptr(codebook), _ptr(signs), _ptr(idx), _ptr(q), _ptr(mu),
+                                                       _ptr(delta), _stream(stream)))
 
 
 def sage_abs_error(A: PackedMatrix, W, energy, ws: Workspace, stream=None) -> float:

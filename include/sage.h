@@ -277,6 +277,33 @@ int sage_decoder_layer_forward(const sage_decoder_layer* L, const uint16_t* h, i
                                const sage_decoder_outputs* out, void* ws, size_t ws_bytes, sage_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The encoder's per-row stage on the GPU (Sec. 3.1-3.2): for a given stored
+ * codebook, every subvector's signs, its Eq. 6 direction
+ *   z = argmax_k (sum_i w_i p_i c_ki)^2 / sum_i w_i c_ki^2,  p = |W subvector|,
+ * (ties to the smallest k; an all-zero score gives z = 0, r* = 0) with fitted
+ * radius r* = sum w p c / sum w c^2, the Eq. 14 grid of every row group of 16
+ * (mu = min r*, delta = (max r* - min r*) / (2^V - 1), both rounded to fp16,
+ * nearest even) and the Eq. 2 codes q = clamp(floor((r* - mu) / delta + 0.5),
+ * 0, 2^V - 1) against the stored grid (delta = 0: q = 0).  fp64 with every
+ * product, sum and quotient rounded separately, in the CPU encoder's order:
+ * the fields equal sage_encode's bit for bit for the same codebook,
+ * permutation and weights.
+ *   W: device fp64 [d_out][d_in], original column order;
+ *   perm: device int32 [d_in] (storage column p holds original channel
+ *     perm[p], e.g. sage_esg_permutation's);
+ *   omega: device fp64 [d_in], the Eq. 4 weight of each storage column
+ *     (omega of subvector group j over storage columns 8j .. 8j + 7);
+ *   codebook: device fp16 [K][8], K = 2^log2K (the stored codebook);
+ *   signs, idx, q: device u8 / u16 / u8 [d_out][d_in/8]; mu, delta: device
+ *     fp16 [d_out][d_in/128] (outputs).
+ * The codebook itself (weighted spherical k-means on sampled subvectors) is
+ * sage_encode's.  Errors: INVALID_ARGUMENT (null), UNSUPPORTED (d_in % 128,
+ * log2K outside 4..8), CUDA. */
+int sage_encode_rows(int d_out, int d_in, int log2K, const double* W, const int32_t* perm, const double* omega,
+                     const uint16_t* codebook, uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu,
+                     uint16_t* delta, sage_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Adaptive bit splitting (Sec. 3.3, Eqs. 7-9).  Each matrix chooses its
  * (K, V) split among the 18-bit candidates by the energy-weighted relative
  * reconstruction error in ORIGINAL channel order (Eq. 8),

@@ -215,3 +215,10 @@ def test_abs_argument_errors(lib):
     B = (sage.sage_matrix * 2)(A, sage.sage_matrix(64, 512, 6, 0x100000, 0x200000, 0x300000, None))
     best = C.c_int()
     assert lib.sage_abs_select(B, 2, 0x400000, 0x500000, ws, need.value, C.byref(best), None, None) == sage.SAGE_ERR_UNSUPPORTED
+
+
+def test_encode_rows_argument_errors(lib):
+    a = [0x100000 * (i + 1) for i in range(10)]
+    assert lib.sage_encode_rows(8, 128, 6, None, *a[1:10], None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_encode_rows(8, 100, 6, *a, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_encode_rows(8, 128, 9, *a, None) == sage.SAGE_ERR_UNSUPPORTED
