@@ -1,16 +1,16 @@
 #!/usr/bin/env python
 """Benchmark: batch-1 packed SAGE GEMV over a Qwen3-4B-shaped decoder layer on B200.
 
-A step is the packed GEMV work of one decoder layer at batch 1: its seven
-projections (q, k, v, o, gate, up, down; hidden 2560) computed straight from
-2.25-bit codes in ONE launch of the libsage engine (sage_gemv_grouped over the
-seven matrices, each with its own synthetic fp16 input row).  Every step reads
-a different copy of the layer's packed planes, so the working set (> 4 x the
-126 MB L2) comes from HBM.  Reported alongside (under "extra"): the same layer
-as its four dependent stages in one launch with the operations between them
-fused (sage_decoder_layer_forward), the four stages as four launches, the
-4096 -> 12288 batch sweep through the GEMV and tcgen05 paths, and the
-grouped-expert MoE GEMV.
+A step is one Qwen3-4B-shaped decoder layer at batch 1 (hidden 2560): its
+seven projections (q, k, v, o, gate, up, down) computed straight from 2.25-bit
+codes, with the operations between them fused (RMSNorm, attention over one
+cached position, residual adds, SiLU * up), in ONE launch of the libsage engine
+(sage_decoder_layer_forward).  Every step reads a different copy of the layer's
+packed planes, so the working set (> 4 x the 126 MB L2) comes from HBM.
+Reported alongside (under "extra"): the seven projections as one grouped launch
+with independent inputs, the four dependency stages as four launches, the
+4096 -> 12288 batch sweep through the GEMV and tcgen05 paths, the grouped-expert
+MoE GEMV, and the encoder / blockwise-optimisation kernels.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -661,10 +661,32 @@ def bench_encode_rows(stream, reps=10):
     oracle.encode_rows(inp.W[:256], r["perm"], om, r["codebook"], inp.log2K)
     cpu_s = (time.perf_counter() - t0) * 16  # 256 of 4096 rows
     us = float(np.median(t))
+    # the weighted spherical k-means on the same layer's 65,536 samples
+    S_ = inp.W.shape[1] // 8
+    o_, j_ = inp.sample // S_, inp.sample % S_
+    P = np.ascontiguousarray(np.abs(inp.W[o_[:, None], r["perm"].reshape(S_, 8)[j_]]))
+    Wt = np.ascontiguousarray(om.reshape(S_, 8)[j_])
+    Pd, Wd, initd = dev(P), dev(Wt), dev(inp.init)
+    sage.sage_kmeans(Pd, Wd, inp.log2K, initd, inp.iters, stream)
+    km = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        sage.sage_kmeans(Pd, Wd, inp.log2K, initd, inp.iters, stream)
+        b.record(stream)
+        b.synchronize()
+        km.append(a.elapsed_time(b) * 1e3)
+    t0 = time.perf_counter()
+    oracle.kmeans(P, Wt, 1 << inp.log2K, inp.init, 1)
+    km_cpu_s = (time.perf_counter() - t0) * inp.iters  # one round, scaled by the rounds
     return {"workload": "encoder row stage (Eq. 6 over 64 codewords in fp64, Eq. 14, Eq. 2), 4096 x 4096",
             "us": dist_summary(t), "subvectors_per_s": round(4096 * 512 / (us * 1e-6) / 1e9, 3),
             "unit": "G subvectors/s", "oracle_one_core_s_extrapolated": round(cpu_s, 3),
-            "oracle_sample": "rows 0-255, scaled by 16"}
+            "oracle_sample": "rows 0-255, scaled by 16",
+            "kmeans": {"workload": f"weighted spherical k-means, {len(inp.sample)} samples, K = {1 << inp.log2K}, "
+                                   f"{inp.iters} rounds (synchronous call)",
+                       "us": dist_summary(km), "oracle_one_core_s_extrapolated": round(km_cpu_s, 3),
+                       "oracle_sample": f"one round, scaled by {inp.iters}"}}
 
 
 def oracle_beside(pool_1):

@@ -36,7 +36,8 @@ EXPORTS = (
     "sage_esg_permutation", "sage_encode", "sage_workspace_size", "sage_gemv", "sage_gemv_grouped",
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
     "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
-    "sage_qdq_forward", "sage_abs_error", "sage_abs_select", "sage_encode_rows",
+    "sage_qdq_forward", "sage_abs_error", "sage_abs_select", "sage_encode_rows", "sage_kmeans_workspace_size",
+    "sage_kmeans",
 )
 
 
@@ -102,6 +103,8 @@ def load(path: str = LIB_PATH):
         "sage_abs_error": ([MP, P, P, P, SZ, C.POINTER(C.c_double), P], I),
         "sage_abs_select": ([MP, I, P, P, P, SZ, C.POINTER(I), P, P], I),
         "sage_encode_rows": ([I, I, I, P, P, P, P, P, P, P, P, P, P], I),
+        "sage_kmeans_workspace_size": ([I], C.c_size_t),
+        "sage_kmeans": ([I, I, P, P, P, I, P, P, P, C.c_size_t, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -329,6 +332,20 @@ def sage_encode_rows(d_out: int, d_in: int, log2K: int, W, perm, omega, codebook
     _check("sage_encode_rows", load().sage_encode_rows(d_out, d_in, log2K, _ptr(W), _ptr(perm), _ptr(omega),
                                                        _ptr(codebook), _ptr(signs), _ptr(idx), _ptr(q), _ptr(mu),
                                                        _ptr(delta), _stream(stream)))
+
+
+def sage_kmeans(P, Wt, log2K: int, init, iters: int, stream=None):
+    """Weighted spherical k-means on the GPU (device tensors: P, Wt fp64 [n][8],
+    init int64 [K]) -> (codebook fp64 [K][8], codebook fp16 bits [K][8]) on the device."""
+    import torch
+    n = int(P.shape[0])
+    K = 1 << log2K
+    cb = torch.empty((K, 8), dtype=torch.float64, device=P.device)
+    cb16 = torch.empty((K, 8), dtype=torch.int16, device=P.device)
+    ws = Workspace(load().sage_kmeans_workspace_size(n))
+    _check("sage_kmeans", load().sage_kmeans(n, log2K, _ptr(P), _ptr(Wt), _ptr(init), iters, _ptr(cb), _ptr(cb16),
+                                             ws.ptr, ws.nbytes, _stream(stream)))
+    return cb, cb16
 
 
 def sage_abs_error(A: PackedMatrix, W, energy, ws: Workspace, stream=None) -> float:

@@ -296,12 +296,38 @@ int sage_decoder_layer_forward(const sage_decoder_layer* L, const uint16_t* h, i
  *   codebook: device fp16 [K][8], K = 2^log2K (the stored codebook);
  *   signs, idx, q: device u8 / u16 / u8 [d_out][d_in/8]; mu, delta: device
  *     fp16 [d_out][d_in/128] (outputs).
- * The codebook itself (weighted spherical k-means on sampled subvectors) is
- * sage_encode's.  Errors: INVALID_ARGUMENT (null), UNSUPPORTED (d_in % 128,
- * log2K outside 4..8), CUDA. */
+ * The codebook itself comes from sage_kmeans (GPU) or sage_encode (CPU).
+ * Errors: INVALID_ARGUMENT (null), UNSUPPORTED (d_in % 128, log2K outside
+ * 4..8), CUDA. */
 int sage_encode_rows(int d_out, int d_in, int log2K, const double* W, const int32_t* perm, const double* omega,
                      const uint16_t* codebook, uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu,
                      uint16_t* delta, sage_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The encoder's weighted spherical k-means on the GPU (Sec. 3.2 "Weighted
+ * Quantizer Fitting"; Sec. 4.1 sets 65,536 sampled subvectors): K = 2^log2K
+ * unit codewords start as the unit directions of the samples init[0..K)
+ * (an all-zero sample gives the direction 1/sqrt(8) in every component);
+ * each of `iters` rounds assigns every sample by Eq. 6 (as sage_encode_rows,
+ * against the fp64 codewords) and moves each codeword to the normalised sum
+ * of its members' w * p / |p| (members in sample order; all-zero samples add
+ * nothing; an empty cluster keeps its codeword).  fp64 with every operation
+ * rounded separately, in the CPU encoder's order: the codebook equals
+ * sage_encode's k-means bit for bit on the same samples.
+ *   P, Wt: device fp64 [n][8]: the sampled subvectors' magnitudes |W| in
+ *     storage column order and their Eq. 4 weights;
+ *   init: device int64 [K], positions into the n samples;
+ *   cb: device fp64 [K][8] (output); cb16: device fp16 [K][8], the codebook
+ *     rounded to nearest even (output; may be null);
+ *   ws: device memory of sage_kmeans_workspace_size(n) bytes, 16-byte aligned,
+ *     owned by the caller, not shared with a concurrent call.
+ * Synchronous: returns after the stream has finished the work.  Errors:
+ * INVALID_ARGUMENT (null pointer; an init entry outside [0, n), found on the
+ * device -- the codebook is then undefined), UNSUPPORTED (n < 1, iters < 0,
+ * log2K outside 4..8), MISALIGNED, WORKSPACE, CUDA. */
+size_t sage_kmeans_workspace_size(int n);
+int sage_kmeans(int n, int log2K, const double* P, const double* Wt, const int64_t* init, int iters, double* cb,
+                uint16_t* cb16, void* ws, size_t ws_bytes, sage_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Adaptive bit splitting (Sec. 3.3, Eqs. 7-9).  Each matrix chooses its

@@ -222,3 +222,20 @@ def test_encode_rows_argument_errors(lib):
     assert lib.sage_encode_rows(8, 128, 6, None, *a[1:10], None) == sage.SAGE_ERR_INVALID_ARGUMENT
     assert lib.sage_encode_rows(8, 100, 6, *a, None) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_encode_rows(8, 128, 9, *a, None) == sage.SAGE_ERR_UNSUPPORTED
+
+
+def test_kmeans_argument_errors(lib):
+    """Checks that return before any device work (no GPU here)."""
+    n = 1000
+    need = lib.sage_kmeans_workspace_size(n)
+    assert need >= 64 * n and lib.sage_kmeans_workspace_size(0) == 0
+    a = [0x100000 * (i + 1) for i in range(4)]  # P, Wt, init, cb (never dereferenced)
+    ws = 0x800000
+    assert lib.sage_kmeans(n, 6, None, a[1], a[2], 3, a[3], None, ws, need, None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_kmeans(n, 6, a[0], a[1], a[2], 3, None, None, ws, need, None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_kmeans(0, 6, *a[:3], 3, a[3], None, ws, need, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_kmeans(n, 3, *a[:3], 3, a[3], None, ws, need, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_kmeans(n, 6, *a[:3], -1, a[3], None, ws, need, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_kmeans(n, 6, *a[:3], 3, a[3], None, None, need, None) == sage.SAGE_ERR_WORKSPACE
+    assert lib.sage_kmeans(n, 6, *a[:3], 3, a[3], None, ws + 8, need, None) == sage.SAGE_ERR_MISALIGNED
+    assert lib.sage_kmeans(n, 6, *a[:3], 3, a[3], None, ws, need - 1, None) == sage.SAGE_ERR_WORKSPACE

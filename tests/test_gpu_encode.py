@@ -1,8 +1,9 @@
-"""GPU parity of the encoder's per-row stage (sage_encode_rows: Eq. 6
-assignment, Eq. 14 grid, Eq. 2 codes for a given stored codebook; Sec.
-3.1-3.2): bit-exact against the oracle's stage and against the library's CPU
-encoder at full size, through the C ABI (integer and fp16-bit outputs, so the
-bar is equality)."""
+"""GPU parity of the encoder (Sec. 3.1-3.2): its per-row stage
+(sage_encode_rows: Eq. 6 assignment, Eq. 14 grid, Eq. 2 codes for a given
+stored codebook) and its weighted spherical k-means (sage_kmeans), bit-exact
+against the oracle and against the library's CPU encoder at full size, through
+the C ABI (integer, fp16-bit and fp64 outputs computed with separately rounded
+fp64 operations in the same order, so the bar is equality)."""
 import numpy as np
 import pytest
 
@@ -70,5 +71,80 @@ def test_encode_rows_matches_cpu_encoder_full_size():
     r = sage.sage_encode(inp.W, inp.energies, inp.log2K, inp.gamma, inp.sample, inp.init, inp.iters)
     om = oracle.omega_columns(inp.energies, r["perm"], inp.gamma)
     got = _gpu_rows(inp.W, r["perm"], om, r["codebook"], inp.log2K)
+    for k in ("signs", "idx", "q", "mu", "delta"):
+        assert np.array_equal(got[k], r[k]), k
+
+
+def _samples(W, perm, om, sample):
+    """Magnitudes and Eq. 4 weights of the sampled subvectors (storage order)."""
+    S = W.shape[1] // 8
+    o, j = sample // S, sample % S
+    cols = perm.reshape(S, 8)[j]                      # [n][8] original channels
+    P = np.abs(W[o[:, None], cols])
+    Wt = om.reshape(S, 8)[j]
+    return np.ascontiguousarray(P), np.ascontiguousarray(Wt)
+
+
+@pytest.mark.parametrize("log2K", [4, 5, 6, 7, 8])
+def test_kmeans_matches_oracle(log2K):
+    """Random samples with all-zero ones among them, an initial codeword on a
+    zero sample (the 1/sqrt(8) direction) and a repeated initial pick (two equal
+    codewords: the later one stays empty and keeps its codeword)."""
+    g = np.random.default_rng(80 + log2K)
+    n, K = 3000, 1 << log2K
+    P = np.abs(g.standard_normal((n, 8))) * g.lognormal(0.0, 1.0, (n, 1))
+    P[g.choice(n, 40, replace=False)] = 0.0
+    Wt = g.lognormal(0.0, 0.7, (n, 8))
+    init = g.choice(n, K, replace=False).astype(np.int64)
+    zero = int(np.flatnonzero(P.sum(axis=1) == 0)[0])
+    init[1] = zero
+    init[K - 1] = init[2]
+    ref = oracle.kmeans(P, Wt, K, init, 4)
+    cb, cb16 = sage.sage_kmeans(_dev(P), _dev(Wt), log2K, _dev(init), 4)
+    got = cb.cpu().numpy()
+    assert np.array_equal(got.view(np.uint64), ref.view(np.uint64))
+    want16 = np.array([oracle.double_to_half(float(v)) for v in ref.reshape(-1)], np.uint16).reshape(K, 8)
+    assert np.array_equal(cb16.cpu().numpy().view(np.uint16), want16)
+    # one round: the repeated pick's later cluster is empty (ties go to the smaller
+    # index) and keeps its initial codeword; the zero sample's codeword starts uniform
+    cb1, _ = sage.sage_kmeans(_dev(P), _dev(Wt), log2K, _dev(init), 1)
+    ref0 = oracle.kmeans(P, Wt, K, init, 0)
+    assert np.array_equal(cb1.cpu().numpy()[K - 1].view(np.uint64), ref0[K - 1].view(np.uint64))
+    assert np.all(ref0[1] == 1.0 / np.sqrt(8.0))
+
+
+def test_kmeans_zero_rounds_is_the_initialisation():
+    g = np.random.default_rng(90)
+    P = np.abs(g.standard_normal((100, 8)))
+    Wt = np.ones((100, 8))
+    init = np.arange(16, dtype=np.int64) * 3
+    cb, _ = sage.sage_kmeans(_dev(P), _dev(Wt), 4, _dev(init), 0)
+    ref = oracle.kmeans(P, Wt, 16, init, 0)
+    assert np.array_equal(cb.cpu().numpy().view(np.uint64), ref.view(np.uint64))
+
+
+def test_kmeans_rejects_init_outside_the_samples():
+    """An init position >= n is found on the device (the kernel reads sample 0
+    in its place) and reported as INVALID_ARGUMENT."""
+    P = np.ones((50, 8))
+    init = np.arange(16, dtype=np.int64)
+    init[5] = 50
+    with pytest.raises(sage.SageError) as e:
+        sage.sage_kmeans(_dev(P), _dev(P), 4, _dev(init), 2)
+    assert e.value.status == sage.SAGE_ERR_INVALID_ARGUMENT
+
+
+def test_gpu_encoder_matches_cpu_encoder_full_size():
+    """The weight-derived 4096 x 4096 layer (65,536 samples): the GPU k-means on
+    the CPU encoder's samples gives its codebook bit for bit, and the GPU row
+    stage with that codebook gives every field."""
+    inp, _ = synth.config2()
+    r = sage.sage_encode(inp.W, inp.energies, inp.log2K, inp.gamma, inp.sample, inp.init, inp.iters)
+    om = oracle.omega_columns(inp.energies, r["perm"], inp.gamma)
+    P, Wt = _samples(inp.W, r["perm"], om, inp.sample)
+    _, cb16 = sage.sage_kmeans(_dev(P), _dev(Wt), inp.log2K, _dev(inp.init), inp.iters)
+    cb16 = cb16.cpu().numpy().view(np.uint16)
+    assert np.array_equal(cb16, r["codebook"])
+    got = _gpu_rows(inp.W, r["perm"], om, cb16, inp.log2K)
     for k in ("signs", "idx", "q", "mu", "delta"):
         assert np.array_equal(got[k], r[k]), k
