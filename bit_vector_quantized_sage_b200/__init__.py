@@ -334,18 +334,20 @@ def sage_encode_rows(d_out: int, d_in: int, log2K: int, W, perm, omega, codebook
                                                        _ptr(delta), _stream(stream)))
 
 
-def sage_kmeans(P, Wt, log2K: int, init, iters: int, stream=None):
+def sage_kmeans(P, Wt, log2K: int, init, iters: int, ws: "Workspace | None" = None, stream=None):
     """Weighted spherical k-means on the GPU (device tensors: P, Wt fp64 [n][8],
-    init int64 [K]) -> (codebook fp64 [K][8], codebook fp16 bits [K][8]) on the device."""
+    init int64 [K]) -> (codebook fp64 [K][8], codebook fp16 bits [K][8], workspace);
+    asynchronous: sage_query_status(workspace) reports a bad init entry."""
     import torch
     n = int(P.shape[0])
     K = 1 << log2K
     cb = torch.empty((K, 8), dtype=torch.float64, device=P.device)
     cb16 = torch.empty((K, 8), dtype=torch.int16, device=P.device)
-    ws = Workspace(load().sage_kmeans_workspace_size(n))
+    if ws is None:
+        ws = Workspace(load().sage_kmeans_workspace_size(n))
     _check("sage_kmeans", load().sage_kmeans(n, log2K, _ptr(P), _ptr(Wt), _ptr(init), iters, _ptr(cb), _ptr(cb16),
                                              ws.ptr, ws.nbytes, _stream(stream)))
-    return cb, cb16
+    return cb, cb16, ws
 
 
 def sage_abs_error(A: PackedMatrix, W, energy, ws: Workspace, stream=None) -> float:

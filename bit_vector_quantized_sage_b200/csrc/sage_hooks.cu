@@ -172,6 +172,7 @@ int read_and_clear_status(void* ws, sage_stream_t stream) {
     if (v == 0) return SAGE_OK;
     if (cudaMemset(ws, 0, sizeof(v)) != cudaSuccess) return SAGE_ERR_CUDA;
     if (v & kDevTimeout) return SAGE_ERR_TIMEOUT;
+    if (v & kDevBadInput) return SAGE_ERR_INVALID_ARGUMENT;
     return SAGE_ERR_UNSUPPORTED;
 }
 

@@ -18,6 +18,7 @@ constexpr int kBlockOct = 32;   // row octets per storage block (256 rows)
 
 // Device status word bits (first word of the workspace).
 constexpr uint32_t kDevTimeout = 1u;
+constexpr uint32_t kDevBadInput = 4u;  // an input value found invalid on the device
 constexpr uint32_t kDevUnsupported = 2u;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kKmThreads = 256;   // prep / init / assignment kernels
 constexpr int kUpdThreads = 512;  // update kernel: samples scanned per round
-constexpr size_t kKmHeader = 256; // workspace header: word 0 = bad-init flag
+constexpr size_t kKmHeader = 256; // workspace header: word 0 = the status word
 
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -76,15 +76,15 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_prep_kernel(int n, const do
 }
 
 // Codeword k = unit direction of sample init[k] (all-zero sample: the uniform
-// direction 1 / sqrt(8)).  An init entry outside [0, n) raises the flag and
-// uses sample 0.
+// direction 1 / sqrt(8)).  An init entry outside [0, n) is recorded in the
+// status word and sample 0 is used in its place.
 __global__ void kmeans_init_kernel(int n, int K, const double* __restrict__ P, const int64_t* __restrict__ init,
                                    double* __restrict__ cb, uint32_t* flag) {
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= K) return;
     long long id = init[k];
     if (id < 0 || id >= n) {
-        atomicOr(flag, 1u);
+        atomicOr(flag, kDevBadInput);
         id = 0;
     }
     const double* p = P + (size_t)id * 8;
@@ -264,7 +264,6 @@ extern "C" int sage_kmeans(int n, int log2K, const double* P, const double* Wt, 
             return SAGE_ERR_CUDA;
         smem_set[dev] = true;
     }
-    if (cudaMemsetAsync(w.flag, 0, sizeof(uint32_t), s) != cudaSuccess) return SAGE_ERR_CUDA;
     kmeans_prep_kernel<<<grid, kKmThreads, 0, s>>>(n, P, Wt, w.live, w.v);
     kmeans_init_kernel<<<(K + 63) / 64, 64, 0, s>>>(n, K, P, init, cb, w.flag);
     for (int it = 0; it < iters; ++it) {
@@ -272,10 +271,5 @@ extern "C" int sage_kmeans(int n, int log2K, const double* P, const double* Wt, 
         kmeans_update_kernel<<<K, kUpdThreads, kUpdSmem, s>>>(n, w.z, w.live, w.v, cb);
     }
     if (cb16) kmeans_half_kernel<<<(K * 8 + 255) / 256, 256, 0, s>>>(K * 8, cb, cb16);
-    if (cudaGetLastError() != cudaSuccess) return SAGE_ERR_CUDA;
-    uint32_t flag = 0;
-    if (cudaMemcpyAsync(&flag, w.flag, sizeof(flag), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
-        return SAGE_ERR_CUDA;
-    return flag ? SAGE_ERR_INVALID_ARGUMENT : SAGE_OK;
+    return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

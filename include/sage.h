@@ -320,11 +320,13 @@ int sage_encode_rows(int d_out, int d_in, int log2K, const double* W, const int3
  *   cb: device fp64 [K][8] (output); cb16: device fp16 [K][8], the codebook
  *     rounded to nearest even (output; may be null);
  *   ws: device memory of sage_kmeans_workspace_size(n) bytes, 16-byte aligned,
- *     owned by the caller, not shared with a concurrent call.
- * Synchronous: returns after the stream has finished the work.  Errors:
- * INVALID_ARGUMENT (null pointer; an init entry outside [0, n), found on the
- * device -- the codebook is then undefined), UNSUPPORTED (n < 1, iters < 0,
- * log2K outside 4..8), MISALIGNED, WORKSPACE, CUDA. */
+ *     zero-filled once before first use (word 0 is its status word), owned by
+ *     the caller, not shared with a concurrent call.
+ * Asynchronous on `stream`.  Errors: INVALID_ARGUMENT (null pointer),
+ * UNSUPPORTED (n < 1, iters < 0, log2K outside 4..8), MISALIGNED, WORKSPACE,
+ * CUDA; an init entry outside [0, n) is found on the device (sample 0 is read
+ * in its place, the codebook is then meaningless) and sage_query_status(ws)
+ * returns INVALID_ARGUMENT for it. */
 size_t sage_kmeans_workspace_size(int n);
 int sage_kmeans(int n, int log2K, const double* P, const double* Wt, const int64_t* init, int iters, double* cb,
                 uint16_t* cb16, void* ws, size_t ws_bytes, sage_stream_t stream);
@@ -398,7 +400,9 @@ int sage_permute_x(const uint16_t* x, const int32_t* perm, int M, int d_in, uint
 
 /* Synchronises `stream`, reads and clears the workspace status word.
  * Returns SAGE_OK, SAGE_ERR_TIMEOUT (a bounded device wait gave up),
- * SAGE_ERR_UNSUPPORTED (a device-side limit was exceeded) or SAGE_ERR_CUDA. */
+ * SAGE_ERR_INVALID_ARGUMENT (an input value found invalid on the device, e.g.
+ * a sage_kmeans init entry), SAGE_ERR_UNSUPPORTED (a device-side limit was
+ * exceeded) or SAGE_ERR_CUDA. */
 int sage_query_status(void* ws, sage_stream_t stream);
 
 #ifdef __cplusplus

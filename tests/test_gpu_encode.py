@@ -100,14 +100,15 @@ def test_kmeans_matches_oracle(log2K):
     init[1] = zero
     init[K - 1] = init[2]
     ref = oracle.kmeans(P, Wt, K, init, 4)
-    cb, cb16 = sage.sage_kmeans(_dev(P), _dev(Wt), log2K, _dev(init), 4)
+    cb, cb16, ws = sage.sage_kmeans(_dev(P), _dev(Wt), log2K, _dev(init), 4)
+    assert sage.sage_query_status(ws) == 0
     got = cb.cpu().numpy()
     assert np.array_equal(got.view(np.uint64), ref.view(np.uint64))
     want16 = np.array([oracle.double_to_half(float(v)) for v in ref.reshape(-1)], np.uint16).reshape(K, 8)
     assert np.array_equal(cb16.cpu().numpy().view(np.uint16), want16)
     # one round: the repeated pick's later cluster is empty (ties go to the smaller
     # index) and keeps its initial codeword; the zero sample's codeword starts uniform
-    cb1, _ = sage.sage_kmeans(_dev(P), _dev(Wt), log2K, _dev(init), 1)
+    cb1, _, _ = sage.sage_kmeans(_dev(P), _dev(Wt), log2K, _dev(init), 1)
     ref0 = oracle.kmeans(P, Wt, K, init, 0)
     assert np.array_equal(cb1.cpu().numpy()[K - 1].view(np.uint64), ref0[K - 1].view(np.uint64))
     assert np.all(ref0[1] == 1.0 / np.sqrt(8.0))
@@ -118,20 +119,21 @@ def test_kmeans_zero_rounds_is_the_initialisation():
     P = np.abs(g.standard_normal((100, 8)))
     Wt = np.ones((100, 8))
     init = np.arange(16, dtype=np.int64) * 3
-    cb, _ = sage.sage_kmeans(_dev(P), _dev(Wt), 4, _dev(init), 0)
+    cb, _, _ = sage.sage_kmeans(_dev(P), _dev(Wt), 4, _dev(init), 0)
     ref = oracle.kmeans(P, Wt, 16, init, 0)
     assert np.array_equal(cb.cpu().numpy().view(np.uint64), ref.view(np.uint64))
 
 
 def test_kmeans_rejects_init_outside_the_samples():
     """An init position >= n is found on the device (the kernel reads sample 0
-    in its place) and reported as INVALID_ARGUMENT."""
+    in its place) and reported through the workspace status word; the word is
+    cleared by the query."""
     P = np.ones((50, 8))
     init = np.arange(16, dtype=np.int64)
     init[5] = 50
-    with pytest.raises(sage.SageError) as e:
-        sage.sage_kmeans(_dev(P), _dev(P), 4, _dev(init), 2)
-    assert e.value.status == sage.SAGE_ERR_INVALID_ARGUMENT
+    _, _, ws = sage.sage_kmeans(_dev(P), _dev(P), 4, _dev(init), 2)
+    assert sage.sage_query_status(ws) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert sage.sage_query_status(ws) == 0
 
 
 def test_gpu_encoder_matches_cpu_encoder_full_size():
@@ -142,7 +144,7 @@ def test_gpu_encoder_matches_cpu_encoder_full_size():
     r = sage.sage_encode(inp.W, inp.energies, inp.log2K, inp.gamma, inp.sample, inp.init, inp.iters)
     om = oracle.omega_columns(inp.energies, r["perm"], inp.gamma)
     P, Wt = _samples(inp.W, r["perm"], om, inp.sample)
-    _, cb16 = sage.sage_kmeans(_dev(P), _dev(Wt), inp.log2K, _dev(inp.init), inp.iters)
+    _, cb16, _ = sage.sage_kmeans(_dev(P), _dev(Wt), inp.log2K, _dev(inp.init), inp.iters)
     cb16 = cb16.cpu().numpy().view(np.uint16)
     assert np.array_equal(cb16, r["codebook"])
     got = _gpu_rows(inp.W, r["perm"], om, cb16, inp.log2K)
