@@ -608,9 +608,14 @@ def bench_abs(stream, reps=10):
     import synth
     import bit_vector_quantized_sage_b200 as sage
     packed = []
+    inits = {}
+    t_cpu_enc = 0.0
     for log2K in (4, 5, 6, 7, 8):
         inp, _ = synth.config2(d_out=4096, d_in=4096, n_samples=65536, iters=10, log2K=log2K)
+        inits[log2K] = inp.init
+        t0 = time.perf_counter()
         r = sage.sage_encode(inp.W, inp.energies, log2K, inp.gamma, inp.sample, inp.init, inp.iters)
+        t_cpu_enc += time.perf_counter() - t0
         f = synth.Fields(4096, 4096, log2K, r["signs"], r["idx"], r["q"], r["mu"], r["delta"], r["codebook"],
                          r["perm"], f"K=2^{log2K}")
         packed.append(sage.PackedMatrix.from_fields(f))
@@ -629,11 +634,51 @@ def bench_abs(stream, reps=10):
     us = float(np.median(t))
     nbytes = packed[0].packed_bytes + 4096 * 4 + 4096 * 4096 * 4 + 4096 * 4
     hbm, _ = _peaks()
+    # the same selection with the five encodings made on the GPU (k-means, row
+    # stage, device packer), from the host-side inputs (permutation, Eq. 4 weights,
+    # samples), which are computed once per matrix
+    t0 = time.perf_counter()
+    x = sage.sage_encode_inputs(inp.W, inp.energies, inp.gamma, inp.sample)
+    t_inputs = time.perf_counter() - t0
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    Wd, Pd, Wtd, permd, omd = dev(inp.W), dev(x["P"]), dev(x["Wt"]), dev(x["perm"]), dev(x["omega"])
+    initd = {k: dev(v) for k, v in inits.items()}
+    kws = sage.Workspace(sage.sage_kmeans_workspace_size(Pd.shape[0]))
+    fl = [torch.empty((4096, 512), dtype=torch.uint8, device="cuda"), torch.empty((4096, 512), dtype=torch.int16, device="cuda"),
+          torch.empty((4096, 512), dtype=torch.uint8, device="cuda"), torch.empty((4096, 32), dtype=torch.int16, device="cuda"),
+          torch.empty((4096, 32), dtype=torch.int16, device="cuda")]
+
+    def gpu_abs():
+        cands = []
+        for log2K in (4, 5, 6, 7, 8):
+            _, cb16, _ = sage.sage_kmeans(Pd, Wtd, log2K, initd[log2K], 10, kws, stream)
+            sage.sage_encode_rows(4096, 4096, log2K, Wd, permd, omd, cb16, *fl, stream)
+            main, meta = sage.sage_pack_device(4096, 4096, log2K, *fl, stream)
+            cands.append(sage.PackedMatrix(4096, 4096, log2K, main, meta, cb16.reshape(-1), permd))
+        return sage.sage_abs_select(cands, W, e, ws, stream)
+
+    g_best, g_errs = gpu_abs()
+    tg = []
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gpu_abs()
+        e1.record(stream)
+        e1.synchronize()
+        tg.append(e0.elapsed_time(e1) * 1e3)
+    assert sage.sage_query_status(kws) == 0
     return {"workload": "Eq. 8 score of the five split encodings of the weight-derived 4096 x 4096 layer, Eq. 9 choice",
             "best_log2K": 4 + best, "errors": [round(x, 6) for x in errs],
             "us_per_candidate": dist_summary(t), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
             "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
-            "note": "synchronous calls (each adds its CTAs' partial sums on the host)"}
+            "note": "synchronous calls (each adds its CTAs' partial sums on the host)",
+            "gpu_encoder_end_to_end": {
+                "what": "the five encodings on the GPU (sage_kmeans 10 rounds, sage_encode_rows, sage_pack_device) "
+                        "and the Eq. 8 scores / Eq. 9 choice",
+                "us": dist_summary(tg), "best_log2K": 4 + g_best, "same_errors_as_cpu_encoder": g_errs == errs,
+                "host_inputs_s": round(t_inputs, 3),
+                "cpu_encoder_s": round(t_cpu_enc, 3), "cpu_encoder_cores": host_cores(),
+                "cpu_encoder_what": "the five sage_encode calls (all host cores), packing excluded"}}
 
 
 def bench_encode_rows(stream, reps=10):

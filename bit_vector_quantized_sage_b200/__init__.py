@@ -37,7 +37,7 @@ EXPORTS = (
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
     "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
     "sage_qdq_forward", "sage_abs_error", "sage_abs_select", "sage_encode_rows", "sage_kmeans_workspace_size",
-    "sage_kmeans",
+    "sage_kmeans", "sage_pack_device", "sage_encode_inputs",
 )
 
 
@@ -104,6 +104,8 @@ def load(path: str = LIB_PATH):
         "sage_abs_select": ([MP, I, P, P, P, SZ, C.POINTER(I), P, P], I),
         "sage_encode_rows": ([I, I, I, P, P, P, P, P, P, P, P, P, P], I),
         "sage_kmeans_workspace_size": ([I], C.c_size_t),
+        "sage_pack_device": ([I, I, I, P, P, P, P, P, P, P, P], I),
+        "sage_encode_inputs": ([I, I, P, P, C.c_double, I, P, P, P, P, P], I),
         "sage_kmeans": ([I, I, P, P, P, I, P, P, P, C.c_size_t, P], I),
     }
     for name, (args, res) in sig.items():
@@ -334,6 +336,36 @@ def sage_encode_rows(d_out: int, d_in: int, log2K: int, W, perm, omega, codebook
                                                        _ptr(delta), _stream(stream)))
 
 
+def sage_encode_inputs(W, energy, gamma: float, sample):
+    """Host: ESG permutation, Eq. 4 weights per storage column and the sampled
+    subvectors' magnitudes / weights -> dict(perm, omega, P, Wt) (numpy)."""
+    W, pW = _np(W, np.float64)
+    e, pe = _np(energy, np.float64)
+    sm, psm = _np(sample, np.int64)
+    d_out, d_in = W.shape
+    n = sm.shape[0]
+    out = dict(perm=np.zeros(d_in, np.int32), omega=np.zeros(d_in), P=np.zeros((n, 8)), Wt=np.zeros((n, 8)))
+    _check("sage_encode_inputs", load().sage_encode_inputs(d_out, d_in, pW, pe, gamma, n, psm,
+                                                           *(o.ctypes.data for o in out.values())))
+    return out
+
+
+def sage_kmeans_workspace_size(n: int) -> int:
+    return int(load().sage_kmeans_workspace_size(n))
+
+
+def sage_pack_device(d_out: int, d_in: int, log2K: int, signs, idx, q, mu, delta, stream=None):
+    """The packer on the device (device field tensors) -> (main, meta) int32 device planes."""
+    import torch
+    mb, tb = C.c_size_t(), C.c_size_t()
+    _check("sage_packed_sizes", load().sage_packed_sizes(d_out, d_in, log2K, C.byref(mb), C.byref(tb)))
+    main = torch.empty(mb.value // 4, dtype=torch.int32, device=signs.device)
+    meta = torch.empty(tb.value // 4, dtype=torch.int32, device=signs.device)
+    _check("sage_pack_device", load().sage_pack_device(d_out, d_in, log2K, _ptr(signs), _ptr(idx), _ptr(q), _ptr(mu),
+                                                       _ptr(delta), _ptr(main), _ptr(meta), _stream(stream)))
+    return main, meta
+
+
 def sage_kmeans(P, Wt, log2K: int, init, iters: int, ws: "Workspace | None" = None, stream=None):
     """Weighted spherical k-means on the GPU (device tensors: P, Wt fp64 [n][8],
     init int64 [K]) -> (codebook fp64 [K][8], codebook fp16 bits [K][8], workspace);
@@ -344,7 +376,7 @@ def sage_kmeans(P, Wt, log2K: int, init, iters: int, ws: "Workspace | None" = No
     cb = torch.empty((K, 8), dtype=torch.float64, device=P.device)
     cb16 = torch.empty((K, 8), dtype=torch.int16, device=P.device)
     if ws is None:
-        ws = Workspace(load().sage_kmeans_workspace_size(n))
+        ws = Workspace(sage_kmeans_workspace_size(n))
     _check("sage_kmeans", load().sage_kmeans(n, log2K, _ptr(P), _ptr(Wt), _ptr(init), iters, _ptr(cb), _ptr(cb16),
                                              ws.ptr, ws.nbytes, _stream(stream)))
     return cb, cb16, ws

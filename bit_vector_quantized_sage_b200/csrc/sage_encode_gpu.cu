@@ -10,7 +10,8 @@
 // permutation and Eq. 4 weights.  One persistent grid; each CTA holds the
 // codebook in fp64 in shared memory and gives 16 threads to a row group
 // (one subvector each); the group's radius range is a 16-lane shuffle
-// reduction.
+// reduction.  sage_pack_device then writes the packed planes from the fields
+// on the device, word for word what the host packer writes.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -104,10 +105,104 @@ __global__ void __launch_bounds__(kEncThreads) encode_rows_kernel(int d_out, int
     }
 }
 
+// Packed format v2 on the device (the host packer's layout): blocks of 32
+// row octets stored contiguously, subvector-column major inside a block.
+__device__ __forceinline__ int pk_octets(int R8, int blk) { return min(32, R8 - blk * 32); }
+
+// One thread per 16-byte main record word (octet b, column j, word u): word u
+// holds rows 2u (row A) and 2u + 1 (row B) of the octet.  Row A: z at bits
+// 7.., q at bits 23 - V..; row B: z at bits 23.., q at bits 7 - V..; sign
+// bits 0-5 of row A / B in the three slot pairs (p, p + 16) of its half.
+__global__ void pack_main_kernel(int d_out, int S, int log2K, const uint8_t* __restrict__ signs,
+                                 const uint16_t* __restrict__ idx, const uint8_t* __restrict__ q,
+                                 uint32_t* __restrict__ main_out) {
+    const int V = 10 - log2K, R8 = (d_out + 7) >> 3;
+    const uint32_t zm = (1u << log2K) - 1u, qm = (1u << V) - 1u;
+    const long long total = (long long)R8 * S * 4;
+    for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < total;
+         id += (long long)gridDim.x * blockDim.x) {
+        const int u = (int)(id & 3);
+        const long long r = id >> 2;            // record: block-major, then column, then octet
+        const int blk = (int)(r / ((long long)S * 32));
+        const int nB = pk_octets(R8, blk);
+        const long long in_blk = r - (long long)blk * S * 32;
+        const int j = (int)(in_blk / nB), ob = (int)(in_blk - (long long)j * nB);
+        if (j >= S) continue;  // the last block is shorter: no record there
+        uint32_t w = 0;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int o = (blk * 32 + ob) * 8 + 2 * u + half;
+            if (o >= d_out) continue;
+            const size_t e = (size_t)o * S + j;
+            const uint32_t z = idx[e] & zm, qq = q[e] & qm, sb = signs[e];
+            w |= half ? (z << 23) | (qq << (7 - V)) : (z << 7) | (qq << (23 - V));
+#pragma unroll
+            for (int n = 0; n < 3; ++n) {
+                const int k = n + 3 * half;  // sign slots {0 .. 6 - V} then {17 - V .. 15}
+                const int pos = k <= 6 - V ? k : (17 - V) + (k - (7 - V));
+                w |= ((sb >> (2 * n)) & 1u) << pos;
+                w |= ((sb >> (2 * n + 1)) & 1u) << (pos + 16);
+            }
+        }
+        main_out[(size_t)blk * S * 128 + ((size_t)j * nB + ob) * 4 + u] = w;
+    }
+}
+
+// One thread per 8-byte meta entry (octet b, group g, row t): the group's 16
+// sign bits 6 (bits 0-15) and 7 (bits 16-31) of row 8b + t, then mu | delta << 16.
+__global__ void pack_meta_kernel(int d_out, int S, int G, const uint8_t* __restrict__ signs,
+                                 const uint16_t* __restrict__ mu, const uint16_t* __restrict__ delta,
+                                 uint2* __restrict__ meta_out) {
+    const int R8 = (d_out + 7) >> 3;
+    const long long total = (long long)R8 * G * 8;
+    for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < total;
+         id += (long long)gridDim.x * blockDim.x) {
+        const int t = (int)(id & 7);
+        const long long r = id >> 3;
+        const int blk = (int)(r / ((long long)G * 32));
+        const int nB = pk_octets(R8, blk);
+        const long long in_blk = r - (long long)blk * G * 32;
+        const int g = (int)(in_blk / nB), ob = (int)(in_blk - (long long)g * nB);
+        if (g >= G) continue;
+        const int o = (blk * 32 + ob) * 8 + t;
+        uint2 m = make_uint2(0u, 0u);
+        if (o < d_out) {
+            const uint8_t* sr = signs + (size_t)o * S + g * 16;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const uint32_t sb = sr[jj];
+                m.x |= ((sb >> 6) & 1u) << jj;
+                m.x |= ((sb >> 7) & 1u) << (jj + 16);
+            }
+            m.y = (uint32_t)mu[(size_t)o * G + g] | ((uint32_t)delta[(size_t)o * G + g] << 16);
+        }
+        meta_out[(size_t)blk * G * 256 + ((size_t)g * nB + ob) * 8 + t] = m;
+    }
+}
+
 }  // namespace
 }  // namespace sage
 
 using namespace sage;
+
+extern "C" int sage_pack_device(int d_out, int d_in, int log2K, const uint8_t* signs, const uint16_t* idx,
+                                const uint8_t* q, const uint16_t* mu, const uint16_t* delta, uint32_t* main_out,
+                                uint32_t* meta_out, sage_stream_t stream) {
+    if (!signs || !idx || !q || !mu || !delta || !main_out || !meta_out) return SAGE_ERR_INVALID_ARGUMENT;
+    if (d_out < 1 || d_in < 128 || d_in % 128 || log2K < 4 || log2K > 8) return SAGE_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(meta_out) % 8 || reinterpret_cast<uintptr_t>(main_out) % 4)
+        return SAGE_ERR_MISALIGNED;
+    const int S = d_in / 8, G = d_in / 128;
+    const long long R8 = (d_out + 7) / 8;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int cap = 8 * current_sm_count();
+    const long long nm = R8 * S * 4, nt = R8 * G * 8;
+    pack_main_kernel<<<(int)std::max<long long>(1, std::min<long long>((nm + 255) / 256, cap)), 256, 0, s>>>(
+        d_out, S, log2K, signs, idx, q, main_out);
+    pack_meta_kernel<<<(int)std::max<long long>(1, std::min<long long>((nt + 255) / 256, cap)), 256, 0, s>>>(
+        d_out, S, G, signs, mu, delta, reinterpret_cast<uint2*>(meta_out));
+    return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
 
 extern "C" int sage_encode_rows(int d_out, int d_in, int log2K, const double* W, const int32_t* perm,
                                 const double* omega, const uint16_t* codebook, uint8_t* signs, uint16_t* idx,

@@ -255,6 +255,42 @@ void parallel_for(int n, int n_threads, F&& f) {
 
 }  // namespace
 
+namespace {
+// Eq. 4: omega of storage column 8j + i = e^gamma / mean over the subvector's
+// 8 channels of e^gamma, e the energies in storage order.
+void omega_columns(int d_in, const double* energy, const int32_t* perm, double gamma, double* omega) {
+    for (int j = 0; j < d_in / kSV; ++j) {
+        double eg[kSV], mean = 0.0;
+        for (int i = 0; i < kSV; ++i) { eg[i] = std::pow(energy[perm[j * kSV + i]], gamma); mean += eg[i]; }
+        mean /= kSV;
+        for (int i = 0; i < kSV; ++i) omega[(size_t)j * kSV + i] = eg[i] / mean;
+    }
+}
+}  // namespace
+
+extern "C" int sage_encode_inputs(int d_out, int d_in, const double* W, const double* energy, double gamma,
+                                  int n_samples, const int64_t* sample, int32_t* perm_out, double* omega_out,
+                                  double* P_out, double* Wt_out) {
+    if (!W || !energy || !sample || !perm_out || !omega_out || !P_out || !Wt_out) return SAGE_ERR_INVALID_ARGUMENT;
+    if (d_out < 1 || d_in < 1 || n_samples < 1) return SAGE_ERR_INVALID_ARGUMENT;
+    if (d_in % 128) return SAGE_ERR_UNSUPPORTED;
+    const int S = d_in / kSV;
+    const int64_t n_sv = (int64_t)d_out * S;
+    for (int s = 0; s < n_samples; ++s)
+        if (sample[s] < 0 || sample[s] >= n_sv) return SAGE_ERR_INVALID_ARGUMENT;
+    const int rc = sage_esg_permutation(d_in, energy, perm_out);
+    if (rc) return rc;
+    omega_columns(d_in, energy, perm_out, gamma, omega_out);
+    for (int s = 0; s < n_samples; ++s) {
+        const int64_t o = sample[s] / S, j = sample[s] % S;
+        for (int i = 0; i < kSV; ++i) {
+            P_out[(size_t)s * kSV + i] = std::fabs(W[o * d_in + perm_out[j * kSV + i]]);
+            Wt_out[(size_t)s * kSV + i] = omega_out[(size_t)j * kSV + i];
+        }
+    }
+    return SAGE_OK;
+}
+
 extern "C" int sage_encode(int d_out, int d_in, int log2K, const double* W, const double* energy, double gamma,
                            int n_samples, const int64_t* sample, const int64_t* init, int iters, int n_threads,
                            int32_t* perm_out, uint16_t* codebook_out, uint8_t* signs, uint16_t* idx, uint8_t* q,
@@ -276,12 +312,7 @@ extern "C" int sage_encode(int d_out, int d_in, int log2K, const double* W, cons
 
     // Eq. 4 weights per storage column (same for every row), e in permuted order.
     std::vector<double> omega((size_t)d_in);
-    for (int j = 0; j < S; ++j) {
-        double eg[kSV], mean = 0.0;
-        for (int i = 0; i < kSV; ++i) { eg[i] = std::pow(energy[perm_out[j * kSV + i]], gamma); mean += eg[i]; }
-        mean /= kSV;
-        for (int i = 0; i < kSV; ++i) omega[(size_t)j * kSV + i] = eg[i] / mean;
-    }
+    omega_columns(d_in, energy, perm_out, gamma, omega.data());
     auto magnitudes = [&](int64_t sv, double* p) {
         const int64_t o = sv / S, j = sv % S;
         for (int i = 0; i < kSV; ++i) p[i] = std::fabs(W[o * d_in + perm_out[j * kSV + i]]);

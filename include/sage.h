@@ -150,6 +150,18 @@ int sage_encode(int d_out, int d_in, int log2K, const double* W, const double* e
                 int32_t* perm_out, uint16_t* codebook_out,
                 uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu, uint16_t* delta);
 
+/* HOST.  The inputs of the GPU encoder (sage_kmeans, sage_encode_rows) for
+ * one matrix, as sage_encode computes them before its k-means: the ESG
+ * permutation (as sage_esg_permutation), the Eq. 4 weight of every storage
+ * column (omega_out [d_in], exponent gamma; the weights of subvector column j
+ * are omega_out[8j .. 8j + 7]) and, for the listed sample subvectors
+ * (ids o*(d_in/8)+j), their magnitudes |W| in storage column order and their
+ * weights (P_out, Wt_out: fp64 [n_samples][8]).
+ * Errors: INVALID_ARGUMENT (null, sizes, sample ids), UNSUPPORTED (d_in % 128). */
+int sage_encode_inputs(int d_out, int d_in, const double* W, const double* energy, double gamma,
+                       int n_samples, const int64_t* sample, int32_t* perm_out, double* omega_out,
+                       double* P_out, double* Wt_out);
+
 /* Device workspace bytes for one call of `op` over the n matrices `mats`
  * (host array: the single matrix of sage_gemv / sage_gemm, all matrices of a
  * sage_gemv_grouped call, or all experts of a sage_moe_gemv call) at batch M
@@ -302,6 +314,20 @@ int sage_decoder_layer_forward(const sage_decoder_layer* L, const uint16_t* h, i
 int sage_encode_rows(int d_out, int d_in, int log2K, const double* W, const int32_t* perm, const double* omega,
                      const uint16_t* codebook, uint8_t* signs, uint16_t* idx, uint8_t* q, uint16_t* mu,
                      uint16_t* delta, sage_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The packer on the device: the same planes as sage_pack (format v2), word
+ * for word, from device fields, so that an encoding made on the GPU is
+ * packed without a round trip through the host.  Shapes and field layouts as
+ * sage_pack; main_out / meta_out: device buffers of sage_packed_sizes()
+ * bytes, every word written.  Unlike sage_pack, which rejects them, field
+ * values wider than their bits (idx >= K, q >= 2^V) are masked to their
+ * widths.  Asynchronous on `stream`.  Errors: INVALID_ARGUMENT (null),
+ * UNSUPPORTED (d_in % 128, log2K outside 4..8), MISALIGNED (main_out not
+ * 4-byte or meta_out not 8-byte aligned), CUDA. */
+int sage_pack_device(int d_out, int d_in, int log2K, const uint8_t* signs, const uint16_t* idx, const uint8_t* q,
+                     const uint16_t* mu, const uint16_t* delta, uint32_t* main_out, uint32_t* meta_out,
+                     sage_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * The encoder's weighted spherical k-means on the GPU (Sec. 3.2 "Weighted

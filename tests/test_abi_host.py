@@ -239,3 +239,33 @@ def test_kmeans_argument_errors(lib):
     assert lib.sage_kmeans(n, 6, *a[:3], 3, a[3], None, None, need, None) == sage.SAGE_ERR_WORKSPACE
     assert lib.sage_kmeans(n, 6, *a[:3], 3, a[3], None, ws + 8, need, None) == sage.SAGE_ERR_MISALIGNED
     assert lib.sage_kmeans(n, 6, *a[:3], 3, a[3], None, ws, need - 1, None) == sage.SAGE_ERR_WORKSPACE
+
+
+def test_encode_inputs_match_oracle():
+    """The GPU encoder's host-side inputs: ESG permutation, Eq. 4 weights per
+    storage column and the sampled subvectors' magnitudes / weights, against the
+    oracle's definitions (bit for bit: the same fp64 operations)."""
+    g = np.random.default_rng(17)
+    d_out, d_in = 40, 256
+    W = g.standard_normal((d_out, d_in))
+    e = synth.lognormal_energies(g, d_in, 1.5)
+    sample = np.sort(g.choice(d_out * d_in // 8, 300, replace=False)).astype(np.int64)
+    r = sage.sage_encode_inputs(W, e, 0.75, sample)
+    assert np.array_equal(r["perm"], oracle.esg_perm(e))
+    om = oracle.omega_columns(e, r["perm"], 0.75)
+    assert np.array_equal(r["omega"], om)
+    S = d_in // 8
+    o, j = sample // S, sample % S
+    assert np.array_equal(r["P"], np.abs(W[o[:, None], r["perm"].reshape(S, 8)[j]]))
+    assert np.array_equal(r["Wt"], om.reshape(S, 8)[j])
+    with pytest.raises(sage.SageError):
+        sage.sage_encode_inputs(W, e, 0.75, np.array([d_out * S], np.int64))
+
+
+def test_pack_device_argument_errors(lib):
+    a = [0x100000 * (i + 1) for i in range(7)]
+    assert lib.sage_pack_device(8, 128, 6, None, *a[1:], None) == sage.SAGE_ERR_INVALID_ARGUMENT
+    assert lib.sage_pack_device(8, 100, 6, *a, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_pack_device(8, 128, 9, *a, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_pack_device(8, 128, 6, *a[:5], a[5] + 2, a[6], None) == sage.SAGE_ERR_MISALIGNED
+    assert lib.sage_pack_device(8, 128, 6, *a[:6], a[6] + 4, None) == sage.SAGE_ERR_MISALIGNED

@@ -77,3 +77,44 @@ def test_abs_select_matches_oracle(shape):
         assert abs(a - b) <= 1e-5 * b, (a, b)
     assert best == ref_best, (errs, ref_errs)
     assert 0.0 < min(errs) < 1.0
+
+
+def _gpu_encoding(inp, log2K, x):
+    """One split encoded on the GPU from the host-side inputs x (permutation,
+    Eq. 4 weights, samples): k-means, row stage, device packer."""
+    import torch
+    d_out, d_in = inp.W.shape
+    S, G = d_in // 8, d_in // 128
+    _, cb16, ws = sage.sage_kmeans(_dev(x["P"]), _dev(x["Wt"]), log2K, _dev(inp.init), inp.iters)
+    fl = dict(signs=torch.empty((d_out, S), dtype=torch.uint8, device="cuda"),
+              idx=torch.empty((d_out, S), dtype=torch.int16, device="cuda"),
+              q=torch.empty((d_out, S), dtype=torch.uint8, device="cuda"),
+              mu=torch.empty((d_out, G), dtype=torch.int16, device="cuda"),
+              delta=torch.empty((d_out, G), dtype=torch.int16, device="cuda"))
+    sage.sage_encode_rows(d_out, d_in, log2K, _dev(inp.W), _dev(x["perm"]), _dev(x["omega"]), cb16, *fl.values())
+    main, meta = sage.sage_pack_device(d_out, d_in, log2K, *fl.values())
+    assert sage.sage_query_status(ws) == 0
+    return sage.PackedMatrix(d_out, d_in, log2K, main, meta, cb16.reshape(-1), _dev(x["perm"]), f"K=2^{log2K}")
+
+
+def test_abs_select_with_the_gpu_encoder():
+    """Adaptive bit splitting end to end on the GPU: the five splits encoded by
+    sage_kmeans + sage_encode_rows + sage_pack_device give the CPU encoder's
+    planes and codebooks word for word, hence the same Eq. 8 errors (bit for
+    bit) and the same Eq. 9 choice."""
+    d_out, d_in, n_samples = 512, 1024, 8192
+    inp, fields = _encodings(d_out, d_in, n_samples)
+    x = sage.sage_encode_inputs(inp.W, inp.energies, inp.gamma, inp.sample)
+    gpu, cpu = [], []
+    for log2K, f in zip(SPLITS, fields):
+        i2, _ = synth.config2(d_out=d_out, d_in=d_in, n_samples=n_samples, iters=5, log2K=log2K)
+        A = _gpu_encoding(i2, log2K, x)
+        B = sage.PackedMatrix.from_fields(f)
+        assert np.array_equal(A.main.cpu().numpy(), B.main.cpu().numpy()), log2K
+        assert np.array_equal(A.meta.cpu().numpy(), B.meta.cpu().numpy()), log2K
+        assert np.array_equal(A.codebook.cpu().numpy(), B.codebook.cpu().numpy()), log2K
+        gpu.append(A)
+        cpu.append(B)
+    W32, e32 = _dev(inp.W.astype(np.float32)), _dev(inp.energies.astype(np.float32))
+    ws = workspace_for(sage.SAGE_OP_ABS, gpu[0], 1)
+    assert sage.sage_abs_select(gpu, W32, e32, ws) == sage.sage_abs_select(cpu, W32, e32, ws)

@@ -150,3 +150,18 @@ def test_gpu_encoder_matches_cpu_encoder_full_size():
     got = _gpu_rows(inp.W, r["perm"], om, cb16, inp.log2K)
     for k in ("signs", "idx", "q", "mu", "delta"):
         assert np.array_equal(got[k], r[k]), k
+
+
+@pytest.mark.parametrize("log2K", [4, 5, 6, 7, 8])
+def test_pack_device_matches_host_packer(log2K):
+    """Random fields on two storage blocks (the second one short: 300 rows are
+    38 row octets) and a ragged last octet: the device planes equal the host
+    packer's word for word."""
+    g = np.random.default_rng(70 + log2K)
+    d_out, d_in = 300, 384
+    f = synth.random_fields(g, d_out, d_in, log2K)
+    main, meta = sage.sage_pack(d_out, d_in, log2K, f.signs, f.idx, f.q, f.mu, f.delta)
+    dm, dt = sage.sage_pack_device(d_out, d_in, log2K, _dev(f.signs), _dev(f.idx.view(np.int16)), _dev(f.q),
+                                   _dev(f.mu.view(np.int16)), _dev(f.delta.view(np.int16)))
+    assert np.array_equal(dm.cpu().numpy().view(np.uint32), np.asarray(main).view(np.uint32).reshape(-1))
+    assert np.array_equal(dt.cpu().numpy().view(np.uint32), np.asarray(meta).view(np.uint32).reshape(-1))
