@@ -80,6 +80,8 @@ def lib():
             L.oracle_add.restype = None
             L.oracle_silu_mul.argtypes = [sz, P, P, P]
             L.oracle_silu_mul.restype = None
+            L.oracle_moe_combine.argtypes = [i32, i32, i32, P, P, P]
+            L.oracle_moe_combine.restype = None
             L.oracle_attend_one_position.argtypes = [i32, i32, i32, i32, P, P]
             L.oracle_attend_one_position.restype = None
             L.oracle_qdq_angle.argtypes = [f64]
@@ -305,6 +307,16 @@ def silu_mul(gate16: np.ndarray, up16: np.ndarray) -> np.ndarray:
     g, u = _c(gate16, np.uint16), _c(up16, np.uint16)
     out = np.zeros_like(g)
     lib().oracle_silu_mul(g.size, _p(g), _p(u), _p(out))
+    return out
+
+
+def moe_combine(y16: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Router-weighted combine: y16 fp16 bits [T*topk][d], w [T][topk] -> fp16 bits [T][d]."""
+    w = _c(np.atleast_2d(w), np.float64)
+    T, topk = w.shape
+    y = _c(y16, np.uint16).reshape(T * topk, -1)
+    out = np.zeros((T, y.shape[1]), np.uint16)
+    lib().oracle_moe_combine(T, topk, y.shape[1], _p(y), _p(w), _p(out))
     return out
 
 

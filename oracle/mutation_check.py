@@ -40,6 +40,10 @@ _UNROUNDED = ("            for (int t = 0; t < GROUP_SV; ++t)\n"
               "                q[(size_t)o * S + g * GROUP_SV + t] = (uint8_t)qq; } }")
 
 PLANTS = {
+    "moe_combine_unweighted": ("                acc += w[(size_t)t * topk + k] * oracle_half_to_double(y[((size_t)t * topk + k) * d + c]);",
+                               "                acc += oracle_half_to_double(y[((size_t)t * topk + k) * d + c]);"),
+    "moe_combine_wrong_token": ("                acc += w[(size_t)t * topk + k] * oracle_half_to_double(y[((size_t)t * topk + k) * d + c]);",
+                                "                acc += w[(size_t)t * topk + k] * oracle_half_to_double(y[((size_t)k * T + t) * d + c]);"),
     "dequant_sign_flip": ("const double sgn = ((s >> i) & 1) ? -1.0 : 1.0;", "const double sgn = ((s >> i) & 1) ? 1.0 : -1.0;"),
     "dequant_group_index": ("            const int g = j / GROUP_SV;", "            const int g = j / 8;"),
     "dequant_radius_no_q": ("const double r_hat = m + (double)q[(size_t)o * S + j] * d;", "const double r_hat = m + (double)q[(size_t)o * S + j] * d * 0.5;"),

@@ -531,6 +531,20 @@ void oracle_silu_mul(size_t n, const uint16_t* gate, const uint16_t* up, uint16_
     }
 }
 
+/* Router-weighted combine of a mixture-of-experts projection: token t's
+ * output is the sum over its top-k slots of the router weight times the
+ * slot's expert output, out[t] = fp16( sum_k w[t][k] * y[t*topk + k] ),
+ * summed in slot order in fp64.  y: [T*topk][d]; w: [T][topk]; out: [T][d]. */
+void oracle_moe_combine(int T, int topk, int d, const uint16_t* y, const double* w, uint16_t* out) {
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int k = 0; k < topk; ++k)
+                acc += w[(size_t)t * topk + k] * oracle_half_to_double(y[((size_t)t * topk + k) * d + c]);
+            out[(size_t)t * d + c] = oracle_double_to_half(acc);
+        }
+}
+
 /* Attention over a single cached position (the first token of a sequence):
  * the softmax over one key is 1, so query head h returns the value vector of
  * its key/value head h / (n_heads / n_kv) (grouped-query attention).

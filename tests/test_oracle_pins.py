@@ -818,3 +818,22 @@ def test_encode_rows_is_the_encoders_row_part():
         rows = oracle.encode_rows(inp.W, ref["perm"], om, ref["codebook"], log2K)
         for k in rows:
             assert np.array_equal(rows[k], ref[k]), (log2K, k)
+
+
+def test_moe_combine_closed_forms():
+    """Router-weighted combine: one slot with weight 1 is the identity; equal
+    slot outputs with weights summing to 1 give that output; a hand-worked
+    token (exact in fp16 and fp64); the slots are those of their own token."""
+    g = np.random.default_rng(5)
+    y = _h(g.standard_normal((6, 32)))
+    assert np.array_equal(oracle.moe_combine(y, np.ones((6, 1))), y)
+    rows = np.repeat(y[:1], 4, axis=0)
+    assert np.array_equal(oracle.moe_combine(rows, np.array([[0.125, 0.375, 0.25, 0.25]])), y[:1])
+    # token 0: 0.25 * 1 + 0.75 * 2 = 1.75 ; token 1: 0.5 * -4 + 0.5 * 3 = -0.5
+    y2 = _h([[1.0, 0.0], [2.0, 8.0], [-4.0, 1.0], [3.0, 1.0]])
+    got = oracle.moe_combine(y2, np.array([[0.25, 0.75], [0.5, 0.5]])).view(np.float16)
+    assert np.array_equal(got, np.array([[1.75, 6.0], [-0.5, 1.0]], np.float16))
+    # against a direct fp64 sum with one rounding
+    w = g.random((3, 2))
+    want = _h((w[:, :, None] * y.view(np.float16).astype(np.float64).reshape(3, 2, 32)).sum(axis=1))
+    assert np.array_equal(oracle.moe_combine(y, w), want)
