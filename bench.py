@@ -563,9 +563,20 @@ def bench_moe(stream, reps=20):
             nbytes = sum(packed[e].packed_bytes + (1 << packed[e].log2K) * 16 for e in active)
             nbytes += xb.nbytes + n_pairs * d_out * 2
             us = float(np.median(t))
-            out.append({"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size), "us": dist_summary(t),
-                        "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
-                        "us_cold": dist_summary(tc)})
+            pt = {"proj": synth.MOE_PROJ[proj][0], "T": T, "experts": int(active.size), "us": dist_summary(t),
+                  "gbs": round(nbytes / (us * 1e-6) / 1e9, 1), "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
+                  "us_cold": dist_summary(tc)}
+            if proj == 2:  # the down projection followed by the router-weighted combine
+                wr = torch.from_numpy(np.random.default_rng(T).dirichlet(np.ones(synth.MOE_TOPK), size=T)
+                                      .astype(np.float32)).cuda()
+                yt = torch.zeros((T, d_out), dtype=torch.int16, device="cuda")
+                fc = [lambda st, E=E: (sage.sage_moe_gemv(E, pe, xr, n_pairs, x, y, ws, st),
+                                       sage.sage_moe_combine(T, synth.MOE_TOPK, y, wr, yt, st)) for E in sets]
+                for fn in fc:
+                    fn(stream)
+                pt["us_with_combine"] = dist_summary(per_call_us(fc, stream))
+                assert sage.sage_query_status(ws) == sage.SAGE_OK
+            out.append(pt)
         del sets
     del flush
     return {"workload": "128 experts, top-8, one projection per call (in-kernel routing + grouped GEMV)",

@@ -37,7 +37,7 @@ EXPORTS = (
     "sage_gemm", "sage_moe_gemv", "sage_dequant", "sage_unpack_device", "sage_permute_x",
     "sage_query_status", "sage_gemv_static", "sage_decoder_layer_workspace_size", "sage_decoder_layer_forward",
     "sage_qdq_forward", "sage_abs_error", "sage_abs_select", "sage_encode_rows", "sage_kmeans_workspace_size",
-    "sage_kmeans", "sage_pack_device", "sage_encode_inputs",
+    "sage_kmeans", "sage_pack_device", "sage_encode_inputs", "sage_moe_combine",
 )
 
 
@@ -105,6 +105,7 @@ def load(path: str = LIB_PATH):
         "sage_encode_rows": ([I, I, I, P, P, P, P, P, P, P, P, P, P], I),
         "sage_kmeans_workspace_size": ([I], C.c_size_t),
         "sage_pack_device": ([I, I, I, P, P, P, P, P, P, P, P], I),
+        "sage_moe_combine": ([I, I, I, P, P, P, P], I),
         "sage_encode_inputs": ([I, I, P, P, C.c_double, I, P, P, P, P, P], I),
         "sage_kmeans": ([I, I, P, P, P, I, P, P, P, C.c_size_t, P], I),
     }
@@ -348,6 +349,13 @@ def sage_encode_inputs(W, energy, gamma: float, sample):
     _check("sage_encode_inputs", load().sage_encode_inputs(d_out, d_in, pW, pe, gamma, n, psm,
                                                            *(o.ctypes.data for o in out.values())))
     return out
+
+
+def sage_moe_combine(T: int, topk: int, y_pairs, weights, y, stream=None):
+    """Router-weighted combine (device tensors: y_pairs fp16 bits [T*topk][d_out],
+    weights fp32 [T][topk], y fp16 bits [T][d_out])."""
+    _check("sage_moe_combine", load().sage_moe_combine(T, topk, int(y.shape[-1]), _ptr(y_pairs), _ptr(weights),
+                                                       _ptr(y), _stream(stream)))
 
 
 def sage_kmeans_workspace_size(n: int) -> int:

@@ -239,6 +239,20 @@ int sage_moe_gemv(const sage_matrix* experts, int n_experts,
                   const int32_t* pair_expert, const int32_t* pair_xrow, int n_pairs,
                   const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes, sage_stream_t stream);
 
+/* Router-weighted combine of a mixture-of-experts projection (the step after
+ * the down projection of a top-k routed MLP): for every token t,
+ *   y[t][c] = fp16( sum_k weights[t][k] * y_pairs[t * topk + k][c] ),
+ * summed in fp32 in slot order (k = 0, 1, ...).  y_pairs: device fp16
+ * [T * topk][d_out] (pair p = t * topk + k, the layout sage_moe_gemv writes for
+ * pairs listed token by token); weights: device fp32 [T][topk]; y: device fp16
+ * [T][d_out] (output).  Launched with programmatic dependent launch: it may
+ * start while the preceding kernel on `stream` drains and waits for it before
+ * reading.  Errors: INVALID_ARGUMENT (null, T/topk/d_out < 1), UNSUPPORTED
+ * (d_out % 8), MISALIGNED (y_pairs or y not 16-byte aligned, weights not
+ * 4-byte aligned), CUDA. */
+int sage_moe_combine(int T, int topk, int d_out, const uint16_t* y_pairs, const float* weights, uint16_t* y,
+                     sage_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Fused decoder layer.  The packed projections of one transformer decoder
  * layer run as ONE launch of four dependent stages, with the operations

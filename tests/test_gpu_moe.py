@@ -67,3 +67,63 @@ def test_moe_many_pairs_on_one_expert():
     for p in range(n_pairs):
         y_ref, B = oracle.gemv(experts_f[pe[p]], x[xrow[p]:xrow[p] + 1])
         assert_within_bound(yb[p:p + 1], y_ref, B, f"pair {p}")
+
+
+def _combine_bound(yp16, w):
+    """|GPU - oracle| allowed for the router-weighted combine: the fp32 sum of
+    topk terms errs by at most topk * 2^-24 * sum_k |w y| (< 1e-6 of it here),
+    which can move the fp16 rounding of the result by one ulp."""
+    T, topk = w.shape
+    a = np.abs(w)[:, :, None] * np.abs(yp16.view(np.float16).astype(np.float64).reshape(T, topk, -1))
+    return a.sum(axis=1)
+
+
+def _check_combine(got16, ref16, bound):
+    got = got16.view(np.float16).astype(np.float64)
+    ref = ref16.view(np.float16).astype(np.float64)
+    ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= ulp + 1e-6 * bound), np.max(np.abs(got - ref) - ulp)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_moe_combine_matches_oracle(T):
+    import torch
+    g = np.random.default_rng(30 + T)
+    d_out, topk = 2048, synth.MOE_TOPK
+    yp = g.standard_normal((T * topk, d_out)).astype(np.float16).view(np.uint16)
+    w = g.dirichlet(np.ones(topk), size=T).astype(np.float32)
+    y = torch.zeros((T, d_out), dtype=torch.int16, device="cuda")
+    sage.sage_moe_combine(T, topk, dev_u16(yp), torch.from_numpy(w).cuda(), y)
+    torch.cuda.synchronize()
+    ref = oracle.moe_combine(yp, w.astype(np.float64))
+    _check_combine(host_u16(y), ref, _combine_bound(yp, w.astype(np.float64)))
+
+
+def test_moe_down_projection_then_combine():
+    """The MoE down projection of config 4 at T = 16 followed by the combine
+    (back to back on one stream, the combine launched as a dependent launch):
+    each token's output against the oracle's per-pair GEMV outputs combined by
+    the oracle.  The GPU pair outputs themselves are checked by test_moe_config4;
+    here the combine consumes exactly what the GEMV wrote."""
+    import torch
+    T = 16
+    spec = synth.config4(T)
+    experts_f = [spec.expert(e, 2) for e in range(synth.MOE_EXPERTS)]
+    packed = [sage.PackedMatrix.from_fields(f) for f in experts_f]
+    n_pairs = T * synth.MOE_TOPK
+    pe = spec.routes.reshape(-1).astype(np.int32)
+    xrow = np.arange(n_pairs, dtype=np.int32)
+    d_out = synth.MOE_PROJ[2][1]
+    g = np.random.default_rng(99)
+    w = g.dirichlet(np.ones(synth.MOE_TOPK), size=T).astype(np.float32)
+    yp = torch.zeros((n_pairs, d_out), dtype=torch.int16, device="cuda")
+    y = torch.zeros((T, d_out), dtype=torch.int16, device="cuda")
+    ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_MOE, packed, n_pairs))
+    sage.sage_moe_gemv(packed, torch.from_numpy(pe).cuda(), torch.from_numpy(xrow).cuda(), n_pairs,
+                       dev_u16(spec.x_down), yp, ws)
+    sage.sage_moe_combine(T, synth.MOE_TOPK, yp, torch.from_numpy(w).cuda(), y)
+    torch.cuda.synchronize()
+    assert sage.sage_query_status(ws) == sage.SAGE_OK
+    ypb = host_u16(yp)
+    _check_combine(host_u16(y), oracle.moe_combine(ypb, w.astype(np.float64)),
+                   _combine_bound(ypb, w.astype(np.float64)))
