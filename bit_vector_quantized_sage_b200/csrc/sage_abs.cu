@@ -4,13 +4,17 @@
 // its original weights, in original channel order (Eq. 8), and the choice of
 // the split with the smallest error among candidate encodings (Eq. 9).
 //
-// One persistent grid walks the (row octet, subvector column) records of the
-// packed planes.  A thread rebuilds its record's 8 rows x 8 weights in fp32
-// (r^ = mu + q delta times the signed fp16 codeword, as the GEMV does), reads
-// the 8 original channels perm[8j .. 8j + 7] of each row of W and their
-// energies, and adds e (w - w^)^2 and e w^2 in fp64.  Each CTA reduces its
-// sums and stores them; the host adds the CTAs' partials in CTA order (the
-// result is deterministic) and divides.
+// One persistent grid, one CTA per SM, walks the row octets; within an octet
+// a thread takes subvector columns j = tid, tid + blockDim, ...  A thread
+// rebuilds its record's 8 rows x 8 weights in fp32 (r^ = mu + q delta times
+// the signed fp16 codeword, as the GEMV does), reads the 8 original channels
+// perm[8j .. 8j + 7] of each row of W and their energies, and adds
+// e (w - w^)^2 and e w^2 in fp64.  The permutation scatters a thread's W
+// reads over the octet's 8 rows, but the CTA as a whole reads every element
+// of those rows once, so they stay in L1 (8 rows of fp32 W) and each W
+// sector comes from HBM once.  Each CTA reduces its sums and stores them; the
+// host adds the CTAs' partials in CTA order (the result is deterministic)
+// and divides.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -23,10 +27,9 @@ namespace sage {
 using namespace dev;
 namespace {
 
-constexpr int kAbsThreads = 256;
-constexpr int kAbsCtasPerSm = 4;
+constexpr int kAbsThreads = 512;
 
-int abs_ctas() { return kAbsCtasPerSm * current_sm_count(); }
+int abs_ctas() { return 2 * current_sm_count(); }
 
 template <int V>
 __global__ void __launch_bounds__(kAbsThreads) abs_error_kernel(sage_matrix A, const float* __restrict__ W,
@@ -36,10 +39,8 @@ __global__ void __launch_bounds__(kAbsThreads) abs_error_kernel(sage_matrix A, c
     const int R8 = (A.d_out + 7) >> 3, S = A.d_in >> 3, G = A.d_in >> 7;
     const uint4* cb = reinterpret_cast<const uint4*>(A.codebook);
     double num = 0.0, den = 0.0;
-    const long long n = (long long)R8 * S;
-    for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < n;
-         id += (long long)gridDim.x * blockDim.x) {
-        const int b = (int)(id % R8), j = (int)(id / R8);
+    for (int b = blockIdx.x; b < R8; b += gridDim.x)
+    for (int j = threadIdx.x; j < S; j += blockDim.x) {
         const int blk = b >> 5, ob = b & 31, g = j >> 4, t = j & 15;
         const uint4 rec = __ldg(reinterpret_cast<const uint4*>(A.main + main_word(R8, S, blk, j, ob, 0)));
         const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
