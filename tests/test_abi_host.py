@@ -260,6 +260,9 @@ def test_encode_inputs_match_oracle():
     assert np.array_equal(r["Wt"], om.reshape(S, 8)[j])
     with pytest.raises(sage.SageError):
         sage.sage_encode_inputs(W, e, 0.75, np.array([d_out * S], np.int64))
+    with pytest.raises(sage.SageError) as err:
+        sage.sage_encode_inputs(W[:, :200], e[:200], 0.75, sample[:4])
+    assert err.value.status == sage.SAGE_ERR_UNSUPPORTED
 
 
 def test_pack_device_argument_errors(lib):

@@ -165,3 +165,19 @@ def test_pack_device_matches_host_packer(log2K):
                                    _dev(f.mu.view(np.int16)), _dev(f.delta.view(np.int16)))
     assert np.array_equal(dm.cpu().numpy().view(np.uint32), np.asarray(main).view(np.uint32).reshape(-1))
     assert np.array_equal(dt.cpu().numpy().view(np.uint32), np.asarray(meta).view(np.uint32).reshape(-1))
+
+
+def test_pack_device_masks_wide_fields():
+    """Field values wider than their bits (idx >= K, q >= 2^V) are masked on the
+    device, where the host packer rejects them: the planes equal the host
+    packer's planes of the masked fields."""
+    g = np.random.default_rng(77)
+    d_out, d_in, log2K = 24, 128, 5
+    f = synth.random_fields(g, d_out, d_in, log2K)
+    wide_idx = (f.idx.astype(np.uint32) | (1 << log2K)).astype(np.uint16)
+    wide_q = (f.q.astype(np.uint32) | (1 << (10 - log2K))).astype(np.uint8)
+    main, meta = sage.sage_pack(d_out, d_in, log2K, f.signs, f.idx, f.q, f.mu, f.delta)
+    dm, dt = sage.sage_pack_device(d_out, d_in, log2K, _dev(f.signs), _dev(wide_idx.view(np.int16)), _dev(wide_q),
+                                   _dev(f.mu.view(np.int16)), _dev(f.delta.view(np.int16)))
+    assert np.array_equal(dm.cpu().numpy().view(np.uint32), np.asarray(main).view(np.uint32).reshape(-1))
+    assert np.array_equal(dt.cpu().numpy().view(np.uint32), np.asarray(meta).view(np.uint32).reshape(-1))
