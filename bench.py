@@ -807,6 +807,32 @@ def run_reference(args):
     return 0
 
 
+EXTRAS = {
+    "gemm": ("up_proj_4096x12288_batch_sweep", lambda st: bench_gemm(st)),
+    "moe": ("moe_128_experts", lambda st: bench_moe(st)),
+    "qdq": ("qdq_forward_4096x4096", lambda st: bench_qdq(st)),
+    "abs": ("abs_select_4096x4096", lambda st: bench_abs(st)),
+    "encoder": ("encode_rows_4096x4096", lambda st: bench_encode_rows(st)),
+}
+
+
+def run_extras(names):
+    """The listed extra measurements alone, on one GPU (one JSON line)."""
+    import torch
+    import bit_vector_quantized_sage_b200 as sage
+    from bit_vector_quantized_sage_b200 import build as sage_build
+    sage_build.build()
+    sage.load()
+    stream = torch.cuda.Stream()
+    out = {}
+    with torch.cuda.stream(stream):
+        for n in names:
+            key, fn = EXTRAS[n]
+            out[key] = fn(stream)
+    print(json.dumps({"extra": out}))
+    return 0
+
+
 def run_gpu(args):
     import torch
     import bit_vector_quantized_sage_b200 as sage
@@ -911,11 +937,8 @@ def run_gpu(args):
     extra = {"layer_modes": layer_modes}
     if rank == 0 and world == 1 and not args.no_extra:
         with torch.cuda.stream(stream):
-            extra["up_proj_4096x12288_batch_sweep"] = bench_gemm(stream)
-            extra["moe_128_experts"] = bench_moe(stream)
-            extra["qdq_forward_4096x4096"] = bench_qdq(stream)
-            extra["abs_select_4096x4096"] = bench_abs(stream)
-            extra["encode_rows_4096x4096"] = bench_encode_rows(stream)
+            for key, fn in EXTRAS.values():
+                extra[key] = fn(stream)
 
     peak, peak_kind = _peaks()
     traffic, traffic_note = traffic_for(args.layer)
@@ -982,9 +1005,14 @@ def main():
                     help="how the layer's seven projections are launched (default: the fused decoder layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the batch sweep and MoE measurements")
+    ap.add_argument("--only-extra", default="",
+                    help="comma list of extras to run alone (gemm, moe, qdq, abs, encoder), without the layer "
+                         "measurement; prints {\"extra\": ...} (for profiling those kernels)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only_extra:
+        return run_extras(args.only_extra.split(","))
     return run_gpu(args)
 
 
