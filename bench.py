@@ -587,7 +587,7 @@ def bench_qdq(stream):
     """The continuous-parameter decode (blockwise optimisation forward) of a
     4096 x 4096 matrix at (K, V) = (64, 4): per subvector it reads rho, the
     sign byte and the index (7 B) and writes 8 fp32 weights and the radius code
-    (33 B).  HBM-bound on those writes."""
+    (33 B); reported as GB/s of those bytes against the HBM copy rate."""
     import torch
     import synth
     import bit_vector_quantized_sage_b200 as sage
