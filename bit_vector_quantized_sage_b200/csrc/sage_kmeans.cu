@@ -239,14 +239,14 @@ __global__ void kmeans_half_kernel(int n, const double* __restrict__ cb, uint16_
 using namespace sage;
 
 extern "C" size_t sage_kmeans_workspace_size(int n) {
-    if (n < 1) return 0;
+    if (n < 1 || n > (1 << 30)) return 0;
     return kKmHeader + round256((size_t)n * 4) + round256((size_t)n) + (size_t)n * 64;
 }
 
 extern "C" int sage_kmeans(int n, int log2K, const double* P, const double* Wt, const int64_t* init, int iters,
                            double* cb, uint16_t* cb16, void* ws, size_t ws_bytes, sage_stream_t stream) {
     if (!P || !Wt || !init || !cb) return SAGE_ERR_INVALID_ARGUMENT;
-    if (n < 1 || iters < 0 || log2K < 4 || log2K > 8) return SAGE_ERR_UNSUPPORTED;
+    if (n < 1 || n > (1 << 30) || iters < 0 || log2K < 4 || log2K > 8) return SAGE_ERR_UNSUPPORTED;
     if (!ws) return SAGE_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) % 16) return SAGE_ERR_MISALIGNED;
     if (ws_bytes < sage_kmeans_workspace_size(n)) return SAGE_ERR_WORKSPACE;

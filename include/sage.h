@@ -363,11 +363,11 @@ int sage_pack_device(int d_out, int d_in, int log2K, const uint8_t* signs, const
  *     zero-filled once before first use (word 0 is its status word), owned by
  *     the caller, not shared with a concurrent call.
  * Asynchronous on `stream`.  Errors: INVALID_ARGUMENT (null pointer),
- * UNSUPPORTED (n < 1, iters < 0, log2K outside 4..8), MISALIGNED, WORKSPACE,
+ * UNSUPPORTED (n outside 1..2^30, iters < 0, log2K outside 4..8), MISALIGNED, WORKSPACE,
  * CUDA; an init entry outside [0, n) is found on the device (sample 0 is read
  * in its place, the codebook is then meaningless) and sage_query_status(ws)
  * returns INVALID_ARGUMENT for it. */
-size_t sage_kmeans_workspace_size(int n);
+size_t sage_kmeans_workspace_size(int n);  /* 0 for n outside 1..2^30 */
 int sage_kmeans(int n, int log2K, const double* P, const double* Wt, const int64_t* init, int iters, double* cb,
                 uint16_t* cb16, void* ws, size_t ws_bytes, sage_stream_t stream);
 

@@ -229,6 +229,9 @@ def test_kmeans_argument_errors(lib):
     n = 1000
     need = lib.sage_kmeans_workspace_size(n)
     assert need >= 64 * n and lib.sage_kmeans_workspace_size(0) == 0
+    assert lib.sage_kmeans_workspace_size((1 << 30) + 1) == 0
+    assert lib.sage_kmeans((1 << 30) + 1, 6, 0x100000, 0x200000, 0x300000, 3, 0x400000, None, 0x800000, 1 << 40,
+                           None) == sage.SAGE_ERR_UNSUPPORTED
     a = [0x100000 * (i + 1) for i in range(4)]  # P, Wt, init, cb (never dereferenced)
     ws = 0x800000
     assert lib.sage_kmeans(n, 6, None, a[1], a[2], 3, a[3], None, ws, need, None) == sage.SAGE_ERR_INVALID_ARGUMENT
