@@ -632,7 +632,7 @@ def bench_abs(stream, reps=10):
         packed.append(sage.PackedMatrix.from_fields(f))
     W = torch.from_numpy(inp.W.astype(np.float32)).cuda()
     e = torch.from_numpy(inp.energies.astype(np.float32)).cuda()
-    ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_ABS, packed[0], 1))
+    ws = sage.Workspace(sage.sage_workspace_size(sage.SAGE_OP_ABS, packed, 1))  # all five: one sync
     best, errs = sage.sage_abs_select(packed, W, e, ws, stream)
     t = []
     for _ in range(reps):
@@ -682,7 +682,7 @@ def bench_abs(stream, reps=10):
             "best_log2K": 4 + best, "errors": [round(x, 6) for x in errs],
             "us_per_candidate": dist_summary(t), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
             "hbm_frac": round(nbytes / (us * 1e-6) / 1e9 / hbm, 4),
-            "note": "synchronous calls (each adds its CTAs' partial sums on the host)",
+            "note": "one synchronous sage_abs_select over the five candidates (the host adds each one's CTA partials)",
             "gpu_encoder_end_to_end": {
                 "what": "the five encodings on the GPU (sage_kmeans 10 rounds, sage_encode_rows, sage_pack_device) "
                         "and the Eq. 8 scores / Eq. 9 choice",

@@ -114,23 +114,13 @@ __global__ void __launch_bounds__(kAbsThreads) abs_error_kernel(sage_matrix A, c
 
 }  // namespace
 
-size_t abs_workspace_bytes() { return 256 + (size_t)abs_ctas() * 2 * sizeof(double); }
+size_t abs_partials_bytes() { return (size_t)abs_ctas() * 2 * sizeof(double); }
+size_t abs_workspace_bytes(int n) { return 256 + (size_t)(n < 1 ? 1 : n) * abs_partials_bytes(); }
 
-}  // namespace sage
+namespace {
 
-using namespace sage;
-
-extern "C" int sage_abs_error(const sage_matrix* A, const float* W, const float* energy, void* ws, size_t ws_bytes,
-                              double* err, sage_stream_t stream) {
-    int rc = check_matrix(A);
-    if (rc) return rc;
-    if (!W || !energy || !err) return SAGE_ERR_INVALID_ARGUMENT;
-    if (!ws) return SAGE_ERR_WORKSPACE;
-    if (!aligned16(ws) || !aligned16(W)) return SAGE_ERR_MISALIGNED;
-    if (ws_bytes < abs_workspace_bytes()) return SAGE_ERR_WORKSPACE;
+int abs_launch(const sage_matrix* A, const float* W, const float* energy, double* partials, cudaStream_t s) {
     const int grid = abs_ctas();
-    double* partials = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + 256);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (A->log2K) {
         case 4: abs_error_kernel<6><<<grid, kAbsThreads, 0, s>>>(*A, W, energy, partials); break;
         case 5: abs_error_kernel<5><<<grid, kAbsThreads, 0, s>>>(*A, W, energy, partials); break;
@@ -138,13 +128,13 @@ extern "C" int sage_abs_error(const sage_matrix* A, const float* W, const float*
         case 7: abs_error_kernel<3><<<grid, kAbsThreads, 0, s>>>(*A, W, energy, partials); break;
         default: abs_error_kernel<2><<<grid, kAbsThreads, 0, s>>>(*A, W, energy, partials); break;
     }
-    if (cudaGetLastError() != cudaSuccess) return SAGE_ERR_CUDA;
-    std::vector<double> h((size_t)grid * 2);
-    if (cudaMemcpyAsync(h.data(), partials, h.size() * sizeof(double), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
-        return SAGE_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+// Eq. 8 from one candidate's CTA partials, added in CTA order (deterministic).
+int abs_finish(const double* h, double* err) {
     double num = 0.0, den = 0.0;
-    for (int c = 0; c < grid; ++c) {  // CTA order: deterministic
+    for (int c = 0; c < abs_ctas(); ++c) {
         num += h[2 * c];
         den += h[2 * c + 1];
     }
@@ -153,23 +143,66 @@ extern "C" int sage_abs_error(const sage_matrix* A, const float* W, const float*
     return SAGE_OK;
 }
 
+// Scores candidates [0, n): as many per round as the workspace holds partials
+// for, one copy back and one synchronisation per round.
+int abs_score(const sage_matrix* cands, int n, const float* W, const float* energy, void* ws, size_t ws_bytes,
+              double* errs, sage_stream_t stream) {
+    if (!W || !energy || !errs) return SAGE_ERR_INVALID_ARGUMENT;
+    if (!ws) return SAGE_ERR_WORKSPACE;
+    if (!aligned16(ws) || !aligned16(W)) return SAGE_ERR_MISALIGNED;
+    if (ws_bytes < abs_workspace_bytes(1)) return SAGE_ERR_WORKSPACE;
+    for (int i = 0; i < n; ++i) {
+        const int rc = check_matrix(&cands[i]);
+        if (rc) return rc;
+    }
+    const size_t per = abs_partials_bytes();
+    const int batch = (int)std::min<size_t>((size_t)n, (ws_bytes - 256) / per);
+    double* partials = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + 256);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::vector<double> h(per / sizeof(double) * (size_t)batch);
+    for (int i0 = 0; i0 < n; i0 += batch) {
+        const int nb = std::min(batch, n - i0);
+        for (int b = 0; b < nb; ++b) {
+            const int rc = abs_launch(&cands[i0 + b], W, energy, partials + b * (per / sizeof(double)), s);
+            if (rc) return rc;
+        }
+        if (cudaMemcpyAsync(h.data(), partials, per * nb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return SAGE_ERR_CUDA;
+        for (int b = 0; b < nb; ++b) {
+            const int rc = abs_finish(h.data() + b * (per / sizeof(double)), &errs[i0 + b]);
+            if (rc) return rc;
+        }
+    }
+    return SAGE_OK;
+}
+
+}  // namespace
+
+}  // namespace sage
+
+using namespace sage;
+
+extern "C" int sage_abs_error(const sage_matrix* A, const float* W, const float* energy, void* ws, size_t ws_bytes,
+                              double* err, sage_stream_t stream) {
+    if (!A) return SAGE_ERR_INVALID_ARGUMENT;
+    if (!err) return SAGE_ERR_INVALID_ARGUMENT;
+    return abs_score(A, 1, W, energy, ws, ws_bytes, err, stream);
+}
+
 extern "C" int sage_abs_select(const sage_matrix* cands, int n, const float* W, const float* energy, void* ws,
                                size_t ws_bytes, int* best, double* errs, sage_stream_t stream) {
     if (!cands || n < 1 || !best) return SAGE_ERR_INVALID_ARGUMENT;
     for (int i = 0; i < n; ++i)
         if (cands[i].d_out != cands[0].d_out || cands[i].d_in != cands[0].d_in) return SAGE_ERR_UNSUPPORTED;
-    int arg = -1;
-    double emin = 0.0;
-    for (int i = 0; i < n; ++i) {
-        double e = 0.0;
-        const int rc = sage_abs_error(&cands[i], W, energy, ws, ws_bytes, &e, stream);
-        if (rc) return rc;
-        if (errs) errs[i] = e;
-        if (arg < 0 || e < emin) {  // Eq. 9; ties keep the earlier candidate
-            arg = i;
-            emin = e;
-        }
-    }
+    std::vector<double> e((size_t)n);
+    const int rc = abs_score(cands, n, W, energy, ws, ws_bytes, e.data(), stream);
+    if (rc) return rc;
+    int arg = 0;
+    for (int i = 1; i < n; ++i)
+        if (e[i] < e[arg]) arg = i;  // Eq. 9; ties keep the earlier candidate
+    if (errs)
+        for (int i = 0; i < n; ++i) errs[i] = e[i];
     *best = arg;
     return SAGE_OK;
 }

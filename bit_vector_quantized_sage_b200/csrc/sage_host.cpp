@@ -411,7 +411,7 @@ int sage_workspace_size(int op, const sage_matrix* mats, int n, int M, size_t* b
             return SAGE_OK;
         }
         case SAGE_OP_MOE: *bytes = moe_workspace_bytes(mats, n, M); return SAGE_OK;
-        case SAGE_OP_ABS: *bytes = abs_workspace_bytes(); return SAGE_OK;
+        case SAGE_OP_ABS: *bytes = abs_workspace_bytes(n); return SAGE_OK;
         default: return SAGE_ERR_INVALID_ARGUMENT;
     }
 }

@@ -65,7 +65,7 @@ int launch_moe(const sage_matrix* experts, int n_experts, const int32_t* pair_ex
                const int32_t* pair_xrow, int n_pairs, const uint16_t* x, uint16_t* y,
                void* ws, size_t ws_bytes, sage_stream_t stream);
 size_t moe_workspace_bytes(const sage_matrix* experts, int n_experts, int n_pairs);
-size_t abs_workspace_bytes();
+size_t abs_workspace_bytes(int n);  // partials for n candidates scored per synchronisation
 
 int launch_gemm(const sage_matrix* A, const uint16_t* x, int M, uint16_t* y,
                 void* ws, size_t ws_bytes, sage_stream_t stream);

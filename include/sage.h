@@ -384,11 +384,15 @@ int sage_kmeans(int n, int log2K, const double* P, const double* Wt, const int64
  *     energies `energy` (device fp32 [d_in]); *err is a HOST double.
  *     Synchronous: it waits for the stream and adds the CTAs' partial sums on
  *     the host in a fixed order (deterministic).  ws: device workspace of
- *     sage_workspace_size(SAGE_OP_ABS, ...) bytes.
+ *     sage_workspace_size(SAGE_OP_ABS, mats, n, ...) bytes: partial sums for
+ *     n candidates (n = 1 suffices for every call; sized for all of a
+ *     sage_abs_select's candidates, that call scores them all before one
+ *     synchronisation, otherwise as many per synchronisation as fit).
  *   sage_abs_select: Eq. 9, the index of the candidate encoding with the
  *     smallest E (ties: the earlier candidate); cands: host array of n packed
  *     encodings of the same W (one per split); errs: host double [n] or null.
- * The encodings themselves come from sage_encode, one call per split.
+ * The encodings come from sage_encode (CPU) or, on the GPU, from
+ * sage_kmeans + sage_encode_rows + sage_pack_device, one per split.
  * Errors: INVALID_ARGUMENT (null pointers, zero-energy W), UNSUPPORTED
  * (candidates of different shapes), MISALIGNED, WORKSPACE, CUDA. */
 int sage_abs_error(const sage_matrix* A, const float* W, const float* energy, void* ws, size_t ws_bytes,

@@ -72,6 +72,10 @@ def test_abs_select_matches_oracle(shape):
     packed = [sage.PackedMatrix.from_fields(f) for f in fields]
     ws = workspace_for(sage.SAGE_OP_ABS, packed[0], 1)
     best, errs = sage.sage_abs_select(packed, _dev(W32), _dev(e32), ws)
+    # a workspace for all five: scored before one synchronisation, the same bits
+    ws5 = workspace_for(sage.SAGE_OP_ABS, packed, 1)
+    assert ws5.nbytes > ws.nbytes
+    assert sage.sage_abs_select(packed, _dev(W32), _dev(e32), ws5) == (best, errs)
     ref_best, ref_errs = oracle.abs_select(fields, W32.astype(np.float64), e32.astype(np.float64))
     for a, b in zip(errs, ref_errs):
         assert abs(a - b) <= 1e-5 * b, (a, b)
