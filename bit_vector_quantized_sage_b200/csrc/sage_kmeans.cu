@@ -135,12 +135,15 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_assign_kernel(int n, int K,
 // Cluster blockIdx.x: the sum of its live members' terms in sample order
 // (threads 0..7 hold one component each), then the normalisation.  Samples
 // are scanned in chunks of kUpdChunk: the chunk's members are compacted in
-// order (warp ballots), their terms staged in shared memory by all threads
-// (one round trip for the chunk), and added in order from there; the next
-// chunk's assignments are loaded while the current one is summed.
-constexpr int kUpdPer = 2;                         // samples per thread and chunk
-constexpr int kUpdChunk = kUpdThreads * kUpdPer;   // 1024
-constexpr int kUpdSmem = kUpdChunk * 8 * 8 + kUpdChunk * 4;  // member terms + member list
+// order (warp ballots and one scan of the per-warp counts), their terms
+// staged in shared memory by all threads, up to kUpdVals members per round
+// trip, and added in order from there; the next chunk's assignments are
+// loaded while the current one is summed.
+constexpr int kUpdPer = 8;                         // samples per thread and chunk
+constexpr int kUpdChunk = kUpdThreads * kUpdPer;   // 4096
+constexpr int kUpdVals = 1024;                     // member terms staged per round trip
+constexpr int kUpdSmem = kUpdVals * 8 * 8 + kUpdChunk * 4;  // member terms + member list
+static_assert((kUpdThreads / 32) * kUpdPer == 128, "the count scan takes 4 counts per lane of one warp");
 
 __global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(int n, const int32_t* __restrict__ z,
                                                                     const uint8_t* __restrict__ live,
@@ -148,14 +151,14 @@ __global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(int n, const
                                                                     double* __restrict__ cb) {
     constexpr int NW = kUpdThreads / 32;
     extern __shared__ __align__(16) uint8_t km_smem[];
-    double* vals = reinterpret_cast<double*>(km_smem);                   // [kUpdChunk][8]
-    int* list = reinterpret_cast<int*>(km_smem + kUpdChunk * 8 * 8);   // [kUpdChunk]
-    __shared__ int wcount[NW * kUpdPer];
+    double* vals = reinterpret_cast<double*>(km_smem);                  // [kUpdVals][8]
+    int* list = reinterpret_cast<int*>(km_smem + kUpdVals * 8 * 8);    // [kUpdChunk]
+    __shared__ int wcount[NW * kUpdPer + 1];  // counts per (r, warp), then their exclusive prefix; [last] = total
     __shared__ double a[8];
     __shared__ double s_nn;
     const int k = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     double acc = 0.0;
-    // sample c0 + r * kUpdThreads + tid is this thread's r-th of the chunk
+    // sample c0 + r * kUpdThreads + tid is this thread's r-th of the chunk: (r, warp, lane) is sample order
     bool nf[kUpdPer];
 #pragma unroll
     for (int r = 0; r < kUpdPer; ++r) {
@@ -164,58 +167,73 @@ __global__ void __launch_bounds__(kUpdThreads) kmeans_update_kernel(int n, const
     }
     for (int c0 = 0; c0 < n; c0 += kUpdChunk) {
         bool f[kUpdPer];
+        unsigned bal[kUpdPer];
 #pragma unroll
         for (int r = 0; r < kUpdPer; ++r) {
             f[r] = nf[r];
             const int s = c0 + kUpdChunk + r * kUpdThreads + tid;  // the next chunk's
             nf[r] = s < n ? (live[s] != 0) & (z[s] == k) : false;
-        }
-        unsigned bal[kUpdPer];
-#pragma unroll
-        for (int r = 0; r < kUpdPer; ++r) {
             bal[r] = __ballot_sync(0xffffffffu, f[r]);
             if (lane == 0) wcount[r * NW + w] = __popc(bal[r]);
         }
         __syncthreads();
-        int total = 0, base[kUpdPer];
-        for (int q = 0; q < NW * kUpdPer; ++q) {  // members ordered by (r, warp, lane) = sample order
-            const int c = wcount[q];
+        if (w == 0) {  // exclusive scan of the 128 counts in (r, warp) order, 4 per lane
+            int c[4], sum = 0;
 #pragma unroll
-            for (int r = 0; r < kUpdPer; ++r)
-                if (q == r * NW + w) base[r] = total;
-            total += c;
+            for (int u = 0; u < 4; ++u) {
+                c[u] = wcount[lane * 4 + u];
+                sum += c[u];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            int ex = incl - sum;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                wcount[lane * 4 + u] = ex;
+                ex += c[u];
+            }
+            if (lane == 31) wcount[NW * kUpdPer] = incl;
         }
+        __syncthreads();
+        const int total = wcount[NW * kUpdPer];
 #pragma unroll
         for (int r = 0; r < kUpdPer; ++r)
-            if (f[r]) list[base[r] + __popc(bal[r] & ((1u << lane) - 1u))] = c0 + r * kUpdThreads + tid;
+            if (f[r]) list[wcount[r * NW + w] + __popc(bal[r] & ((1u << lane) - 1u))] = c0 + r * kUpdThreads + tid;
         __syncthreads();
-        if (total == 0) continue;  // uniform: every thread read the same counts
-        for (int e0 = tid; e0 < total * 8; e0 += 4 * kUpdThreads) {  // up to four terms in flight per thread
-            double t[4];
+        for (int m0 = 0; m0 < total; m0 += kUpdVals) {  // uniform: every thread read the same total
+            const int cnt = min(kUpdVals, total - m0);
+            for (int e0 = tid; e0 < cnt * 8; e0 += 4 * kUpdThreads) {  // up to four terms in flight per thread
+                double t[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * kUpdThreads;
-                t[u] = e < total * 8 ? v[(size_t)list[e >> 3] * 8 + (e & 7)] : 0.0;
-            }
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u * kUpdThreads;
+                    t[u] = e < cnt * 8 ? v[(size_t)list[m0 + (e >> 3)] * 8 + (e & 7)] : 0.0;
+                }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * kUpdThreads;
-                if (e < total * 8) vals[e] = t[u];
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u * kUpdThreads;
+                    if (e < cnt * 8) vals[e] = t[u];
+                }
             }
+            __syncthreads();
+            if (tid < 8) {
+                int m = 0;
+                for (; m + 8 <= cnt; m += 8) {
+                    double t[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) t[u] = vals[(m + u) * 8 + tid];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc = __dadd_rn(acc, t[u]);  // member order
+                }
+                for (; m < cnt; ++m) acc = __dadd_rn(acc, vals[m * 8 + tid]);
+            }
+            __syncthreads();  // the terms are rewritten next round
         }
-        __syncthreads();
-        if (tid < 8) {
-            int m = 0;
-            for (; m + 8 <= total; m += 8) {
-                double t[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) t[u] = vals[(m + u) * 8 + tid];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) acc = __dadd_rn(acc, t[u]);  // member order
-            }
-            for (; m < total; ++m) acc = __dadd_rn(acc, vals[m * 8 + tid]);
-        }
-        __syncthreads();  // list and terms are rewritten next chunk
+        // the list and the counts are rewritten next chunk only after the barriers above
     }
     if (tid < 8) a[tid] = acc;
     __syncthreads();
