@@ -14,8 +14,8 @@
 // subvector's 8 fp32 weights as two 16-byte stores (a group's 16 threads
 // write 512 contiguous bytes).  Per subvector it reads 7 bytes (rho, sign
 // byte, index) and writes 32; a 64 MB output stays in L2 during the launch,
-// so the pass is bound by each thread's dependent chain (loads, softplus,
-// group shuffles, stores) rather than by HBM.
+// so HBM is not the limit: the L1 pipe is, through the random codeword reads
+// from shared memory (hence the bank-spread layout) and the stores.
 #include <cuda_runtime.h>
 
 #include <algorithm>
