@@ -53,7 +53,8 @@ PLANTS = {
     "assign_radius_wrong": ("best_r = num / den; }", "best_r = num; }"),
     "grid_off_by_one": ("*delta16 = oracle_double_to_half((hi - lo) / (double)((1 << V) - 1));", "*delta16 = oracle_double_to_half((hi - lo) / (double)(1 << V));"),
     "quantize_truncate": ("    double qq = floor((r - mu) / d + 0.5);", "    double qq = floor((r - mu) / d);"),
-    "quantize_no_clamp_top": ("    if (qq > (double)((1 << V) - 1)) qq = (double)((1 << V) - 1);", "    if (qq > (double)((1 << V))) qq = (double)((1 << V));"),
+    "quantize_no_clamp_top": ("    if (qq < 0.0) qq = 0.0;\n    if (qq > (double)((1 << V) - 1)) qq = (double)((1 << V) - 1);",
+                              "    if (qq < 0.0) qq = 0.0;\n    if (qq > (double)((1 << V))) qq = (double)((1 << V));"),
     "omega_no_gamma": ("    for (int i = 0; i < SV; ++i) w8[i] = pow(e8[i], gamma) / mean;", "    for (int i = 0; i < SV; ++i) w8[i] = e8[i] / mean;"),
     "esg_ascending": ("    if (ea > eb) return -1;\n    if (ea < eb) return 1;", "    if (ea > eb) return 1;\n    if (ea < eb) return -1;"),
     "half_ties_away": ("    double s = nearbyint(ldexp(a, 10 - e));", "    double s = floor(ldexp(a, 10 - e) + 0.5);"),

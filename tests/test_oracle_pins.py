@@ -837,3 +837,17 @@ def test_moe_combine_closed_forms():
     w = g.random((3, 2))
     want = _h((w[:, :, None] * y.view(np.float16).astype(np.float64).reshape(3, 2, 32)).sum(axis=1))
     assert np.array_equal(oracle.moe_combine(y, w), want)
+
+
+def test_mutation_plants_apply_once():
+    """Every planted mistake of oracle/mutation_check.py names a passage that
+    occurs exactly once in the oracle's source, so the check plants what it
+    says (a second copy of a line elsewhere would make the plant ambiguous)."""
+    import importlib.util
+    import os
+    here = os.path.dirname(os.path.abspath(__file__))
+    spec = importlib.util.spec_from_file_location("mutation_check", os.path.join(here, "..", "oracle", "mutation_check.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    src = open(m.SRC).read()
+    assert {n: src.count(a) for n, (a, _) in m.PLANTS.items() if src.count(a) != 1} == {}
